@@ -1,0 +1,183 @@
+"""Seeded synthetic inputs for the DSA step, shared by the tests, the bench and
+the smoke check.
+
+This module only draws numbers and lays them out; it holds none of the
+method's arithmetic.  Every array is NumPy: bf16 tensors are raw uint16 bit
+patterns (round-to-nearest-even from float32), index tensors are int32,
+weights float32.
+
+Recipe (all configs): a NumPy Generator(PCG64(seed)) draws, in this order,
+  q_idx   integers in [-3, 3]            -> bf16   [n_q, H_I, D_I]
+  k_pages integers in [-3, 3]            -> bf16   [num_pages, 64, D_I]
+  w       integers in [0, 3]             -> float32 [n_q, H_I]
+  q       float32 standard normal        -> bf16   [n_q, H, R + P]
+  latent  float32 standard normal        -> bf16   [num_pages, 64, R + P]
+  then, when `shuffle_pages`, a permutation of the physical pages.
+Normals are drawn in fixed chunks of 2**22 values.  Sequence lengths of the
+ragged batched config are drawn first, from their own Generator(PCG64(1)),
+uniformly in [2048, 65536].  Integer index queries/keys make every fp32
+indexer score exact, as in the workloads the step is quoted on.
+"""
+
+from __future__ import annotations
+
+import math
+from dataclasses import dataclass, field, replace
+
+import numpy as np
+
+PAGE_SIZE = 64
+_CHUNK = 1 << 22
+
+
+@dataclass(frozen=True)
+class Workload:
+    name: str
+    mode: str                 # "decode" or "prefill"
+    seq_lens: tuple           # decode: per-sequence context (incl. current token)
+    n_q: int                  # query rows (decode: B; prefill: T)
+    H_I: int
+    D_I: int
+    topk: int
+    H: int
+    R: int
+    P: int
+    scale: float
+    seed: int = 0
+    shuffle_pages: bool = False
+    q_pos0: int = 0           # prefill: absolute position of query row 0
+    value_kind: str = "int"   # "int": index q/k integers; "normal": bf16 N(0,1)
+    description: str = ""
+
+    @property
+    def W(self) -> int:
+        return self.R + self.P
+
+    @property
+    def num_seqs(self) -> int:
+        return len(self.seq_lens)
+
+
+def ragged_lengths(batch: int, lo: int, hi: int, seed: int) -> tuple:
+    rng = np.random.Generator(np.random.PCG64(seed))
+    return tuple(int(x) for x in rng.integers(lo, hi + 1, size=batch))
+
+
+CONFIGS = {
+    "tiny_decode": Workload(
+        name="tiny_decode", mode="decode", seq_lens=(4096,), n_q=1, H_I=4, D_I=32,
+        topk=256, H=4, R=64, P=16, scale=1.0 / math.sqrt(80.0), seed=0,
+        description="batch 1, context 4,096; indexer 4x32; top-k 256; MLA 4 heads, latent 64+16"),
+    "glm5_decode_8k": Workload(
+        name="glm5_decode_8k", mode="decode", seq_lens=(8192,), n_q=1, H_I=32, D_I=128,
+        topk=2048, H=64, R=512, P=64, scale=1.0 / math.sqrt(192.0), seed=0,
+        description="batch 1, context 8,192; indexer 32x128; top-k 2,048; MLA 64 heads, 512+64"),
+    "glm5_decode_b32_ragged": Workload(
+        name="glm5_decode_b32_ragged", mode="decode",
+        seq_lens=ragged_lengths(32, 2048, 65536, 1), n_q=32, H_I=32, D_I=128,
+        topk=2048, H=64, R=512, P=64, scale=1.0 / math.sqrt(192.0), seed=2,
+        shuffle_pages=True,
+        description="batch 32, contexts U[2,048, 65,536] (seed 1), shuffled 64-token pages"),
+    "glm5_prefill_2300": Workload(
+        name="glm5_prefill_2300", mode="prefill", seq_lens=(2300,), n_q=2300, H_I=32,
+        D_I=128, topk=2048, H=64, R=512, P=64, scale=1.0 / math.sqrt(192.0), seed=0,
+        description="causal prefill chunk of 2,300 tokens; top-k 2,048 per row"),
+    "glm5_decode_4x128k": Workload(
+        name="glm5_decode_4x128k", mode="decode", seq_lens=(131072,) * 4, n_q=4, H_I=32,
+        D_I=128, topk=2048, H=64, R=512, P=64, scale=1.0 / math.sqrt(192.0), seed=0,
+        description="batch 4, context 131,072 each; indexer key scan dominates"),
+}
+CONFIG_ORDER = ["tiny_decode", "glm5_decode_8k", "glm5_decode_b32_ragged",
+                "glm5_prefill_2300", "glm5_decode_4x128k"]
+
+
+def f32_to_bf16_bits(x: np.ndarray) -> np.ndarray:
+    """Round float32 values to bf16 (round to nearest, ties to even); uint16 bits."""
+    u = np.ascontiguousarray(x, dtype=np.float32).view(np.uint32)
+    rounding = ((u >> 16) & 1) + np.uint32(0x7FFF)
+    return ((u + rounding) >> 16).astype(np.uint16)
+
+
+def _ints_bf16(rng, lo, hi, shape):
+    vals = rng.integers(lo, hi + 1, size=shape).astype(np.float32)
+    return f32_to_bf16_bits(vals)
+
+
+def _normal_bf16(rng, shape):
+    n = int(np.prod(shape))
+    out = np.empty(n, dtype=np.uint16)
+    for start in range(0, n, _CHUNK):
+        m = min(_CHUNK, n - start)
+        out[start:start + m] = f32_to_bf16_bits(rng.standard_normal(m, dtype=np.float32))
+    return out.reshape(shape)
+
+
+def pages_needed(n_tokens: int) -> int:
+    return (n_tokens + PAGE_SIZE - 1) // PAGE_SIZE
+
+
+def make_inputs(wl: Workload) -> dict:
+    """Draw the arrays of one workload.  Returns a dict of NumPy arrays and scalars."""
+    rng = np.random.Generator(np.random.PCG64(wl.seed))
+    if wl.mode == "decode":
+        lens = list(wl.seq_lens)
+        assert len(lens) == wl.n_q
+    else:
+        lens = [wl.q_pos0 + wl.n_q]
+    npages = [pages_needed(n) for n in lens]
+    num_pages = int(sum(npages))
+    max_pages = max(1, max(npages))
+
+    if wl.value_kind == "int":
+        q_idx = _ints_bf16(rng, -3, 3, (wl.n_q, wl.H_I, wl.D_I))
+        k_pages = _ints_bf16(rng, -3, 3, (num_pages, PAGE_SIZE, wl.D_I))
+    else:
+        q_idx = _normal_bf16(rng, (wl.n_q, wl.H_I, wl.D_I))
+        k_pages = _normal_bf16(rng, (num_pages, PAGE_SIZE, wl.D_I))
+    w = rng.integers(0, 4, size=(wl.n_q, wl.H_I)).astype(np.float32)
+    q = _normal_bf16(rng, (wl.n_q, wl.H, wl.W))
+    latent_pages = _normal_bf16(rng, (num_pages, PAGE_SIZE, wl.W))
+
+    phys = np.arange(num_pages, dtype=np.int64)
+    if wl.shuffle_pages:
+        phys = rng.permutation(num_pages)
+    block_table = np.full((len(lens), max_pages), -1, dtype=np.int32)
+    start = 0
+    for b, npg in enumerate(npages):
+        block_table[b, :npg] = phys[start:start + npg]
+        start += npg
+
+    return {
+        "mode": wl.mode,
+        "q_idx": q_idx, "w": w, "k_pages": k_pages,
+        "q": q, "latent_pages": latent_pages,
+        "block_table": block_table,
+        "seq_lens": np.asarray(lens, dtype=np.int32),
+        "topk": wl.topk, "R": wl.R, "P": wl.P, "H": wl.H,
+        "H_I": wl.H_I, "D_I": wl.D_I, "scale": wl.scale,
+        "q_pos0": wl.q_pos0, "n_q": wl.n_q,
+    }
+
+
+def small_decode(seq_lens, *, H_I=4, D_I=32, topk=64, H=8, R=64, P=16, seed=0,
+                 shuffle_pages=True, value_kind="int", scale=None) -> Workload:
+    """A small decode workload for parity tests (several tiles, ragged tails)."""
+    W = R + P
+    return Workload(name="small_decode", mode="decode", seq_lens=tuple(seq_lens),
+                    n_q=len(seq_lens), H_I=H_I, D_I=D_I, topk=topk, H=H, R=R, P=P,
+                    scale=(1.0 / math.sqrt(W)) if scale is None else scale, seed=seed,
+                    shuffle_pages=shuffle_pages, value_kind=value_kind)
+
+
+def small_prefill(T, *, q_pos0=0, H_I=4, D_I=32, topk=64, H=8, R=64, P=16, seed=0,
+                  shuffle_pages=True, value_kind="int", scale=None) -> Workload:
+    W = R + P
+    return Workload(name="small_prefill", mode="prefill", seq_lens=(q_pos0 + T,), n_q=T,
+                    H_I=H_I, D_I=D_I, topk=topk, H=H, R=R, P=P,
+                    scale=(1.0 / math.sqrt(W)) if scale is None else scale, seed=seed,
+                    shuffle_pages=shuffle_pages, q_pos0=q_pos0, value_kind=value_kind)
+
+
+__all__ = ["Workload", "CONFIGS", "CONFIG_ORDER", "make_inputs", "f32_to_bf16_bits",
+           "small_decode", "small_prefill", "ragged_lengths", "pages_needed", "PAGE_SIZE",
+           "replace", "field"]

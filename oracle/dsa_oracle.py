@@ -1,0 +1,258 @@
+"""Float64 CPU oracle for the DSA sparse-attention step (TEST INFRASTRUCTURE ONLY).
+
+This module is the plain, slow definition that the CUDA library is checked
+against.  Only the test suite, the smoke check and the CPU-baseline leg of the
+benchmark may import it; the product path never does, and this module imports
+nothing from the product.  It shares no code, tables or constants with the CUDA
+kernels: inputs arrive as NumPy arrays (bf16 values as raw uint16 bits) and
+every step is written out in float64.
+
+What it computes (one query row):
+
+1. Indexer scores.  "GLM on an A100, in Vx", section "The model": a separate
+   indexer scores every earlier token; section "How do we know it is right?":
+   the indexer applies a ReLU per indexer head before the heads are combined.
+   Reading used here: score[s] = sum_h w[h] * max(0, q_idx[h] . k_idx[s]),
+   one index key per token shared by all indexer heads, no extra scale.
+2. Exact top-k.  Same page, "The model": each query keeps the 2,048 highest
+   scores, everything when fewer tokens exist; "How do we know it is right?":
+   ties resolve like a stable argsort of -scores (lower token index first).
+   "Self-contained GLM-5 serving stack ..." names exact heap selection among
+   its implemented optimizations; the oracle selects with a heap.
+   The kept indices are emitted in ascending token order, padded with -1.
+3. Absorbed MLA attention over the compressed latent rows of the kept tokens
+   only.  "Self-contained GLM-5 serving stack ...", file list (glm_vx/model.py):
+   absorbed MLA decode over compressed request-local KV; "GLM on an A100, in
+   Vx", "The model": keys and values are compressed into one small latent
+   vector per token.  Each latent row is [c_kv (R) | k_rope (P)]; the absorbed
+   query has the same layout; V is the c_kv part.
+   z[h, j] = scale * q[h, :] . L[sel_j, :];  p = softmax_j(z);
+   out[h, :] = sum_j p[h, j] * L[sel_j, :R];  lse[h] = log sum_j exp(z[h, j]).
+
+Every function here is pinned by tests that do not re-type its formula:
+hand-computed golden values, closed forms, brute force over all subsets on
+tiny inputs, the stable-argsort library rule, dense-vs-sparse and
+absorbed-vs-non-absorbed identities, and special cases.
+"""
+
+from __future__ import annotations
+
+import heapq
+import math
+
+import numpy as np
+
+PAGE_SIZE = 64
+
+
+# --------------------------------------------------------------------------
+# bf16 decoding of the input bits (exact widening)
+# --------------------------------------------------------------------------
+
+def bf16_to_f64(bits: np.ndarray) -> np.ndarray:
+    """Widen raw bf16 bit patterns (uint16) to float64 exactly.
+
+    A bf16 value is the upper half of an IEEE binary32; placing the 16 bits
+    in the high half of a 32-bit word and reading it as float32 is exact, and
+    float32 -> float64 is exact.
+    """
+    bits = np.asarray(bits, dtype=np.uint16)
+    return (bits.astype(np.uint32) << 16).view(np.float32).astype(np.float64)
+
+
+# --------------------------------------------------------------------------
+# paged cache lookup
+# --------------------------------------------------------------------------
+
+def gather_paged_rows(pages: np.ndarray, block_table_row: np.ndarray,
+                      positions) -> np.ndarray:
+    """Rows of a paged cache at the given token positions of one sequence.
+
+    pages: [num_pages, PAGE_SIZE, width]; block_table_row: physical page id of
+    each logical page of the sequence.  Token position s lives in logical page
+    s // PAGE_SIZE, slot s % PAGE_SIZE.
+    """
+    pos = np.asarray(positions, dtype=np.int64).reshape(-1)
+    phys = np.asarray(block_table_row, dtype=np.int64)[pos // PAGE_SIZE]
+    return pages[phys, pos % PAGE_SIZE]
+
+
+# --------------------------------------------------------------------------
+# step 1: indexer scores
+# --------------------------------------------------------------------------
+
+def indexer_scores(q_idx: np.ndarray, w: np.ndarray, k_idx: np.ndarray) -> np.ndarray:
+    """score[s] = sum_h w[h] * relu(q_idx[h] . k_idx[s]) in float64.
+
+    q_idx: [H_I, D_I] float64; w: [H_I] float64; k_idx: [n, D_I] float64.
+    Returns [n] float64.
+    """
+    q_idx = np.asarray(q_idx, dtype=np.float64)
+    k_idx = np.asarray(k_idx, dtype=np.float64)
+    w = np.asarray(w, dtype=np.float64)
+    dots = k_idx @ q_idx.T                 # [n, H_I]: one dot per key and head
+    relu = np.where(dots > 0.0, dots, 0.0)  # ReLU per indexer head
+    return relu @ w                         # head-weighted sum
+
+
+# --------------------------------------------------------------------------
+# step 2: exact top-k with the stable tie rule
+# --------------------------------------------------------------------------
+
+def topk_select(scores, k: int) -> np.ndarray:
+    """Indices of the k best tokens, ascending, padded with -1 to length k.
+
+    "Best" follows a stable argsort of -scores: a higher score first, and at
+    equal scores the lower token index first.  With n <= k every token is kept.
+    Scores are compared as float64 values, so -0.0 and +0.0 are equal.
+    """
+    scores = [float(x) for x in scores]
+    n = len(scores)
+    out = np.full(k, -1, dtype=np.int64)
+    if n <= k:
+        out[:n] = np.arange(n)
+        return out
+    # a heap selection of the k smallest keys (-score, index)
+    chosen = heapq.nsmallest(k, range(n), key=lambda s: (-scores[s], s))
+    out[:] = sorted(chosen)
+    return out
+
+
+# --------------------------------------------------------------------------
+# step 3: absorbed MLA over the selected latent rows
+# --------------------------------------------------------------------------
+
+def mla_attention(q: np.ndarray, rows: np.ndarray, R: int, scale: float):
+    """Absorbed MLA attention of one query row over the given latent rows.
+
+    q: [H, W] float64 absorbed query ([latent part R | rope part P]);
+    rows: [n, W] float64 latent rows, n >= 1.
+    Returns (out [H, R], lse [H], p [H, n]) in float64, lse in natural log.
+    """
+    q = np.asarray(q, dtype=np.float64)
+    rows = np.asarray(rows, dtype=np.float64)
+    z = scale * (q @ rows.T)                       # [H, n] logits
+    m = z.max(axis=1, keepdims=True)               # stable softmax: subtract the max
+    e = np.exp(z - m)
+    l = e.sum(axis=1, keepdims=True)
+    p = e / l
+    out = p @ rows[:, :R]                          # V is the c_kv part of the latent
+    lse = m[:, 0] + np.log(l[:, 0])
+    return out, lse, p
+
+
+def dense_mla_attention(q: np.ndarray, latent: np.ndarray, R: int, scale: float):
+    """MLA attention of one query over ALL given latent rows, no selection.
+
+    Written separately from mla_attention (explicit per-head loops over the
+    keys) so that the sparse == dense identity below the top-k size compares
+    two independent routines.
+    """
+    q = np.asarray(q, dtype=np.float64)
+    latent = np.asarray(latent, dtype=np.float64)
+    H = q.shape[0]
+    n = latent.shape[0]
+    out = np.zeros((H, R))
+    lse = np.zeros(H)
+    for h in range(H):
+        logits = [scale * float(np.dot(q[h], latent[j])) for j in range(n)]
+        top = max(logits)
+        weights = [math.exp(x - top) for x in logits]
+        total = math.fsum(weights)
+        acc = np.zeros(R)
+        for j in range(n):
+            acc += (weights[j] / total) * latent[j, :R]
+        out[h] = acc
+        lse[h] = top + math.log(total)
+    return out, lse
+
+
+def mla_attention_nonabsorbed(q_nope, q_rope, c_kv, k_rope, W_UK, W_UV, scale):
+    """Standard (non-absorbed) multi-head attention that MLA absorption rewrites.
+
+    Per head h: k_h[s] = [W_UK[h] @ c_kv[s] | k_rope[s]], v_h[s] = c_kv[s] @ W_UV[h],
+    q_h = [q_nope[h] | q_rope[h]]; out_h = softmax(scale * q_h . k_h) @ v_h.
+    q_nope [H, d_nope], q_rope [H, P], c_kv [n, R], k_rope [n, P],
+    W_UK [H, d_nope, R], W_UV [H, R, d_v].  Returns (out [H, d_v], lse [H]).
+    """
+    H = q_nope.shape[0]
+    n = c_kv.shape[0]
+    d_v = W_UV.shape[2]
+    out = np.zeros((H, d_v))
+    lse = np.zeros(H)
+    for h in range(H):
+        k_nope = c_kv @ W_UK[h].T                   # [n, d_nope]
+        keys = np.concatenate([k_nope, k_rope], axis=1)
+        query = np.concatenate([q_nope[h], q_rope[h]])
+        values = c_kv @ W_UV[h]                     # [n, d_v]
+        z = scale * (keys @ query)
+        m = z.max()
+        e = np.exp(z - m)
+        out[h] = (e / e.sum()) @ values
+        lse[h] = m + np.log(e.sum())
+    return out, lse
+
+
+def absorb_query(q_nope, q_rope, W_UK):
+    """Absorbed query [H, R + P]: q_lat[h] = W_UK[h]^T q_nope[h], rope part unchanged."""
+    H = q_nope.shape[0]
+    q_lat = np.stack([W_UK[h].T @ q_nope[h] for h in range(H)])
+    return np.concatenate([q_lat, q_rope], axis=1)
+
+
+# --------------------------------------------------------------------------
+# the whole step
+# --------------------------------------------------------------------------
+
+def dsa_query(q_idx, w, k_rows, q, latent_of, k: int, R: int, scale: float):
+    """One query row of the DSA step over its own context (float64 inputs).
+
+    q_idx [H_I, D_I], w [H_I], k_rows [n, D_I] (index keys of tokens 0..n-1),
+    q [H, W]; latent_of(positions) returns the float64 latent rows [len, W] of
+    those token positions.  Returns dict(scores, idx, out, lse).
+    """
+    scores = indexer_scores(q_idx, w, k_rows)
+    idx = topk_select(scores, k)
+    sel = idx[idx >= 0]
+    out, lse, _ = mla_attention(q, latent_of(sel), R, scale)
+    return {"scores": scores, "idx": idx, "out": out, "lse": lse}
+
+
+def _query_row(inp, r, table_row, n):
+    k_rows = bf16_to_f64(gather_paged_rows(inp["k_pages"], table_row, np.arange(n)))
+
+    def latent_of(sel):
+        return bf16_to_f64(gather_paged_rows(inp["latent_pages"], table_row, sel))
+
+    return dsa_query(bf16_to_f64(inp["q_idx"][r]), np.asarray(inp["w"][r], np.float64),
+                     k_rows, bf16_to_f64(inp["q"][r]), latent_of,
+                     int(inp["topk"]), int(inp["R"]), float(inp["scale"]))
+
+
+def dsa_decode(inp: dict, rows=None) -> dict:
+    """Decode step over a paged cache, from the raw input arrays.
+
+    inp keys: q_idx [B, H_I, D_I] u16, w [B, H_I] f32, k_pages [pages, 64, D_I] u16,
+    q [B, H, W] u16, latent_pages [pages, 64, W] u16, block_table [B, maxp] i32,
+    seq_lens [B] i32, topk, R, scale.  The query of sequence b sits at position
+    seq_lens[b] - 1 and sees tokens 0..seq_lens[b]-1.  `rows` restricts the
+    computation to those sequences.
+    """
+    B = inp["q_idx"].shape[0]
+    rows = range(B) if rows is None else rows
+    return {int(b): _query_row(inp, b, inp["block_table"][b], int(inp["seq_lens"][b]))
+            for b in rows}
+
+
+def dsa_prefill(inp: dict, rows=None) -> dict:
+    """Causal prefill of one sequence: query row t sits at position q_pos0 + t
+    and sees tokens 0..q_pos0+t (diagonal included).
+
+    inp keys as in dsa_decode, with q_idx [T, H_I, D_I], w [T, H_I], q [T, H, W],
+    a single block-table row block_table [1, maxp] and q_pos0.
+    """
+    T = inp["q_idx"].shape[0]
+    rows = range(T) if rows is None else rows
+    q_pos0 = int(inp.get("q_pos0", 0))
+    return {int(t): _query_row(inp, t, inp["block_table"][0], q_pos0 + int(t) + 1)
+            for t in rows}
