@@ -1,0 +1,468 @@
+#!/usr/bin/env python
+"""Benchmark of the DSA sparse-attention step on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+                    [--config NAME] [--no-extra]
+
+One step = one dsa_attention_forward call (indexer scores -> exact top-k ->
+sparse MLA -> split combine) over one batch of synthetic GLM-5-shaped input
+already resident in HBM.  The headline workload is the GLM-5-width decode
+(batch 1, context 8,192); every other workload is measured too and reported
+under "per_config".  L2 is flushed (a 512 MB write) before every timed step;
+each step is timed with CUDA events on the launching stream; multi-GPU runs
+are independent replicas (weak scaling) timed as the max over ranks.
+
+`--impl reference` times the float64 CPU oracle on this host's cores on the
+same workload (bounded samples), with the same JSON keys.
+"""
+
+from __future__ import annotations
+
+import argparse
+import json
+import math
+import os
+import statistics
+import sys
+import threading
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import dsa_inputs as di  # noqa: E402
+
+HEADLINE = "glm5_decode_8k"
+EXTRA = ["tiny_decode", "glm5_decode_b32_ragged", "glm5_prefill_2300", "glm5_decode_4x128k"]
+NOMINAL_HBM_GBS = 8000.0
+FLUSH_BYTES = 512 << 20
+
+
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            d = json.load(f)
+        return {"hbm_gbs": float(d["hbm_gbs"]), "bf16_tflops": float(d["bf16_tflops"]),
+                "bf16_tflops_sustained": float(d.get("bf16_tflops_sustained", d["bf16_tflops"])),
+                "source": "measured"}
+    except Exception:
+        return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0,
+                "source": "fallback"}
+
+
+# ---------------------------------------------------------------------------
+# workload arithmetic (algorithmic bytes / flops)
+# ---------------------------------------------------------------------------
+
+def row_lengths(wl):
+    if wl.mode == "prefill":
+        return [wl.q_pos0 + t + 1 for t in range(wl.n_q)]
+    return list(wl.seq_lens)
+
+
+def algorithmic(wl):
+    """Must-move bytes and flops of one step (scores and page tables excluded)."""
+    lens = row_lengths(wl)
+    keys = sum(lens)
+    sel = sum(min(wl.topk, n) for n in lens)
+    b_keys = keys * wl.D_I * 2
+    b_lat = sel * wl.W * 2
+    b_small = wl.n_q * (wl.H * wl.W * 2 + wl.H_I * wl.D_I * 2 + wl.H_I * 4 + wl.H * wl.R * 4
+                        + wl.H * 4)
+    if wl.mode == "prefill":   # every row reads the same (L2-resident) cache
+        b_keys = (wl.q_pos0 + wl.n_q) * wl.D_I * 2
+        b_lat = (wl.q_pos0 + wl.n_q) * wl.W * 2
+    flops_idx = 2 * wl.H_I * wl.D_I * keys
+    flops_mla = sel * wl.H * 2 * (wl.W + wl.R)
+    # indexer kernel alone: key rows read + fp32 score per key written
+    b_indexer = keys * (wl.D_I * 2 + 4) + wl.n_q * wl.H_I * (wl.D_I * 2 + 4)
+    if wl.mode == "prefill":
+        b_indexer = (wl.q_pos0 + wl.n_q) * wl.D_I * 2 + keys * 4
+    return {"bytes": b_keys + b_lat + b_small, "bytes_keys": b_keys, "bytes_latent": b_lat,
+            "flops": flops_idx + flops_mla, "flops_indexer": flops_idx, "flops_mla": flops_mla,
+            "bytes_indexer": b_indexer, "keys": keys, "selected": sel}
+
+
+# ---------------------------------------------------------------------------
+# clocks (NVML, read only)
+# ---------------------------------------------------------------------------
+
+class ClockSampler:
+    REASONS = {"hw_slowdown": 0x8, "sw_thermal_slowdown": 0x20, "hw_thermal_slowdown": 0x40,
+               "sw_power_cap": 0x4, "hw_power_brake_slowdown": 0x80}
+
+    def __init__(self, device_index: int, period_s: float = 0.01):
+        self.samples, self.reasons = [], set()
+        self.max_mhz = None
+        self._stop = threading.Event()
+        self._ok = False
+        try:
+            import pynvml
+            pynvml.nvmlInit()
+            self._nv = pynvml
+            self._h = pynvml.nvmlDeviceGetHandleByIndex(device_index)
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self._h, pynvml.NVML_CLOCK_SM)
+            self._ok = True
+        except Exception:
+            self._nv = None
+        self._period = period_s
+        self._thr = threading.Thread(target=self._run, daemon=True)
+
+    def _run(self):
+        while not self._stop.is_set():
+            try:
+                self.samples.append(self._nv.nvmlDeviceGetClockInfo(self._h, self._nv.NVML_CLOCK_SM))
+                r = self._nv.nvmlDeviceGetCurrentClocksEventReasons(self._h)
+                for name, bit in self.REASONS.items():
+                    if r & bit:
+                        self.reasons.add(name)
+            except Exception:
+                pass
+            time.sleep(self._period)
+
+    def __enter__(self):
+        if self._ok:
+            self._thr.start()
+        return self
+
+    def __exit__(self, *a):
+        self._stop.set()
+        if self._ok:
+            self._thr.join()
+
+    def summary(self):
+        if not self.samples:
+            return {"sm_mhz": None, "sm_max_mhz": self.max_mhz, "reasons": sorted(self.reasons),
+                    "samples": 0}
+        return {"sm_mhz": float(statistics.median(self.samples)), "sm_max_mhz": self.max_mhz,
+                "reasons": sorted(self.reasons), "samples": len(self.samples)}
+
+
+# ---------------------------------------------------------------------------
+# GPU arm
+# ---------------------------------------------------------------------------
+
+class Case:
+    """Device-resident inputs, outputs and workspace of one workload."""
+
+    def __init__(self, wl, torch, dsa, seed_offset=0):
+        if seed_offset:
+            wl = di.replace(wl, seed=wl.seed + seed_offset)
+        self.wl = wl
+        self.inp = di.make_inputs(wl)
+        inp = self.inp
+        dev = "cuda"
+
+        def bf(x):
+            return torch.from_numpy(np.ascontiguousarray(x).view(np.int16)).view(torch.bfloat16).to(dev)
+
+        self.t = {"q_idx": bf(inp["q_idx"]), "k_pages": bf(inp["k_pages"]), "q": bf(inp["q"]),
+                  "latent_pages": bf(inp["latent_pages"]), "w": torch.from_numpy(inp["w"]).to(dev),
+                  "block_table": torch.from_numpy(inp["block_table"]).to(dev),
+                  "seq_lens": torch.from_numpy(inp["seq_lens"]).to(dev)}
+        self.cache = dsa.PagedCache(self.t["seq_lens"], self.t["block_table"],
+                                    num_pages=int(inp["k_pages"].shape[0]),
+                                    max_seq_len=int(inp["seq_lens"].max()))
+        self.dims = dsa.Dims(n_q=wl.n_q, H_I=wl.H_I, D_I=wl.D_I, topk=wl.topk, H=wl.H, R=wl.R,
+                             P=wl.P, causal=int(wl.mode == "prefill"), q_pos0=wl.q_pos0,
+                             scale=wl.scale)
+        self.idx = torch.empty((wl.n_q, wl.topk), dtype=torch.int32, device=dev)
+        self.out = torch.empty((wl.n_q, wl.H, wl.R), dtype=torch.float32, device=dev)
+        self.lse = torch.empty((wl.n_q, wl.H), dtype=torch.float32, device=dev)
+        self.ws = dsa.workspace(dsa.OP_ATTENTION_FORWARD, self.dims, self.cache)
+        ld = max(4, (max(row_lengths(wl)) + 3) // 4 * 4)
+        self.scores = torch.empty((wl.n_q, ld), dtype=torch.float32, device=dev)
+        self.dsa = dsa
+        self.torch = torch
+
+    def step(self):
+        t = self.t
+        self.dsa.dsa_attention_forward(t["q_idx"], t["w"], t["k_pages"], t["q"], t["latent_pages"],
+                                       self.cache, self.dims, self.idx, self.out, self.lse, self.ws)
+
+    def indexer(self):
+        t = self.t
+        self.dsa.dsa_indexer_scores(t["q_idx"], t["w"], t["k_pages"], self.cache, self.dims,
+                                    self.scores, self.ws)
+
+    def launches_per_step(self):
+        # indexer + top-k + MLA, plus the split combine when a row is split
+        # (the same split rule as the library's launcher)
+        n_q, topk = self.wl.n_q, self.wl.topk
+        sms = self.torch.cuda.get_device_properties(0).multi_processor_count
+        nchunks = (topk + 127) // 128
+        want = max(1, min((sms + n_q - 1) // n_q, min(nchunks, 64)))
+        cps = (nchunks + want - 1) // want
+        nsplit = (nchunks + cps - 1) // cps
+        return 3 + (1 if nsplit > 1 else 0)
+
+
+def timed_events(torch, fn, steps, warmup, flush_buf):
+    """Mean ms of fn over `steps` runs, each preceded (untimed) by an L2 flush."""
+    for _ in range(warmup):
+        flush_buf.add_(1)
+        fn()
+    torch.cuda.synchronize()
+    starts = [torch.cuda.Event(enable_timing=True) for _ in range(steps)]
+    ends = [torch.cuda.Event(enable_timing=True) for _ in range(steps)]
+    for i in range(steps):
+        flush_buf.add_(1)
+        starts[i].record()
+        fn()
+        ends[i].record()
+    torch.cuda.synchronize()
+    times = [s.elapsed_time(e) for s, e in zip(starts, ends)]
+    return sum(times) / len(times), times
+
+
+def measure(case, torch, steps, warmup, flush_buf, peaks):
+    wl = case.wl
+    alg = algorithmic(wl)
+    ms, _ = timed_events(torch, case.step, steps, warmup, flush_buf)
+    st, info = case.dsa.workspace_check(case.ws)
+    if st != 0:
+        raise RuntimeError(f"device status {st} ({info:#x}) on {wl.name}")
+    ms_idx, _ = timed_events(torch, case.indexer, steps, warmup, flush_buf)
+    s = ms * 1e-3
+    res = {
+        "workload": wl.name, "mode": wl.mode, "us_per_step": ms * 1e3,
+        "tokens_per_s": wl.n_q / s,
+        "alg_bytes": alg["bytes"], "alg_gbs": alg["bytes"] / s / 1e9,
+        "frac_of_8tbs": alg["bytes"] / s / 1e9 / NOMINAL_HBM_GBS,
+        "frac_of_measured_hbm": alg["bytes"] / s / 1e9 / peaks["hbm_gbs"],
+        "tflops": alg["flops"] / s / 1e12,
+        "frac_of_bf16_peak": alg["flops"] / s / 1e12 / peaks["bf16_tflops"],
+        "indexer_us": ms_idx * 1e3,
+        "indexer_alg_bytes": alg["bytes_indexer"],
+        "indexer_gbs": alg["bytes_indexer"] / (ms_idx * 1e-3) / 1e9,
+        "indexer_frac_of_measured_hbm": alg["bytes_indexer"] / (ms_idx * 1e-3) / 1e9 / peaks["hbm_gbs"],
+        "launches_per_step": case.launches_per_step(),
+    }
+    return res
+
+
+def measure_e2e(case, torch, steps, warmup):
+    """Same metric through the public API with host buffers: pinned-host
+    inputs copied in and results copied out inside the timed region."""
+    t = case.t
+    names_in = ["q_idx", "w", "q", "seq_lens", "block_table"]
+    host_in = {k: t[k].cpu().pin_memory() for k in names_in}
+    host_out = {"idx": torch.empty_like(case.idx, device="cpu").pin_memory(),
+                "out": torch.empty_like(case.out, device="cpu").pin_memory(),
+                "lse": torch.empty_like(case.lse, device="cpu").pin_memory()}
+    h2d = sum(v.numel() * v.element_size() for v in host_in.values())
+    d2h = sum(v.numel() * v.element_size() for v in host_out.values())
+
+    def one():
+        for k in names_in:
+            t[k].copy_(host_in[k], non_blocking=True)
+        case.step()
+        host_out["idx"].copy_(case.idx, non_blocking=True)
+        host_out["out"].copy_(case.out, non_blocking=True)
+        host_out["lse"].copy_(case.lse, non_blocking=True)
+
+    for _ in range(warmup):
+        one()
+    torch.cuda.synchronize()
+    ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    ev0.record()
+    for _ in range(steps):
+        one()
+    ev1.record()
+    torch.cuda.synchronize()
+    ms = ev0.elapsed_time(ev1) / steps
+    return {"value": case.wl.n_q / (ms * 1e-3), "unit": "tokens/s", "ms_per_step": ms,
+            "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h)}
+
+
+def oracle_rows_per_s(wl, budget_s: float):
+    """Time the float64 oracle on whole query rows of `wl` for ~budget_s."""
+    from oracle import dsa_oracle as orc
+    inp = di.make_inputs(wl)
+    fn = orc.dsa_prefill if wl.mode == "prefill" else orc.dsa_decode
+    rows = list(range(wl.n_q))
+    if wl.mode == "prefill":   # rows past the top-k size exercise the selection
+        rows = rows[::-1]
+    done, t0 = 0, time.perf_counter()
+    while True:
+        fn(inp, [rows[done % len(rows)]])
+        done += 1
+        el = time.perf_counter() - t0
+        if el >= budget_s:
+            break
+    return done / el, done, el
+
+
+def blas_threads():
+    try:
+        from threadpoolctl import threadpool_info
+        info = threadpool_info()
+        n = [i.get("num_threads", 1) for i in info if i.get("user_api") == "blas"]
+        return int(max(n)) if n else 1
+    except Exception:
+        return os.cpu_count() or 1
+
+
+def cpu_baseline(wl, budget_s=10.0):
+    rate, n, el = oracle_rows_per_s(wl, budget_s)
+    return {"value": rate, "unit": "tokens/s", "cores": blas_threads(), "kind": "oracle",
+            "sample": f"{n} query rows of {wl.name} through the float64 oracle in {el:.1f} s "
+                      f"(host: {os.cpu_count()} logical cores)"}
+
+
+def run_ours(args):
+    import torch
+    import torch.distributed as dist
+
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    torch.cuda.set_device(local)
+    if world > 1:
+        from datetime import timedelta
+        dist.init_process_group("nccl", timeout=timedelta(seconds=300),
+                                device_id=torch.device("cuda", local))
+    import sparse_attention_scores_b200 as dsa
+    dsa.lib()
+    peaks = load_peaks()
+    flush_buf = torch.empty(FLUSH_BYTES // 4, dtype=torch.float32, device="cuda")
+
+    wl = di.CONFIGS[args.config]
+    # weak scaling: every rank runs its own replica of the workload (its own batch)
+    case = Case(wl, torch, dsa, seed_offset=1000 * rank)
+    case.step()
+    torch.cuda.synchronize()
+
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    with ClockSampler(local) as clk:
+        head = measure(case, torch, args.steps, args.warmup, flush_buf, peaks)
+        # keep the sampler on the same work long enough for NVML to see it
+        t_end = time.perf_counter() + 1.0
+        while time.perf_counter() < t_end:
+            case.step()
+        torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    ms = head["us_per_step"] / 1e3
+    if world > 1:
+        tt = torch.tensor([ms], device="cuda")
+        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
+        ms = float(tt.item())
+    e2e = measure_e2e(case, torch, args.steps, args.warmup)
+    if world > 1:
+        tt = torch.tensor([e2e["ms_per_step"]], device="cuda")
+        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
+        e2e["ms_per_step"] = float(tt.item())
+        e2e["value"] = wl.n_q * world / (e2e["ms_per_step"] * 1e-3)
+
+    per_config = {}
+    if not args.no_extra:
+        for name in EXTRA:
+            c = Case(di.CONFIGS[name], torch, dsa, seed_offset=1000 * rank)
+            c.step()
+            torch.cuda.synchronize()
+            r = measure(c, torch, args.steps, args.warmup, flush_buf, peaks)
+            if world > 1:
+                tt = torch.tensor([r["us_per_step"]], device="cuda")
+                dist.all_reduce(tt, op=dist.ReduceOp.MAX)
+                r["us_per_step"] = float(tt.item())
+            per_config[name] = r
+            del c
+            torch.cuda.empty_cache()
+
+    if rank == 0:
+        alg = algorithmic(wl)
+        idx_s = head["indexer_us"] * 1e-6
+        line = {
+            "metric": "DSA attention decode tokens/s (one layer's DSA step: indexer, exact "
+                      "top-2048, sparse absorbed MLA)",
+            "value": wl.n_q * world / (ms * 1e-3),
+            "unit": "tokens/s",
+            "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": ms, "us_per_step": ms * 1e3,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+            "dtype": "bf16 inputs, fp32 accumulate/outputs",
+            "data": "synthetic (seeded GLM-5-shaped inputs; integer indexer q/k)",
+            "config": {"workload": wl.name, "description": wl.description,
+                       "global_batch": wl.n_q * world, "seq_len": max(wl.seq_lens),
+                       "parallelism": f"replicas x{world}",
+                       "l2": "flushed (512 MB write) before every timed step",
+                       "alg_bytes_per_step": alg["bytes"],
+                       "achieved_gbs": alg["bytes"] / (ms * 1e-3) / 1e9,
+                       "frac_of_8tbs": alg["bytes"] / (ms * 1e-3) / 1e9 / NOMINAL_HBM_GBS},
+            "roofline": {"kernel": "indexer (tcgen05 + TMA)", "bound": "hbm",
+                         "achieved": alg["bytes_indexer"] / idx_s / 1e9,
+                         "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                         "frac": alg["bytes_indexer"] / idx_s / 1e9 / peaks["hbm_gbs"],
+                         "traffic": None, "peak_source": peaks["source"],
+                         "alg_bytes_per_launch": alg["bytes_indexer"],
+                         "launch_us": head["indexer_us"]},
+            "e2e": e2e,
+            "gpu_launches": head["launches_per_step"] * args.steps,
+            "clocks": clk.summary(),
+            "per_config": per_config,
+        }
+        if args.cpu_baseline_s > 0 and world == 1:
+            line["cpu_baseline"] = cpu_baseline(wl, args.cpu_baseline_s)
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+
+
+def run_reference(args):
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return
+    wl = di.CONFIGS[args.config]
+    for _ in range(args.warmup):
+        oracle_rows_per_s(wl, 0.0)
+    times = []
+    for _ in range(args.steps):
+        rate, n, el = oracle_rows_per_s(wl, 0.0)   # one step = one whole query row
+        times.append(el / n)
+    s = sum(times) / len(times)
+    value = 1.0 / s   # query rows (decode tokens) per second
+    line = {
+        "impl": "reference",
+        "metric": "DSA attention decode tokens/s (one layer's DSA step: indexer, exact "
+                  "top-2048, sparse absorbed MLA)",
+        "value": value, "unit": "tokens/s", "n_gpus": int(os.environ.get("WORLD_SIZE", "1")),
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": s * 1e3,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+        "data": "synthetic (seeded GLM-5-shaped inputs)",
+        "config": {"workload": wl.name, "description": wl.description},
+        "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": blas_threads(),
+                         "kind": "oracle",
+                         "sample": f"{args.steps} steps, each one whole query row of {wl.name}"},
+        "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0,
+                "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=50)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--config", default=HEADLINE, choices=list(di.CONFIGS))
+    ap.add_argument("--no-extra", action="store_true", help="skip the other workloads")
+    ap.add_argument("--cpu-baseline-s", type=float, default=10.0)
+    args = ap.parse_args()
+    if args.warmup < 3:
+        args.warmup = 3
+    if args.impl == "reference":
+        run_reference(args)
+    else:
+        run_ours(args)
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,201 @@
+/*
+ * dsa.h - C ABI of the DSA sparse-attention step for NVIDIA B200 (sm_100a).
+ *
+ * The step (GLM-5 decoder attention with DeepSeek-style sparse attention):
+ *   1. indexer scores   score[s] = sum_h w[h] * max(0, q_idx[h] . k_idx[s])
+ *   2. exact top-k      keep the k best tokens (all of them when fewer exist);
+ *                       equal scores resolve to the lower token index
+ *   3. absorbed MLA     attention in the compressed latent space over the
+ *                       kept tokens only:
+ *                         z[h,j]   = scale * q[h,:] . L[idx_j, :]      (all R+P columns)
+ *                         out[h,:] = sum_j softmax_j(z[h,:]) * L[idx_j, 0:R]
+ *                         lse[h]   = log sum_j exp(z[h,j])            (natural log)
+ *
+ * Sources: "GLM on an A100, in Vx", section "The model" (an indexer scores
+ * every earlier token; each query attends to the 2,048 highest-scoring tokens;
+ * below 2,048 tokens everything is kept; keys and values share one latent
+ * vector per token) and section "How do we know it is right?" (ReLU inside the
+ * indexer; ties follow a stable argsort of -scores).  "Self-contained GLM-5
+ * serving stack: Just Vx kernels compiled to PTX", file list (absorbed MLA
+ * decode, compressed request-local KV, DSA indexer selection) and GPU-code
+ * paragraph (split online-softmax compressed MLA).
+ *
+ * Conventions shared by every entry point
+ * ---------------------------------------
+ *  - bf16 tensors are passed as raw 16-bit patterns (uint16_t).
+ *  - Every tensor pointer is DEVICE memory owned by the caller.  The library
+ *    allocates nothing, keeps no mutable global state and is thread-safe.
+ *  - Every call is asynchronous on `stream`.  A NULL stream means the
+ *    per-thread default stream, never the legacy default stream.
+ *  - Arguments (shapes, ranges, 16-byte alignment) are checked on the host
+ *    before anything is launched; a rejected call has no side effects and
+ *    returns DSA_ERR_INVALID_ARG or DSA_ERR_UNSUPPORTED.  Launch failures
+ *    return DSA_ERR_CUDA.  No C++ exception crosses this interface.
+ *  - Checks made on the device (a page id or token index out of range, a
+ *    bounded wait that gave up) never fault: the kernel skips the access,
+ *    records the event in the workspace status block and finishes.  Read it
+ *    with dsa_workspace_check().
+ *
+ * Paged caches
+ * ------------
+ * Both caches are pools of 64-token pages that share one block table:
+ *   k_idx_pages   [num_pages, 64, D_I]   bf16  indexer keys, one per token
+ *   latent_pages  [num_pages, 64, R + P] bf16  latent rows [c_kv (R) | k_rope (P)]
+ * Token s of sequence b lives in physical page block_table[b, s / 64], slot s % 64.
+ *
+ * Query rows
+ * ----------
+ * Decode (dims.causal == 0): row b is the newest token of sequence b; it sits
+ *   at position seq_lens[b] - 1 and sees tokens 0 .. seq_lens[b]-1.
+ * Prefill (dims.causal == 1): the rows are T consecutive tokens of sequence 0;
+ *   row t sits at position q_pos0 + t and sees tokens 0 .. q_pos0 + t.
+ *
+ * Index output: the kept token positions of each row in ascending order,
+ * padded with -1 when the row sees fewer than k tokens.
+ */
+#ifndef DSA_H_
+#define DSA_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#if defined(__GNUC__)
+#define DSA_API __attribute__((visibility("default")))
+#else
+#define DSA_API
+#endif
+
+/* cudaStream_t without pulling in the CUDA headers. */
+typedef struct CUstream_st *dsa_stream_t;
+
+typedef enum {
+  DSA_OK = 0,
+  DSA_ERR_INVALID_ARG = 1,  /* bad pointer, shape, alignment or range (host check) */
+  DSA_ERR_UNSUPPORTED = 2,  /* valid request outside what the kernels implement   */
+  DSA_ERR_CUDA = 3,         /* a CUDA runtime call or a launch failed              */
+  DSA_ERR_WORKSPACE = 4,    /* workspace missing, misaligned or too small          */
+  DSA_ERR_TIMEOUT = 5,      /* a bounded device-side wait gave up (from the status block) */
+  DSA_ERR_DEVICE_CHECK = 6  /* a device-side range check failed (from the status block)   */
+} dsa_status_t;
+
+/* Paged-cache view.  Pointers are device memory. */
+typedef struct {
+  int32_t num_seqs;            /* sequences (decode: B; prefill: 1)                  */
+  const int32_t *seq_lens;     /* [num_seqs] tokens in the cache, current included   */
+  const int32_t *block_table;  /* [num_seqs, max_pages] physical page ids             */
+  int32_t max_pages;           /* row stride of block_table                           */
+  int32_t page_size;           /* tokens per page; must be 64                          */
+  int32_t num_pages;           /* physical pages in each pool (device range check)    */
+  int32_t max_seq_len;         /* host-side upper bound on every seq_lens[b]; sizes grids */
+} dsa_cache_t;
+
+/* Problem dimensions. */
+typedef struct {
+  int32_t n_q;     /* query rows: decode B (== num_seqs); prefill T                 */
+  int32_t H_I;     /* indexer heads, 1..64                                            */
+  int32_t D_I;     /* indexer head dim: 32, 64 or 128                                 */
+  int32_t topk;    /* k: 1..4096                                                      */
+  int32_t H;       /* MLA heads, 1..64 (tiles always hold 64 head columns)            */
+  int32_t R;       /* latent (kv_lora) rank, multiple of 64, <= 512                   */
+  int32_t P;       /* rope part, multiple of 16, R + P <= 576                          */
+  int32_t causal;  /* 0 = decode rows, 1 = causal prefill rows of sequence 0           */
+  int32_t q_pos0;  /* prefill: position of row 0                                       */
+  float scale;     /* softmax scale applied to q . L                                   */
+} dsa_dims_t;
+
+/* Operation ids for dsa_workspace_bytes(). */
+typedef enum {
+  DSA_OP_INDEXER_SCORES = 0,
+  DSA_OP_TOPK = 1,
+  DSA_OP_SPARSE_MLA_DECODE = 2,
+  DSA_OP_SPARSE_MLA_PREFILL = 3,
+  DSA_OP_ATTENTION_FORWARD = 4
+} dsa_op_t;
+
+/* Library version (major * 10000 + minor * 100 + patch). */
+DSA_API int dsa_version(void);
+
+/* Human-readable name of a status code (static string). */
+DSA_API const char *dsa_status_string(dsa_status_t status);
+
+/* Bytes of device workspace `op` needs for these dims and cache.  Every
+ * workspace starts with a 256-byte status block; the rest is scratch whose
+ * contents are undefined between calls.  Returns 0 for invalid input. */
+DSA_API size_t dsa_workspace_bytes(dsa_op_t op, const dsa_dims_t *dims, const dsa_cache_t *cache);
+
+/* Clear the status block of a workspace (asynchronous on `stream`).  Call it
+ * once after allocating a workspace and after reading an error. */
+DSA_API dsa_status_t dsa_workspace_init(void *ws, size_t ws_bytes, dsa_stream_t stream);
+
+/* Wait for `stream`, then read the status block: DSA_OK, DSA_ERR_TIMEOUT or
+ * DSA_ERR_DEVICE_CHECK.  `info` (may be NULL) receives the first recorded
+ * event code.  Synchronous. */
+DSA_API dsa_status_t dsa_workspace_check(const void *ws, dsa_stream_t stream, uint32_t *info);
+
+/* Step 1 - indexer scores ("GLM on an A100, in Vx", "The model"; ReLU per
+ * indexer head from "How do we know it is right?").
+ *   q_idx        [n_q, H_I, D_I] bf16
+ *   w            [n_q, H_I]      fp32 head weights (any 1/sqrt scale folded in)
+ *   k_idx_pages  [num_pages, 64, D_I] bf16, rows 16-byte aligned
+ *   scores       [n_q, ld] fp32 output; entry (r, s) is written for every
+ *                token s the row sees (s < seq_lens[r], or s <= q_pos0 + r);
+ *                entries past that are left untouched.  ld >= max tokens seen,
+ *                multiple of 4.
+ * Uses tcgen05 tensor-core tiles fed by TMA; exact for integer-valued inputs
+ * whose partial sums stay below 2^24. */
+DSA_API dsa_status_t dsa_indexer_scores(const uint16_t *q_idx, const float *w,
+                                const uint16_t *k_idx_pages, const dsa_cache_t *cache,
+                                const dsa_dims_t *dims, float *scores, int64_t ld,
+                                void *ws, size_t ws_bytes, dsa_stream_t stream);
+
+/* Step 2 - exact top-k with the stable lower-index tie rule ("GLM on an A100,
+ * in Vx", "The model" and "How do we know it is right?").
+ *   scores     [n_q, ld] fp32; row r uses its first len(r) entries, where
+ *              len(r) = valid_len[r] if valid_len != NULL, else causal_base + r + 1
+ *              (clamped to [0, ld]).  -0.0 and +0.0 compare equal; NaN is undefined.
+ *   idx        [n_q, k] int32 output: kept positions ascending, -1 padded.
+ * Scores are read, never modified. */
+DSA_API dsa_status_t dsa_topk(const float *scores, int64_t ld, int32_t n_q, const int32_t *valid_len,
+                      int32_t causal_base, int32_t k, int32_t *idx, void *ws, size_t ws_bytes,
+                      dsa_stream_t stream);
+
+/* Step 3 - absorbed MLA decode over the kept latent rows ("Self-contained
+ * GLM-5 serving stack ...", file list and GPU-code paragraph).
+ *   q            [n_q, H, R + P] bf16 absorbed queries, rows 16-byte aligned
+ *   latent_pages [num_pages, 64, R + P] bf16
+ *   idx          [n_q, topk] int32 token positions (-1 = unused slot); a position
+ *                outside the row's context is skipped and flagged on the device
+ *   out          [n_q, H, R] fp32, lse [n_q, H] fp32 (natural log).  A row with
+ *                no kept token gets out = 0 and lse = -inf.
+ * dims.causal must be 0; row b reads sequence b of the cache. */
+DSA_API dsa_status_t dsa_sparse_mla_decode(const uint16_t *q, const uint16_t *latent_pages,
+                                   const dsa_cache_t *cache, const int32_t *idx,
+                                   const dsa_dims_t *dims, float *out, float *lse,
+                                   void *ws, size_t ws_bytes, dsa_stream_t stream);
+
+/* Step 3 for causal prefill rows: as dsa_sparse_mla_decode with dims.causal == 1;
+ * every row reads sequence 0 of the cache and may only keep tokens <= q_pos0 + t. */
+DSA_API dsa_status_t dsa_sparse_mla_prefill(const uint16_t *q, const uint16_t *latent_pages,
+                                    const dsa_cache_t *cache, const int32_t *idx,
+                                    const dsa_dims_t *dims, float *out, float *lse,
+                                    void *ws, size_t ws_bytes, dsa_stream_t stream);
+
+/* The whole step: indexer scores -> exact top-k -> sparse MLA, one call, all
+ * launches on `stream`.  idx_out [n_q, topk] (may be NULL) receives the kept
+ * positions; out/lse as above.  Bit-identical to calling the three steps in
+ * order with the same workspace sizes. */
+DSA_API dsa_status_t dsa_attention_forward(const uint16_t *q_idx, const float *w,
+                                   const uint16_t *k_idx_pages, const uint16_t *q,
+                                   const uint16_t *latent_pages, const dsa_cache_t *cache,
+                                   const dsa_dims_t *dims, int32_t *idx_out, float *out,
+                                   float *lse, void *ws, size_t ws_bytes, dsa_stream_t stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* DSA_H_ */

@@ -1,0 +1,204 @@
+"""Python binding of libdsa, the B200 (sm_100a) DSA sparse-attention step.
+
+Argument marshalling only: every function below forwards torch tensors'
+device pointers to the C ABI of include/dsa.h, on the current CUDA stream,
+and raises DsaError on a non-OK status.  There is no fallback: when the
+compiled library is missing, loading it raises.
+
+    import sparse_attention_scores_b200 as dsa
+    cache = dsa.PagedCache(seq_lens, block_table, num_pages, max_seq_len)
+    dims = dsa.Dims(n_q, H_I, D_I, topk, H, R, P, causal, q_pos0, scale)
+    ws = dsa.workspace(dsa.OP_ATTENTION_FORWARD, dims, cache)
+    dsa.dsa_attention_forward(q_idx, w, k_pages, q, latent_pages, cache, dims,
+                              idx_out, out, lse, ws)
+"""
+
+from __future__ import annotations
+
+import ctypes
+import os
+from dataclasses import dataclass
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libdsa.so")
+
+OP_INDEXER_SCORES = 0
+OP_TOPK = 1
+OP_SPARSE_MLA_DECODE = 2
+OP_SPARSE_MLA_PREFILL = 3
+OP_ATTENTION_FORWARD = 4
+
+STATUS_NAMES = {0: "DSA_OK", 1: "DSA_ERR_INVALID_ARG", 2: "DSA_ERR_UNSUPPORTED",
+                3: "DSA_ERR_CUDA", 4: "DSA_ERR_WORKSPACE", 5: "DSA_ERR_TIMEOUT",
+                6: "DSA_ERR_DEVICE_CHECK"}
+
+EXPORTED = ["dsa_version", "dsa_status_string", "dsa_workspace_bytes", "dsa_workspace_init",
+            "dsa_workspace_check", "dsa_indexer_scores", "dsa_topk", "dsa_sparse_mla_decode",
+            "dsa_sparse_mla_prefill", "dsa_attention_forward"]
+
+
+class DsaError(RuntimeError):
+    def __init__(self, status: int, where: str):
+        self.status = status
+        super().__init__(f"{where}: {STATUS_NAMES.get(status, status)}")
+
+
+class CacheStruct(ctypes.Structure):
+    _fields_ = [("num_seqs", ctypes.c_int32), ("seq_lens", ctypes.c_void_p),
+                ("block_table", ctypes.c_void_p), ("max_pages", ctypes.c_int32),
+                ("page_size", ctypes.c_int32), ("num_pages", ctypes.c_int32),
+                ("max_seq_len", ctypes.c_int32)]
+
+
+class DimsStruct(ctypes.Structure):
+    _fields_ = [("n_q", ctypes.c_int32), ("H_I", ctypes.c_int32), ("D_I", ctypes.c_int32),
+                ("topk", ctypes.c_int32), ("H", ctypes.c_int32), ("R", ctypes.c_int32),
+                ("P", ctypes.c_int32), ("causal", ctypes.c_int32), ("q_pos0", ctypes.c_int32),
+                ("scale", ctypes.c_float)]
+
+
+_lib = None
+
+
+def lib() -> ctypes.CDLL:
+    """Load libdsa.so (built in place by __graft_entry__.build or
+    `python -m sparse_attention_scores_b200.build`).  Raises if it is missing."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(LIB_PATH):
+            raise RuntimeError(f"libdsa.so not built ({LIB_PATH}); run "
+                               "`python -m sparse_attention_scores_b200.build`")
+        L = ctypes.CDLL(LIB_PATH)
+        vp, sz, i32, i64 = ctypes.c_void_p, ctypes.c_size_t, ctypes.c_int32, ctypes.c_int64
+        pc, pd = ctypes.POINTER(CacheStruct), ctypes.POINTER(DimsStruct)
+        sigs = {
+            "dsa_version": ([], ctypes.c_int),
+            "dsa_status_string": ([ctypes.c_int], ctypes.c_char_p),
+            "dsa_workspace_bytes": ([ctypes.c_int, pd, pc], sz),
+            "dsa_workspace_init": ([vp, sz, vp], ctypes.c_int),
+            "dsa_workspace_check": ([vp, vp, ctypes.POINTER(ctypes.c_uint32)], ctypes.c_int),
+            "dsa_indexer_scores": ([vp, vp, vp, pc, pd, vp, i64, vp, sz, vp], ctypes.c_int),
+            "dsa_topk": ([vp, i64, i32, vp, i32, i32, vp, vp, sz, vp], ctypes.c_int),
+            "dsa_sparse_mla_decode": ([vp, vp, pc, vp, pd, vp, vp, vp, sz, vp], ctypes.c_int),
+            "dsa_sparse_mla_prefill": ([vp, vp, pc, vp, pd, vp, vp, vp, sz, vp], ctypes.c_int),
+            "dsa_attention_forward": ([vp, vp, vp, vp, vp, pc, pd, vp, vp, vp, vp, sz, vp],
+                                      ctypes.c_int),
+        }
+        for name, (args, res) in sigs.items():
+            fn = getattr(L, name)
+            fn.argtypes = args
+            fn.restype = res
+        _lib = L
+    return _lib
+
+
+@dataclass
+class Dims:
+    n_q: int
+    H_I: int
+    D_I: int
+    topk: int
+    H: int
+    R: int
+    P: int
+    causal: int = 0
+    q_pos0: int = 0
+    scale: float = 1.0
+
+    def struct(self) -> DimsStruct:
+        return DimsStruct(self.n_q, self.H_I, self.D_I, self.topk, self.H, self.R, self.P,
+                          self.causal, self.q_pos0, self.scale)
+
+
+@dataclass
+class PagedCache:
+    """Device-side view of the paged caches: seq_lens [B] int32 and
+    block_table [B, max_pages] int32 CUDA tensors, plus host-side sizes."""
+    seq_lens: object
+    block_table: object
+    num_pages: int
+    max_seq_len: int
+    page_size: int = 64
+
+    def struct(self) -> CacheStruct:
+        return CacheStruct(int(self.seq_lens.shape[0]), _ptr(self.seq_lens),
+                           _ptr(self.block_table), int(self.block_table.shape[1]),
+                           self.page_size, int(self.num_pages), int(self.max_seq_len))
+
+
+def _ptr(t) -> int | None:
+    return None if t is None else int(t.data_ptr())
+
+
+def _stream(stream) -> int | None:
+    if stream is None:
+        import torch
+        return int(torch.cuda.current_stream().cuda_stream) or None
+    return int(stream.cuda_stream) if hasattr(stream, "cuda_stream") else int(stream)
+
+
+def _check(status: int, where: str) -> None:
+    if status != 0:
+        raise DsaError(status, where)
+
+
+def workspace_bytes(op: int, dims: Dims, cache: PagedCache | None) -> int:
+    c = ctypes.byref(cache.struct()) if cache is not None else None
+    return int(lib().dsa_workspace_bytes(op, ctypes.byref(dims.struct()), c))
+
+
+def workspace(op: int, dims: Dims, cache: PagedCache | None, device="cuda", stream=None):
+    """Allocate (with torch) and initialise a workspace for `op`."""
+    import torch
+    n = workspace_bytes(op, dims, cache)
+    if n == 0:
+        raise DsaError(1, "dsa_workspace_bytes")
+    ws = torch.empty(n, dtype=torch.uint8, device=device)
+    _check(lib().dsa_workspace_init(_ptr(ws), n, _stream(stream)), "dsa_workspace_init")
+    return ws
+
+
+def workspace_check(ws, stream=None) -> tuple[int, int]:
+    info = ctypes.c_uint32(0)
+    st = lib().dsa_workspace_check(_ptr(ws), _stream(stream), ctypes.byref(info))
+    return int(st), int(info.value)
+
+
+def dsa_indexer_scores(q_idx, w, k_idx_pages, cache: PagedCache, dims: Dims, scores, ws,
+                       stream=None) -> None:
+    _check(lib().dsa_indexer_scores(_ptr(q_idx), _ptr(w), _ptr(k_idx_pages),
+                                    ctypes.byref(cache.struct()), ctypes.byref(dims.struct()),
+                                    _ptr(scores), int(scores.stride(0)), _ptr(ws), ws.numel(),
+                                    _stream(stream)), "dsa_indexer_scores")
+
+
+def dsa_topk(scores, valid_len, causal_base: int, k: int, idx, ws, stream=None) -> None:
+    _check(lib().dsa_topk(_ptr(scores), int(scores.stride(0)), int(scores.shape[0]),
+                          _ptr(valid_len), int(causal_base), int(k), _ptr(idx), _ptr(ws),
+                          ws.numel(), _stream(stream)), "dsa_topk")
+
+
+def dsa_sparse_mla_decode(q, latent_pages, cache: PagedCache, idx, dims: Dims, out, lse, ws,
+                          stream=None) -> None:
+    _check(lib().dsa_sparse_mla_decode(_ptr(q), _ptr(latent_pages), ctypes.byref(cache.struct()),
+                                       _ptr(idx), ctypes.byref(dims.struct()), _ptr(out),
+                                       _ptr(lse), _ptr(ws), ws.numel(), _stream(stream)),
+           "dsa_sparse_mla_decode")
+
+
+def dsa_sparse_mla_prefill(q, latent_pages, cache: PagedCache, idx, dims: Dims, out, lse, ws,
+                           stream=None) -> None:
+    _check(lib().dsa_sparse_mla_prefill(_ptr(q), _ptr(latent_pages),
+                                        ctypes.byref(cache.struct()), _ptr(idx),
+                                        ctypes.byref(dims.struct()), _ptr(out), _ptr(lse),
+                                        _ptr(ws), ws.numel(), _stream(stream)),
+           "dsa_sparse_mla_prefill")
+
+
+def dsa_attention_forward(q_idx, w, k_idx_pages, q, latent_pages, cache: PagedCache, dims: Dims,
+                          idx_out, out, lse, ws, stream=None) -> None:
+    _check(lib().dsa_attention_forward(_ptr(q_idx), _ptr(w), _ptr(k_idx_pages), _ptr(q),
+                                       _ptr(latent_pages), ctypes.byref(cache.struct()),
+                                       ctypes.byref(dims.struct()), _ptr(idx_out), _ptr(out),
+                                       _ptr(lse), _ptr(ws), ws.numel(), _stream(stream)),
+           "dsa_attention_forward")

@@ -1,0 +1,380 @@
+// The C ABI of libdsa: argument checks on the host, workspace layout, and the
+// launch sequence of each entry point.  See include/dsa.h for the contract.
+#include <math.h>
+#include <stdlib.h>
+#include <string.h>
+
+#include <algorithm>
+
+#include "dsa_internal.h"
+
+namespace dsa {
+
+uint64_t wait_limit_ns() {
+  static const uint64_t v = [] {
+    const char *s = getenv("DSA_WAIT_LIMIT_NS");
+    if (s != nullptr && *s != '\0') return static_cast<uint64_t>(strtoull(s, nullptr, 10));
+    return static_cast<uint64_t>(1000000000ull);
+  }();
+  return v;
+}
+
+namespace {
+constexpr int kMaxDevices = 64;
+int g_sm_count[kMaxDevices];
+size_t g_smem_optin[kMaxDevices];
+
+int current_device() {
+  int d = 0;
+  if (cudaGetDevice(&d) != cudaSuccess || d < 0 || d >= kMaxDevices) return -1;
+  return d;
+}
+}  // namespace
+
+int device_sm_count() {
+  const int d = current_device();
+  if (d < 0) return 148;
+  if (g_sm_count[d] == 0) {
+    int v = 0;
+    if (cudaDeviceGetAttribute(&v, cudaDevAttrMultiProcessorCount, d) != cudaSuccess || v <= 0)
+      return 148;
+    g_sm_count[d] = v;
+  }
+  return g_sm_count[d];
+}
+
+size_t device_max_smem_optin() {
+  const int d = current_device();
+  if (d < 0) return 232448;
+  if (g_smem_optin[d] == 0) {
+    int v = 0;
+    if (cudaDeviceGetAttribute(&v, cudaDevAttrMaxSharedMemoryPerBlockOptin, d) != cudaSuccess ||
+        v <= 0)
+      return 232448;
+    g_smem_optin[d] = static_cast<size_t>(v);
+  }
+  return g_smem_optin[d];
+}
+
+namespace {
+
+constexpr size_t kStatusBytes = sizeof(DevStatus);
+
+size_t align256(size_t x) { return (x + 255) & ~static_cast<size_t>(255); }
+bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+bool aligned4(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 3u) == 0; }
+cudaStream_t as_stream(dsa_stream_t s) {
+  return s ? reinterpret_cast<cudaStream_t>(s) : cudaStreamPerThread;
+}
+
+// tokens the longest query row sees
+int64_t max_keys(const dsa_dims_t &d, const dsa_cache_t &c) {
+  return d.causal ? static_cast<int64_t>(d.q_pos0) + d.n_q : static_cast<int64_t>(c.max_seq_len);
+}
+int64_t scores_ld(const dsa_dims_t &d, const dsa_cache_t &c) {
+  return std::max<int64_t>(4, (max_keys(d, c) + 3) & ~static_cast<int64_t>(3));
+}
+
+dsa_status_t check_dims_common(const dsa_dims_t *d) {
+  if (d == nullptr) return DSA_ERR_INVALID_ARG;
+  if (d->n_q < 0 || d->causal < 0 || d->causal > 1 || d->q_pos0 < 0) return DSA_ERR_INVALID_ARG;
+  if (d->causal == 0 && d->q_pos0 != 0) return DSA_ERR_INVALID_ARG;
+  return DSA_OK;
+}
+
+dsa_status_t check_cache(const dsa_cache_t *c, const dsa_dims_t &d) {
+  if (c == nullptr) return DSA_ERR_INVALID_ARG;
+  if (c->seq_lens == nullptr || c->block_table == nullptr) return DSA_ERR_INVALID_ARG;
+  if (!aligned4(c->seq_lens) || !aligned4(c->block_table)) return DSA_ERR_INVALID_ARG;
+  if (c->page_size != kPageSize) return DSA_ERR_UNSUPPORTED;
+  if (c->num_seqs < 1 || c->max_pages < 1 || c->num_pages < 1) return DSA_ERR_INVALID_ARG;
+  if (c->max_seq_len < 0) return DSA_ERR_INVALID_ARG;
+  if (static_cast<int64_t>(c->max_seq_len) > static_cast<int64_t>(c->max_pages) * kPageSize)
+    return DSA_ERR_INVALID_ARG;
+  if (static_cast<int64_t>(c->num_pages) * kPageSize > INT32_MAX) return DSA_ERR_UNSUPPORTED;
+  if (d.causal == 0) {
+    if (c->num_seqs != d.n_q) return DSA_ERR_INVALID_ARG;
+  } else {
+    if (static_cast<int64_t>(d.q_pos0) + d.n_q > static_cast<int64_t>(c->max_pages) * kPageSize)
+      return DSA_ERR_INVALID_ARG;
+  }
+  return DSA_OK;
+}
+
+dsa_status_t check_indexer_dims(const dsa_dims_t &d) {
+  if (d.H_I < 1 || d.H_I > 64) return DSA_ERR_UNSUPPORTED;
+  if (d.D_I != 32 && d.D_I != 64 && d.D_I != 128) return DSA_ERR_UNSUPPORTED;
+  // the indexer walks row groups out of a shared-memory table
+  const int64_t groups = d.causal ? (d.n_q + 3) / 4 : d.n_q;
+  if (groups > 8192) return DSA_ERR_UNSUPPORTED;
+  return DSA_OK;
+}
+
+dsa_status_t check_mla_dims(const dsa_dims_t &d) {
+  if (d.topk < 1 || d.topk > 65536) return DSA_ERR_UNSUPPORTED;
+  if (d.H < 1 || d.H > 64) return DSA_ERR_UNSUPPORTED;
+  if (d.R < 64 || d.R > 512 || d.R % 64 != 0) return DSA_ERR_UNSUPPORTED;
+  if (d.P < 0 || d.P % 16 != 0 || d.R + d.P > 576) return DSA_ERR_UNSUPPORTED;
+  if (!isfinite(d.scale)) return DSA_ERR_INVALID_ARG;
+  if (d.n_q > 65535) return DSA_ERR_UNSUPPORTED;  // grid.y
+  return DSA_OK;
+}
+
+DevStatus *status_of(void *ws) { return static_cast<DevStatus *>(ws); }
+
+dsa_status_t check_ws(void *ws, size_t ws_bytes, size_t need) {
+  if (ws == nullptr || (reinterpret_cast<uintptr_t>(ws) & 255u) != 0) return DSA_ERR_WORKSPACE;
+  if (ws_bytes < need) return DSA_ERR_WORKSPACE;
+  return DSA_OK;
+}
+
+#define DSA_TRY(expr)                        \
+  do {                                       \
+    const dsa_status_t st__ = (expr);        \
+    if (st__ != DSA_OK) return st__;         \
+  } while (0)
+
+size_t ws_bytes_for(dsa_op_t op, const dsa_dims_t &d, const dsa_cache_t &c) {
+  switch (op) {
+    case DSA_OP_INDEXER_SCORES:
+    case DSA_OP_TOPK:
+      return kStatusBytes;
+    case DSA_OP_SPARSE_MLA_DECODE:
+    case DSA_OP_SPARSE_MLA_PREFILL:
+      return kStatusBytes + align256(mla_scratch_bytes(d.n_q, d.topk, d.R));
+    case DSA_OP_ATTENTION_FORWARD: {
+      const size_t scores = static_cast<size_t>(d.n_q) * scores_ld(d, c) * 4;
+      const size_t idx = static_cast<size_t>(d.n_q) * d.topk * 4;
+      return kStatusBytes + align256(scores) + align256(idx) +
+             align256(mla_scratch_bytes(d.n_q, d.topk, d.R));
+    }
+  }
+  return 0;
+}
+
+dsa_status_t run_indexer(const uint16_t *q_idx, const float *w, const uint16_t *k_pages,
+                         const dsa_cache_t &c, const dsa_dims_t &d, float *scores, int64_t ld,
+                         DevStatus *st, cudaStream_t s) {
+  IndexerLaunch a;
+  a.q_idx = q_idx;
+  a.w = w;
+  a.k_pages = k_pages;
+  a.seq_lens = c.seq_lens;
+  a.block_table = c.block_table;
+  a.scores = scores;
+  a.ld = ld;
+  a.n_q = d.n_q;
+  a.H_I = d.H_I;
+  a.D_I = d.D_I;
+  a.causal = d.causal;
+  a.q_pos0 = d.q_pos0;
+  a.num_seqs = c.num_seqs;
+  a.max_pages = c.max_pages;
+  a.num_pages = c.num_pages;
+  a.max_seq_len = c.max_seq_len;
+  a.status = st;
+  return launch_indexer(a, s);
+}
+
+dsa_status_t run_topk(const float *scores, int64_t ld, int n_q, const int32_t *valid_len,
+                      int causal_base, int k, int32_t *idx, int max_len, DevStatus *st,
+                      cudaStream_t s) {
+  TopkLaunch a;
+  a.scores = scores;
+  a.ld = ld;
+  a.n_q = n_q;
+  a.valid_len = valid_len;
+  a.causal_base = causal_base;
+  a.k = k;
+  a.idx = idx;
+  a.max_len = max_len;
+  a.status = st;
+  return launch_topk(a, s);
+}
+
+dsa_status_t run_mla(const uint16_t *q, const uint16_t *latent, const dsa_cache_t &c,
+                     const int32_t *idx, const dsa_dims_t &d, float *out, float *lse, void *scratch,
+                     size_t scratch_bytes, DevStatus *st, cudaStream_t s) {
+  MlaLaunch a;
+  a.q = q;
+  a.latent = latent;
+  a.idx = idx;
+  a.seq_lens = c.seq_lens;
+  a.block_table = c.block_table;
+  a.out = out;
+  a.lse = lse;
+  a.n_q = d.n_q;
+  a.H = d.H;
+  a.R = d.R;
+  a.P = d.P;
+  a.topk = d.topk;
+  a.causal = d.causal;
+  a.q_pos0 = d.q_pos0;
+  a.max_pages = c.max_pages;
+  a.num_pages = c.num_pages;
+  a.scale = d.scale;
+  a.scratch = scratch;
+  a.scratch_bytes = scratch_bytes;
+  a.status = st;
+  return launch_mla(a, s);
+}
+
+dsa_status_t mla_entry(const uint16_t *q, const uint16_t *latent_pages, const dsa_cache_t *cache,
+                       const int32_t *idx, const dsa_dims_t *dims, float *out, float *lse,
+                       void *ws, size_t ws_bytes, dsa_stream_t stream, int want_causal) {
+  DSA_TRY(check_dims_common(dims));
+  if (dims->causal != want_causal) return DSA_ERR_INVALID_ARG;
+  DSA_TRY(check_mla_dims(*dims));
+  DSA_TRY(check_cache(cache, *dims));
+  if (q == nullptr || latent_pages == nullptr || idx == nullptr || out == nullptr || lse == nullptr)
+    return DSA_ERR_INVALID_ARG;
+  if (!aligned16(q) || !aligned16(latent_pages) || !aligned4(idx) || !aligned4(out) ||
+      !aligned4(lse))
+    return DSA_ERR_INVALID_ARG;
+  const size_t need = ws_bytes_for(want_causal ? DSA_OP_SPARSE_MLA_PREFILL : DSA_OP_SPARSE_MLA_DECODE,
+                                   *dims, *cache);
+  DSA_TRY(check_ws(ws, ws_bytes, need));
+  if (dims->n_q == 0) return DSA_OK;
+  return run_mla(q, latent_pages, *cache, idx, *dims, out, lse,
+                 static_cast<uint8_t *>(ws) + kStatusBytes, ws_bytes - kStatusBytes, status_of(ws),
+                 as_stream(stream));
+}
+
+}  // namespace
+}  // namespace dsa
+
+using namespace dsa;
+
+extern "C" {
+
+int dsa_version(void) { return 100; }
+
+const char *dsa_status_string(dsa_status_t s) {
+  switch (s) {
+    case DSA_OK: return "ok";
+    case DSA_ERR_INVALID_ARG: return "invalid argument";
+    case DSA_ERR_UNSUPPORTED: return "unsupported shape or configuration";
+    case DSA_ERR_CUDA: return "CUDA error";
+    case DSA_ERR_WORKSPACE: return "workspace missing, misaligned or too small";
+    case DSA_ERR_TIMEOUT: return "a bounded device-side wait timed out";
+    case DSA_ERR_DEVICE_CHECK: return "a device-side range check failed";
+  }
+  return "unknown status";
+}
+
+size_t dsa_workspace_bytes(dsa_op_t op, const dsa_dims_t *dims, const dsa_cache_t *cache) {
+  if (check_dims_common(dims) != DSA_OK) return 0;
+  if (op == DSA_OP_INDEXER_SCORES || op == DSA_OP_TOPK) return kStatusBytes;
+  if (check_mla_dims(*dims) != DSA_OK) return 0;
+  if (op == DSA_OP_ATTENTION_FORWARD && (cache == nullptr || check_cache(cache, *dims) != DSA_OK))
+    return 0;
+  dsa_cache_t empty = {};
+  return ws_bytes_for(op, *dims, cache ? *cache : empty);
+}
+
+dsa_status_t dsa_workspace_init(void *ws, size_t ws_bytes, dsa_stream_t stream) {
+  DSA_TRY(check_ws(ws, ws_bytes, kStatusBytes));
+  if (cudaMemsetAsync(ws, 0, kStatusBytes, as_stream(stream)) != cudaSuccess) return DSA_ERR_CUDA;
+  return DSA_OK;
+}
+
+dsa_status_t dsa_workspace_check(const void *ws, dsa_stream_t stream, uint32_t *info) {
+  if (ws == nullptr) return DSA_ERR_WORKSPACE;
+  DevStatus host;
+  cudaStream_t s = as_stream(stream);
+  if (cudaMemcpyAsync(&host, ws, sizeof(host), cudaMemcpyDeviceToHost, s) != cudaSuccess)
+    return DSA_ERR_CUDA;
+  if (cudaStreamSynchronize(s) != cudaSuccess) return DSA_ERR_CUDA;
+  if (info) *info = host.first;
+  if (host.flags & kErrTimeout) return DSA_ERR_TIMEOUT;
+  if (host.flags != 0u) return DSA_ERR_DEVICE_CHECK;
+  return DSA_OK;
+}
+
+dsa_status_t dsa_indexer_scores(const uint16_t *q_idx, const float *w, const uint16_t *k_idx_pages,
+                                const dsa_cache_t *cache, const dsa_dims_t *dims, float *scores,
+                                int64_t ld, void *ws, size_t ws_bytes, dsa_stream_t stream) {
+  DSA_TRY(check_dims_common(dims));
+  DSA_TRY(check_indexer_dims(*dims));
+  DSA_TRY(check_cache(cache, *dims));
+  if (q_idx == nullptr || w == nullptr || k_idx_pages == nullptr || scores == nullptr)
+    return DSA_ERR_INVALID_ARG;
+  if (!aligned16(q_idx) || !aligned16(k_idx_pages) || !aligned16(scores) || !aligned4(w))
+    return DSA_ERR_INVALID_ARG;
+  if (ld < max_keys(*dims, *cache) || ld % 4 != 0 || ld <= 0) return DSA_ERR_INVALID_ARG;
+  DSA_TRY(check_ws(ws, ws_bytes, kStatusBytes));
+  if (dims->n_q == 0) return DSA_OK;
+  return run_indexer(q_idx, w, k_idx_pages, *cache, *dims, scores, ld, status_of(ws),
+                     as_stream(stream));
+}
+
+dsa_status_t dsa_topk(const float *scores, int64_t ld, int32_t n_q, const int32_t *valid_len,
+                      int32_t causal_base, int32_t k, int32_t *idx, void *ws, size_t ws_bytes,
+                      dsa_stream_t stream) {
+  if (scores == nullptr || idx == nullptr) return DSA_ERR_INVALID_ARG;
+  if (n_q < 0 || k < 1 || ld < 1 || ld > INT32_MAX) return DSA_ERR_INVALID_ARG;
+  if (!aligned4(scores) || !aligned4(idx) || (valid_len && !aligned4(valid_len)))
+    return DSA_ERR_INVALID_ARG;
+  if (valid_len == nullptr && causal_base < -1) return DSA_ERR_INVALID_ARG;
+  if (n_q > 262144) return DSA_ERR_UNSUPPORTED;  // grid.x with 8-CTA clusters
+  DSA_TRY(check_ws(ws, ws_bytes, kStatusBytes));
+  if (n_q == 0) return DSA_OK;
+  // without a host-side bound on the lengths, size the kernel for the full row
+  const int max_len = static_cast<int>(
+      valid_len ? ld : std::min<int64_t>(ld, static_cast<int64_t>(causal_base) + n_q));
+  return run_topk(scores, ld, n_q, valid_len, causal_base, k, idx, max_len, status_of(ws),
+                  as_stream(stream));
+}
+
+dsa_status_t dsa_sparse_mla_decode(const uint16_t *q, const uint16_t *latent_pages,
+                                   const dsa_cache_t *cache, const int32_t *idx,
+                                   const dsa_dims_t *dims, float *out, float *lse, void *ws,
+                                   size_t ws_bytes, dsa_stream_t stream) {
+  return mla_entry(q, latent_pages, cache, idx, dims, out, lse, ws, ws_bytes, stream, 0);
+}
+
+dsa_status_t dsa_sparse_mla_prefill(const uint16_t *q, const uint16_t *latent_pages,
+                                    const dsa_cache_t *cache, const int32_t *idx,
+                                    const dsa_dims_t *dims, float *out, float *lse, void *ws,
+                                    size_t ws_bytes, dsa_stream_t stream) {
+  return mla_entry(q, latent_pages, cache, idx, dims, out, lse, ws, ws_bytes, stream, 1);
+}
+
+dsa_status_t dsa_attention_forward(const uint16_t *q_idx, const float *w,
+                                   const uint16_t *k_idx_pages, const uint16_t *q,
+                                   const uint16_t *latent_pages, const dsa_cache_t *cache,
+                                   const dsa_dims_t *dims, int32_t *idx_out, float *out,
+                                   float *lse, void *ws, size_t ws_bytes, dsa_stream_t stream) {
+  DSA_TRY(check_dims_common(dims));
+  DSA_TRY(check_indexer_dims(*dims));
+  DSA_TRY(check_mla_dims(*dims));
+  DSA_TRY(check_cache(cache, *dims));
+  if (q_idx == nullptr || w == nullptr || k_idx_pages == nullptr || q == nullptr ||
+      latent_pages == nullptr || out == nullptr || lse == nullptr)
+    return DSA_ERR_INVALID_ARG;
+  if (!aligned16(q_idx) || !aligned16(k_idx_pages) || !aligned16(q) || !aligned16(latent_pages) ||
+      !aligned4(w) || !aligned4(out) || !aligned4(lse) || (idx_out && !aligned4(idx_out)))
+    return DSA_ERR_INVALID_ARG;
+  const dsa_dims_t &d = *dims;
+  const dsa_cache_t &c = *cache;
+  DSA_TRY(check_ws(ws, ws_bytes, ws_bytes_for(DSA_OP_ATTENTION_FORWARD, d, c)));
+  if (d.n_q == 0) return DSA_OK;
+
+  uint8_t *base = static_cast<uint8_t *>(ws);
+  DevStatus *st = status_of(ws);
+  const int64_t ld = scores_ld(d, c);
+  float *scores = reinterpret_cast<float *>(base + kStatusBytes);
+  int32_t *idx_ws = reinterpret_cast<int32_t *>(
+      base + kStatusBytes + align256(static_cast<size_t>(d.n_q) * ld * 4));
+  uint8_t *scratch = reinterpret_cast<uint8_t *>(idx_ws) + align256(static_cast<size_t>(d.n_q) * d.topk * 4);
+  const size_t scratch_bytes = ws_bytes - static_cast<size_t>(scratch - base);
+  int32_t *idx = idx_out ? idx_out : idx_ws;
+  cudaStream_t s = as_stream(stream);
+
+  DSA_TRY(run_indexer(q_idx, w, k_idx_pages, c, d, scores, ld, st, s));
+  DSA_TRY(run_topk(scores, ld, d.n_q, d.causal ? nullptr : c.seq_lens, d.q_pos0, d.topk, idx,
+                   static_cast<int>(max_keys(d, c)), st, s));
+  return run_mla(q, latent_pages, c, idx, d, out, lse, scratch, scratch_bytes, st, s);
+}
+
+}  // extern "C"

@@ -1,0 +1,69 @@
+// Host-side launchers of the DSA kernels (internal to libdsa; not part of the ABI).
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "../../include/dsa.h"
+#include "dsa_common.cuh"
+
+namespace dsa {
+
+// Wall-time limit of every bounded device-side wait, in nanoseconds.  One
+// second by default; the environment variable DSA_WAIT_LIMIT_NS overrides it
+// (read once), which lets a test force the time-out path.
+uint64_t wait_limit_ns();
+// Fixed limit used while draining copies/MMAs in flight on the error path.
+constexpr uint64_t kDrainLimitNs = 1000000000ull;
+
+int device_sm_count();
+size_t device_max_smem_optin();
+
+struct IndexerLaunch {
+  const uint16_t *q_idx;
+  const float *w;
+  const uint16_t *k_pages;
+  const int32_t *seq_lens;
+  const int32_t *block_table;
+  float *scores;
+  int64_t ld;
+  int n_q, H_I, D_I, causal, q_pos0;
+  int num_seqs, max_pages, num_pages, max_seq_len;
+  DevStatus *status;
+};
+dsa_status_t launch_indexer(const IndexerLaunch &a, cudaStream_t stream);
+
+struct TopkLaunch {
+  const float *scores;
+  int64_t ld;
+  int n_q;
+  const int32_t *valid_len;
+  int causal_base;
+  int k;
+  int32_t *idx;
+  int max_len;  // host upper bound on any row's length
+  DevStatus *status;
+};
+dsa_status_t launch_topk(const TopkLaunch &a, cudaStream_t stream);
+
+struct MlaLaunch {
+  const uint16_t *q;
+  const uint16_t *latent;
+  const int32_t *idx;
+  const int32_t *seq_lens;
+  const int32_t *block_table;
+  float *out;
+  float *lse;
+  int n_q, H, R, P, topk, causal, q_pos0;
+  int max_pages, num_pages;
+  float scale;
+  void *scratch;        // partial results when the keys are split over CTAs
+  size_t scratch_bytes;
+  DevStatus *status;
+};
+// Number of key splits the launcher uses and the scratch bytes it needs.
+int mla_num_splits(int n_q, int topk);
+size_t mla_scratch_bytes(int n_q, int topk, int R);
+dsa_status_t launch_mla(const MlaLaunch &a, cudaStream_t stream);
+
+}  // namespace dsa

@@ -1,0 +1,450 @@
+// Step 1 of the DSA step: indexer scores on tcgen05 tensor cores.
+//
+//   score[r, s] = sum_h w[r, h] * max(0, q_idx[r, h, :] . k_idx[s, :])
+//
+// ("GLM on an A100, in Vx", section "The model": a separate indexer scores
+// every earlier token; section "How do we know it is right?": ReLU per
+// indexer head before the heads are combined.)
+//
+// Design (sm_100a): one persistent CTA per SM walks a contiguous range of
+// work units.  A unit is one tile of 128 keys of one row group (decode: one
+// sequence; causal prefill: G consecutive query rows, which share their keys).
+// The key tile is the A operand (M = 128 keys, K = D_I), the queries of the
+// group are the B operand (N = G * H_I), so one MMA chain per tile yields
+// every (key, row, head) dot product in tensor memory.  Warp roles:
+//   warp 0     TMA producer: 64-key pages straight from the paged cache
+//              (two per tile) into a ring of shared-memory stages; the
+//              query tile when the row group changes
+//   warp 1     tcgen05.mma issuer (one thread), double-buffered accumulators
+//   warps 2-5  epilogue: tcgen05.ld of a 128-lane accumulator, ReLU,
+//              head-weighted sum, coalesced fp32 stores
+// Every wait is bounded in wall time; a time-out records an error in the
+// status block, drains what is in flight, frees tensor memory and returns.
+#include <algorithm>
+#include <cudaTypedefs.h>
+
+#include "dsa_internal.h"
+
+namespace dsa {
+namespace {
+
+constexpr int kThreads = 192;
+constexpr int kTileKeys = 128;
+constexpr int kLookahead = 16;  // units whose page ids the producer fetches at once
+
+struct IndexerParams {
+  const float *w;
+  const int32_t *seq_lens;
+  const int32_t *block_table;
+  float *scores;
+  int64_t ld;
+  int n_q, H_I, D_I, causal, q_pos0;
+  int max_pages, num_pages;
+  int num_groups;
+  int stages;
+  uint64_t wait_ns;
+  DevStatus *status;
+};
+
+// Tokens a row group must score (the longest row of the group).
+template <int G>
+__device__ __forceinline__ int group_keys(const IndexerParams &p, int g) {
+  int n;
+  if (!p.causal) {
+    n = p.seq_lens[g];
+  } else {
+    const int last = min(g * G + G, p.n_q) - 1;
+    n = p.q_pos0 + last + 1;
+  }
+  return max(0, min(min(n, p.max_pages * kPageSize), static_cast<int>(p.ld)));
+}
+// Tokens row r sees.
+__device__ __forceinline__ int row_keys(const IndexerParams &p, int r) {
+  const int n = p.causal ? p.q_pos0 + r + 1 : p.seq_lens[r];
+  return max(0, min(min(n, p.max_pages * kPageSize), static_cast<int>(p.ld)));
+}
+
+// group containing unit u: the largest g with tile_start[g] <= u
+__device__ __forceinline__ int locate(const int *tile_start, int ng, int u) {
+  int lo = 0, hi = ng - 1;
+  while (lo < hi) {
+    const int mid = (lo + hi + 1) >> 1;
+    if (tile_start[mid] <= u) lo = mid; else hi = mid - 1;
+  }
+  return lo;
+}
+
+template <int G, int AW>
+__global__ void __launch_bounds__(kThreads, 1)
+    indexer_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmQ,
+                   const IndexerParams p) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                              ~static_cast<uintptr_t>(1023));
+  const int S = p.stages;
+  const int natoms = p.D_I * 2 / AW;            // swizzle atoms along K
+  const int stage_bytes = kTileKeys * p.D_I * 2;
+  const int ncols = G * p.H_I;                  // useful accumulator columns
+  const int n_mma = (ncols + 15) & ~15;         // MMA N (multiple of 16)
+  const int q_bytes = natoms * n_mma * AW;
+  const uint32_t acc_stride = (n_mma + 31) & ~31;
+  uint32_t tmem_cols = 32;
+  while (tmem_cols < 2 * acc_stride) tmem_cols <<= 1;
+
+  uint8_t *stage_base = smem;
+  uint8_t *q_base = smem + S * stage_bytes;
+  uint64_t *bars = reinterpret_cast<uint64_t *>(q_base + 2 * q_bytes);
+  uint64_t *full = bars;
+  uint64_t *empty = bars + S;
+  uint64_t *qfull = bars + 2 * S;
+  uint64_t *qempty = qfull + 2;
+  uint64_t *tfull = qempty + 2;
+  uint64_t *tempty = tfull + 2;
+  uint64_t *drain = tempty + 2;
+  uint32_t *misc = reinterpret_cast<uint32_t *>(drain + 1);  // [0] tmem base, [1] abort
+  int *scan_tmp = reinterpret_cast<int *>(misc + 4);          // [kThreads]
+  int *tile_start = scan_tmp + kThreads;                      // [num_groups + 1]
+
+  const int warp = warp_id(), lane = lane_id();
+  const int NG = p.num_groups;
+
+  if (threadIdx.x == 0) {
+    for (int i = 0; i < S; ++i) { mbar_init(&full[i], 1); mbar_init(&empty[i], 1); }
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(&qfull[i], 1); mbar_init(&qempty[i], 1);
+      mbar_init(&tfull[i], 1); mbar_init(&tempty[i], 4);
+    }
+    mbar_init(drain, 1);
+    misc[1] = 0u;
+    fence_barrier_init();
+  }
+  if (warp == 0 && lane == 0) { tma_prefetch_desc(&tmK); tma_prefetch_desc(&tmQ); }
+  if (warp == 1) { tmem_alloc(&misc[0], tmem_cols); tmem_relinquish(); }
+
+  // tile prefix over row groups (every CTA computes the same table)
+  {
+    const int per = (NG + kThreads - 1) / kThreads;
+    const int g0 = min(NG, static_cast<int>(threadIdx.x) * per), g1 = min(NG, g0 + per);
+    int local = 0;
+    for (int g = g0; g < g1; ++g) local += (group_keys<G>(p, g) + kTileKeys - 1) / kTileKeys;
+    scan_tmp[threadIdx.x] = local;
+    __syncthreads();
+    if (threadIdx.x == 0) {
+      int run = 0;
+      for (int i = 0; i < kThreads; ++i) { const int v = scan_tmp[i]; scan_tmp[i] = run; run += v; }
+      tile_start[NG] = run;
+    }
+    __syncthreads();
+    int run = scan_tmp[threadIdx.x];
+    for (int g = g0; g < g1; ++g) {
+      tile_start[g] = run;
+      run += (group_keys<G>(p, g) + kTileKeys - 1) / kTileKeys;
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem_base = misc[0];
+  volatile uint32_t *abort_flag = &misc[1];
+
+  const int total = tile_start[NG];
+  const int u0 = static_cast<int>((static_cast<int64_t>(total) * blockIdx.x) / gridDim.x);
+  const int u1 = static_cast<int>((static_cast<int64_t>(total) * (blockIdx.x + 1)) / gridDim.x);
+  const uint32_t layout = (AW == 128) ? kLayoutSW128 : kLayoutSW64;
+
+  if (warp == 0) {
+    // ------------------------------------------------------------ producer
+    int stage = 0, qslot = 0, cur = -1;
+    uint32_t phase = 0, qphase = 0;
+    uint32_t armed = 0, armed_par = 0;  // stages with loads in flight, their phase parity
+    bool ok = true;
+    for (int ub = u0; ub < u1 && ok; ub += kLookahead) {
+      // lane-parallel lookahead: lane l fetches page (l & 1) of unit ub + l/2
+      const int my_u = ub + (lane >> 1);
+      int my_g = -1, my_id = -1;
+      if (my_u < u1) {
+        my_g = locate(tile_start, NG, my_u);
+        const int t = my_u - tile_start[my_g];
+        const int pg = 2 * t + (lane & 1);
+        if (pg * kPageSize < group_keys<G>(p, my_g)) {
+          const int b = p.causal ? 0 : my_g;
+          const int id = p.block_table[static_cast<int64_t>(b) * p.max_pages + pg];
+          if (id < 0 || id >= p.num_pages)
+            report(p.status, kErrBadPage, (kKernIndexer << 24) | (pg & 0xFFFF));
+          else
+            my_id = id;
+        }
+      }
+      const int nb = min(kLookahead, u1 - ub);
+      for (int i = 0; i < nb; ++i) {
+        const int g = __shfl_sync(0xffffffffu, my_g, 2 * i);
+        const int id0 = __shfl_sync(0xffffffffu, my_id, 2 * i);
+        const int id1 = __shfl_sync(0xffffffffu, my_id, 2 * i + 1);
+        int okl = 1;
+        if (lane == 0) {
+          if (*abort_flag) okl = 0;
+          if (okl && g != cur) {
+            if (!mbar_wait(&qempty[qslot], qphase ^ 1u, p.wait_ns)) {
+              okl = 0;
+            } else {
+              mbar_arrive_expect_tx(&qfull[qslot], static_cast<uint32_t>(natoms * ncols * AW));
+              for (int a = 0; a < natoms; ++a)
+                tma_load_2d(q_base + qslot * q_bytes + a * n_mma * AW, &tmQ, a * (AW / 2),
+                            g * ncols, &qfull[qslot]);
+            }
+          }
+          if (okl && !mbar_wait(&empty[stage], phase ^ 1u, p.wait_ns)) okl = 0;
+          if (okl) {
+            const uint32_t page_bytes = kPageSize * p.D_I * 2;
+            const uint32_t bytes = ((id0 >= 0) + (id1 >= 0)) * page_bytes;
+            uint8_t *dst = stage_base + stage * stage_bytes;
+            if (bytes == 0) {
+              mbar_arrive(&full[stage]);
+            } else {
+              mbar_arrive_expect_tx(&full[stage], bytes);
+              for (int a = 0; a < natoms; ++a) {
+                if (id0 >= 0)
+                  tma_load_2d(dst + a * kTileKeys * AW, &tmK, a * (AW / 2), id0 * kPageSize,
+                              &full[stage]);
+                if (id1 >= 0)
+                  tma_load_2d(dst + a * kTileKeys * AW + kPageSize * AW, &tmK, a * (AW / 2),
+                              id1 * kPageSize, &full[stage]);
+              }
+              armed |= 1u << stage;
+              armed_par = (armed_par & ~(1u << stage)) | (phase << stage);
+            }
+          }
+        }
+        okl = __shfl_sync(0xffffffffu, okl, 0);
+        if (!okl) { ok = false; break; }
+        if (g != cur) {
+          cur = g;
+          qslot ^= 1;
+          if (qslot == 0) qphase ^= 1u;
+        }
+        if (++stage == S) { stage = 0; phase ^= 1u; }
+      }
+    }
+    if (lane == 0) {
+      if (!ok && !*abort_flag) {
+        *abort_flag = 1u;
+        report(p.status, kErrTimeout, (kKernIndexer << 24) | 0x1);
+      }
+      for (int s = 0; s < S; ++s)  // drain loads in flight
+        if (armed & (1u << s)) mbar_wait(&full[s], (armed_par >> s) & 1u, kDrainLimitNs);
+    }
+  } else if (warp == 1) {
+    // ------------------------------------------------------------ MMA issuer
+    if (lane == 0) {
+      const uint32_t idesc = idesc_bf16_f32(kTileKeys, n_mma, 0, 0);
+      int stage = 0, qslot = 0, cur = -1, cur_slot = 0, acc = 0;
+      uint32_t phase = 0, qphase = 0, aphase = 0;
+      bool ok = true;
+      int g = (u0 < u1) ? locate(tile_start, NG, u0) : 0;
+      for (int u = u0; u < u1; ++u) {
+        while (tile_start[g + 1] <= u) ++g;
+        if (*abort_flag) { ok = false; break; }
+        if (g != cur) {
+          if (!mbar_wait(&qfull[qslot], qphase, p.wait_ns)) { ok = false; break; }
+          cur = g;
+          cur_slot = qslot;
+          qslot ^= 1;
+          if (qslot == 0) qphase ^= 1u;
+        }
+        if (!mbar_wait(&full[stage], phase, p.wait_ns)) { ok = false; break; }
+        if (!mbar_wait(&tempty[acc], aphase ^ 1u, p.wait_ns)) { ok = false; break; }
+        tc_fence_after();
+        const uint32_t d = tmem_base + acc * acc_stride;
+        const uint32_t a_base = smem_u32(stage_base + stage * stage_bytes);
+        const uint32_t b_base = smem_u32(q_base + cur_slot * q_bytes);
+        for (int a = 0; a < natoms; ++a) {
+          for (int kk = 0; kk < AW / 32; ++kk) {
+            const uint64_t adesc = smem_desc(a_base + a * kTileKeys * AW + kk * 32, 16, 8 * AW, layout);
+            const uint64_t bdesc = smem_desc(b_base + a * n_mma * AW + kk * 32, 16, 8 * AW, layout);
+            mma_bf16(d, adesc, bdesc, idesc, (a | kk) != 0 ? 1u : 0u);
+          }
+        }
+        mma_commit(&empty[stage]);
+        mma_commit(&tfull[acc]);
+        const bool last_of_group = (u + 1 == u1) || (tile_start[g + 1] <= u + 1);
+        if (last_of_group) mma_commit(&qempty[cur_slot]);
+        if (++stage == S) { stage = 0; phase ^= 1u; }
+        acc ^= 1;
+        if (acc == 0) aphase ^= 1u;
+      }
+      if (!ok && !*abort_flag) {
+        *abort_flag = 1u;
+        report(p.status, kErrTimeout, (kKernIndexer << 24) | 0x2);
+      }
+      mma_commit(drain);  // every MMA issued above has completed once this fires
+      mbar_wait(drain, 0, kDrainLimitNs);
+    }
+  } else {
+    // ------------------------------------------------------------ epilogue
+    const int quad = warp & 3;           // tensor-memory lane quadrant of this warp
+    const int key_in_tile = quad * 32 + lane;
+    const int nchunks = (ncols + 31) / 32;
+    int acc = 0;
+    uint32_t aphase = 0;
+    bool ok = true;
+    int g = (u0 < u1) ? locate(tile_start, NG, u0) : 0;
+    for (int u = u0; u < u1; ++u) {
+      while (tile_start[g + 1] <= u) ++g;
+      if (__any_sync(0xffffffffu, *abort_flag != 0u)) { ok = false; break; }
+      if (!__all_sync(0xffffffffu, mbar_wait(&tfull[acc], aphase, p.wait_ns))) { ok = false; break; }
+      tc_fence_after();
+      float s[G];
+#pragma unroll
+      for (int j = 0; j < G; ++j) s[j] = 0.f;
+      const uint32_t taddr = tmem_base + (static_cast<uint32_t>(quad * 32) << 16) + acc * acc_stride;
+      for (int c = 0; c < nchunks; ++c) {
+        uint32_t v[32];
+        tmem_ld_32x32b_x32(taddr + c * 32, v);
+        tmem_ld_wait();
+        float part = 0.f;
+#pragma unroll
+        for (int i = 0; i < 32; ++i) {
+          const int col = c * 32 + i;
+          if (col < ncols) {
+            const int r = min(g * G + col / p.H_I, p.n_q - 1);
+            const float wv = __ldg(&p.w[static_cast<int64_t>(r) * p.H_I + (col % p.H_I)]);
+            const float x = __uint_as_float(v[i]);
+            part += wv * (x > 0.f ? x : 0.f);
+          }
+        }
+        if (G == 1) {
+          s[0] += part;
+        } else {
+          const int j = (c * 32) / p.H_I;  // H_I is a multiple of 32 when G > 1
+#pragma unroll
+          for (int jj = 0; jj < G; ++jj)
+            if (jj == j) s[jj] += part;
+        }
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&tempty[acc]);
+      const int t = u - tile_start[g];
+      const int key = t * kTileKeys + key_in_tile;
+#pragma unroll
+      for (int j = 0; j < G; ++j) {
+        const int r = p.causal ? g * G + j : g;
+        if (r < p.n_q && key < row_keys(p, r)) p.scores[static_cast<int64_t>(r) * p.ld + key] = s[j];
+      }
+      acc ^= 1;
+      if (acc == 0) aphase ^= 1u;
+    }
+    if (!ok && lane == 0 && !*abort_flag) {
+      *abort_flag = 1u;
+      report(p.status, kErrTimeout, (kKernIndexer << 24) | 0x3);
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  if (warp == 1) {
+    __syncwarp();
+    tmem_dealloc(tmem_base, tmem_cols);
+  }
+}
+
+// ---------------------------------------------------------------------------
+// host side
+// ---------------------------------------------------------------------------
+PFN_cuTensorMapEncodeTiled_v12000 get_encode_fn() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  static bool tried = false;
+  if (!tried) {
+    tried = true;
+    void *ptr = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) ==
+            cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(ptr);
+  }
+  return fn;
+}
+
+// 2-D bf16 tensor map: `rows` rows of `cols` elements, box of box_cols x box_rows.
+bool make_map_2d(CUtensorMap *map, const void *base, uint64_t cols, uint64_t rows,
+                 uint32_t box_cols, uint32_t box_rows, int aw) {
+  auto encode = get_encode_fn();
+  if (encode == nullptr) return false;
+  cuuint64_t dims[2] = {cols, rows};
+  cuuint64_t strides[1] = {cols * 2};
+  cuuint32_t box[2] = {box_cols, box_rows};
+  cuuint32_t estr[2] = {1, 1};
+  CUresult r = encode(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void *>(base), dims,
+                      strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                      aw == 128 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_64B,
+                      CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
+template <int G, int AW>
+dsa_status_t launch_impl(const IndexerLaunch &a, cudaStream_t stream) {
+  const int natoms = a.D_I * 2 / AW;
+  const int ncols = G * a.H_I;
+  const int n_mma = (ncols + 15) & ~15;
+  const int num_groups = a.causal ? (a.n_q + G - 1) / G : a.n_q;
+  CUtensorMap tmK, tmQ;
+  if (!make_map_2d(&tmK, a.k_pages, a.D_I, static_cast<uint64_t>(a.num_pages) * kPageSize, AW / 2,
+                   kPageSize, AW))
+    return DSA_ERR_CUDA;
+  if (!make_map_2d(&tmQ, a.q_idx, a.D_I, static_cast<uint64_t>(a.n_q) * a.H_I, AW / 2, ncols, AW))
+    return DSA_ERR_CUDA;
+  (void)natoms;
+
+  const size_t stage_bytes = static_cast<size_t>(kTileKeys) * a.D_I * 2;
+  const size_t q_bytes = static_cast<size_t>(natoms) * n_mma * AW;
+  const size_t fixed = 1024 /*align*/ + 2 * q_bytes + 8 * (2 * 8 + 9) + 16 + 4 * kThreads +
+                       4 * ((num_groups + 4) & ~3) + 64;
+  const size_t max_smem = device_max_smem_optin();
+  int stages = static_cast<int>((max_smem - fixed) / stage_bytes);
+  stages = std::min(stages, 8);
+  if (stages < 2) return DSA_ERR_UNSUPPORTED;
+  const size_t smem = fixed + stages * stage_bytes;
+
+  static bool attr_set = false;  // per template instantiation
+  if (!attr_set) {
+    if (cudaFuncSetAttribute(indexer_kernel<G, AW>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             static_cast<int>(max_smem)) != cudaSuccess)
+      return DSA_ERR_CUDA;
+    attr_set = true;
+  }
+  const int64_t max_keys = a.causal ? static_cast<int64_t>(a.q_pos0) + a.n_q : a.max_seq_len;
+  const int64_t max_units = static_cast<int64_t>(num_groups) * ((max_keys + kTileKeys - 1) / kTileKeys);
+  const int grid = static_cast<int>(std::max<int64_t>(1, std::min<int64_t>(device_sm_count(), max_units)));
+
+  IndexerParams p;
+  p.w = a.w;
+  p.seq_lens = a.seq_lens;
+  p.block_table = a.block_table;
+  p.scores = a.scores;
+  p.ld = a.ld;
+  p.n_q = a.n_q;
+  p.H_I = a.H_I;
+  p.D_I = a.D_I;
+  p.causal = a.causal;
+  p.q_pos0 = a.q_pos0;
+  p.max_pages = a.max_pages;
+  p.num_pages = a.num_pages;
+  p.num_groups = num_groups;
+  p.stages = stages;
+  p.wait_ns = wait_limit_ns();
+  p.status = a.status;
+  indexer_kernel<G, AW><<<grid, kThreads, smem, stream>>>(tmK, tmQ, p);
+  return cudaGetLastError() == cudaSuccess ? DSA_OK : DSA_ERR_CUDA;
+}
+
+}  // namespace
+
+dsa_status_t launch_indexer(const IndexerLaunch &a, cudaStream_t stream) {
+  const bool grouped = a.causal && (a.H_I % 32 == 0) && (4 * a.H_I <= 256);
+  if (a.D_I == 32) return grouped ? launch_impl<4, 64>(a, stream) : launch_impl<1, 64>(a, stream);
+  return grouped ? launch_impl<4, 128>(a, stream) : launch_impl<1, 128>(a, stream);
+}
+
+}  // namespace dsa

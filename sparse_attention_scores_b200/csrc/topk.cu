@@ -1,0 +1,265 @@
+// Step 2 of the DSA step: exact top-k with the stable lower-index tie rule.
+//
+// ("GLM on an A100, in Vx", section "The model": each query keeps the 2,048
+// highest-scoring tokens, all of them below 2,048; section "How do we know it
+// is right?": ties resolve as a stable argsort of -scores does, i.e. the lower
+// token index wins.)
+//
+// Design: one thread-block cluster of C CTAs per row.  Each CTA owns a
+// contiguous segment of the row and keeps the order-preserving 32-bit keys of
+// its scores in shared memory (re-reading global memory only when a segment
+// is larger than shared memory).  Three radix passes (11 + 11 + 10 bits) find
+// the exact k-th largest key T: every CTA builds a shared-memory histogram
+// (warp-aggregated atomics), the cluster barrier publishes it, and every CTA
+// sums all C histograms through distributed shared memory and runs the same
+// deterministic suffix scan.  The kept set is {key > T} plus the first
+// (k - #{key > T}) keys equal to T in index order, which a block-wide scan
+// compacts in ascending index order: output position = number of kept tokens
+// with a lower index.  No sort, no global atomics, no global scratch.
+#include <algorithm>
+
+#include "dsa_internal.h"
+
+namespace dsa {
+namespace {
+
+constexpr int kThreads = 512;
+constexpr int kWarps = kThreads / 32;
+constexpr int kBins = 2048;
+
+struct TopkParams {
+  const float *scores;
+  int64_t ld;
+  int n_q;
+  const int32_t *valid_len;
+  int causal_base;
+  int k;
+  int32_t *idx;
+  int seg_cap;  // keys a CTA can keep in shared memory
+  DevStatus *status;
+};
+
+// exclusive block-wide prefix sum of v; *total receives the block sum
+__device__ __forceinline__ int block_exclusive_scan(int v, int *warp_sums, int *total) {
+  const int lane = lane_id(), warp = warp_id();
+  int x = v;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const int y = __shfl_up_sync(0xffffffffu, x, o);
+    if (lane >= o) x += y;
+  }
+  if (lane == 31) warp_sums[warp] = x;
+  __syncthreads();
+  if (warp == 0) {
+    int s = (lane < kWarps) ? warp_sums[lane] : 0;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int y = __shfl_up_sync(0xffffffffu, s, o);
+      if (lane >= o) s += y;
+    }
+    if (lane < kWarps) warp_sums[lane] = s;
+  }
+  __syncthreads();
+  const int before = (warp > 0) ? warp_sums[warp - 1] : 0;
+  *total = warp_sums[kWarps - 1];
+  __syncthreads();
+  return before + x - v;
+}
+
+// exclusive suffix sum (sum over threads with a higher id)
+__device__ __forceinline__ int block_exclusive_suffix(int v, int *warp_sums) {
+  const int lane = lane_id(), warp = warp_id();
+  int x = v;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const int y = __shfl_down_sync(0xffffffffu, x, o);
+    if (lane + o < 32) x += y;
+  }
+  if (lane == 0) warp_sums[warp] = x;
+  __syncthreads();
+  if (warp == 0) {
+    int s = (lane < kWarps) ? warp_sums[lane] : 0;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int y = __shfl_down_sync(0xffffffffu, s, o);
+      if (lane + o < 32) s += y;
+    }
+    if (lane < kWarps) warp_sums[lane] = s;
+  }
+  __syncthreads();
+  const int after = (warp + 1 < kWarps) ? warp_sums[warp + 1] : 0;
+  __syncthreads();
+  return after + x - v;
+}
+
+__global__ void __launch_bounds__(kThreads, 1) topk_kernel(const TopkParams p) {
+  extern __shared__ uint32_t sm[];
+  uint32_t *hist = sm;                                         // [kBins]
+  int *warp_sums = reinterpret_cast<int *>(sm + kBins);        // [32]
+  int *bcast = warp_sums + 32;                                 // [8]
+  uint32_t *cnts = reinterpret_cast<uint32_t *>(bcast + 8);    // [2] per-CTA gt / eq counts
+  uint32_t *keys = cnts + 8;                                   // [seg_cap]
+
+  const uint32_t C = cluster_nctarank();
+  const uint32_t c = cluster_ctarank();
+  const int row = blockIdx.x / C;
+  const int tid = threadIdx.x;
+  const int k = p.k;
+  int32_t *out = p.idx + static_cast<int64_t>(row) * k;
+
+  int n = p.valid_len ? p.valid_len[row] : p.causal_base + row + 1;
+  if (static_cast<int64_t>(n) > p.ld) n = static_cast<int>(p.ld);
+  if (n < 0) n = 0;
+
+  if (n <= k) {  // every token is kept: 0..n-1, then -1
+    for (int i = c * kThreads + tid; i < k; i += C * kThreads) out[i] = (i < n) ? i : -1;
+    return;  // the whole cluster takes this branch; no shared memory was shared
+  }
+
+  const float *srow = p.scores + static_cast<int64_t>(row) * p.ld;
+  const int seg = ((n + C - 1) / C + 3) & ~3;
+  const int lo = min(n, static_cast<int>(c) * seg);
+  const int cnt = max(0, min(n, lo + seg) - lo);
+  const bool cached = seg <= p.seg_cap;
+  if (cached) {
+    for (int i = tid; i < cnt; i += kThreads) keys[i] = score_key(srow[lo + i]);
+  }
+  __syncthreads();
+  auto key_at = [&](int i) -> uint32_t { return cached ? keys[i] : score_key(srow[lo + i]); };
+
+  uint32_t prefix = 0, pmask = 0;
+  int krem = k;
+#pragma unroll 1
+  for (int pass = 0; pass < 3; ++pass) {
+    const int shift = (pass == 0) ? 21 : (pass == 1 ? 10 : 0);
+    const uint32_t bmask = (pass < 2) ? 0x7FFu : 0x3FFu;
+    for (int i = tid; i < kBins; i += kThreads) hist[i] = 0u;
+    __syncthreads();
+    for (int base = 0; base < cnt; base += kThreads) {
+      const int i = base + tid;
+      bool match = false;
+      uint32_t bin = 0xFFFFFFFFu;
+      if (i < cnt) {
+        const uint32_t u = key_at(i);
+        match = (u & pmask) == prefix;
+        if (match) bin = (u >> shift) & bmask;
+      }
+      const uint32_t peers = __match_any_sync(0xffffffffu, bin);
+      if (match && lane_id() == __ffs(peers) - 1) atomicAdd(&hist[bin], __popc(peers));
+    }
+    cluster_sync();  // all histograms of this pass are complete
+    // global histogram: thread t owns bins 4t .. 4t+3
+    uint32_t gh[4] = {0u, 0u, 0u, 0u};
+    for (uint32_t r = 0; r < C; ++r) {
+#pragma unroll
+      for (int q = 0; q < 4; ++q)
+        gh[q] += ld_dsmem_u32(map_to_rank(smem_u32(&hist[4 * tid + q]), r));
+    }
+    const int mine = static_cast<int>(gh[0] + gh[1] + gh[2] + gh[3]);
+    int above = block_exclusive_suffix(mine, warp_sums);
+    // the bin where the running count from the top reaches krem
+#pragma unroll
+    for (int q = 3; q >= 0; --q) {
+      const int h = static_cast<int>(gh[q]);
+      if (above < krem && krem <= above + h) { bcast[0] = 4 * tid + q; bcast[1] = krem - above; }
+      above += h;
+    }
+    cluster_sync();  // peers finished reading this CTA's histogram; bcast is visible
+    const uint32_t sel = static_cast<uint32_t>(bcast[0]);
+    krem = bcast[1];
+    prefix |= sel << shift;
+    pmask |= bmask << shift;
+  }
+  const uint32_t T = prefix;   // the k-th largest key
+  const int need_eq = krem;    // how many keys equal to T are kept
+
+  // per-CTA counts of keys above / equal to T, shared through the cluster
+  int gt_l = 0, eq_l = 0;
+  for (int i = tid; i < cnt; i += kThreads) {
+    const uint32_t u = key_at(i);
+    gt_l += (u > T);
+    eq_l += (u == T);
+  }
+  int tot;
+  block_exclusive_scan(gt_l, warp_sums, &tot);
+  if (tid == 0) cnts[0] = static_cast<uint32_t>(tot);
+  block_exclusive_scan(eq_l, warp_sums, &tot);
+  if (tid == 0) cnts[1] = static_cast<uint32_t>(tot);
+  cluster_sync();
+  if (tid == 0) {
+    uint32_t gt_before = 0, eq_before = 0;
+    for (uint32_t r = 0; r < c; ++r) {
+      gt_before += ld_dsmem_u32(map_to_rank(smem_u32(&cnts[0]), r));
+      eq_before += ld_dsmem_u32(map_to_rank(smem_u32(&cnts[1]), r));
+    }
+    bcast[2] = static_cast<int>(eq_before);
+    bcast[3] = static_cast<int>(gt_before + umin(eq_before, static_cast<uint32_t>(need_eq)));
+  }
+  __syncthreads();
+  int carry_eq = bcast[2], carry_sel = bcast[3];
+  for (int base = 0; base < cnt; base += kThreads) {
+    const int i = base + tid;
+    uint32_t u = 0;
+    if (i < cnt) u = key_at(i);
+    const int gt = (i < cnt) && (u > T);
+    const int eq = (i < cnt) && (u == T);
+    int eq_tot;
+    const int eq_rank = carry_eq + block_exclusive_scan(eq, warp_sums, &eq_tot);
+    const int keep = gt || (eq && eq_rank < need_eq);
+    int sel_tot;
+    const int pos = carry_sel + block_exclusive_scan(keep, warp_sums, &sel_tot);
+    if (keep && pos < k) out[pos] = lo + i;
+    carry_eq += eq_tot;
+    carry_sel += sel_tot;
+  }
+  cluster_sync();  // keep this CTA's shared memory alive until peers are done
+}
+
+}  // namespace
+
+dsa_status_t launch_topk(const TopkLaunch &a, cudaStream_t stream) {
+  const int max_len = std::max(1, a.max_len);
+  int C = (max_len + 4095) / 4096;
+  C = std::max(1, std::min(C, 8));
+  const int seg = ((max_len + C - 1) / C + 3) & ~3;
+  const size_t fixed = 4 * (kBins + 32 + 8 + 8) + 64;
+  const size_t max_smem = device_max_smem_optin();
+  const int cap_max = static_cast<int>((max_smem - fixed) / 4);
+  const int seg_cap = std::min(seg, cap_max);
+  const size_t smem = fixed + 4 * static_cast<size_t>(seg_cap);
+
+  static bool attr_set = false;
+  if (!attr_set) {
+    if (cudaFuncSetAttribute(topk_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             static_cast<int>(max_smem)) != cudaSuccess)
+      return DSA_ERR_CUDA;
+    attr_set = true;
+  }
+  TopkParams p;
+  p.scores = a.scores;
+  p.ld = a.ld;
+  p.n_q = a.n_q;
+  p.valid_len = a.valid_len;
+  p.causal_base = a.causal_base;
+  p.k = a.k;
+  p.idx = a.idx;
+  p.seg_cap = seg_cap;
+  p.status = a.status;
+
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(static_cast<unsigned>(a.n_q) * C, 1, 1);
+  cfg.blockDim = dim3(kThreads, 1, 1);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = C;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  if (cudaLaunchKernelEx(&cfg, topk_kernel, p) != cudaSuccess) return DSA_ERR_CUDA;
+  return DSA_OK;
+}
+
+}  // namespace dsa
