@@ -19,6 +19,14 @@ uint64_t wait_limit_ns() {
   return v;
 }
 
+int debug_stall() {
+  static const int v = [] {
+    const char *s = getenv("DSA_DEBUG_STALL");
+    return (s != nullptr && *s != '\0') ? atoi(s) : 0;
+  }();
+  return v;
+}
+
 namespace {
 constexpr int kMaxDevices = 64;
 int g_sm_count[kMaxDevices];

@@ -13,6 +13,11 @@ namespace dsa {
 // second by default; the environment variable DSA_WAIT_LIMIT_NS overrides it
 // (read once), which lets a test force the time-out path.
 uint64_t wait_limit_ns();
+// Test hook (environment variable DSA_DEBUG_STALL, read once): a kernel id
+// (1 = indexer, 3 = sparse MLA) whose CTAs first wait on a barrier that
+// nothing arrives at, so that the bounded wait runs out and the kernel takes
+// its error path.  0 (the default) disables it.
+int debug_stall();
 // Fixed limit used while draining copies/MMAs in flight on the error path.
 constexpr uint64_t kDrainLimitNs = 1000000000ull;
 

@@ -43,6 +43,7 @@ struct IndexerParams {
   int num_groups;
   int stages;
   uint64_t wait_ns;
+  int debug_stall;  // the MMA issuer first waits on a barrier nothing arrives at
   DevStatus *status;
 };
 
@@ -240,8 +241,9 @@ __global__ void __launch_bounds__(kThreads, 1)
       int stage = 0, qslot = 0, cur = -1, cur_slot = 0, acc = 0;
       uint32_t phase = 0, qphase = 0, aphase = 0;
       bool ok = true;
+      if (p.debug_stall && !mbar_wait(drain, 0, p.wait_ns)) ok = false;
       int g = (u0 < u1) ? locate(tile_start, NG, u0) : 0;
-      for (int u = u0; u < u1; ++u) {
+      for (int u = u0; u < u1 && ok; ++u) {
         while (tile_start[g + 1] <= u) ++g;
         if (*abort_flag) { ok = false; break; }
         if (g != cur) {
@@ -434,6 +436,7 @@ dsa_status_t launch_impl(const IndexerLaunch &a, cudaStream_t stream) {
   p.num_groups = num_groups;
   p.stages = stages;
   p.wait_ns = wait_limit_ns();
+  p.debug_stall = debug_stall() == kKernIndexer ? 1 : 0;
   p.status = a.status;
   indexer_kernel<G, AW><<<grid, kThreads, smem, stream>>>(tmK, tmQ, p);
   return cudaGetLastError() == cudaSuccess ? DSA_OK : DSA_ERR_CUDA;

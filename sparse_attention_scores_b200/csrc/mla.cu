@@ -23,6 +23,7 @@
 //   O^T     += tcgen05.mma, M = 128 latent columns (R/128 blocks), N = 64
 //            heads, K = 128 keys; the same shared tile serves as V^T
 //            (MN-major view), P is written as bf16 over the rope atom
+// PV uses p = hi + lo (two bf16 terms) for near-fp32 weights.
 // A row split over several CTAs writes (m, l, O) partials that a second
 // kernel merges by log-sum-exp weights.
 #include <algorithm>
@@ -55,6 +56,7 @@ struct MlaParams {
   int nsplit, chunks_per_split;
   float scale_log2;
   uint64_t wait_ns;
+  int debug_stall;  // wait once on a barrier nothing arrives at (tests the time-out path)
   DevStatus *status;
 };
 
@@ -79,8 +81,8 @@ __device__ __forceinline__ void tmem_st_wait() {
 // at once.  Each butterfly step halves the heads a lane keeps and exchanges
 // the other half with its partner; afterwards lane L holds the reductions of
 // heads 2L and 2L+1 in o[0], o[1].  62 shuffles instead of 64 x 5.
-template <bool kMax>
-__device__ __forceinline__ void butterfly64(const float (&v)[64], float (&o)[2]) {
+template <bool kMax, typename Get>
+__device__ __forceinline__ void butterfly64(Get v, float (&o)[2]) {
   const int lane = lane_id();
   auto op = [](float a, float b) { return kMax ? fmaxf(a, b) : a + b; };
   float a[32];
@@ -88,8 +90,9 @@ __device__ __forceinline__ void butterfly64(const float (&v)[64], float (&o)[2])
     const bool up = lane & 16;
 #pragma unroll
     for (int i = 0; i < 32; ++i) {
-      const float send = up ? v[i] : v[i + 32];
-      const float keep = up ? v[i + 32] : v[i];
+      const float lo_h = v(i), hi_h = v(i + 32);
+      const float send = up ? lo_h : hi_h;
+      const float keep = up ? hi_h : lo_h;
       a[i] = op(keep, __shfl_xor_sync(0xffffffffu, send, 16));
     }
   }
@@ -170,6 +173,7 @@ __global__ void __launch_bounds__(kThreads, 1) mla_kernel(const MlaParams p) {
     mbar_init(&bars[0], 1);
     mbar_init(&bars[1], 1);
     mbar_init(&bars[2], 1);
+    mbar_init(&bars[3], 1);
     misc[1] = 0u;
     misc[2] = 0u;
     fence_barrier_init();
@@ -197,10 +201,15 @@ __global__ void __launch_bounds__(kThreads, 1) mla_kernel(const MlaParams p) {
   const uint32_t lane_off = static_cast<uint32_t>(warp * 32) << 16;
   const uint32_t idesc_s = idesc_bf16_f32(kChunk, kHeads, 0, 0);
   const uint32_t idesc_pv = idesc_bf16_f32(kChunk, kHeads, 1, 1);
-  uint32_t phase = 0;
+  uint32_t phase = 0, pv_phase = 0;
   bool have_o = false;
   bool failed = false;
 
+  if (p.debug_stall) {
+    if (!mbar_wait(&bars[3], 0u, p.wait_ns)) misc[2] = 1u;
+    __syncthreads();
+    if (misc[2]) failed = true;
+  }
   for (int ch = c_begin; ch < c_end && !failed; ++ch) {
     // resolve the 128 selected positions of this chunk
     {
@@ -276,7 +285,7 @@ __global__ void __launch_bounds__(kThreads, 1) mla_kernel(const MlaParams p) {
     // per-head chunk max over the 128 keys
     {
       float o[2];
-      butterfly64<true>(z, o);
+      butterfly64<true>([&](int h) { return z[h]; }, o);
       red[warp * kHeads + 2 * lane] = o[0];
       red[warp * kHeads + 2 * lane + 1] = o[1];
     }
@@ -292,29 +301,29 @@ __global__ void __launch_bounds__(kThreads, 1) mla_kernel(const MlaParams p) {
       if (a != 1.f && have_o) misc[1] = 1u;
     }
     __syncthreads();
-    // probabilities (bf16 for the PV product; sums use the rounded values)
-    float pf[64];
-    {
+    // probabilities, split into a bf16 head and a bf16 tail: p = hi + lo to
+    // about 2^-17, so the PV product keeps near-fp32 weights even when a few
+    // keys dominate.  Sums use hi + lo.
+    uint32_t phi[32], plo[32];  // packed bf16 pairs of heads (2i, 2i+1)
 #pragma unroll
-      for (int j = 0; j < 8; ++j) {
-        uint32_t packed[4];
-#pragma unroll
-        for (int e = 0; e < 8; e += 2) {
-          const int h = 8 * j + e;
-          const float p0 = (z[h] == -INFINITY) ? 0.f : exp2f(z[h] - mrun[h]);
-          const float p1 = (z[h + 1] == -INFINITY) ? 0.f : exp2f(z[h + 1] - mrun[h + 1]);
-          const __nv_bfloat162 pb = __floats2bfloat162_rn(p0, p1);
-          pf[h] = __low2float(pb);
-          pf[h + 1] = __high2float(pb);
-          packed[e >> 1] = *reinterpret_cast<const uint32_t *>(&pb);
-        }
-        const uint32_t dst = smem_u32(Ps) + tid * 128 + ((j ^ (tid & 7)) << 4);
-        asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(dst), "r"(packed[0]),
-                     "r"(packed[1]), "r"(packed[2]), "r"(packed[3])
-                     : "memory");
-      }
+    for (int i = 0; i < 32; ++i) {
+      const int h = 2 * i;
+      const float p0 = (z[h] == -INFINITY) ? 0.f : exp2f(z[h] - mrun[h]);
+      const float p1 = (z[h + 1] == -INFINITY) ? 0.f : exp2f(z[h + 1] - mrun[h + 1]);
+      const __nv_bfloat162 hi = __floats2bfloat162_rn(p0, p1);
+      const __nv_bfloat162 lo =
+          __floats2bfloat162_rn(p0 - __low2float(hi), p1 - __high2float(hi));
+      phi[i] = *reinterpret_cast<const uint32_t *>(&hi);
+      plo[i] = *reinterpret_cast<const uint32_t *>(&lo);
     }
     {
+      // p of head h as the PV product sees it: hi + lo
+      auto pf = [&](int h) {
+        const uint32_t a = phi[h >> 1], b = plo[h >> 1];
+        const uint32_t ha = (h & 1) ? (a & 0xFFFF0000u) : (a << 16);
+        const uint32_t hb = (h & 1) ? (b & 0xFFFF0000u) : (b << 16);
+        return __uint_as_float(ha) + __uint_as_float(hb);
+      };
       float o[2];
       butterfly64<false>(pf, o);
       red[warp * kHeads + 2 * lane] = o[0];
@@ -340,28 +349,48 @@ __global__ void __launch_bounds__(kThreads, 1) mla_kernel(const MlaParams p) {
         }
       tmem_st_wait();
     }
-    fence_proxy_async_smem();
-    tc_fence_before();
-    __syncthreads();
-    tc_fence_after();
-    // O^T += L^T . P^T  (M = 128 latent columns per block, N = 64 heads, K = 128 keys)
-    if (tid == 0) {
-      const uint32_t ls = smem_u32(Ls), ps = smem_u32(Ps);
-      for (int mb = 0; mb < nmb; ++mb)
-        for (int ks = 0; ks < kChunk / 16; ++ks)
-          mma_bf16(tmem_o + mb * kHeads,
-                   smem_desc(ls + 2 * mb * kAtomL + ks * 2048, kAtomL, 1024, kLayoutSW128),
-                   smem_desc(ps + ks * 2048, kAtomQ, 1024, kLayoutSW128), idesc_pv,
-                   (have_o || ks > 0) ? 1u : 0u);
-      mma_commit(&bars[1]);
+    // O^T += L^T . P^T  (M = 128 latent columns per block, N = 64 heads), in two
+    // halves of 64 keys; each half multiplies by the hi and by the lo terms.
+    // The 16 KB P region holds [hi | lo] for the 64 keys of one half.
+    bool pv_failed = false;
+    for (int half = 0; half < 2; ++half) {
+      if ((warp >> 1) == half) {
+        const int rk = tid & 63;
+        const uint32_t base = smem_u32(Ps) + rk * 128;
+#pragma unroll
+        for (int j = 0; j < 8; ++j) {
+          const uint32_t off = ((j ^ (rk & 7)) << 4);
+          asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(base + off),
+                       "r"(phi[4 * j]), "r"(phi[4 * j + 1]), "r"(phi[4 * j + 2]), "r"(phi[4 * j + 3])
+                       : "memory");
+          asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(base + 8192 + off),
+                       "r"(plo[4 * j]), "r"(plo[4 * j + 1]), "r"(plo[4 * j + 2]), "r"(plo[4 * j + 3])
+                       : "memory");
+        }
+      }
+      fence_proxy_async_smem();
+      tc_fence_before();
+      __syncthreads();
+      tc_fence_after();
+      if (tid == 0) {
+        const uint32_t ls = smem_u32(Ls), ps = smem_u32(Ps);
+        for (int mb = 0; mb < nmb; ++mb)
+          for (int part = 0; part < 2; ++part)
+            for (int ks = 0; ks < 4; ++ks)
+              mma_bf16(tmem_o + mb * kHeads,
+                       smem_desc(ls + 2 * mb * kAtomL + (half * 4 + ks) * 2048, kAtomL, 1024,
+                                 kLayoutSW128),
+                       smem_desc(ps + part * 8192 + ks * 2048, kAtomQ, 1024, kLayoutSW128),
+                       idesc_pv, (have_o || half || part || ks) ? 1u : 0u);
+        mma_commit(&bars[1]);
+      }
+      if (!mbar_wait(&bars[1], pv_phase, p.wait_ns)) misc[2] = 1u;
+      pv_phase ^= 1u;
+      tc_fence_after();
+      __syncthreads();
+      if (misc[2]) { pv_failed = true; break; }
     }
-    if (!mbar_wait(&bars[1], phase, p.wait_ns)) {
-      failed = true;
-      misc[2] = 1u;
-    }
-    tc_fence_after();
-    __syncthreads();
-    if (misc[2]) failed = true;
+    if (pv_failed) failed = true;
     have_o = true;
     phase ^= 1u;
   }
@@ -518,6 +547,7 @@ dsa_status_t launch_mla(const MlaLaunch &a, cudaStream_t stream) {
   p.chunks_per_split = cps;
   p.scale_log2 = static_cast<float>(static_cast<double>(a.scale) * 1.4426950408889634);
   p.wait_ns = wait_limit_ns();
+  p.debug_stall = debug_stall() == kKernMla ? 1 : 0;
   p.status = a.status;
   mla_kernel<<<dim3(nsplit, a.n_q), kThreads, smem, stream>>>(p);
   if (cudaGetLastError() != cudaSuccess) return DSA_ERR_CUDA;

@@ -290,16 +290,19 @@ def test_bad_page_id_is_reported_not_faulted():
     assert_row_matches(1, ref[1], idx2, out2, lse2)
 
 
-def test_bounded_wait_timeout_path():
-    # a zero wall-time limit makes every wait that is not already satisfied
-    # give up: the kernels must report DSA_ERR_TIMEOUT and leave the context
-    # usable (run in a child process, which reads the limit at load time)
+@pytest.mark.parametrize("kernel", [1, 3], ids=["indexer", "mla"])
+def test_bounded_wait_timeout_path(kernel):
+    # DSA_DEBUG_STALL makes the chosen kernel wait once on a barrier that
+    # nothing arrives at; with a 50 ms limit the wait runs out, the kernel
+    # records DSA_ERR_TIMEOUT, drains what is in flight, frees its tensor
+    # memory and returns, and the context stays usable (child process: the
+    # library reads both variables once, at first use)
     code = r"""
 import sys, numpy as np, torch
 sys.path.insert(0, %r)
 import dsa_inputs as di
 import sparse_attention_scores_b200 as dsa
-from tests.dsa_testutil import upload, cache_of, dims_of
+from tests.dsa_testutil import upload, cache_of, dims_of, run_forward
 wl = di.small_decode([5000, 3000], H_I=32, D_I=128, topk=2048, H=64, R=512, P=64, seed=1)
 inp = di.make_inputs(wl); t = upload(inp)
 cache, dims = cache_of(inp, t), dims_of(inp)
@@ -312,11 +315,12 @@ st, info = dsa.workspace_check(ws)
 x = torch.ones(1000, device="cuda").sum().item()
 print("STATUS", st, hex(info), x)
 """ % ROOT
-    env = dict(os.environ, DSA_WAIT_LIMIT_NS="0")
+    env = dict(os.environ, DSA_WAIT_LIMIT_NS="50000000", DSA_DEBUG_STALL=str(kernel))
     res = subprocess.run([sys.executable, "-c", code], capture_output=True, text=True, env=env,
                          timeout=300, cwd=ROOT)
     assert res.returncode == 0, res.stderr[-2000:]
     line = [l for l in res.stdout.splitlines() if l.startswith("STATUS")][0]
-    st = int(line.split()[1])
+    st, info = int(line.split()[1]), int(line.split()[2], 16)
     assert st == 5, line     # DSA_ERR_TIMEOUT
+    assert info >> 24 == kernel, line
     assert line.endswith("1000.0")
