@@ -302,22 +302,24 @@ __global__ void __launch_bounds__(kThreads, 1)
       for (int c = 0; c < nchunks; ++c) {
         uint32_t v[32];
         tmem_ld_32x32b_x32(taddr + c * 32, v);
+        // the 32 columns of a chunk belong to one row of the group (H_I is a
+        // multiple of 32 when G > 1): row j, heads h0 .. h0 + nvalid - 1
+        const int j = (G == 1) ? 0 : (c * 32) / p.H_I;
+        const int h0 = c * 32 - j * p.H_I;
+        const int nvalid = min(32, p.H_I - h0);
+        const float *wrow = p.w + static_cast<int64_t>(min(g * G + j, p.n_q - 1)) * p.H_I + h0;
         tmem_ld_wait();
         float part = 0.f;
 #pragma unroll
         for (int i = 0; i < 32; ++i) {
-          const int col = c * 32 + i;
-          if (col < ncols) {
-            const int r = min(g * G + col / p.H_I, p.n_q - 1);
-            const float wv = __ldg(&p.w[static_cast<int64_t>(r) * p.H_I + (col % p.H_I)]);
+          if (i < nvalid) {
             const float x = __uint_as_float(v[i]);
-            part += wv * (x > 0.f ? x : 0.f);
+            part += __ldg(wrow + i) * (x > 0.f ? x : 0.f);
           }
         }
         if (G == 1) {
           s[0] += part;
         } else {
-          const int j = (c * 32) / p.H_I;  // H_I is a multiple of 32 when G > 1
 #pragma unroll
           for (int jj = 0; jj < G; ++jj)
             if (jj == j) s[jj] += part;

@@ -185,11 +185,14 @@ __global__ void __launch_bounds__(kThreads, 1) mla_kernel(const MlaParams p) {
   {
     const uint16_t *qrow = p.q + static_cast<int64_t>(row) * p.H * W;
     const uint32_t qs = smem_u32(Qs);
-    for (int i = tid; i < kHeads * cpr; i += kThreads) {
-      const int h = i / cpr, cc = i - h * cpr;
+    // warp w copies heads w, w+4, ...; its lanes walk the 16-byte pieces of a row
+    for (int h = warp; h < kHeads; h += kThreads / 32) {
       const bool ok = h < p.H;
-      const uint16_t *src = ok ? qrow + h * W + cc * 8 : p.q;
-      cp_async_16(qs + (cc >> 3) * kAtomQ + h * 128 + (((cc & 7) ^ (h & 7)) << 4), src, ok ? 16u : 0u);
+      for (int cc = lane; cc < cpr; cc += 32) {
+        const uint16_t *src = ok ? qrow + h * W + cc * 8 : p.q;
+        cp_async_16(qs + (cc >> 3) * kAtomQ + h * 128 + (((cc & 7) ^ (h & 7)) << 4), src,
+                    ok ? 16u : 0u);
+      }
     }
     cp_async_commit();
   }
@@ -234,11 +237,11 @@ __global__ void __launch_bounds__(kThreads, 1) mla_kernel(const MlaParams p) {
     // gather the latent rows (invalid slots are zero-filled)
     {
       const uint32_t ls = smem_u32(Ls);
-      for (int i = tid; i < kChunk * cpr; i += kThreads) {
-        const int key = i / cpr, cc = i - key * cpr;
+      for (int key = warp; key < kChunk; key += kThreads / 32) {
         const uint16_t *src = rowp[key];
-        cp_async_16(ls + (cc >> 3) * kAtomL + key * 128 + (((cc & 7) ^ (key & 7)) << 4),
-                    src ? src + cc * 8 : p.latent, src ? 16u : 0u);
+        for (int cc = lane; cc < cpr; cc += 32)
+          cp_async_16(ls + (cc >> 3) * kAtomL + key * 128 + (((cc & 7) ^ (key & 7)) << 4),
+                      src ? src + cc * 8 : p.latent, src ? 16u : 0u);
       }
       cp_async_commit();
       cp_async_wait_all();

@@ -39,33 +39,6 @@ struct TopkParams {
   DevStatus *status;
 };
 
-// exclusive block-wide prefix sum of v; *total receives the block sum
-__device__ __forceinline__ int block_exclusive_scan(int v, int *warp_sums, int *total) {
-  const int lane = lane_id(), warp = warp_id();
-  int x = v;
-#pragma unroll
-  for (int o = 1; o < 32; o <<= 1) {
-    const int y = __shfl_up_sync(0xffffffffu, x, o);
-    if (lane >= o) x += y;
-  }
-  if (lane == 31) warp_sums[warp] = x;
-  __syncthreads();
-  if (warp == 0) {
-    int s = (lane < kWarps) ? warp_sums[lane] : 0;
-#pragma unroll
-    for (int o = 1; o < 32; o <<= 1) {
-      const int y = __shfl_up_sync(0xffffffffu, s, o);
-      if (lane >= o) s += y;
-    }
-    if (lane < kWarps) warp_sums[lane] = s;
-  }
-  __syncthreads();
-  const int before = (warp > 0) ? warp_sums[warp - 1] : 0;
-  *total = warp_sums[kWarps - 1];
-  __syncthreads();
-  return before + x - v;
-}
-
 // exclusive suffix sum (sum over threads with a higher id)
 __device__ __forceinline__ int block_exclusive_suffix(int v, int *warp_sums) {
   const int lane = lane_id(), warp = warp_id();
@@ -95,8 +68,8 @@ __device__ __forceinline__ int block_exclusive_suffix(int v, int *warp_sums) {
 __global__ void __launch_bounds__(kThreads, 1) topk_kernel(const TopkParams p) {
   extern __shared__ uint32_t sm[];
   uint32_t *hist = sm;                                         // [kBins]
-  int *warp_sums = reinterpret_cast<int *>(sm + kBins);        // [32]
-  int *bcast = warp_sums + 32;                                 // [8]
+  int *warp_sums = reinterpret_cast<int *>(sm + kBins);        // [2 * kWarps]
+  int *bcast = warp_sums + 2 * kWarps;                         // [8]
   uint32_t *cnts = reinterpret_cast<uint32_t *>(bcast + 8);    // [2] per-CTA gt / eq counts
   uint32_t *keys = cnts + 8;                                   // [seg_cap]
 
@@ -173,18 +146,36 @@ __global__ void __launch_bounds__(kThreads, 1) topk_kernel(const TopkParams p) {
   const uint32_t T = prefix;   // the k-th largest key
   const int need_eq = krem;    // how many keys equal to T are kept
 
-  // per-CTA counts of keys above / equal to T, shared through the cluster
-  int gt_l = 0, eq_l = 0;
-  for (int i = tid; i < cnt; i += kThreads) {
-    const uint32_t u = key_at(i);
-    gt_l += (u > T);
-    eq_l += (u == T);
+  // Ordered compaction.  Warp w owns the contiguous run [w*run, (w+1)*run) of
+  // this CTA's segment and walks it in 32-key strips, so index order is
+  // (CTA, warp, strip, lane).  Pass A counts keys above / equal to T per warp;
+  // the CTA totals go to the cluster; pass B emits each kept index at
+  // position = kept tokens with a lower index, found by ballots.
+  const int warp = warp_id(), lane = lane_id();
+  const uint32_t lt_mask = (1u << lane) - 1u;
+  const int run = ((cnt + kWarps * 32 - 1) / (kWarps * 32)) * 32;
+  const int w_lo = min(cnt, warp * run), w_hi = min(cnt, w_lo + run);
+  int gt_w = 0, eq_w = 0;
+  for (int base = w_lo; base < w_hi; base += 32) {
+    const int i = base + lane;
+    const uint32_t u = (i < w_hi) ? key_at(i) : 0u;
+    gt_w += __popc(__ballot_sync(0xffffffffu, i < w_hi && u > T));
+    eq_w += __popc(__ballot_sync(0xffffffffu, i < w_hi && u == T));
   }
-  int tot;
-  block_exclusive_scan(gt_l, warp_sums, &tot);
-  if (tid == 0) cnts[0] = static_cast<uint32_t>(tot);
-  block_exclusive_scan(eq_l, warp_sums, &tot);
-  if (tid == 0) cnts[1] = static_cast<uint32_t>(tot);
+  int *wgt = warp_sums;        // [kWarps] per-warp counts, then exclusive prefixes
+  int *weq = warp_sums + kWarps;
+  if (lane == 0) { wgt[warp] = gt_w; weq[warp] = eq_w; }
+  __syncthreads();
+  if (tid == 0) {
+    int g = 0, e = 0;
+    for (int w = 0; w < kWarps; ++w) {
+      const int a = wgt[w], b = weq[w];
+      wgt[w] = g; weq[w] = e;
+      g += a; e += b;
+    }
+    cnts[0] = static_cast<uint32_t>(g);
+    cnts[1] = static_cast<uint32_t>(e);
+  }
   cluster_sync();
   if (tid == 0) {
     uint32_t gt_before = 0, eq_before = 0;
@@ -192,25 +183,26 @@ __global__ void __launch_bounds__(kThreads, 1) topk_kernel(const TopkParams p) {
       gt_before += ld_dsmem_u32(map_to_rank(smem_u32(&cnts[0]), r));
       eq_before += ld_dsmem_u32(map_to_rank(smem_u32(&cnts[1]), r));
     }
-    bcast[2] = static_cast<int>(eq_before);
-    bcast[3] = static_cast<int>(gt_before + umin(eq_before, static_cast<uint32_t>(need_eq)));
+    bcast[2] = static_cast<int>(gt_before);
+    bcast[3] = static_cast<int>(eq_before);
   }
   __syncthreads();
-  int carry_eq = bcast[2], carry_sel = bcast[3];
-  for (int base = 0; base < cnt; base += kThreads) {
-    const int i = base + tid;
-    uint32_t u = 0;
-    if (i < cnt) u = key_at(i);
-    const int gt = (i < cnt) && (u > T);
-    const int eq = (i < cnt) && (u == T);
-    int eq_tot;
-    const int eq_rank = carry_eq + block_exclusive_scan(eq, warp_sums, &eq_tot);
-    const int keep = gt || (eq && eq_rank < need_eq);
-    int sel_tot;
-    const int pos = carry_sel + block_exclusive_scan(keep, warp_sums, &sel_tot);
-    if (keep && pos < k) out[pos] = lo + i;
-    carry_eq += eq_tot;
-    carry_sel += sel_tot;
+  int erank = bcast[3] + weq[warp];                              // equal keys before this warp
+  int pos = bcast[2] + wgt[warp] + min(erank, need_eq);          // kept keys before this warp
+  for (int base = w_lo; base < w_hi; base += 32) {
+    const int i = base + lane;
+    const uint32_t u = (i < w_hi) ? key_at(i) : 0u;
+    const bool gt = i < w_hi && u > T;
+    const bool eq = i < w_hi && u == T;
+    const uint32_t eqm = __ballot_sync(0xffffffffu, eq);
+    const bool keep = gt || (eq && erank + __popc(eqm & lt_mask) < need_eq);
+    const uint32_t km = __ballot_sync(0xffffffffu, keep);
+    if (keep) {
+      const int o = pos + __popc(km & lt_mask);
+      if (o < k) out[o] = lo + i;
+    }
+    pos += __popc(km);
+    erank += __popc(eqm);
   }
   cluster_sync();  // keep this CTA's shared memory alive until peers are done
 }
@@ -222,7 +214,7 @@ dsa_status_t launch_topk(const TopkLaunch &a, cudaStream_t stream) {
   int C = (max_len + 4095) / 4096;
   C = std::max(1, std::min(C, 8));
   const int seg = ((max_len + C - 1) / C + 3) & ~3;
-  const size_t fixed = 4 * (kBins + 32 + 8 + 8) + 64;
+  const size_t fixed = 4 * (kBins + 2 * kWarps + 8 + 8) + 64;
   const size_t max_smem = device_max_smem_optin();
   const int cap_max = static_cast<int>((max_smem - fixed) / 4);
   const int seg_cap = std::min(seg, cap_max);
