@@ -194,6 +194,38 @@ DSA_API dsa_status_t dsa_attention_forward(const uint16_t *q_idx, const float *w
                                    const dsa_dims_t *dims, int32_t *idx_out, float *out,
                                    float *lse, void *ws, size_t ws_bytes, dsa_stream_t stream);
 
+/* Sparse MLA decode for callers that cannot allocate device memory.
+ *
+ * The pages have no counterpart of this entry point: it exists for callers
+ * that cannot call cudaMalloc (or any allocator) at the point where they run
+ * the step, e.g. code inside a memory pool that must not grow, or a host that
+ * hands the library only its input and output buffers.  It computes exactly
+ * what dsa_sparse_mla_decode computes (same kernels, same launch shapes) but
+ * takes no workspace: its scratch (the per-split partial results and a status
+ * block) is a fixed 32 MiB array in the library's own device memory, present
+ * on every GPU that loads the library until the process exits.
+ *
+ *   Arguments as for dsa_sparse_mla_decode, without ws / ws_bytes.
+ *   Returns DSA_ERR_WORKSPACE when the partial results of this call would not
+ *   fit in the 32 MiB array (n_q * splits * 64 * R * 4 bytes plus small
+ *   change; e.g. batch 32 at R = 512 and top-k 2,048 fits), before launching
+ *   anything.
+ *
+ * The first call on a device looks up the array's device address (once per
+ * device, with that device current); make that first call before any stream
+ * capture.  All calls on a device share the one array, and it keeps the last
+ * call's contents: calls whose executions overlap on the GPU (different
+ * streams, or different host threads) race on it and must be ordered by the
+ * caller.  Device-side range-check events of this call are recorded in the
+ * array's status block, which is cleared at the start of every call and is
+ * not reported back; validate indices on the host, or use
+ * dsa_sparse_mla_decode with a workspace when that check is needed.
+ * Allocates nothing: no cudaMalloc, no cudaFree, no allocating library call. */
+DSA_API dsa_status_t dsa_sparse_mla_decode_noalloc(const uint16_t *q, const uint16_t *latent_pages,
+                                           const dsa_cache_t *cache, const int32_t *idx,
+                                           const dsa_dims_t *dims, float *out, float *lse,
+                                           dsa_stream_t stream);
+
 #ifdef __cplusplus
 }
 #endif

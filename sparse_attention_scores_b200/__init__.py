@@ -34,7 +34,7 @@ STATUS_NAMES = {0: "DSA_OK", 1: "DSA_ERR_INVALID_ARG", 2: "DSA_ERR_UNSUPPORTED",
 
 EXPORTED = ["dsa_version", "dsa_status_string", "dsa_workspace_bytes", "dsa_workspace_init",
             "dsa_workspace_check", "dsa_indexer_scores", "dsa_topk", "dsa_sparse_mla_decode",
-            "dsa_sparse_mla_prefill", "dsa_attention_forward"]
+            "dsa_sparse_mla_prefill", "dsa_attention_forward", "dsa_sparse_mla_decode_noalloc"]
 
 
 class DsaError(RuntimeError):
@@ -83,6 +83,7 @@ def lib() -> ctypes.CDLL:
             "dsa_sparse_mla_prefill": ([vp, vp, pc, vp, pd, vp, vp, vp, sz, vp], ctypes.c_int),
             "dsa_attention_forward": ([vp, vp, vp, vp, vp, pc, pd, vp, vp, vp, vp, sz, vp],
                                       ctypes.c_int),
+            "dsa_sparse_mla_decode_noalloc": ([vp, vp, pc, vp, pd, vp, vp, vp], ctypes.c_int),
         }
         for name, (args, res) in sigs.items():
             fn = getattr(L, name)
@@ -193,6 +194,17 @@ def dsa_sparse_mla_prefill(q, latent_pages, cache: PagedCache, idx, dims: Dims, 
                                         ctypes.byref(dims.struct()), _ptr(out), _ptr(lse),
                                         _ptr(ws), ws.numel(), _stream(stream)),
            "dsa_sparse_mla_prefill")
+
+
+def dsa_sparse_mla_decode_noalloc(q, latent_pages, cache: PagedCache, idx, dims: Dims, out, lse,
+                                  stream=None) -> None:
+    """Sparse MLA decode without a workspace, for callers that cannot allocate
+    device memory: the scratch is a fixed array inside the library (see
+    include/dsa.h for its limits and sharing rules)."""
+    _check(lib().dsa_sparse_mla_decode_noalloc(_ptr(q), _ptr(latent_pages),
+                                               ctypes.byref(cache.struct()), _ptr(idx),
+                                               ctypes.byref(dims.struct()), _ptr(out), _ptr(lse),
+                                               _stream(stream)), "dsa_sparse_mla_decode_noalloc")
 
 
 def dsa_attention_forward(q_idx, w, k_idx_pages, q, latent_pages, cache: PagedCache, dims: Dims,

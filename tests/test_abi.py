@@ -27,7 +27,7 @@ def _declared_symbols():
 
 def test_every_declared_symbol_is_exported(L):
     declared = _declared_symbols()
-    assert len(declared) == 10
+    assert len(declared) == 11
     assert sorted(declared) == sorted(dsa.EXPORTED)
     out = subprocess.run(["nm", "-D", "--defined-only", dsa.LIB_PATH], capture_output=True,
                          text=True, check=True).stdout
@@ -68,7 +68,30 @@ def test_workspace_bytes_host_only(L):
     assert L.dsa_workspace_bytes(dsa.OP_ATTENTION_FORWARD, ctypes.byref(bad), ctypes.byref(c)) == 0
 
 
+def _no_device():
+    # the fake addresses below must never reach a kernel: these host-only
+    # checks run where there is no CUDA device
+    try:
+        import torch
+        if torch.cuda.is_available():
+            pytest.skip("host-only validation test; a CUDA device is present")
+    except ImportError:
+        pass
+
+
+def test_noalloc_size_check_host_only(L):
+    _no_device()
+    # 140 rows x 2 splits x 64 heads x 512 x 4 B = 36.7 MB > the 32 MiB array
+    d = _dims(n_q=140, topk=65536)
+    c = _cache(num_seqs=140, max_pages=1024, num_pages=1024, max_seq_len=65536)
+    fake = ctypes.c_void_p(0x300000)
+    st = L.dsa_sparse_mla_decode_noalloc(fake, fake, ctypes.byref(c), fake, ctypes.byref(d),
+                                         fake, fake, None)
+    assert st == 4
+
+
 def test_host_validation_rejects_without_launch(L):
+    _no_device()
     d, c = _dims(), _cache()
     fake = ctypes.c_void_p(0x300000)
     ws = ctypes.c_void_p(0x400000)

@@ -1,0 +1,95 @@
+"""The sparse MLA decode entry point that allocates nothing.
+
+Some callers cannot allocate device memory where they run the step (a
+memory pool that must not grow, a host that only hands over its input and
+output buffers).  dsa_sparse_mla_decode_noalloc serves them: its scratch is a
+fixed array inside the library.  This test calls it through the C ABI and
+checks it against dsa_sparse_mla_decode (the entry point with a caller
+workspace) on two calls in a row, within the tolerances of the other tests.
+This file is named so that pytest collects it last.
+"""
+
+import ctypes
+
+import numpy as np
+import pytest
+import torch
+
+import dsa_inputs as di
+import sparse_attention_scores_b200 as dsa
+from tests.dsa_testutil import LSE_TOL, OUT_TOL, cache_of, dims_of, norm_err, upload
+
+pytestmark = pytest.mark.gpu
+
+
+def _selection(rng, lengths, k):
+    idx = np.full((len(lengths), k), -1, np.int32)
+    for r, n in enumerate(lengths):
+        m = min(n, k)
+        idx[r, :m] = np.sort(rng.choice(n, size=m, replace=False))
+    return idx
+
+
+def test_noalloc_matches_workspace_entry_point():
+    if not torch.cuda.is_available():
+        pytest.skip("no CUDA device")
+    L = dsa.lib()
+    rng = np.random.default_rng(77)
+    # batch 4 at GLM-5 width: the rows are split over several CTAs, so the
+    # built-in scratch array holds real partial results
+    lengths = [9000, 2500, 4100, 700]
+    wl = di.small_decode(lengths, H_I=4, D_I=32, topk=2048, H=64, R=512, P=64, seed=5)
+    inp = di.make_inputs(wl)
+    t = upload(inp)
+    cache, dims = cache_of(inp, t), dims_of(inp)
+    B = wl.n_q
+    ws = dsa.workspace(dsa.OP_SPARSE_MLA_DECODE, dims, cache)
+    for call in range(2):
+        idx = torch.from_numpy(_selection(rng, lengths, wl.topk)).cuda()
+        ref_out = torch.empty((B, wl.H, wl.R), device="cuda")
+        ref_lse = torch.empty((B, wl.H), device="cuda")
+        dsa.dsa_sparse_mla_decode(t["q"], t["latent_pages"], cache, idx, dims, ref_out, ref_lse, ws)
+        out = torch.full((B, wl.H, wl.R), float("nan"), device="cuda")
+        lse = torch.full((B, wl.H), float("nan"), device="cuda")
+        stream = torch.cuda.current_stream().cuda_stream or None
+        st = L.dsa_sparse_mla_decode_noalloc(
+            ctypes.c_void_p(t["q"].data_ptr()), ctypes.c_void_p(t["latent_pages"].data_ptr()),
+            ctypes.byref(cache.struct()), ctypes.c_void_p(idx.data_ptr()),
+            ctypes.byref(dims.struct()), ctypes.c_void_p(out.data_ptr()),
+            ctypes.c_void_p(lse.data_ptr()), stream)
+        assert st == 0, dsa.STATUS_NAMES.get(st, st)
+        torch.cuda.synchronize()
+        assert dsa.workspace_check(ws)[0] == 0
+        o, l = out.cpu().numpy(), lse.cpu().numpy()
+        ro, rl = ref_out.cpu().numpy().astype(np.float64), ref_lse.cpu().numpy().astype(np.float64)
+        for b in range(B):
+            assert norm_err(o[b], ro[b]) <= OUT_TOL, (call, b)
+            assert np.max(np.abs(l[b] - rl[b])) <= LSE_TOL, (call, b)
+
+
+def test_noalloc_rejects_oversize_request():
+    # 140 rows at R = 512 with a 65,536-token selection split in two per row
+    # need 36.7 MB of partials: more than the 32 MiB array, so the call must
+    # return DSA_ERR_WORKSPACE before launching.  Real, correctly sized buffers
+    # (every slot unused) keep the call memory-safe regardless.
+    if not torch.cuda.is_available():
+        pytest.skip("no CUDA device")
+    L = dsa.lib()
+    B, k, H, R, P = 140, 65536, 64, 512, 64
+    q = torch.zeros((B, H, R + P), dtype=torch.bfloat16, device="cuda")
+    latent = torch.zeros((1, 64, R + P), dtype=torch.bfloat16, device="cuda")
+    idx = torch.full((B, k), -1, dtype=torch.int32, device="cuda")
+    out = torch.empty((B, H, R), device="cuda")
+    lse = torch.empty((B, H), device="cuda")
+    seq_lens = torch.ones(B, dtype=torch.int32, device="cuda")
+    table = torch.zeros((B, 1), dtype=torch.int32, device="cuda")
+    cache = dsa.PagedCache(seq_lens, table, num_pages=1, max_seq_len=1)
+    dims = dsa.Dims(n_q=B, H_I=4, D_I=32, topk=k, H=H, R=R, P=P, scale=0.1)
+    stream = torch.cuda.current_stream().cuda_stream or None
+    st = L.dsa_sparse_mla_decode_noalloc(
+        ctypes.c_void_p(q.data_ptr()), ctypes.c_void_p(latent.data_ptr()),
+        ctypes.byref(cache.struct()), ctypes.c_void_p(idx.data_ptr()),
+        ctypes.byref(dims.struct()), ctypes.c_void_p(out.data_ptr()),
+        ctypes.c_void_p(lse.data_ptr()), stream)
+    torch.cuda.synchronize()
+    assert st == 4, dsa.STATUS_NAMES.get(st, st)   # DSA_ERR_WORKSPACE
