@@ -202,8 +202,9 @@ dsa_status_t run_topk(const float *scores, int64_t ld, int n_q, const int32_t *v
 
 dsa_status_t run_mla(const uint16_t *q, const uint16_t *latent, const dsa_cache_t &c,
                      const int32_t *idx, const dsa_dims_t &d, float *out, float *lse, void *scratch,
-                     size_t scratch_bytes, DevStatus *st, cudaStream_t s) {
+                     size_t scratch_bytes, DevStatus *st, cudaStream_t s, int early_q = 0) {
   MlaLaunch a;
+  a.early_q = early_q;
   a.q = q;
   a.latent = latent;
   a.idx = idx;
@@ -382,7 +383,8 @@ dsa_status_t dsa_attention_forward(const uint16_t *q_idx, const float *w,
   DSA_TRY(run_indexer(q_idx, w, k_idx_pages, c, d, scores, ld, st, s));
   DSA_TRY(run_topk(scores, ld, d.n_q, d.causal ? nullptr : c.seq_lens, d.q_pos0, d.topk, idx,
                    static_cast<int>(max_keys(d, c)), st, s));
-  return run_mla(q, latent_pages, c, idx, d, out, lse, scratch, scratch_bytes, st, s);
+  return run_mla(q, latent_pages, c, idx, d, out, lse, scratch, scratch_bytes, st, s,
+                 /*early_q=*/1);
 }
 
 }  // extern "C"

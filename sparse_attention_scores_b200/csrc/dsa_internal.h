@@ -4,6 +4,8 @@
 #include <cuda_runtime.h>
 #include <stdint.h>
 
+#include <utility>
+
 #include "../../include/dsa.h"
 #include "dsa_common.cuh"
 
@@ -22,6 +24,34 @@ int debug_stall();
 constexpr uint64_t kDrainLimitNs = 1000000000ull;
 
 int device_sm_count();
+
+// Launch `kernel` on `stream` with programmatic stream serialization (the
+// kernel calls griddep_wait() before its first dependent read), optionally
+// as clusters of cluster_x CTAs.
+template <typename... KArgs, typename... Args>
+cudaError_t launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem,
+                       cudaStream_t stream, unsigned cluster_x, Args &&...args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[2];
+  int n = 0;
+  attr[n].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[n].val.programmaticStreamSerializationAllowed = 1;
+  ++n;
+  if (cluster_x > 1) {
+    attr[n].id = cudaLaunchAttributeClusterDimension;
+    attr[n].val.clusterDim.x = cluster_x;
+    attr[n].val.clusterDim.y = 1;
+    attr[n].val.clusterDim.z = 1;
+    ++n;
+  }
+  cfg.attrs = attr;
+  cfg.numAttrs = n;
+  return cudaLaunchKernelEx(&cfg, kernel, std::forward<Args>(args)...);
+}
 size_t device_max_smem_optin();
 
 struct IndexerLaunch {
@@ -65,6 +95,10 @@ struct MlaLaunch {
   void *scratch;        // partial results when the keys are split over CTAs
   size_t scratch_bytes;
   DevStatus *status;
+  // 1 when q is known to be complete before the kernel preceding this one in
+  // the stream started (the fused forward): the query tile is then loaded
+  // before waiting on that kernel, overlapping its tail
+  int early_q = 0;
 };
 // Number of key splits the launcher uses and the scratch bytes it needs.
 int mla_num_splits(int n_q, int topk);

@@ -16,8 +16,9 @@
 //              (two per tile) into a ring of shared-memory stages; the
 //              query tile when the row group changes
 //   warp 1     tcgen05.mma issuer (one thread), double-buffered accumulators
-//   warps 2-5  epilogue: tcgen05.ld of a 128-lane accumulator, ReLU,
-//              head-weighted sum, coalesced fp32 stores
+//   warps 2-9  epilogue, two warpgroups taking alternate tiles: tcgen05.ld
+//              of a 128-lane accumulator, ReLU, head-weighted sum, coalesced
+//              fp32 stores; up to 8 accumulators let the MMA run ahead
 // Every wait is bounded in wall time; a time-out records an error in the
 // status block, drains what is in flight, frees tensor memory and returns.
 #include <algorithm>
@@ -28,7 +29,8 @@
 namespace dsa {
 namespace {
 
-constexpr int kThreads = 192;
+constexpr int kThreads = 320;      // producer warp, MMA warp, two epilogue warpgroups
+constexpr int kMaxAcc = 8;         // accumulator buffers in tensor memory
 constexpr int kTileKeys = 128;
 constexpr int kLookahead = 16;  // units whose page ids the producer fetches at once
 
@@ -89,8 +91,11 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int n_mma = (ncols + 15) & ~15;         // MMA N (multiple of 16)
   const int q_bytes = natoms * n_mma * AW;
   const uint32_t acc_stride = (n_mma + 31) & ~31;
+  // as many accumulators as fit 512 columns (<= 8): the MMA warp runs that
+  // many tiles ahead of the epilogue
+  const int nacc = min(kMaxAcc, static_cast<int>(512u / acc_stride));
   uint32_t tmem_cols = 32;
-  while (tmem_cols < 2 * acc_stride) tmem_cols <<= 1;
+  while (tmem_cols < nacc * acc_stride) tmem_cols <<= 1;
 
   uint8_t *stage_base = smem;
   uint8_t *q_base = smem + S * stage_bytes;
@@ -100,8 +105,8 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint64_t *qfull = bars + 2 * S;
   uint64_t *qempty = qfull + 2;
   uint64_t *tfull = qempty + 2;
-  uint64_t *tempty = tfull + 2;
-  uint64_t *drain = tempty + 2;
+  uint64_t *tempty = tfull + kMaxAcc;
+  uint64_t *drain = tempty + kMaxAcc;
   uint32_t *misc = reinterpret_cast<uint32_t *>(drain + 1);  // [0] tmem base, [1] abort
   int *scan_tmp = reinterpret_cast<int *>(misc + 4);          // [kThreads]
   int *tile_start = scan_tmp + kThreads;                      // [num_groups + 1]
@@ -111,10 +116,8 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   if (threadIdx.x == 0) {
     for (int i = 0; i < S; ++i) { mbar_init(&full[i], 1); mbar_init(&empty[i], 1); }
-    for (int i = 0; i < 2; ++i) {
-      mbar_init(&qfull[i], 1); mbar_init(&qempty[i], 1);
-      mbar_init(&tfull[i], 1); mbar_init(&tempty[i], 4);
-    }
+    for (int i = 0; i < 2; ++i) { mbar_init(&qfull[i], 1); mbar_init(&qempty[i], 1); }
+    for (int i = 0; i < kMaxAcc; ++i) { mbar_init(&tfull[i], 1); mbar_init(&tempty[i], 4); }
     mbar_init(drain, 1);
     misc[1] = 0u;
     fence_barrier_init();
@@ -122,6 +125,9 @@ __global__ void __launch_bounds__(kThreads, 1)
   if (warp == 0 && lane == 0) { tma_prefetch_desc(&tmK); tma_prefetch_desc(&tmQ); }
   if (warp == 1) { tmem_alloc(&misc[0], tmem_cols); tmem_relinquish(); }
 
+  // everything below may read what earlier work in the stream wrote
+  griddep_wait();
+  griddep_launch_dependents();
   // tile prefix over row groups (every CTA computes the same table)
   {
     const int per = (NG + kThreads - 1) / kThreads;
@@ -238,8 +244,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     // ------------------------------------------------------------ MMA issuer
     if (lane == 0) {
       const uint32_t idesc = idesc_bf16_f32(kTileKeys, n_mma, 0, 0);
-      int stage = 0, qslot = 0, cur = -1, cur_slot = 0, acc = 0;
-      uint32_t phase = 0, qphase = 0, aphase = 0;
+      int stage = 0, qslot = 0, cur = -1, cur_slot = 0;
+      uint32_t phase = 0, qphase = 0;
       bool ok = true;
       if (p.debug_stall && !mbar_wait(drain, 0, p.wait_ns)) ok = false;
       int g = (u0 < u1) ? locate(tile_start, NG, u0) : 0;
@@ -253,6 +259,10 @@ __global__ void __launch_bounds__(kThreads, 1)
           qslot ^= 1;
           if (qslot == 0) qphase ^= 1u;
         }
+        // accumulator of the i-th unit of this CTA: i % nacc, its (i / nacc)-th use
+        const int i_unit = u - u0;
+        const int acc = i_unit % nacc;
+        const uint32_t aphase = static_cast<uint32_t>(i_unit / nacc) & 1u;
         if (!mbar_wait(&full[stage], phase, p.wait_ns)) { ok = false; break; }
         if (!mbar_wait(&tempty[acc], aphase ^ 1u, p.wait_ns)) { ok = false; break; }
         tc_fence_after();
@@ -271,8 +281,6 @@ __global__ void __launch_bounds__(kThreads, 1)
         const bool last_of_group = (u + 1 == u1) || (tile_start[g + 1] <= u + 1);
         if (last_of_group) mma_commit(&qempty[cur_slot]);
         if (++stage == S) { stage = 0; phase ^= 1u; }
-        acc ^= 1;
-        if (acc == 0) aphase ^= 1u;
       }
       if (!ok && !*abort_flag) {
         *abort_flag = 1u;
@@ -283,15 +291,28 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
   } else {
     // ------------------------------------------------------------ epilogue
-    const int quad = warp & 3;           // tensor-memory lane quadrant of this warp
+    // two warpgroups take alternate tiles; within a group, warp w reads the
+    // tensor-memory lane quadrant w % 4 (keys 32*quad .. 32*quad+31 of the tile)
+    const int quad = warp & 3;
+    const int eg = (warp - 2) >> 2;
     const int key_in_tile = quad * 32 + lane;
     const int nchunks = (ncols + 31) / 32;
-    int acc = 0;
-    uint32_t aphase = 0;
+    const bool w_in_regs = (G == 1) && (p.H_I <= 32);
+    float wreg[32];
+    int wgroup = -1;
     bool ok = true;
     int g = (u0 < u1) ? locate(tile_start, NG, u0) : 0;
-    for (int u = u0; u < u1; ++u) {
+    for (int u = u0 + eg; u < u1; u += 2) {
       while (tile_start[g + 1] <= u) ++g;
+      const int i_unit = u - u0;
+      const int acc = i_unit % nacc;
+      const uint32_t aphase = static_cast<uint32_t>(i_unit / nacc) & 1u;
+      if (w_in_regs && g != wgroup) {
+#pragma unroll
+        for (int i = 0; i < 32; ++i)
+          wreg[i] = (i < p.H_I) ? __ldg(p.w + static_cast<int64_t>(g) * p.H_I + i) : 0.f;
+        wgroup = g;
+      }
       if (__any_sync(0xffffffffu, *abort_flag != 0u)) { ok = false; break; }
       if (!__all_sync(0xffffffffu, mbar_wait(&tfull[acc], aphase, p.wait_ns))) { ok = false; break; }
       tc_fence_after();
@@ -299,30 +320,41 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
       for (int j = 0; j < G; ++j) s[j] = 0.f;
       const uint32_t taddr = tmem_base + (static_cast<uint32_t>(quad * 32) << 16) + acc * acc_stride;
-      for (int c = 0; c < nchunks; ++c) {
+      if (w_in_regs) {
         uint32_t v[32];
-        tmem_ld_32x32b_x32(taddr + c * 32, v);
-        // the 32 columns of a chunk belong to one row of the group (H_I is a
-        // multiple of 32 when G > 1): row j, heads h0 .. h0 + nvalid - 1
-        const int j = (G == 1) ? 0 : (c * 32) / p.H_I;
-        const int h0 = c * 32 - j * p.H_I;
-        const int nvalid = min(32, p.H_I - h0);
-        const float *wrow = p.w + static_cast<int64_t>(min(g * G + j, p.n_q - 1)) * p.H_I + h0;
+        tmem_ld_32x32b_x32(taddr, v);
         tmem_ld_wait();
-        float part = 0.f;
 #pragma unroll
         for (int i = 0; i < 32; ++i) {
-          if (i < nvalid) {
-            const float x = __uint_as_float(v[i]);
-            part += __ldg(wrow + i) * (x > 0.f ? x : 0.f);
-          }
+          const float x = __uint_as_float(v[i]);
+          if (i < p.H_I) s[0] += wreg[i] * (x > 0.f ? x : 0.f);
         }
-        if (G == 1) {
-          s[0] += part;
-        } else {
+      } else {
+        for (int c = 0; c < nchunks; ++c) {
+          uint32_t v[32];
+          tmem_ld_32x32b_x32(taddr + c * 32, v);
+          // the 32 columns of a chunk belong to one row of the group (H_I is a
+          // multiple of 32 when G > 1): row j, heads h0 .. h0 + nvalid - 1
+          const int j = (G == 1) ? 0 : (c * 32) / p.H_I;
+          const int h0 = c * 32 - j * p.H_I;
+          const int nvalid = min(32, p.H_I - h0);
+          const float *wrow = p.w + static_cast<int64_t>(min(g * G + j, p.n_q - 1)) * p.H_I + h0;
+          tmem_ld_wait();
+          float part = 0.f;
 #pragma unroll
-          for (int jj = 0; jj < G; ++jj)
-            if (jj == j) s[jj] += part;
+          for (int i = 0; i < 32; ++i) {
+            if (i < nvalid) {
+              const float x = __uint_as_float(v[i]);
+              part += __ldg(wrow + i) * (x > 0.f ? x : 0.f);
+            }
+          }
+          if (G == 1) {
+            s[0] += part;
+          } else {
+#pragma unroll
+            for (int jj = 0; jj < G; ++jj)
+              if (jj == j) s[jj] += part;
+          }
         }
       }
       tc_fence_before();
@@ -335,8 +367,6 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int r = p.causal ? g * G + j : g;
         if (r < p.n_q && key < row_keys(p, r)) p.scores[static_cast<int64_t>(r) * p.ld + key] = s[j];
       }
-      acc ^= 1;
-      if (acc == 0) aphase ^= 1u;
     }
     if (!ok && lane == 0 && !*abort_flag) {
       *abort_flag = 1u;
@@ -403,7 +433,7 @@ dsa_status_t launch_impl(const IndexerLaunch &a, cudaStream_t stream) {
 
   const size_t stage_bytes = static_cast<size_t>(kTileKeys) * a.D_I * 2;
   const size_t q_bytes = static_cast<size_t>(natoms) * n_mma * AW;
-  const size_t fixed = 1024 /*align*/ + 2 * q_bytes + 8 * (2 * 8 + 9) + 16 + 4 * kThreads +
+  const size_t fixed = 1024 /*align*/ + 2 * q_bytes + 8 * (2 * 8 + 5 + 2 * kMaxAcc) + 16 + 4 * kThreads +
                        4 * ((num_groups + 4) & ~3) + 64;
   const size_t max_smem = device_max_smem_optin();
   int stages = static_cast<int>((max_smem - fixed) / stage_bytes);
@@ -440,8 +470,10 @@ dsa_status_t launch_impl(const IndexerLaunch &a, cudaStream_t stream) {
   p.wait_ns = wait_limit_ns();
   p.debug_stall = debug_stall() == kKernIndexer ? 1 : 0;
   p.status = a.status;
-  indexer_kernel<G, AW><<<grid, kThreads, smem, stream>>>(tmK, tmQ, p);
-  return cudaGetLastError() == cudaSuccess ? DSA_OK : DSA_ERR_CUDA;
+  if (launch_pdl(indexer_kernel<G, AW>, dim3(grid), dim3(kThreads), smem, stream, 1, tmK, tmQ, p) !=
+      cudaSuccess)
+    return DSA_ERR_CUDA;
+  return DSA_OK;
 }
 
 }  // namespace

@@ -57,6 +57,7 @@ struct MlaParams {
   float scale_log2;
   uint64_t wait_ns;
   int debug_stall;  // wait once on a barrier nothing arrives at (tests the time-out path)
+  int early_q;      // load the query tile before griddep_wait()
   DevStatus *status;
 };
 
@@ -161,7 +162,6 @@ __global__ void __launch_bounds__(kThreads, 1) mla_kernel(const MlaParams p) {
   const int tid = threadIdx.x, warp = warp_id(), lane = lane_id();
   const int split = blockIdx.x, row = blockIdx.y;
   const int b = p.causal ? 0 : row;
-  const int limit = min(p.causal ? p.q_pos0 + row + 1 : p.seq_lens[b], p.max_pages * kPageSize);
   const int nchunks = (p.topk + kChunk - 1) / kChunk;
   const int c_begin = split * p.chunks_per_split;
   const int c_end = min(nchunks, c_begin + p.chunks_per_split);
@@ -181,6 +181,9 @@ __global__ void __launch_bounds__(kThreads, 1) mla_kernel(const MlaParams p) {
   if (tid < kHeads) { mrun[tid] = -INFINITY; lrun[tid] = 0.f; }
   if (warp == 0) { tmem_alloc(&misc[0], tmem_cols); tmem_relinquish(); }
 
+  // earlier work in the stream may have written q, idx or the caches; in the
+  // fused forward q predates the kernel before this one and loads first
+  if (!p.early_q) griddep_wait();
   // the 64-head query tile (heads >= H zero-filled), 128B-swizzled, K-major
   {
     const uint16_t *qrow = p.q + static_cast<int64_t>(row) * p.H * W;
@@ -196,6 +199,9 @@ __global__ void __launch_bounds__(kThreads, 1) mla_kernel(const MlaParams p) {
     }
     cp_async_commit();
   }
+  if (p.early_q) griddep_wait();
+  griddep_launch_dependents();
+  const int limit = min(p.causal ? p.q_pos0 + row + 1 : p.seq_lens[b], p.max_pages * kPageSize);
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
@@ -452,33 +458,49 @@ __global__ void __launch_bounds__(kThreads, 1) mla_kernel(const MlaParams p) {
   }
 }
 
-// Merge the split partials of one (row, head): out = sum_s 2^(m_s - M) O_s / sum_s 2^(m_s - M) l_s.
+// Merge the split partials of one (row, head):
+//   out = sum_s 2^(m_s - M) O_s / sum_s 2^(m_s - M) l_s,  lse = (M + log2 L) ln 2.
+// The first warp loads every split's (m, l) in parallel (nsplit <= 64) and
+// reduces them with shuffles; all threads then stream the partial rows.
 __global__ void __launch_bounds__(128) combine_kernel(const MlaParams p) {
   const int row = blockIdx.x, h = blockIdx.y;
+  griddep_wait();
+  griddep_launch_dependents();
   const float *ml = p.part_ml + static_cast<int64_t>(row) * p.nsplit * 2 * kHeads;
   __shared__ float wgt[64];
-  __shared__ float wsum_sm;
-  if (threadIdx.x == 0) {
-    float M = -INFINITY;
-    for (int s = 0; s < p.nsplit; ++s) M = fmaxf(M, ml[s * 2 * kHeads + h]);
-    float wsum = 0.f;
-    for (int s = 0; s < p.nsplit; ++s) {
-      const float m = ml[s * 2 * kHeads + h];
-      const float wgt_s = (m == -INFINITY) ? 0.f : exp2f(m - M);
-      wgt[s] = wgt_s;
-      wsum += wgt_s * ml[s * 2 * kHeads + kHeads + h];
+  __shared__ float inv_l;
+  if (threadIdx.x < 32) {
+    const int lane = threadIdx.x;
+    const int s0 = lane, s1 = lane + 32;
+    const float m0 = (s0 < p.nsplit) ? ml[s0 * 2 * kHeads + h] : -INFINITY;
+    const float m1 = (s1 < p.nsplit) ? ml[s1 * 2 * kHeads + h] : -INFINITY;
+    const float l0 = (s0 < p.nsplit) ? ml[s0 * 2 * kHeads + kHeads + h] : 0.f;
+    const float l1 = (s1 < p.nsplit) ? ml[s1 * 2 * kHeads + kHeads + h] : 0.f;
+    float M = fmaxf(m0, m1);
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, o));
+    const float w0 = (m0 == -INFINITY) ? 0.f : exp2f(m0 - M);
+    const float w1 = (m1 == -INFINITY) ? 0.f : exp2f(m1 - M);
+    float L = w0 * l0 + w1 * l1;
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) L += __shfl_xor_sync(0xffffffffu, L, o);
+    wgt[s0] = w0;
+    wgt[s1] = w1;
+    if (lane == 0) {
+      inv_l = (L > 0.f) ? 1.f / L : 0.f;
+      p.lse[static_cast<int64_t>(row) * p.H + h] =
+          (L > 0.f) ? (M + log2f(L)) * 0.69314718055994531f : -INFINITY;
     }
-    wsum_sm = wsum;
-    p.lse[static_cast<int64_t>(row) * p.H + h] =
-        (wsum > 0.f) ? (M + log2f(wsum)) * 0.69314718055994531f : -INFINITY;
   }
   __syncthreads();
-  const float wsum = wsum_sm;
+  const float il = inv_l;
+  const float *po = p.part_o + (static_cast<int64_t>(row) * p.nsplit * kHeads + h) * p.R;
+  const int64_t sstride = static_cast<int64_t>(kHeads) * p.R;
   for (int r = threadIdx.x; r < p.R; r += blockDim.x) {
     float acc = 0.f;
-    for (int s = 0; s < p.nsplit; ++s)
-      acc += wgt[s] * p.part_o[((static_cast<int64_t>(row) * p.nsplit + s) * kHeads + h) * p.R + r];
-    p.out[(static_cast<int64_t>(row) * p.H + h) * p.R + r] = (wsum > 0.f) ? acc / wsum : 0.f;
+#pragma unroll 8
+    for (int s = 0; s < p.nsplit; ++s) acc += wgt[s] * po[s * sstride + r];
+    p.out[(static_cast<int64_t>(row) * p.H + h) * p.R + r] = acc * il;
   }
 }
 
@@ -551,12 +573,14 @@ dsa_status_t launch_mla(const MlaLaunch &a, cudaStream_t stream) {
   p.scale_log2 = static_cast<float>(static_cast<double>(a.scale) * 1.4426950408889634);
   p.wait_ns = wait_limit_ns();
   p.debug_stall = debug_stall() == kKernMla ? 1 : 0;
+  p.early_q = a.early_q;
   p.status = a.status;
-  mla_kernel<<<dim3(nsplit, a.n_q), kThreads, smem, stream>>>(p);
-  if (cudaGetLastError() != cudaSuccess) return DSA_ERR_CUDA;
+  if (launch_pdl(mla_kernel, dim3(nsplit, a.n_q), dim3(kThreads), smem, stream, 1, p) !=
+      cudaSuccess)
+    return DSA_ERR_CUDA;
   if (nsplit > 1) {
-    combine_kernel<<<dim3(a.n_q, a.H), 128, 0, stream>>>(p);
-    if (cudaGetLastError() != cudaSuccess) return DSA_ERR_CUDA;
+    if (launch_pdl(combine_kernel, dim3(a.n_q, a.H), dim3(128), 0, stream, 1, p) != cudaSuccess)
+      return DSA_ERR_CUDA;
   }
   return DSA_OK;
 }

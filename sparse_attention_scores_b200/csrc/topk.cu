@@ -67,12 +67,14 @@ __device__ __forceinline__ int block_exclusive_suffix(int v, int *warp_sums) {
 
 __global__ void __launch_bounds__(kThreads, 1) topk_kernel(const TopkParams p) {
   extern __shared__ uint32_t sm[];
-  uint32_t *hist = sm;                                         // [kBins]
-  int *warp_sums = reinterpret_cast<int *>(sm + kBins);        // [2 * kWarps]
+  uint32_t *hist = sm;                                         // [2][kBins]
+  int *warp_sums = reinterpret_cast<int *>(sm + 2 * kBins);    // [2 * kWarps]
   int *bcast = warp_sums + 2 * kWarps;                         // [8]
   uint32_t *cnts = reinterpret_cast<uint32_t *>(bcast + 8);    // [2] per-CTA gt / eq counts
   uint32_t *keys = cnts + 8;                                   // [seg_cap]
 
+  griddep_wait();
+  griddep_launch_dependents();
   const uint32_t C = cluster_nctarank();
   const uint32_t c = cluster_ctarank();
   const int row = blockIdx.x / C;
@@ -95,38 +97,76 @@ __global__ void __launch_bounds__(kThreads, 1) topk_kernel(const TopkParams p) {
   const int cnt = max(0, min(n, lo + seg) - lo);
   const bool cached = seg <= p.seg_cap;
   if (cached) {
-    for (int i = tid; i < cnt; i += kThreads) keys[i] = score_key(srow[lo + i]);
+    // every load of a batch in flight before the first is used
+    const float *src = srow + lo;
+    int done = 0;
+    if ((reinterpret_cast<uintptr_t>(src) & 15u) == 0) {
+      const int nv = cnt >> 2;
+      const float4 *s4 = reinterpret_cast<const float4 *>(src);
+      uint4 *k4 = reinterpret_cast<uint4 *>(keys);
+      for (int base = 0; base < nv; base += kThreads * 8) {
+        float4 v[8];
+#pragma unroll
+        for (int j = 0; j < 8; ++j) {
+          const int i = base + j * kThreads + tid;
+          if (i < nv) v[j] = __ldg(s4 + i);
+        }
+#pragma unroll
+        for (int j = 0; j < 8; ++j) {
+          const int i = base + j * kThreads + tid;
+          if (i < nv)
+            k4[i] = make_uint4(score_key(v[j].x), score_key(v[j].y), score_key(v[j].z),
+                               score_key(v[j].w));
+        }
+      }
+      done = nv << 2;
+    }
+    for (int i = done + tid; i < cnt; i += kThreads) keys[i] = score_key(__ldg(src + i));
   }
   __syncthreads();
   auto key_at = [&](int i) -> uint32_t { return cached ? keys[i] : score_key(srow[lo + i]); };
 
   uint32_t prefix = 0, pmask = 0;
   int krem = k;
+  const int lane = lane_id();
 #pragma unroll 1
   for (int pass = 0; pass < 3; ++pass) {
+    // two histogram buffers: a peer may still read this pass's buffer while
+    // this CTA fills the next one; the cluster barrier of the next pass
+    // separates a buffer's reads from its reuse two passes later
+    uint32_t *hb = hist + (pass & 1) * kBins;
     const int shift = (pass == 0) ? 21 : (pass == 1 ? 10 : 0);
     const uint32_t bmask = (pass < 2) ? 0x7FFu : 0x3FFu;
-    for (int i = tid; i < kBins; i += kThreads) hist[i] = 0u;
+    for (int i = tid; i < kBins; i += kThreads) hb[i] = 0u;
     __syncthreads();
     for (int base = 0; base < cnt; base += kThreads) {
       const int i = base + tid;
       bool match = false;
-      uint32_t bin = 0xFFFFFFFFu;
+      uint32_t bin = 0u;
       if (i < cnt) {
         const uint32_t u = key_at(i);
         match = (u & pmask) == prefix;
-        if (match) bin = (u >> shift) & bmask;
+        bin = (u >> shift) & bmask;
       }
-      const uint32_t peers = __match_any_sync(0xffffffffu, bin);
-      if (match && lane_id() == __ffs(peers) - 1) atomicAdd(&hist[bin], __popc(peers));
+      // lanes with the same bin add once, with the count of the group
+      const uint32_t mm = __ballot_sync(0xffffffffu, match);
+      if (match) {
+        const uint32_t peers = __match_any_sync(mm, bin);
+        if (lane == __ffs(peers) - 1) atomicAdd(&hb[bin], __popc(peers));
+      }
     }
-    cluster_sync();  // all histograms of this pass are complete
-    // global histogram: thread t owns bins 4t .. 4t+3
+    cluster_sync();  // every CTA's histogram of this pass is complete
+    // global histogram: thread t owns bins 4t .. 4t+3; one 16-byte load per peer
     uint32_t gh[4] = {0u, 0u, 0u, 0u};
-    for (uint32_t r = 0; r < C; ++r) {
+    {
+      const uint32_t addr = smem_u32(&hb[4 * tid]);
+      uint4 v[8];
 #pragma unroll
-      for (int q = 0; q < 4; ++q)
-        gh[q] += ld_dsmem_u32(map_to_rank(smem_u32(&hist[4 * tid + q]), r));
+      for (int r = 0; r < 8; ++r)
+        if (r < static_cast<int>(C)) v[r] = ld_dsmem_v4(map_to_rank(addr, r));
+#pragma unroll
+      for (int r = 0; r < 8; ++r)
+        if (r < static_cast<int>(C)) { gh[0] += v[r].x; gh[1] += v[r].y; gh[2] += v[r].z; gh[3] += v[r].w; }
     }
     const int mine = static_cast<int>(gh[0] + gh[1] + gh[2] + gh[3]);
     int above = block_exclusive_suffix(mine, warp_sums);
@@ -137,7 +177,7 @@ __global__ void __launch_bounds__(kThreads, 1) topk_kernel(const TopkParams p) {
       if (above < krem && krem <= above + h) { bcast[0] = 4 * tid + q; bcast[1] = krem - above; }
       above += h;
     }
-    cluster_sync();  // peers finished reading this CTA's histogram; bcast is visible
+    __syncthreads();
     const uint32_t sel = static_cast<uint32_t>(bcast[0]);
     krem = bcast[1];
     prefix |= sel << shift;
@@ -151,7 +191,7 @@ __global__ void __launch_bounds__(kThreads, 1) topk_kernel(const TopkParams p) {
   // (CTA, warp, strip, lane).  Pass A counts keys above / equal to T per warp;
   // the CTA totals go to the cluster; pass B emits each kept index at
   // position = kept tokens with a lower index, found by ballots.
-  const int warp = warp_id(), lane = lane_id();
+  const int warp = warp_id();
   const uint32_t lt_mask = (1u << lane) - 1u;
   const int run = ((cnt + kWarps * 32 - 1) / (kWarps * 32)) * 32;
   const int w_lo = min(cnt, warp * run), w_hi = min(cnt, w_lo + run);
@@ -214,7 +254,7 @@ dsa_status_t launch_topk(const TopkLaunch &a, cudaStream_t stream) {
   int C = (max_len + 4095) / 4096;
   C = std::max(1, std::min(C, 8));
   const int seg = ((max_len + C - 1) / C + 3) & ~3;
-  const size_t fixed = 4 * (kBins + 2 * kWarps + 8 + 8) + 64;
+  const size_t fixed = 4 * (2 * kBins + 2 * kWarps + 8 + 8) + 64;
   const size_t max_smem = device_max_smem_optin();
   const int cap_max = static_cast<int>((max_smem - fixed) / 4);
   const int seg_cap = std::min(seg, cap_max);
@@ -238,19 +278,9 @@ dsa_status_t launch_topk(const TopkLaunch &a, cudaStream_t stream) {
   p.seg_cap = seg_cap;
   p.status = a.status;
 
-  cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3(static_cast<unsigned>(a.n_q) * C, 1, 1);
-  cfg.blockDim = dim3(kThreads, 1, 1);
-  cfg.dynamicSmemBytes = smem;
-  cfg.stream = stream;
-  cudaLaunchAttribute attr[1];
-  attr[0].id = cudaLaunchAttributeClusterDimension;
-  attr[0].val.clusterDim.x = C;
-  attr[0].val.clusterDim.y = 1;
-  attr[0].val.clusterDim.z = 1;
-  cfg.attrs = attr;
-  cfg.numAttrs = 1;
-  if (cudaLaunchKernelEx(&cfg, topk_kernel, p) != cudaSuccess) return DSA_ERR_CUDA;
+  if (launch_pdl(topk_kernel, dim3(static_cast<unsigned>(a.n_q) * C), dim3(kThreads), smem,
+                 stream, static_cast<unsigned>(C), p) != cudaSuccess)
+    return DSA_ERR_CUDA;
   return DSA_OK;
 }
 
