@@ -25,6 +25,13 @@ constexpr uint64_t kDrainLimitNs = 1000000000ull;
 
 int device_sm_count();
 
+// 2-D bf16 tensor map over `rows` rows of `cols` elements (row pitch cols * 2
+// bytes) with a box of box_cols x box_rows and a 128- (aw = 128) or 64-byte
+// (aw = 64) swizzle.  Returns false when the driver entry point is missing or
+// rejects the request.
+bool make_map_2d(CUtensorMap *map, const void *base, uint64_t cols, uint64_t rows,
+                 uint32_t box_cols, uint32_t box_rows, int aw);
+
 // Launch `kernel` on `stream` with programmatic stream serialization (the
 // kernel calls griddep_wait() before its first dependent read), optionally
 // as clusters of cluster_x CTAs.

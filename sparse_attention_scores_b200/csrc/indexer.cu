@@ -22,7 +22,6 @@
 // Every wait is bounded in wall time; a time-out records an error in the
 // status block, drains what is in flight, frees tensor memory and returns.
 #include <algorithm>
-#include <cudaTypedefs.h>
 
 #include "dsa_internal.h"
 
@@ -386,37 +385,6 @@ __global__ void __launch_bounds__(kThreads, 1)
 // ---------------------------------------------------------------------------
 // host side
 // ---------------------------------------------------------------------------
-PFN_cuTensorMapEncodeTiled_v12000 get_encode_fn() {
-  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
-  static bool tried = false;
-  if (!tried) {
-    tried = true;
-    void *ptr = nullptr;
-    cudaDriverEntryPointQueryResult q;
-    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) ==
-            cudaSuccess &&
-        q == cudaDriverEntryPointSuccess)
-      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(ptr);
-  }
-  return fn;
-}
-
-// 2-D bf16 tensor map: `rows` rows of `cols` elements, box of box_cols x box_rows.
-bool make_map_2d(CUtensorMap *map, const void *base, uint64_t cols, uint64_t rows,
-                 uint32_t box_cols, uint32_t box_rows, int aw) {
-  auto encode = get_encode_fn();
-  if (encode == nullptr) return false;
-  cuuint64_t dims[2] = {cols, rows};
-  cuuint64_t strides[1] = {cols * 2};
-  cuuint32_t box[2] = {box_cols, box_rows};
-  cuuint32_t estr[2] = {1, 1};
-  CUresult r = encode(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void *>(base), dims,
-                      strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
-                      aw == 128 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_64B,
-                      CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
-  return r == CUDA_SUCCESS;
-}
-
 template <int G, int AW>
 dsa_status_t launch_impl(const IndexerLaunch &a, cudaStream_t stream) {
   const int natoms = a.D_I * 2 / AW;

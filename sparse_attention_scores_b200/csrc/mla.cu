@@ -9,23 +9,28 @@
 // GPU-code paragraph: split online-softmax compressed MLA; "GLM on an A100,
 // in Vx", "The model": one latent vector per token serves as key and value.)
 //
-// Design (sm_100a): a CTA of 4 warps owns one query row and a contiguous range
+// Design (sm_100a): a CTA of 8 warps owns one query row and a contiguous range
 // of 128-key chunks of its selection.  The 64-head absorbed query stays in
 // shared memory for the whole range.  Per chunk:
-//   gather   the 128 selected latent rows (1,152 B each at R+P = 576) with
-//            16-byte cp.async into a 128B-swizzled K-major tile; unused slots
-//            are zero-filled
+//   gather   TMA tile::gather4 loads (four 128-byte row pieces per
+//            instruction) of the selected latent rows straight into a
+//            128B-swizzled K-major tile, one mbarrier per 64-column atom, so
+//            the first MMAs start while the last atoms are in flight
 //   S^T      tcgen05.mma, M = 128 keys, N = 64 heads, K = R + P, into TMEM
-//   softmax  one thread per key holds its 64 logits; per-head max and sum
-//            over the 128 keys by a transposing butterfly of warp shuffles;
-//            the running max moves only when it grows by more than 2^8, and
-//            then the TMEM accumulator is rescaled
+//   softmax  warp w reads keys 32*(w%4).. and heads 32*(w/4).. of S^T; per-head
+//            max and sum over the 128 keys by a transposing butterfly of warp
+//            shuffles; the running max moves only when it grows by more than
+//            2^8, and then the TMEM accumulator is rescaled
 //   O^T     += tcgen05.mma, M = 128 latent columns (R/128 blocks), N = 64
-//            heads, K = 128 keys; the same shared tile serves as V^T
-//            (MN-major view), P is written as bf16 over the rope atom
-// PV uses p = hi + lo (two bf16 terms) for near-fp32 weights.
-// A row split over several CTAs writes (m, l, O) partials that a second
-// kernel merges by log-sum-exp weights.
+//            heads, K = 128 keys; the latent tile serves as V^T (MN-major view).
+//            P = hi + lo (two bf16 terms, near-fp32 weights), written over the
+//            rope atom, in two halves of 64 keys
+// A row split over several CTAs (up to 16) runs as one thread-block cluster:
+// each CTA pushes its unscaled (m, l, O^T) rows of every head into the shared
+// memory of the CTA that owns the head (fire-and-forget remote stores); after
+// a cluster barrier each owner merges its heads by log-sum-exp weights and
+// writes the final output.  More than 16 splits fall back to (m, l, O)
+// partials in global scratch and a merge kernel.
 #include <algorithm>
 #include <cuda_bf16.h>
 #include <math.h>
@@ -35,25 +40,29 @@
 namespace dsa {
 namespace {
 
-constexpr int kThreads = 128;
-constexpr int kChunk = 128;   // keys per chunk = MMA M
-constexpr int kHeads = 64;    // head columns of every tile = MMA N
+constexpr int kThreads = 256;         // 8 warps
+constexpr int kChunk = 128;           // keys per chunk = MMA M
+constexpr int kHeads = 64;            // head columns of every tile = MMA N
 constexpr int kAtomL = kChunk * 128;  // bytes of one 64-column atom of the latent tile
 constexpr int kAtomQ = kHeads * 128;  // bytes of one 64-column atom of the query tile
+constexpr int kMaxAtoms = 9;          // R + P <= 576
+constexpr int kMaxCluster = 16;
 constexpr float kRescaleLog2 = 8.0f;
+constexpr float kLn2 = 0.69314718055994531f;
+
+enum : int { kMergeNone = 0, kMergeCluster = 1, kMergeGlobal = 2 };
 
 struct MlaParams {
   const uint16_t *q;
-  const uint16_t *latent;
   const int32_t *idx;
   const int32_t *seq_lens;
   const int32_t *block_table;
   float *out;
   float *lse;
-  float *part_o;   // [n_q, nsplit, 64, R]
+  float *part_o;   // [n_q, nsplit, 64, R]   (kMergeGlobal)
   float *part_ml;  // [n_q, nsplit, 2, 64]
   int n_q, H, R, W, topk, causal, q_pos0, max_pages, num_pages;
-  int nsplit, chunks_per_split;
+  int nsplit, chunks_per_split, merge;
   float scale_log2;
   uint64_t wait_ns;
   int debug_stall;  // wait once on a barrier nothing arrives at (tests the time-out path)
@@ -78,67 +87,62 @@ __device__ __forceinline__ void tmem_st_wait() {
   asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
 }
 
-// Reduce 64 per-key values over the 32 keys (lanes) of a warp, for every head
-// at once.  Each butterfly step halves the heads a lane keeps and exchanges
-// the other half with its partner; afterwards lane L holds the reductions of
-// heads 2L and 2L+1 in o[0], o[1].  62 shuffles instead of 64 x 5.
+// TMA gather of four rows (one 64-column atom piece of each) into consecutive
+// 128-byte rows of shared memory; the tensor map's box is one row high.
+__device__ __forceinline__ void tma_gather4(void *dst, const CUtensorMap *map, int x, int r0,
+                                            int r1, int r2, int r3, uint64_t *bar) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.shared::cluster.global.tile::gather4.mbarrier::complete_tx::bytes"
+      " [%0], [%1, {%2, %3, %4, %5, %6}], [%7];" ::"r"(smem_u32(dst)),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(r0), "r"(r1), "r"(r2), "r"(r3),
+      "r"(smem_u32(bar))
+      : "memory");
+}
+
+// Reduce 32 per-key values over the 32 keys (lanes) of a warp, for 32 heads at
+// once: each butterfly step halves the heads a lane keeps and exchanges the
+// other half with its partner; afterwards lane L holds head L's reduction.
+// 31 shuffles instead of 32 x 5.
 template <bool kMax, typename Get>
-__device__ __forceinline__ void butterfly64(Get v, float (&o)[2]) {
+__device__ __forceinline__ float butterfly32(Get v) {
   const int lane = lane_id();
   auto op = [](float a, float b) { return kMax ? fmaxf(a, b) : a + b; };
-  float a[32];
+  float a[16];
   {
     const bool up = lane & 16;
 #pragma unroll
-    for (int i = 0; i < 32; ++i) {
-      const float lo_h = v(i), hi_h = v(i + 32);
-      const float send = up ? lo_h : hi_h;
-      const float keep = up ? hi_h : lo_h;
-      a[i] = op(keep, __shfl_xor_sync(0xffffffffu, send, 16));
+    for (int i = 0; i < 16; ++i) {
+      const float lo_h = v(i), hi_h = v(i + 16);
+      a[i] = op(up ? hi_h : lo_h, __shfl_xor_sync(0xffffffffu, up ? lo_h : hi_h, 16));
     }
   }
-  float b[16];
+  float b[8];
   {
     const bool up = lane & 8;
 #pragma unroll
-    for (int i = 0; i < 16; ++i) {
-      const float send = up ? a[i] : a[i + 16];
-      const float keep = up ? a[i + 16] : a[i];
-      b[i] = op(keep, __shfl_xor_sync(0xffffffffu, send, 8));
-    }
+    for (int i = 0; i < 8; ++i)
+      b[i] = op(up ? a[i + 8] : a[i], __shfl_xor_sync(0xffffffffu, up ? a[i] : a[i + 8], 8));
   }
-  float c[8];
+  float c[4];
   {
     const bool up = lane & 4;
 #pragma unroll
-    for (int i = 0; i < 8; ++i) {
-      const float send = up ? b[i] : b[i + 8];
-      const float keep = up ? b[i + 8] : b[i];
-      c[i] = op(keep, __shfl_xor_sync(0xffffffffu, send, 4));
-    }
+    for (int i = 0; i < 4; ++i)
+      c[i] = op(up ? b[i + 4] : b[i], __shfl_xor_sync(0xffffffffu, up ? b[i] : b[i + 4], 4));
   }
-  float d[4];
+  float d[2];
   {
     const bool up = lane & 2;
 #pragma unroll
-    for (int i = 0; i < 4; ++i) {
-      const float send = up ? c[i] : c[i + 4];
-      const float keep = up ? c[i + 4] : c[i];
-      d[i] = op(keep, __shfl_xor_sync(0xffffffffu, send, 2));
-    }
+    for (int i = 0; i < 2; ++i)
+      d[i] = op(up ? c[i + 2] : c[i], __shfl_xor_sync(0xffffffffu, up ? c[i] : c[i + 2], 2));
   }
-  {
-    const bool up = lane & 1;
-#pragma unroll
-    for (int i = 0; i < 2; ++i) {
-      const float send = up ? d[i] : d[i + 2];
-      const float keep = up ? d[i + 2] : d[i];
-      o[i] = op(keep, __shfl_xor_sync(0xffffffffu, send, 1));
-    }
-  }
+  const bool up = lane & 1;
+  return op(up ? d[1] : d[0], __shfl_xor_sync(0xffffffffu, up ? d[0] : d[1], 1));
 }
 
-__global__ void __launch_bounds__(kThreads, 1) mla_kernel(const MlaParams p) {
+__global__ void __launch_bounds__(kThreads, 1)
+    mla_kernel(const __grid_constant__ CUtensorMap tmL, const MlaParams p) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                               ~static_cast<uintptr_t>(1023));
@@ -151,32 +155,44 @@ __global__ void __launch_bounds__(kThreads, 1) mla_kernel(const MlaParams p) {
   uint8_t *Ls = smem;
   uint8_t *Ps = p_overlays ? (Ls + (2 * nmb) * kAtomL) : (Ls + nL * kAtomL);
   uint8_t *Qs = Ls + nL * kAtomL + (p_overlays ? 0 : kAtomL);
-  const uint16_t **rowp = reinterpret_cast<const uint16_t **>(Qs + nQ * kAtomQ);  // [128]
-  float *red = reinterpret_cast<float *>(rowp + kChunk);  // [4][64]
+  int *rowi = reinterpret_cast<int *>(Qs + nQ * kAtomQ);  // [128] physical row, -1 unused
+  float *red = reinterpret_cast<float *>(rowi + kChunk);  // [4][64]
   float *mrun = red + 4 * kHeads;
   float *lrun = mrun + kHeads;
   float *alpha = lrun + kHeads;
-  uint64_t *bars = reinterpret_cast<uint64_t *>(alpha + kHeads);  // [0] S done, [1] PV done, [2] drain
-  uint32_t *misc = reinterpret_cast<uint32_t *>(bars + 4);        // [0] tmem, [1] rescale, [2] failed
+  float *fscale = alpha + kHeads;
+  float *Mfin = fscale + kHeads;
+  float *Lfin = Mfin + kHeads;
+  uint64_t *bar_atom = reinterpret_cast<uint64_t *>(Lfin + kHeads);  // [kMaxAtoms]
+  uint64_t *bar_s = bar_atom + kMaxAtoms;
+  uint64_t *bar_o = bar_s + 1;
+  uint64_t *bar_drain = bar_o + 1;
+  uint64_t *bar_stall = bar_drain + 1;
+  // [0] tmem base, [1] rescale flag, [2] failed, [3] fallback row
+  uint32_t *misc = reinterpret_cast<uint32_t *>(bar_stall + 1);
 
   const int tid = threadIdx.x, warp = warp_id(), lane = lane_id();
+  const int q4 = warp & 3;   // tensor-memory lane quadrant: keys / rows 32*q4 ..
+  const int hh = warp >> 2;  // head half: heads 32*hh ..
   const int split = blockIdx.x, row = blockIdx.y;
   const int b = p.causal ? 0 : row;
   const int nchunks = (p.topk + kChunk - 1) / kChunk;
   const int c_begin = split * p.chunks_per_split;
   const int c_end = min(nchunks, c_begin + p.chunks_per_split);
-  const int cpr = W / 8;  // 16-byte pieces per latent row
+  const int cpr = W / 8;  // 16-byte pieces per query row
 
   uint32_t tmem_cols = 32;
   while (tmem_cols < static_cast<uint32_t>(kHeads + nmb * kHeads)) tmem_cols <<= 1;
   if (tid == 0) {
-    mbar_init(&bars[0], 1);
-    mbar_init(&bars[1], 1);
-    mbar_init(&bars[2], 1);
-    mbar_init(&bars[3], 1);
+    for (int a = 0; a < kMaxAtoms; ++a) mbar_init(&bar_atom[a], 1);
+    mbar_init(bar_s, 1);
+    mbar_init(bar_o, 1);
+    mbar_init(bar_drain, 1);
+    mbar_init(bar_stall, 1);
     misc[1] = 0u;
     misc[2] = 0u;
     fence_barrier_init();
+    tma_prefetch_desc(&tmL);
   }
   if (tid < kHeads) { mrun[tid] = -INFINITY; lrun[tid] = 0.f; }
   if (warp == 0) { tmem_alloc(&misc[0], tmem_cols); tmem_relinquish(); }
@@ -188,7 +204,6 @@ __global__ void __launch_bounds__(kThreads, 1) mla_kernel(const MlaParams p) {
   {
     const uint16_t *qrow = p.q + static_cast<int64_t>(row) * p.H * W;
     const uint32_t qs = smem_u32(Qs);
-    // warp w copies heads w, w+4, ...; its lanes walk the 16-byte pieces of a row
     for (int h = warp; h < kHeads; h += kThreads / 32) {
       const bool ok = h < p.H;
       for (int cc = lane; cc < cpr; cc += 32) {
@@ -205,26 +220,27 @@ __global__ void __launch_bounds__(kThreads, 1) mla_kernel(const MlaParams p) {
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
-  const uint32_t tmem_s = misc[0];
+  const uint32_t tmem_s = misc[0] + 32u * hh;                     // this warp's S^T columns
   const uint32_t tmem_o = misc[0] + kHeads;
-  const uint32_t lane_off = static_cast<uint32_t>(warp * 32) << 16;
+  const uint32_t lane_off = static_cast<uint32_t>(q4 * 32) << 16;
   const uint32_t idesc_s = idesc_bf16_f32(kChunk, kHeads, 0, 0);
   const uint32_t idesc_pv = idesc_bf16_f32(kChunk, kHeads, 1, 1);
-  uint32_t phase = 0, pv_phase = 0;
+  uint32_t g_phase = 0, s_phase = 0, o_phase = 0;
   bool have_o = false;
   bool failed = false;
 
   if (p.debug_stall) {
-    if (!mbar_wait(&bars[3], 0u, p.wait_ns)) misc[2] = 1u;
+    if (!mbar_wait(bar_stall, 0u, p.wait_ns)) misc[2] = 1u;
     __syncthreads();
     if (misc[2]) failed = true;
   }
   for (int ch = c_begin; ch < c_end && !failed; ++ch) {
-    // resolve the 128 selected positions of this chunk
-    {
+    // resolve the 128 selected positions of this chunk to physical rows
+    int valid = 0;
+    if (tid < kChunk) {
       const int slot = ch * kChunk + tid;
-      int pos = (slot < p.topk) ? p.idx[static_cast<int64_t>(row) * p.topk + slot] : -1;
-      const uint16_t *src = nullptr;
+      const int pos = (slot < p.topk) ? p.idx[static_cast<int64_t>(row) * p.topk + slot] : -1;
+      int phys = -1;
       if (pos >= 0) {
         if (pos >= limit) {
           report(p.status, kErrBadIndex, (kKernMla << 24) | (slot & 0xFFFF));
@@ -233,71 +249,75 @@ __global__ void __launch_bounds__(kThreads, 1) mla_kernel(const MlaParams p) {
           if (page < 0 || page >= p.num_pages)
             report(p.status, kErrBadPage, (kKernMla << 24) | (slot & 0xFFFF));
           else
-            src = p.latent + (static_cast<int64_t>(page) * kPageSize + pos % kPageSize) * W;
+            phys = page * kPageSize + pos % kPageSize;
         }
       }
-      rowp[tid] = src;
+      rowi[tid] = phys;
+      valid = phys >= 0;
+      if (valid) misc[3] = static_cast<uint32_t>(phys);  // any valid row stands in for unused slots
       if (tid == 0) misc[1] = 0u;
     }
-    __syncthreads();
-    // gather the latent rows (invalid slots are zero-filled)
-    {
-      const uint32_t ls = smem_u32(Ls);
-      for (int key = warp; key < kChunk; key += kThreads / 32) {
-        const uint16_t *src = rowp[key];
-        for (int cc = lane; cc < cpr; cc += 32)
-          cp_async_16(ls + (cc >> 3) * kAtomL + key * 128 + (((cc & 7) ^ (key & 7)) << 4),
-                      src ? src + cc * 8 : p.latent, src ? 16u : 0u);
+    if (__syncthreads_count(valid) == 0) continue;  // nothing to attend in this chunk
+    // gather: lane 0 of warp w loads atoms w, w + 8; unused slots repeat a
+    // valid row (their probabilities are zero)
+    if (lane == 0) {
+      const int fb = static_cast<int>(misc[3]);
+      for (int a = warp; a < nQ; a += kThreads / 32) {
+        mbar_arrive_expect_tx(&bar_atom[a], kAtomL);
+        uint8_t *dst = Ls + a * kAtomL;
+#pragma unroll 4
+        for (int g4 = 0; g4 < kChunk / 4; ++g4) {
+          int r[4];
+#pragma unroll
+          for (int k = 0; k < 4; ++k) {
+            const int v = rowi[4 * g4 + k];
+            r[k] = v >= 0 ? v : fb;
+          }
+          tma_gather4(dst + g4 * 512, &tmL, a * 64, r[0], r[1], r[2], r[3], &bar_atom[a]);
+        }
       }
-      cp_async_commit();
-      cp_async_wait_all();
-      fence_proxy_async_smem();
     }
+    if (ch == c_begin) cp_async_wait_all();  // the query tile
+    fence_proxy_async_smem();
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
-    // S^T = L . Q^T  (M = 128 keys, N = 64 heads, K = W)
+    // S^T = L . Q^T  (M = 128 keys, N = 64 heads, K = W), atom by atom as they land
     if (tid == 0) {
       const uint32_t ls = smem_u32(Ls), qs = smem_u32(Qs);
-      for (int a = 0; a < nQ; ++a)
+      bool ok = true;
+      for (int a = 0; a < nQ && ok; ++a) {
+        if (!mbar_wait(&bar_atom[a], g_phase, p.wait_ns)) { ok = false; break; }
+        tc_fence_after();
         for (int kk = 0; kk < 4; ++kk) {
           if (a * 64 + kk * 16 >= W) break;
-          mma_bf16(tmem_s, smem_desc(ls + a * kAtomL + kk * 32, 16, 1024, kLayoutSW128),
+          mma_bf16(misc[0], smem_desc(ls + a * kAtomL + kk * 32, 16, 1024, kLayoutSW128),
                    smem_desc(qs + a * kAtomQ + kk * 32, 16, 1024, kLayoutSW128), idesc_s,
                    (a | kk) != 0 ? 1u : 0u);
         }
-      mma_commit(&bars[0]);
+      }
+      if (!ok) misc[2] = 1u;
+      mma_commit(bar_s);
     }
-    if (!mbar_wait(&bars[0], phase, p.wait_ns)) {
-      failed = true;
-      misc[2] = 1u;
-    }
+    g_phase ^= 1u;
+    if (!mbar_wait(bar_s, s_phase, p.wait_ns)) misc[2] = 1u;
+    s_phase ^= 1u;
     tc_fence_after();
     __syncthreads();
     if (misc[2]) { failed = true; break; }
 
-    // logits of key (warp*32 + lane), log2 units
-    const bool kvalid = rowp[tid] != nullptr;
-    float z[64];
+    // logits of key 32*q4 + lane for heads 32*hh .. 32*hh+31, log2 units
+    const bool kvalid = rowi[q4 * 32 + lane] >= 0;
+    float z[32];
     {
       uint32_t v[32];
       tmem_ld_32x32b_x32(tmem_s + lane_off, v);
       tmem_ld_wait();
 #pragma unroll
       for (int i = 0; i < 32; ++i) z[i] = kvalid ? __uint_as_float(v[i]) * p.scale_log2 : -INFINITY;
-      tmem_ld_32x32b_x32(tmem_s + lane_off + 32, v);
-      tmem_ld_wait();
-#pragma unroll
-      for (int i = 0; i < 32; ++i)
-        z[32 + i] = kvalid ? __uint_as_float(v[i]) * p.scale_log2 : -INFINITY;
     }
     // per-head chunk max over the 128 keys
-    {
-      float o[2];
-      butterfly64<true>([&](int h) { return z[h]; }, o);
-      red[warp * kHeads + 2 * lane] = o[0];
-      red[warp * kHeads + 2 * lane + 1] = o[1];
-    }
+    red[q4 * kHeads + 32 * hh + lane] = butterfly32<true>([&](int i) { return z[i]; });
     __syncthreads();
     if (tid < kHeads) {
       const float mc = fmaxf(fmaxf(red[tid], red[kHeads + tid]),
@@ -313,12 +333,12 @@ __global__ void __launch_bounds__(kThreads, 1) mla_kernel(const MlaParams p) {
     // probabilities, split into a bf16 head and a bf16 tail: p = hi + lo to
     // about 2^-17, so the PV product keeps near-fp32 weights even when a few
     // keys dominate.  Sums use hi + lo.
-    uint32_t phi[32], plo[32];  // packed bf16 pairs of heads (2i, 2i+1)
+    uint32_t phi[16], plo[16];  // packed bf16 pairs of heads (2i, 2i+1) of this half
 #pragma unroll
-    for (int i = 0; i < 32; ++i) {
-      const int h = 2 * i;
-      const float p0 = (z[h] == -INFINITY) ? 0.f : exp2f(z[h] - mrun[h]);
-      const float p1 = (z[h + 1] == -INFINITY) ? 0.f : exp2f(z[h + 1] - mrun[h + 1]);
+    for (int i = 0; i < 16; ++i) {
+      const int h = 32 * hh + 2 * i;
+      const float p0 = (z[2 * i] == -INFINITY) ? 0.f : exp2f(z[2 * i] - mrun[h]);
+      const float p1 = (z[2 * i + 1] == -INFINITY) ? 0.f : exp2f(z[2 * i + 1] - mrun[h + 1]);
       const __nv_bfloat162 hi = __floats2bfloat162_rn(p0, p1);
       const __nv_bfloat162 lo =
           __floats2bfloat162_rn(p0 - __low2float(hi), p1 - __high2float(hi));
@@ -326,17 +346,13 @@ __global__ void __launch_bounds__(kThreads, 1) mla_kernel(const MlaParams p) {
       plo[i] = *reinterpret_cast<const uint32_t *>(&lo);
     }
     {
-      // p of head h as the PV product sees it: hi + lo
-      auto pf = [&](int h) {
-        const uint32_t a = phi[h >> 1], b = plo[h >> 1];
-        const uint32_t ha = (h & 1) ? (a & 0xFFFF0000u) : (a << 16);
-        const uint32_t hb = (h & 1) ? (b & 0xFFFF0000u) : (b << 16);
-        return __uint_as_float(ha) + __uint_as_float(hb);
+      auto pf = [&](int i) {
+        const uint32_t a = phi[i >> 1], c = plo[i >> 1];
+        const uint32_t ha = (i & 1) ? (a & 0xFFFF0000u) : (a << 16);
+        const uint32_t hc = (i & 1) ? (c & 0xFFFF0000u) : (c << 16);
+        return __uint_as_float(ha) + __uint_as_float(hc);
       };
-      float o[2];
-      butterfly64<false>(pf, o);
-      red[warp * kHeads + 2 * lane] = o[0];
-      red[warp * kHeads + 2 * lane + 1] = o[1];
+      red[q4 * kHeads + 32 * hh + lane] = butterfly32<false>(pf);
     }
     __syncthreads();
     if (tid < kHeads) {
@@ -345,17 +361,16 @@ __global__ void __launch_bounds__(kThreads, 1) mla_kernel(const MlaParams p) {
     }
     // rescale the O accumulator when some head's running max moved
     if (misc[1]) {
-      for (int mb = 0; mb < nmb; ++mb)
-        for (int half = 0; half < 2; ++half) {
-          const uint32_t ta = tmem_o + lane_off + mb * kHeads + half * 32;
-          uint32_t v[32];
-          tmem_ld_32x32b_x32(ta, v);
-          tmem_ld_wait();
+      for (int mb = 0; mb < nmb; ++mb) {
+        const uint32_t ta = tmem_o + lane_off + mb * kHeads + 32 * hh;
+        uint32_t v[32];
+        tmem_ld_32x32b_x32(ta, v);
+        tmem_ld_wait();
 #pragma unroll
-          for (int i = 0; i < 32; ++i)
-            v[i] = __float_as_uint(__uint_as_float(v[i]) * alpha[half * 32 + i]);
-          tmem_st_32x32b_x32(ta, v);
-        }
+        for (int i = 0; i < 32; ++i)
+          v[i] = __float_as_uint(__uint_as_float(v[i]) * alpha[32 * hh + i]);
+        tmem_st_32x32b_x32(ta, v);
+      }
       tmem_st_wait();
     }
     // O^T += L^T . P^T  (M = 128 latent columns per block, N = 64 heads), in two
@@ -363,12 +378,12 @@ __global__ void __launch_bounds__(kThreads, 1) mla_kernel(const MlaParams p) {
     // The 16 KB P region holds [hi | lo] for the 64 keys of one half.
     bool pv_failed = false;
     for (int half = 0; half < 2; ++half) {
-      if ((warp >> 1) == half) {
-        const int rk = tid & 63;
+      if ((q4 >> 1) == half) {
+        const int rk = 32 * (q4 & 1) + lane;
         const uint32_t base = smem_u32(Ps) + rk * 128;
 #pragma unroll
-        for (int j = 0; j < 8; ++j) {
-          const uint32_t off = ((j ^ (rk & 7)) << 4);
+        for (int j = 0; j < 4; ++j) {
+          const uint32_t off = (((4 * hh + j) ^ (rk & 7)) << 4);
           asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(base + off),
                        "r"(phi[4 * j]), "r"(phi[4 * j + 1]), "r"(phi[4 * j + 2]), "r"(phi[4 * j + 3])
                        : "memory");
@@ -391,62 +406,149 @@ __global__ void __launch_bounds__(kThreads, 1) mla_kernel(const MlaParams p) {
                                  kLayoutSW128),
                        smem_desc(ps + part * 8192 + ks * 2048, kAtomQ, 1024, kLayoutSW128),
                        idesc_pv, (have_o || half || part || ks) ? 1u : 0u);
-        mma_commit(&bars[1]);
+        mma_commit(bar_o);
       }
-      if (!mbar_wait(&bars[1], pv_phase, p.wait_ns)) misc[2] = 1u;
-      pv_phase ^= 1u;
+      if (!mbar_wait(bar_o, o_phase, p.wait_ns)) misc[2] = 1u;
+      o_phase ^= 1u;
       tc_fence_after();
       __syncthreads();
       if (misc[2]) { pv_failed = true; break; }
     }
     if (pv_failed) failed = true;
     have_o = true;
-    phase ^= 1u;
   }
   cp_async_wait_all();
 
   if (failed) {
     if (tid == 0) {
       report(p.status, kErrTimeout, (kKernMla << 24) | 1u);
-      mma_commit(&bars[2]);  // fires once every MMA issued above has completed
-      mbar_wait(&bars[2], 0u, kDrainLimitNs);
+      mma_commit(bar_drain);  // fires once every MMA issued above has completed
+      mbar_wait(bar_drain, 0u, kDrainLimitNs);
+      // let gathers still in flight land before the shared memory is reused
+      for (int a = 0; a < nQ; ++a) mbar_wait(&bar_atom[a], g_phase ^ 1u, kDrainLimitNs);
+    }
+    if (tid < kHeads) { mrun[tid] = -INFINITY; lrun[tid] = 0.f; }
+    have_o = false;
+    __syncthreads();
+  }
+
+  if (p.merge == kMergeNone) {
+    for (int mb = 0; mb < nmb; ++mb) {
+      uint32_t v[32];
+      if (have_o) {
+        tmem_ld_32x32b_x32(tmem_o + lane_off + mb * kHeads + 32 * hh, v);
+        tmem_ld_wait();
+      }
+      const int r = mb * 128 + q4 * 32 + lane;
+      if (r < R) {
+#pragma unroll
+        for (int i = 0; i < 32; ++i) {
+          const int h = 32 * hh + i;
+          if (h >= p.H) break;
+          const float l = lrun[h];
+          const float o = (have_o && l > 0.f) ? __uint_as_float(v[i]) / l : 0.f;
+          p.out[(static_cast<int64_t>(row) * p.H + h) * R + r] = o;
+        }
+      }
+    }
+    if (tid < p.H) {
+      const float l = lrun[tid];
+      p.lse[static_cast<int64_t>(row) * p.H + tid] =
+          (l > 0.f) ? (mrun[tid] + log2f(l)) * kLn2 : -INFINITY;
+    }
+  } else if (p.merge == kMergeGlobal) {
+    for (int mb = 0; mb < nmb; ++mb) {
+      uint32_t v[32];
+      if (have_o) {
+        tmem_ld_32x32b_x32(tmem_o + lane_off + mb * kHeads + 32 * hh, v);
+        tmem_ld_wait();
+      }
+      const int r = mb * 128 + q4 * 32 + lane;
+      if (r < R) {
+        float *dst = p.part_o + ((static_cast<int64_t>(row) * p.nsplit + split) * kHeads) * R + r;
+#pragma unroll
+        for (int i = 0; i < 32; ++i) {
+          const int h = 32 * hh + i;
+          if (h >= p.H) break;
+          dst[static_cast<int64_t>(h) * R] = have_o ? __uint_as_float(v[i]) : 0.f;
+        }
+      }
+    }
+    if (tid < kHeads) {
+      float *ml = p.part_ml + (static_cast<int64_t>(row) * p.nsplit + split) * 2 * kHeads;
+      ml[tid] = mrun[tid];
+      ml[kHeads + tid] = lrun[tid];
     }
   } else {
-    // write the normalised output (single split) or the partial (m, l, O)
-    const bool direct = p.nsplit == 1;
-    for (int mb = 0; mb < nmb; ++mb)
-      for (int half = 0; half < 2; ++half) {
-        uint32_t v[32];
-        if (have_o) {
-          tmem_ld_32x32b_x32(tmem_o + lane_off + mb * kHeads + half * 32, v);
-          tmem_ld_wait();
-        }
-        const int r = mb * 128 + warp * 32 + lane;
-        if (r < R) {
-#pragma unroll
-          for (int i = 0; i < 32; ++i) {
-            const int h = half * 32 + i;
-            if (h >= p.H) break;
-            const float o = have_o ? __uint_as_float(v[i]) : 0.f;
-            if (direct) {
-              const float l = lrun[h];
-              p.out[(static_cast<int64_t>(row) * p.H + h) * R + r] = (l > 0.f) ? o / l : 0.f;
-            } else {
-              p.part_o[((static_cast<int64_t>(row) * p.nsplit + split) * kHeads + h) * R + r] = o;
-            }
-          }
-        }
-      }
+    // ---- the splits of this row form one cluster: merge through DSMEM ----
+    // Head h belongs to CTA owner(h) = floor((h*C + C - 1) / 64), which owns
+    // heads [h0(o), h1(o)) with h0(o) = floor(o*64 / C).  Every CTA pushes its
+    // unscaled (m, l, O^T) rows of each head into slot `me` of the owner's
+    // shared memory with fire-and-forget remote stores (once every CTA is past
+    // its chunk loop); after the next cluster barrier each owner merges its
+    // heads locally and writes the output.
+    const uint32_t C = cluster_nctarank();
+    const uint32_t me = cluster_ctarank();
+    // slots live in the latent + query tiles, free after the last chunk:
+    //   m, l: [C][hc] (in the reduction scratch), O: [C][hc][R]
+    float *slot_m = red;                    // <= 80 entries
+    float *slot_l = red + 2 * kHeads;       // <= 80 entries
+    float *slot_o = reinterpret_cast<float *>(Ls);
+    auto owner_of = [&](int h) { return static_cast<int>((h * C + C - 1) / kHeads); };
+    auto h0_of = [&](int o) { return static_cast<int>((o * kHeads) / C); };
+    // every CTA of the cluster is past its last chunk: its tiles and reduction
+    // scratch may now receive the pushes
+    cluster_sync();
     if (tid < p.H) {
-      if (direct) {
-        const float l = lrun[tid];
-        p.lse[static_cast<int64_t>(row) * p.H + tid] =
-            (l > 0.f) ? (mrun[tid] + log2f(l)) * 0.69314718055994531f : -INFINITY;
-      } else {
-        float *ml = p.part_ml + (static_cast<int64_t>(row) * p.nsplit + split) * 2 * kHeads;
-        ml[tid] = mrun[tid];
-        ml[kHeads + tid] = lrun[tid];
+      const int o = owner_of(tid), j = tid - h0_of(o), hc = h0_of(o + 1) - h0_of(o);
+      st_dsmem_u32(map_to_rank(smem_u32(&slot_m[me * hc + j]), o), __float_as_uint(mrun[tid]));
+      st_dsmem_u32(map_to_rank(smem_u32(&slot_l[me * hc + j]), o), __float_as_uint(lrun[tid]));
+    }
+    for (int mb = 0; mb < nmb; ++mb) {
+      uint32_t v[32];
+      if (have_o) {
+        tmem_ld_32x32b_x32(tmem_o + lane_off + mb * kHeads + 32 * hh, v);
+        tmem_ld_wait();
       }
+      const int r = mb * 128 + q4 * 32 + lane;
+      if (r < R) {
+#pragma unroll 4
+        for (int i = 0; i < 32; ++i) {
+          const int h = 32 * hh + i;
+          if (h >= p.H) break;
+          const int o = owner_of(h), j = h - h0_of(o), hc = h0_of(o + 1) - h0_of(o);
+          const uint32_t addr = smem_u32(&slot_o[(static_cast<int>(me) * hc + j) * R + r]);
+          st_dsmem_u32(map_to_rank(addr, o), have_o ? v[i] : 0u);
+        }
+      }
+    }
+    cluster_sync();  // every slot of every owner is filled; no remote access follows
+    const int h0 = h0_of(me), hc = h0_of(me + 1) - h0;
+    // per-head merge weights: w_s = 2^(m_s - M) / L with L = sum_s 2^(m_s - M) l_s
+    float *wts = fscale;  // [C][hc] <= 80 entries, reuses fscale + Mfin
+    if (tid < hc && h0 + tid < p.H) {
+      float M = -INFINITY;
+      for (uint32_t s2 = 0; s2 < C; ++s2) M = fmaxf(M, slot_m[s2 * hc + tid]);
+      float L = 0.f;
+      for (uint32_t s2 = 0; s2 < C; ++s2) {
+        const float m = slot_m[s2 * hc + tid];
+        L += (m == -INFINITY) ? 0.f : exp2f(m - M) * slot_l[s2 * hc + tid];
+      }
+      for (uint32_t s2 = 0; s2 < C; ++s2) {
+        const float m = slot_m[s2 * hc + tid];
+        wts[s2 * hc + tid] = (m == -INFINITY || !(L > 0.f)) ? 0.f : exp2f(m - M) / L;
+      }
+      p.lse[static_cast<int64_t>(row) * p.H + h0 + tid] =
+          (L > 0.f) ? (M + log2f(L)) * kLn2 : -INFINITY;
+    }
+    __syncthreads();
+    const int hvalid = max(0, min(hc, p.H - h0));
+    for (int e = tid; e < hvalid * R; e += kThreads) {
+      const int j = e / R, r = e - j * R;
+      float acc = 0.f;
+      for (uint32_t s2 = 0; s2 < C; ++s2)
+        acc += wts[s2 * hc + j] * slot_o[(static_cast<int>(s2) * hc + j) * R + r];
+      p.out[(static_cast<int64_t>(row) * p.H + h0 + j) * R + r] = acc;
     }
   }
   tc_fence_before();
@@ -458,7 +560,8 @@ __global__ void __launch_bounds__(kThreads, 1) mla_kernel(const MlaParams p) {
   }
 }
 
-// Merge the split partials of one (row, head):
+// Merge the split partials of one (row, head) when a row is split over more
+// CTAs than one cluster holds:
 //   out = sum_s 2^(m_s - M) O_s / sum_s 2^(m_s - M) l_s,  lse = (M + log2 L) ln 2.
 // The first warp loads every split's (m, l) in parallel (nsplit <= 64) and
 // reduces them with shuffles; all threads then stream the partial rows.
@@ -488,8 +591,7 @@ __global__ void __launch_bounds__(128) combine_kernel(const MlaParams p) {
     wgt[s1] = w1;
     if (lane == 0) {
       inv_l = (L > 0.f) ? 1.f / L : 0.f;
-      p.lse[static_cast<int64_t>(row) * p.H + h] =
-          (L > 0.f) ? (M + log2f(L)) * 0.69314718055994531f : -INFINITY;
+      p.lse[static_cast<int64_t>(row) * p.H + h] = (L > 0.f) ? (M + log2f(L)) * kLn2 : -INFINITY;
     }
   }
   __syncthreads();
@@ -504,32 +606,81 @@ __global__ void __launch_bounds__(128) combine_kernel(const MlaParams p) {
   }
 }
 
-}  // namespace
+size_t mla_smem_bytes(int R, int P) {
+  const int W = R + P;
+  const int nQ = (W + 63) / 64;
+  const int nmb = (R + 127) / 128;
+  const int nL = std::max(nQ, 2 * nmb);
+  const bool p_overlays = nL > 2 * nmb;
+  return 1024 + static_cast<size_t>(nL) * kAtomL + (p_overlays ? 0 : kAtomL) +
+         static_cast<size_t>(nQ) * kAtomQ + 4 * kChunk + 4 * (10 * kHeads) +
+         8 * (kMaxAtoms + 4) + 16;
+}
 
-int mla_num_splits(int n_q, int topk) {
+// Largest cluster of MLA CTAs the device co-schedules: 16 when the
+// non-portable size is available for this shared-memory size, else 8.
+// Queried once per device.
+int max_cluster_ctas(size_t smem) {
+  static int cached[64];
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return 8;
+  if (cached[dev] == 0) {
+    int best = 8;
+    if (cudaFuncSetAttribute(mla_kernel, cudaFuncAttributeNonPortableClusterSizeAllowed, 1) ==
+        cudaSuccess) {
+      cudaLaunchConfig_t cfg = {};
+      cfg.gridDim = dim3(16, 1, 1);
+      cfg.blockDim = dim3(kThreads, 1, 1);
+      cfg.dynamicSmemBytes = smem;
+      cudaLaunchAttribute attr[1];
+      attr[0].id = cudaLaunchAttributeClusterDimension;
+      attr[0].val.clusterDim.x = 16;
+      attr[0].val.clusterDim.y = 1;
+      attr[0].val.clusterDim.z = 1;
+      cfg.attrs = attr;
+      cfg.numAttrs = 1;
+      int n = 0;
+      if (cudaOccupancyMaxActiveClusters(&n, mla_kernel, &cfg) == cudaSuccess && n > 0) best = 16;
+    }
+    cudaGetLastError();  // clear a rejected query
+    cached[dev] = best;
+  }
+  return cached[dev];
+}
+
+struct SplitPlan {
+  int nsplit, chunks_per_split, merge;
+};
+
+SplitPlan plan_splits(int n_q, int topk, int max_cluster) {
   const int nchunks = (topk + kChunk - 1) / kChunk;
   int want = (device_sm_count() + n_q - 1) / std::max(1, n_q);
   want = std::max(1, std::min(want, std::min(nchunks, 64)));
   const int cps = (nchunks + want - 1) / want;
-  return (nchunks + cps - 1) / cps;
+  const int ns = (nchunks + cps - 1) / cps;
+  SplitPlan s;
+  s.nsplit = ns;
+  s.chunks_per_split = cps;
+  s.merge = (ns == 1) ? kMergeNone : (ns <= max_cluster ? kMergeCluster : kMergeGlobal);
+  return s;
 }
 
+}  // namespace
+
+int mla_num_splits(int n_q, int topk) { return plan_splits(n_q, topk, kMaxCluster).nsplit; }
+
 size_t mla_scratch_bytes(int n_q, int topk, int R) {
-  const int ns = mla_num_splits(n_q, topk);
-  if (ns <= 1) return 0;
-  const size_t o = static_cast<size_t>(n_q) * ns * kHeads * R * 4;
-  const size_t ml = static_cast<size_t>(n_q) * ns * 2 * kHeads * 4;
+  // sized for the smallest cluster limit a device may have (8)
+  const SplitPlan s = plan_splits(n_q, topk, 8);
+  if (s.merge != kMergeGlobal) return 0;
+  const size_t o = static_cast<size_t>(n_q) * s.nsplit * kHeads * R * 4;
+  const size_t ml = static_cast<size_t>(n_q) * s.nsplit * 2 * kHeads * 4;
   return ((o + 255) & ~static_cast<size_t>(255)) + ml;
 }
 
 dsa_status_t launch_mla(const MlaLaunch &a, cudaStream_t stream) {
   const int W = a.R + a.P;
-  const int nQ = (W + 63) / 64;
-  const int nmb = (a.R + 127) / 128;
-  const int nL = std::max(nQ, 2 * nmb);
-  const bool p_overlays = nL > 2 * nmb;
-  const size_t smem = 1024 + static_cast<size_t>(nL) * kAtomL + (p_overlays ? 0 : kAtomL) +
-                      static_cast<size_t>(nQ) * kAtomQ + 8 * kChunk + 4 * (7 * kHeads) + 32 + 16;
+  const size_t smem = mla_smem_bytes(a.R, a.P);
   if (smem > device_max_smem_optin()) return DSA_ERR_UNSUPPORTED;
   static bool attr_set = false;
   if (!attr_set) {
@@ -538,12 +689,14 @@ dsa_status_t launch_mla(const MlaLaunch &a, cudaStream_t stream) {
       return DSA_ERR_CUDA;
     attr_set = true;
   }
-  const int nchunks = (a.topk + kChunk - 1) / kChunk;
-  const int nsplit = mla_num_splits(a.n_q, a.topk);
-  const int cps = (nchunks + nsplit - 1) / nsplit;
+  // a row split in 9..16 runs as one cluster where the device allows it, as
+  // global partials otherwise (the scratch is sized for that case)
+  const SplitPlan sp = plan_splits(a.n_q, a.topk, max_cluster_ctas(smem));
+  CUtensorMap tmL;
+  if (!make_map_2d(&tmL, a.latent, W, static_cast<uint64_t>(a.num_pages) * kPageSize, 64, 1, 128))
+    return DSA_ERR_CUDA;
   MlaParams p;
   p.q = a.q;
-  p.latent = a.latent;
   p.idx = a.idx;
   p.seq_lens = a.seq_lens;
   p.block_table = a.block_table;
@@ -551,10 +704,11 @@ dsa_status_t launch_mla(const MlaLaunch &a, cudaStream_t stream) {
   p.lse = a.lse;
   p.part_o = nullptr;
   p.part_ml = nullptr;
-  if (nsplit > 1) {
-    if (a.scratch == nullptr || a.scratch_bytes < mla_scratch_bytes(a.n_q, a.topk, a.R))
-      return DSA_ERR_WORKSPACE;
-    const size_t o = static_cast<size_t>(a.n_q) * nsplit * kHeads * a.R * 4;
+  if (sp.merge == kMergeGlobal) {
+    const size_t o = static_cast<size_t>(a.n_q) * sp.nsplit * kHeads * a.R * 4;
+    const size_t need = ((o + 255) & ~static_cast<size_t>(255)) +
+                        static_cast<size_t>(a.n_q) * sp.nsplit * 2 * kHeads * 4;
+    if (a.scratch == nullptr || a.scratch_bytes < need) return DSA_ERR_WORKSPACE;
     p.part_o = static_cast<float *>(a.scratch);
     p.part_ml = reinterpret_cast<float *>(static_cast<uint8_t *>(a.scratch) +
                                           ((o + 255) & ~static_cast<size_t>(255)));
@@ -568,17 +722,19 @@ dsa_status_t launch_mla(const MlaLaunch &a, cudaStream_t stream) {
   p.q_pos0 = a.q_pos0;
   p.max_pages = a.max_pages;
   p.num_pages = a.num_pages;
-  p.nsplit = nsplit;
-  p.chunks_per_split = cps;
+  p.nsplit = sp.nsplit;
+  p.chunks_per_split = sp.chunks_per_split;
+  p.merge = sp.merge;
   p.scale_log2 = static_cast<float>(static_cast<double>(a.scale) * 1.4426950408889634);
   p.wait_ns = wait_limit_ns();
   p.debug_stall = debug_stall() == kKernMla ? 1 : 0;
   p.early_q = a.early_q;
   p.status = a.status;
-  if (launch_pdl(mla_kernel, dim3(nsplit, a.n_q), dim3(kThreads), smem, stream, 1, p) !=
-      cudaSuccess)
+  const unsigned cluster = (sp.merge == kMergeCluster) ? static_cast<unsigned>(sp.nsplit) : 1u;
+  if (launch_pdl(mla_kernel, dim3(sp.nsplit, a.n_q), dim3(kThreads), smem, stream, cluster, tmL,
+                 p) != cudaSuccess)
     return DSA_ERR_CUDA;
-  if (nsplit > 1) {
+  if (sp.merge == kMergeGlobal) {
     if (launch_pdl(combine_kernel, dim3(a.n_q, a.H), dim3(128), 0, stream, 1, p) != cudaSuccess)
       return DSA_ERR_CUDA;
   }

@@ -11,10 +11,11 @@
 namespace dsa {
 namespace {
 
-// 32 MiB: the status block plus the split partials of, for example, a batch
-// of 32 rows at R = 512 and top-k 2,048.  Every GPU that loads the library
-// holds it until the process exits.
-constexpr size_t kNoAllocScratchBytes = 32ull << 20;
+// 16 MiB: the status block plus the split partials of a row split over more
+// CTAs than one cluster holds, e.g. one row of top-8,192 at R = 512 in 64
+// splits (8.4 MB).  Every GPU that loads the library holds it until the
+// process exits.
+constexpr size_t kNoAllocScratchBytes = 16ull << 20;
 static __device__ __align__(256) uint8_t g_noalloc_scratch[kNoAllocScratchBytes];
 
 // In host code `g_noalloc_scratch` names a host-side stand-in, not the device

@@ -5,17 +5,22 @@
 // is right?": ties resolve as a stable argsort of -scores does, i.e. the lower
 // token index wins.)
 //
-// Design: one thread-block cluster of C CTAs per row.  Each CTA owns a
-// contiguous segment of the row and keeps the order-preserving 32-bit keys of
-// its scores in shared memory (re-reading global memory only when a segment
-// is larger than shared memory).  Three radix passes (11 + 11 + 10 bits) find
-// the exact k-th largest key T: every CTA builds a shared-memory histogram
-// (warp-aggregated atomics), the cluster barrier publishes it, and every CTA
-// sums all C histograms through distributed shared memory and runs the same
-// deterministic suffix scan.  The kept set is {key > T} plus the first
-// (k - #{key > T}) keys equal to T in index order, which a block-wide scan
-// compacts in ascending index order: output position = number of kept tokens
-// with a lower index.  No sort, no global atomics, no global scratch.
+// Design: one thread-block cluster of C <= 8 CTAs per row.  Each CTA owns a
+// contiguous segment of the row, pulls it into shared memory with one bulk
+// copy and turns it into order-preserving 32-bit keys in place (segments too
+// large for shared memory are re-read from global memory).  Three radix passes
+// (11 + 11 + 10 bits) find the exact k-th largest key T:
+//   - every warp counts its keys into a private shared-memory histogram
+//     (no cross-warp contention, no match/vote aggregation);
+//   - each CTA folds the 16 warp histograms and pushes its non-zero bins into
+//     every CTA's merged histogram with remote reductions
+//     (red.shared::cluster.add): fire-and-forget, no remote loads;
+//   - after one cluster barrier every CTA scans the merged histogram itself.
+// The kept set is {key > T} plus the first (k - #{key > T}) keys equal to T in
+// index order.  Each warp walks a contiguous run of its CTA's segment in
+// 32-key strips; per-CTA counts of keys above / equal to T are pushed to every
+// CTA; each kept index lands at position = number of kept tokens with a lower
+// index.  No sort, no global atomics, no global scratch.
 #include <algorithm>
 
 #include "dsa_internal.h"
@@ -26,6 +31,7 @@ namespace {
 constexpr int kThreads = 512;
 constexpr int kWarps = kThreads / 32;
 constexpr int kBins = 2048;
+constexpr int kMaxC = 8;
 
 struct TopkParams {
   const float *scores;
@@ -36,6 +42,7 @@ struct TopkParams {
   int k;
   int32_t *idx;
   int seg_cap;  // keys a CTA can keep in shared memory
+  uint64_t wait_ns;
   DevStatus *status;
 };
 
@@ -66,21 +73,28 @@ __device__ __forceinline__ int block_exclusive_suffix(int v, int *warp_sums) {
 }
 
 __global__ void __launch_bounds__(kThreads, 1) topk_kernel(const TopkParams p) {
-  extern __shared__ uint32_t sm[];
-  uint32_t *hist = sm;                                         // [2][kBins]
-  int *warp_sums = reinterpret_cast<int *>(sm + 2 * kBins);    // [2 * kWarps]
-  int *bcast = warp_sums + 2 * kWarps;                         // [8]
-  uint32_t *cnts = reinterpret_cast<uint32_t *>(bcast + 8);    // [2] per-CTA gt / eq counts
-  uint32_t *keys = cnts + 8;                                   // [seg_cap]
+  extern __shared__ __align__(16) uint32_t sm[];
+  uint32_t *priv = sm;                                         // [kWarps][kBins]
+  uint32_t *merged = priv + kWarps * kBins;                    // [2][kBins]
+  int *warp_sums = reinterpret_cast<int *>(merged + 2 * kBins);  // [2 * kWarps]
+  int *bcast = warp_sums + 2 * kWarps;                         // [4]
+  uint32_t *cnt_all = reinterpret_cast<uint32_t *>(bcast + 4);   // [kMaxC][2] pushed counts
+  uint64_t *bar = reinterpret_cast<uint64_t *>(cnt_all + 2 * kMaxC);
+  uint32_t *keys = reinterpret_cast<uint32_t *>(bar + 2);      // [seg_cap], 16-byte aligned
 
-  griddep_wait();
-  griddep_launch_dependents();
+  const int tid = threadIdx.x, warp = warp_id(), lane = lane_id();
   const uint32_t C = cluster_nctarank();
   const uint32_t c = cluster_ctarank();
   const int row = blockIdx.x / C;
-  const int tid = threadIdx.x;
   const int k = p.k;
   int32_t *out = p.idx + static_cast<int64_t>(row) * k;
+
+  if (tid == 0) {
+    mbar_init(bar, 1);
+    fence_barrier_init();
+  }
+  griddep_wait();
+  griddep_launch_dependents();
 
   int n = p.valid_len ? p.valid_len[row] : p.causal_base + row + 1;
   if (static_cast<int64_t>(n) > p.ld) n = static_cast<int>(p.ld);
@@ -96,80 +110,77 @@ __global__ void __launch_bounds__(kThreads, 1) topk_kernel(const TopkParams p) {
   const int lo = min(n, static_cast<int>(c) * seg);
   const int cnt = max(0, min(n, lo + seg) - lo);
   const bool cached = seg <= p.seg_cap;
-  if (cached) {
-    // every load of a batch in flight before the first is used
+
+  // zero the histograms; merged[0] must be zero before any peer pushes into it
+  {
+    uint4 *z = reinterpret_cast<uint4 *>(priv);
+    for (int i = tid; i < (kWarps + 2) * kBins / 4; i += kThreads) z[i] = make_uint4(0, 0, 0, 0);
+  }
+  if (cached && cnt > 0) {
     const float *src = srow + lo;
     int done = 0;
-    if ((reinterpret_cast<uintptr_t>(src) & 15u) == 0) {
-      const int nv = cnt >> 2;
-      const float4 *s4 = reinterpret_cast<const float4 *>(src);
-      uint4 *k4 = reinterpret_cast<uint4 *>(keys);
-      for (int base = 0; base < nv; base += kThreads * 8) {
-        float4 v[8];
-#pragma unroll
-        for (int j = 0; j < 8; ++j) {
-          const int i = base + j * kThreads + tid;
-          if (i < nv) v[j] = __ldg(s4 + i);
-        }
-#pragma unroll
-        for (int j = 0; j < 8; ++j) {
-          const int i = base + j * kThreads + tid;
-          if (i < nv)
-            k4[i] = make_uint4(score_key(v[j].x), score_key(v[j].y), score_key(v[j].z),
-                               score_key(v[j].w));
+    if ((reinterpret_cast<uintptr_t>(src) & 15u) == 0 && cnt >= 4) {
+      // one bulk copy of the first cnt & ~3 entries
+      done = cnt & ~3;
+      if (tid == 0) {
+        mbar_arrive_expect_tx(bar, static_cast<uint32_t>(done) * 4u);
+        bulk_load(keys, src, static_cast<uint32_t>(done) * 4u, bar);
+        if (!mbar_wait(bar, 0u, p.wait_ns)) {
+          report(p.status, kErrTimeout, (kKernTopk << 24) | 1u);
+          mbar_wait(bar, 0u, kDrainLimitNs);  // let the copy land before the memory is reused
         }
       }
-      done = nv << 2;
+      __syncthreads();
+      for (int i = tid; i < done; i += kThreads) keys[i] = score_key(__uint_as_float(keys[i]));
     }
     for (int i = done + tid; i < cnt; i += kThreads) keys[i] = score_key(__ldg(src + i));
   }
-  __syncthreads();
+  cluster_sync();  // histograms zeroed everywhere, keys in place
   auto key_at = [&](int i) -> uint32_t { return cached ? keys[i] : score_key(srow[lo + i]); };
 
   uint32_t prefix = 0, pmask = 0;
   int krem = k;
-  const int lane = lane_id();
+  uint32_t *mine = priv + warp * kBins;
 #pragma unroll 1
   for (int pass = 0; pass < 3; ++pass) {
-    // two histogram buffers: a peer may still read this pass's buffer while
-    // this CTA fills the next one; the cluster barrier of the next pass
-    // separates a buffer's reads from its reuse two passes later
-    uint32_t *hb = hist + (pass & 1) * kBins;
     const int shift = (pass == 0) ? 21 : (pass == 1 ? 10 : 0);
     const uint32_t bmask = (pass < 2) ? 0x7FFu : 0x3FFu;
-    for (int i = tid; i < kBins; i += kThreads) hb[i] = 0u;
+    uint32_t *mg = merged + (pass & 1) * kBins;
+    // warp-private counts of the keys that still match the prefix
+    for (int i = tid; i < cnt; i += kThreads) {
+      const uint32_t u = key_at(i);
+      if ((u & pmask) == prefix) atomicAdd(&mine[(u >> shift) & bmask], 1u);
+    }
     __syncthreads();
-    for (int base = 0; base < cnt; base += kThreads) {
-      const int i = base + tid;
-      bool match = false;
-      uint32_t bin = 0u;
-      if (i < cnt) {
-        const uint32_t u = key_at(i);
-        match = (u & pmask) == prefix;
-        bin = (u >> shift) & bmask;
-      }
-      // lanes with the same bin add once, with the count of the group
-      const uint32_t mm = __ballot_sync(0xffffffffu, match);
-      if (match) {
-        const uint32_t peers = __match_any_sync(mm, bin);
-        if (lane == __ffs(peers) - 1) atomicAdd(&hb[bin], __popc(peers));
-      }
-    }
-    cluster_sync();  // every CTA's histogram of this pass is complete
-    // global histogram: thread t owns bins 4t .. 4t+3; one 16-byte load per peer
-    uint32_t gh[4] = {0u, 0u, 0u, 0u};
+    // fold the warp histograms (thread t owns bins 4t .. 4t+3, clearing them
+    // for the next pass) and push non-zero bins into every CTA's merged one
     {
-      const uint32_t addr = smem_u32(&hb[4 * tid]);
-      uint4 v[8];
+      uint32_t v[4] = {0u, 0u, 0u, 0u};
 #pragma unroll
-      for (int r = 0; r < 8; ++r)
-        if (r < static_cast<int>(C)) v[r] = ld_dsmem_v4(map_to_rank(addr, r));
+      for (int w = 0; w < kWarps; ++w) {
+        uint4 *ph = reinterpret_cast<uint4 *>(priv + w * kBins + 4 * tid);
+        const uint4 x = *ph;
+        v[0] += x.x; v[1] += x.y; v[2] += x.z; v[3] += x.w;
+        *ph = make_uint4(0, 0, 0, 0);
+      }
 #pragma unroll
-      for (int r = 0; r < 8; ++r)
-        if (r < static_cast<int>(C)) { gh[0] += v[r].x; gh[1] += v[r].y; gh[2] += v[r].z; gh[3] += v[r].w; }
+      for (int q = 0; q < 4; ++q) {
+        if (v[q] == 0u) continue;
+        const uint32_t addr = smem_u32(&mg[4 * tid + q]);
+        for (uint32_t r = 0; r < C; ++r) red_dsmem_add_u32(map_to_rank(addr, r), v[q]);
+      }
+      // the other buffer is next pass's target: clear it before the barrier
+      // (its last reader, the scan of the previous pass, is behind us)
+      uint32_t *nx = merged + ((pass + 1) & 1) * kBins;
+      *reinterpret_cast<uint4 *>(&nx[4 * tid]) = make_uint4(0, 0, 0, 0);
     }
-    const int mine = static_cast<int>(gh[0] + gh[1] + gh[2] + gh[3]);
-    int above = block_exclusive_suffix(mine, warp_sums);
+    cluster_sync();  // every CTA's counts are in every merged histogram
+    uint32_t gh[4];
+    {
+      const uint4 x = *reinterpret_cast<const uint4 *>(&mg[4 * tid]);
+      gh[0] = x.x; gh[1] = x.y; gh[2] = x.z; gh[3] = x.w;
+    }
+    int above = block_exclusive_suffix(static_cast<int>(gh[0] + gh[1] + gh[2] + gh[3]), warp_sums);
     // the bin where the running count from the top reaches krem
 #pragma unroll
     for (int q = 3; q >= 0; --q) {
@@ -182,16 +193,14 @@ __global__ void __launch_bounds__(kThreads, 1) topk_kernel(const TopkParams p) {
     krem = bcast[1];
     prefix |= sel << shift;
     pmask |= bmask << shift;
+    __syncthreads();  // bcast is rewritten by the next pass
   }
   const uint32_t T = prefix;   // the k-th largest key
   const int need_eq = krem;    // how many keys equal to T are kept
 
   // Ordered compaction.  Warp w owns the contiguous run [w*run, (w+1)*run) of
   // this CTA's segment and walks it in 32-key strips, so index order is
-  // (CTA, warp, strip, lane).  Pass A counts keys above / equal to T per warp;
-  // the CTA totals go to the cluster; pass B emits each kept index at
-  // position = kept tokens with a lower index, found by ballots.
-  const int warp = warp_id();
+  // (CTA, warp, strip, lane).
   const uint32_t lt_mask = (1u << lane) - 1u;
   const int run = ((cnt + kWarps * 32 - 1) / (kWarps * 32)) * 32;
   const int w_lo = min(cnt, warp * run), w_hi = min(cnt, w_lo + run);
@@ -202,7 +211,7 @@ __global__ void __launch_bounds__(kThreads, 1) topk_kernel(const TopkParams p) {
     gt_w += __popc(__ballot_sync(0xffffffffu, i < w_hi && u > T));
     eq_w += __popc(__ballot_sync(0xffffffffu, i < w_hi && u == T));
   }
-  int *wgt = warp_sums;        // [kWarps] per-warp counts, then exclusive prefixes
+  int *wgt = warp_sums;  // [kWarps] per-warp counts, then exclusive prefixes
   int *weq = warp_sums + kWarps;
   if (lane == 0) { wgt[warp] = gt_w; weq[warp] = eq_w; }
   __syncthreads();
@@ -213,22 +222,20 @@ __global__ void __launch_bounds__(kThreads, 1) topk_kernel(const TopkParams p) {
       wgt[w] = g; weq[w] = e;
       g += a; e += b;
     }
-    cnts[0] = static_cast<uint32_t>(g);
-    cnts[1] = static_cast<uint32_t>(e);
-  }
-  cluster_sync();
-  if (tid == 0) {
-    uint32_t gt_before = 0, eq_before = 0;
-    for (uint32_t r = 0; r < c; ++r) {
-      gt_before += ld_dsmem_u32(map_to_rank(smem_u32(&cnts[0]), r));
-      eq_before += ld_dsmem_u32(map_to_rank(smem_u32(&cnts[1]), r));
+    // push this CTA's totals into slot c of every CTA
+    for (uint32_t r = 0; r < C; ++r) {
+      st_dsmem_u32(map_to_rank(smem_u32(&cnt_all[2 * c]), r), static_cast<uint32_t>(g));
+      st_dsmem_u32(map_to_rank(smem_u32(&cnt_all[2 * c + 1]), r), static_cast<uint32_t>(e));
     }
-    bcast[2] = static_cast<int>(gt_before);
-    bcast[3] = static_cast<int>(eq_before);
   }
-  __syncthreads();
-  int erank = bcast[3] + weq[warp];                              // equal keys before this warp
-  int pos = bcast[2] + wgt[warp] + min(erank, need_eq);          // kept keys before this warp
+  cluster_sync();  // counts of every CTA are local; no remote access follows
+  int gt_before = 0, eq_before = 0;
+  for (uint32_t r = 0; r < c; ++r) {
+    gt_before += static_cast<int>(cnt_all[2 * r]);
+    eq_before += static_cast<int>(cnt_all[2 * r + 1]);
+  }
+  int erank = eq_before + weq[warp];                       // equal keys before this warp
+  int pos = gt_before + wgt[warp] + min(erank, need_eq);   // kept keys before this warp
   for (int base = w_lo; base < w_hi; base += 32) {
     const int i = base + lane;
     const uint32_t u = (i < w_hi) ? key_at(i) : 0u;
@@ -244,7 +251,6 @@ __global__ void __launch_bounds__(kThreads, 1) topk_kernel(const TopkParams p) {
     pos += __popc(km);
     erank += __popc(eqm);
   }
-  cluster_sync();  // keep this CTA's shared memory alive until peers are done
 }
 
 }  // namespace
@@ -252,11 +258,11 @@ __global__ void __launch_bounds__(kThreads, 1) topk_kernel(const TopkParams p) {
 dsa_status_t launch_topk(const TopkLaunch &a, cudaStream_t stream) {
   const int max_len = std::max(1, a.max_len);
   int C = (max_len + 4095) / 4096;
-  C = std::max(1, std::min(C, 8));
+  C = std::max(1, std::min(C, kMaxC));
   const int seg = ((max_len + C - 1) / C + 3) & ~3;
-  const size_t fixed = 4 * (2 * kBins + 2 * kWarps + 8 + 8) + 64;
+  const size_t fixed = 4 * ((kWarps + 2) * kBins + 2 * kWarps + 4 + 2 * kMaxC) + 16 + 64;
   const size_t max_smem = device_max_smem_optin();
-  const int cap_max = static_cast<int>((max_smem - fixed) / 4);
+  const int cap_max = static_cast<int>((max_smem - fixed) / 4) & ~3;
   const int seg_cap = std::min(seg, cap_max);
   const size_t smem = fixed + 4 * static_cast<size_t>(seg_cap);
 
@@ -276,8 +282,8 @@ dsa_status_t launch_topk(const TopkLaunch &a, cudaStream_t stream) {
   p.k = a.k;
   p.idx = a.idx;
   p.seg_cap = seg_cap;
+  p.wait_ns = wait_limit_ns();
   p.status = a.status;
-
   if (launch_pdl(topk_kernel, dim3(static_cast<unsigned>(a.n_q) * C), dim3(kThreads), smem,
                  stream, static_cast<unsigned>(C), p) != cudaSuccess)
     return DSA_ERR_CUDA;

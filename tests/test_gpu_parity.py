@@ -161,6 +161,17 @@ def _random_selection(rng, lengths, k):
                                    dict(H=16, R=128, P=32, k=300)])
 @pytest.mark.parametrize("batch", [1, 5, 160])
 def test_sparse_mla_decode(shape, batch):
+    _mla_decode_case(shape, batch)
+
+
+@pytest.mark.parametrize("batch", [1, 2])
+def test_sparse_mla_decode_many_splits(batch):
+    # 64 or 32 splits per row: more than one cluster holds, so the partials
+    # go through global scratch and the merge kernel
+    _mla_decode_case(dict(H=64, R=512, P=64, k=8192), batch)
+
+
+def _mla_decode_case(shape, batch):
     rng = np.random.default_rng(batch * 7 + shape["k"])
     lengths = rng.integers(1, 3 * shape["k"], size=batch).tolist()
     wl = di.small_decode(lengths, H_I=4, D_I=32, topk=shape["k"], H=shape["H"], R=shape["R"],

@@ -30,15 +30,16 @@ def _selection(rng, lengths, k):
     return idx
 
 
-def test_noalloc_matches_workspace_entry_point():
+@pytest.mark.parametrize("lengths,topk", [([9000, 2500, 4100, 700], 2048), ([30000], 8192)],
+                         ids=["batch4_top2048", "batch1_top8192"])
+def test_noalloc_matches_workspace_entry_point(lengths, topk):
     if not torch.cuda.is_available():
         pytest.skip("no CUDA device")
     L = dsa.lib()
     rng = np.random.default_rng(77)
-    # batch 4 at GLM-5 width: the rows are split over several CTAs, so the
-    # built-in scratch array holds real partial results
-    lengths = [9000, 2500, 4100, 700]
-    wl = di.small_decode(lengths, H_I=4, D_I=32, topk=2048, H=64, R=512, P=64, seed=5)
+    # GLM-5 width; with top-8,192 a single row is split over 64 CTAs, whose
+    # partial results go through the built-in scratch array
+    wl = di.small_decode(lengths, H_I=4, D_I=32, topk=topk, H=64, R=512, P=64, seed=5)
     inp = di.make_inputs(wl)
     t = upload(inp)
     cache, dims = cache_of(inp, t), dims_of(inp)
@@ -68,14 +69,14 @@ def test_noalloc_matches_workspace_entry_point():
 
 
 def test_noalloc_rejects_oversize_request():
-    # 140 rows at R = 512 with a 65,536-token selection split in two per row
-    # need 36.7 MB of partials: more than the 32 MiB array, so the call must
-    # return DSA_ERR_WORKSPACE before launching.  Real, correctly sized buffers
-    # (every slot unused) keep the call memory-safe regardless.
+    # 18 rows of top-1,152 split 9 ways need 21.2 MB of partials: more than
+    # the 16 MiB array, so the call must return DSA_ERR_WORKSPACE before
+    # launching.  Real, correctly sized buffers (every slot unused) keep the
+    # call memory-safe regardless.
     if not torch.cuda.is_available():
         pytest.skip("no CUDA device")
     L = dsa.lib()
-    B, k, H, R, P = 140, 65536, 64, 512, 64
+    B, k, H, R, P = 18, 1152, 64, 512, 64
     q = torch.zeros((B, H, R + P), dtype=torch.bfloat16, device="cuda")
     latent = torch.zeros((1, 64, R + P), dtype=torch.bfloat16, device="cuda")
     idx = torch.full((B, k), -1, dtype=torch.int32, device="cuda")
