@@ -202,15 +202,15 @@ DSA_API dsa_status_t dsa_attention_forward(const uint16_t *q_idx, const float *w
  * hands the library only its input and output buffers.  It computes exactly
  * what dsa_sparse_mla_decode computes (same kernels, same launch shapes) but
  * takes no workspace: its scratch (the per-split partial results and a status
- * block) is a fixed 16 MiB array in the library's own device memory, present
+ * block) is a fixed 32 MiB array in the library's own device memory, present
  * on every GPU that loads the library until the process exits.
  *
  *   Arguments as for dsa_sparse_mla_decode, without ws / ws_bytes.
  *   Returns DSA_ERR_WORKSPACE, before launching anything, when the partial
- *   results of this call would not fit in the 16 MiB array.  Partials exist
- *   only when a row is split over more than 8 CTAs (n_q * splits * 64 * R * 4
- *   bytes): one row of top-8,192 at R = 512 needs 8.4 MB and fits; 18 rows of
- *   top-1,152 (9 splits each) need 21 MB and are rejected.
+ *   results of this call (n_q * splits * 64 * R * 4 bytes; rows are split
+ *   when there are fewer rows than SMs) would not fit in the 32 MiB array:
+ *   a batch of 32 at R = 512 and top-2,048 (16.8 MB) fits; 140 rows of
+ *   top-65,536 (two splits each, 36.7 MB) are rejected.
  *
  * The first call on a device looks up the array's device address (once per
  * device, with that device current); make that first call before any stream

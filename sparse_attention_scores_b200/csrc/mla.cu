@@ -25,12 +25,10 @@
 //            heads, K = 128 keys; the latent tile serves as V^T (MN-major view).
 //            P = hi + lo (two bf16 terms, near-fp32 weights), written over the
 //            rope atom, in two halves of 64 keys
-// A row split over several CTAs (up to 16) runs as one thread-block cluster:
-// each CTA pushes its unscaled (m, l, O^T) rows of every head into the shared
-// memory of the CTA that owns the head (fire-and-forget remote stores); after
-// a cluster barrier each owner merges its heads by log-sum-exp weights and
-// writes the final output.  More than 16 splits fall back to (m, l, O)
-// partials in global scratch and a merge kernel.
+// A row split over several CTAs writes its partial (m, l, O) to global
+// scratch (O^T staged in shared memory, written with bulk asynchronous
+// stores); a merge kernel, launched dependent on this one, combines the
+// splits by log-sum-exp weights.
 #include <algorithm>
 #include <cuda_bf16.h>
 #include <math.h>
@@ -46,11 +44,10 @@ constexpr int kHeads = 64;            // head columns of every tile = MMA N
 constexpr int kAtomL = kChunk * 128;  // bytes of one 64-column atom of the latent tile
 constexpr int kAtomQ = kHeads * 128;  // bytes of one 64-column atom of the query tile
 constexpr int kMaxAtoms = 9;          // R + P <= 576
-constexpr int kMaxCluster = 16;
 constexpr float kRescaleLog2 = 8.0f;
 constexpr float kLn2 = 0.69314718055994531f;
 
-enum : int { kMergeNone = 0, kMergeCluster = 1, kMergeGlobal = 2 };
+enum : int { kMergeNone = 0, kMergeGlobal = 1 };
 
 struct MlaParams {
   const uint16_t *q;
@@ -62,7 +59,7 @@ struct MlaParams {
   float *part_o;   // [n_q, nsplit, 64, R]   (kMergeGlobal)
   float *part_ml;  // [n_q, nsplit, 2, 64]
   int n_q, H, R, W, topk, causal, q_pos0, max_pages, num_pages;
-  int nsplit, chunks_per_split, merge;
+  int nsplit, chunks_per_split;
   float scale_log2;
   uint64_t wait_ns;
   int debug_stall;  // wait once on a barrier nothing arrives at (tests the time-out path)
@@ -432,7 +429,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     __syncthreads();
   }
 
-  if (p.merge == kMergeNone) {
+  if (p.nsplit == 1) {
+    // the whole selection ran here: normalise and write the output
     for (int mb = 0; mb < nmb; ++mb) {
       uint32_t v[32];
       if (have_o) {
@@ -456,7 +454,11 @@ __global__ void __launch_bounds__(kThreads, 1)
       p.lse[static_cast<int64_t>(row) * p.H + tid] =
           (l > 0.f) ? (mrun[tid] + log2f(l)) * kLn2 : -INFINITY;
     }
-  } else if (p.merge == kMergeGlobal) {
+  } else {
+    // partial (m, l, O) of this split.  O^T goes through shared memory as
+    // [64 heads][R] fp32 (the latent tile is free now) and leaves with bulk
+    // asynchronous stores, which the load/store units do not throttle.
+    float *Obuf = reinterpret_cast<float *>(Ls);
     for (int mb = 0; mb < nmb; ++mb) {
       uint32_t v[32];
       if (have_o) {
@@ -465,13 +467,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       const int r = mb * 128 + q4 * 32 + lane;
       if (r < R) {
-        float *dst = p.part_o + ((static_cast<int64_t>(row) * p.nsplit + split) * kHeads) * R + r;
 #pragma unroll
-        for (int i = 0; i < 32; ++i) {
-          const int h = 32 * hh + i;
-          if (h >= p.H) break;
-          dst[static_cast<int64_t>(h) * R] = have_o ? __uint_as_float(v[i]) : 0.f;
-        }
+        for (int i = 0; i < 32; ++i) Obuf[(32 * hh + i) * R + r] = have_o ? __uint_as_float(v[i]) : 0.f;
       }
     }
     if (tid < kHeads) {
@@ -479,76 +476,22 @@ __global__ void __launch_bounds__(kThreads, 1)
       ml[tid] = mrun[tid];
       ml[kHeads + tid] = lrun[tid];
     }
-  } else {
-    // ---- the splits of this row form one cluster: merge through DSMEM ----
-    // Head h belongs to CTA owner(h) = floor((h*C + C - 1) / 64), which owns
-    // heads [h0(o), h1(o)) with h0(o) = floor(o*64 / C).  Every CTA pushes its
-    // unscaled (m, l, O^T) rows of each head into slot `me` of the owner's
-    // shared memory with fire-and-forget remote stores (once every CTA is past
-    // its chunk loop); after the next cluster barrier each owner merges its
-    // heads locally and writes the output.
-    const uint32_t C = cluster_nctarank();
-    const uint32_t me = cluster_ctarank();
-    // slots live in the latent + query tiles, free after the last chunk:
-    //   m, l: [C][hc] (in the reduction scratch), O: [C][hc][R]
-    float *slot_m = red;                    // <= 80 entries
-    float *slot_l = red + 2 * kHeads;       // <= 80 entries
-    float *slot_o = reinterpret_cast<float *>(Ls);
-    auto owner_of = [&](int h) { return static_cast<int>((h * C + C - 1) / kHeads); };
-    auto h0_of = [&](int o) { return static_cast<int>((o * kHeads) / C); };
-    // every CTA of the cluster is past its last chunk: its tiles and reduction
-    // scratch may now receive the pushes
-    cluster_sync();
-    if (tid < p.H) {
-      const int o = owner_of(tid), j = tid - h0_of(o), hc = h0_of(o + 1) - h0_of(o);
-      st_dsmem_u32(map_to_rank(smem_u32(&slot_m[me * hc + j]), o), __float_as_uint(mrun[tid]));
-      st_dsmem_u32(map_to_rank(smem_u32(&slot_l[me * hc + j]), o), __float_as_uint(lrun[tid]));
-    }
-    for (int mb = 0; mb < nmb; ++mb) {
-      uint32_t v[32];
-      if (have_o) {
-        tmem_ld_32x32b_x32(tmem_o + lane_off + mb * kHeads + 32 * hh, v);
-        tmem_ld_wait();
-      }
-      const int r = mb * 128 + q4 * 32 + lane;
-      if (r < R) {
-#pragma unroll 4
-        for (int i = 0; i < 32; ++i) {
-          const int h = 32 * hh + i;
-          if (h >= p.H) break;
-          const int o = owner_of(h), j = h - h0_of(o), hc = h0_of(o + 1) - h0_of(o);
-          const uint32_t addr = smem_u32(&slot_o[(static_cast<int>(me) * hc + j) * R + r]);
-          st_dsmem_u32(map_to_rank(addr, o), have_o ? v[i] : 0u);
-        }
-      }
-    }
-    cluster_sync();  // every slot of every owner is filled; no remote access follows
-    const int h0 = h0_of(me), hc = h0_of(me + 1) - h0;
-    // per-head merge weights: w_s = 2^(m_s - M) / L with L = sum_s 2^(m_s - M) l_s
-    float *wts = fscale;  // [C][hc] <= 80 entries, reuses fscale + Mfin
-    if (tid < hc && h0 + tid < p.H) {
-      float M = -INFINITY;
-      for (uint32_t s2 = 0; s2 < C; ++s2) M = fmaxf(M, slot_m[s2 * hc + tid]);
-      float L = 0.f;
-      for (uint32_t s2 = 0; s2 < C; ++s2) {
-        const float m = slot_m[s2 * hc + tid];
-        L += (m == -INFINITY) ? 0.f : exp2f(m - M) * slot_l[s2 * hc + tid];
-      }
-      for (uint32_t s2 = 0; s2 < C; ++s2) {
-        const float m = slot_m[s2 * hc + tid];
-        wts[s2 * hc + tid] = (m == -INFINITY || !(L > 0.f)) ? 0.f : exp2f(m - M) / L;
-      }
-      p.lse[static_cast<int64_t>(row) * p.H + h0 + tid] =
-          (L > 0.f) ? (M + log2f(L)) * kLn2 : -INFINITY;
-    }
+    fence_proxy_async_smem();
     __syncthreads();
-    const int hvalid = max(0, min(hc, p.H - h0));
-    for (int e = tid; e < hvalid * R; e += kThreads) {
-      const int j = e / R, r = e - j * R;
-      float acc = 0.f;
-      for (uint32_t s2 = 0; s2 < C; ++s2)
-        acc += wts[s2 * hc + j] * slot_o[(static_cast<int>(s2) * hc + j) * R + r];
-      p.out[(static_cast<int64_t>(row) * p.H + h0 + j) * R + r] = acc;
+    if (tid == 0) {
+      uint8_t *dst = reinterpret_cast<uint8_t *>(
+          p.part_o + (static_cast<int64_t>(row) * p.nsplit + split) * kHeads * R);
+      const uint32_t total = static_cast<uint32_t>(kHeads * R * 4);
+      for (uint32_t off = 0; off < total; off += 32768u) {
+        const uint32_t n = min(32768u, total - off);
+        asm volatile("cp.async.bulk.global.shared::cta.bulk_group [%0], [%1], %2;" ::"l"(
+                         reinterpret_cast<uint64_t>(dst + off)),
+                     "r"(smem_u32(reinterpret_cast<uint8_t *>(Obuf) + off)), "r"(n)
+                     : "memory");
+      }
+      asm volatile("cp.async.bulk.commit_group;" ::: "memory");
+      // the shared memory must stay valid until the stores have read it
+      asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory");
     }
   }
   tc_fence_before();
@@ -560,8 +503,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   }
 }
 
-// Merge the split partials of one (row, head) when a row is split over more
-// CTAs than one cluster holds:
+// Merge the split partials of one (row, head):
 //   out = sum_s 2^(m_s - M) O_s / sum_s 2^(m_s - M) l_s,  lse = (M + log2 L) ln 2.
 // The first warp loads every split's (m, l) in parallel (nsplit <= 64) and
 // reduces them with shuffles; all threads then stream the partial rows.
@@ -617,42 +559,11 @@ size_t mla_smem_bytes(int R, int P) {
          8 * (kMaxAtoms + 4) + 16;
 }
 
-// Largest cluster of MLA CTAs the device co-schedules: 16 when the
-// non-portable size is available for this shared-memory size, else 8.
-// Queried once per device.
-int max_cluster_ctas(size_t smem) {
-  static int cached[64];
-  int dev = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return 8;
-  if (cached[dev] == 0) {
-    int best = 8;
-    if (cudaFuncSetAttribute(mla_kernel, cudaFuncAttributeNonPortableClusterSizeAllowed, 1) ==
-        cudaSuccess) {
-      cudaLaunchConfig_t cfg = {};
-      cfg.gridDim = dim3(16, 1, 1);
-      cfg.blockDim = dim3(kThreads, 1, 1);
-      cfg.dynamicSmemBytes = smem;
-      cudaLaunchAttribute attr[1];
-      attr[0].id = cudaLaunchAttributeClusterDimension;
-      attr[0].val.clusterDim.x = 16;
-      attr[0].val.clusterDim.y = 1;
-      attr[0].val.clusterDim.z = 1;
-      cfg.attrs = attr;
-      cfg.numAttrs = 1;
-      int n = 0;
-      if (cudaOccupancyMaxActiveClusters(&n, mla_kernel, &cfg) == cudaSuccess && n > 0) best = 16;
-    }
-    cudaGetLastError();  // clear a rejected query
-    cached[dev] = best;
-  }
-  return cached[dev];
-}
-
 struct SplitPlan {
   int nsplit, chunks_per_split, merge;
 };
 
-SplitPlan plan_splits(int n_q, int topk, int max_cluster) {
+SplitPlan plan_splits(int n_q, int topk) {
   const int nchunks = (topk + kChunk - 1) / kChunk;
   int want = (device_sm_count() + n_q - 1) / std::max(1, n_q);
   want = std::max(1, std::min(want, std::min(nchunks, 64)));
@@ -661,17 +572,16 @@ SplitPlan plan_splits(int n_q, int topk, int max_cluster) {
   SplitPlan s;
   s.nsplit = ns;
   s.chunks_per_split = cps;
-  s.merge = (ns == 1) ? kMergeNone : (ns <= max_cluster ? kMergeCluster : kMergeGlobal);
+  s.merge = (ns == 1) ? kMergeNone : kMergeGlobal;
   return s;
 }
 
 }  // namespace
 
-int mla_num_splits(int n_q, int topk) { return plan_splits(n_q, topk, kMaxCluster).nsplit; }
+int mla_num_splits(int n_q, int topk) { return plan_splits(n_q, topk).nsplit; }
 
 size_t mla_scratch_bytes(int n_q, int topk, int R) {
-  // sized for the smallest cluster limit a device may have (8)
-  const SplitPlan s = plan_splits(n_q, topk, 8);
+  const SplitPlan s = plan_splits(n_q, topk);
   if (s.merge != kMergeGlobal) return 0;
   const size_t o = static_cast<size_t>(n_q) * s.nsplit * kHeads * R * 4;
   const size_t ml = static_cast<size_t>(n_q) * s.nsplit * 2 * kHeads * 4;
@@ -689,9 +599,7 @@ dsa_status_t launch_mla(const MlaLaunch &a, cudaStream_t stream) {
       return DSA_ERR_CUDA;
     attr_set = true;
   }
-  // a row split in 9..16 runs as one cluster where the device allows it, as
-  // global partials otherwise (the scratch is sized for that case)
-  const SplitPlan sp = plan_splits(a.n_q, a.topk, max_cluster_ctas(smem));
+  const SplitPlan sp = plan_splits(a.n_q, a.topk);
   CUtensorMap tmL;
   if (!make_map_2d(&tmL, a.latent, W, static_cast<uint64_t>(a.num_pages) * kPageSize, 64, 1, 128))
     return DSA_ERR_CUDA;
@@ -724,15 +632,13 @@ dsa_status_t launch_mla(const MlaLaunch &a, cudaStream_t stream) {
   p.num_pages = a.num_pages;
   p.nsplit = sp.nsplit;
   p.chunks_per_split = sp.chunks_per_split;
-  p.merge = sp.merge;
   p.scale_log2 = static_cast<float>(static_cast<double>(a.scale) * 1.4426950408889634);
   p.wait_ns = wait_limit_ns();
   p.debug_stall = debug_stall() == kKernMla ? 1 : 0;
   p.early_q = a.early_q;
   p.status = a.status;
-  const unsigned cluster = (sp.merge == kMergeCluster) ? static_cast<unsigned>(sp.nsplit) : 1u;
-  if (launch_pdl(mla_kernel, dim3(sp.nsplit, a.n_q), dim3(kThreads), smem, stream, cluster, tmL,
-                 p) != cudaSuccess)
+  if (launch_pdl(mla_kernel, dim3(sp.nsplit, a.n_q), dim3(kThreads), smem, stream, 1, tmL, p) !=
+      cudaSuccess)
     return DSA_ERR_CUDA;
   if (sp.merge == kMergeGlobal) {
     if (launch_pdl(combine_kernel, dim3(a.n_q, a.H), dim3(128), 0, stream, 1, p) != cudaSuccess)

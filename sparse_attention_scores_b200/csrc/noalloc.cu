@@ -11,11 +11,11 @@
 namespace dsa {
 namespace {
 
-// 16 MiB: the status block plus the split partials of a row split over more
-// CTAs than one cluster holds, e.g. one row of top-8,192 at R = 512 in 64
-// splits (8.4 MB).  Every GPU that loads the library holds it until the
-// process exits.
-constexpr size_t kNoAllocScratchBytes = 16ull << 20;
+// 32 MiB: the status block plus the split partials of, e.g., a batch of 32
+// rows at R = 512 and top-2,048 (4 splits each, 16.8 MB) or one row of
+// top-8,192 (64 splits, 8.4 MB).  Every GPU that loads the library holds it
+// until the process exits.
+constexpr size_t kNoAllocScratchBytes = 32ull << 20;
 static __device__ __align__(256) uint8_t g_noalloc_scratch[kNoAllocScratchBytes];
 
 // In host code `g_noalloc_scratch` names a host-side stand-in, not the device

@@ -18,9 +18,10 @@
 //   - after one cluster barrier every CTA scans the merged histogram itself.
 // The kept set is {key > T} plus the first (k - #{key > T}) keys equal to T in
 // index order.  Each warp walks a contiguous run of its CTA's segment in
-// 32-key strips; per-CTA counts of keys above / equal to T are pushed to every
-// CTA; each kept index lands at position = number of kept tokens with a lower
-// index.  No sort, no global atomics, no global scratch.
+// 32-key strips (the histogram passes walk the same order, so the last pass
+// yields each warp's counts above / equal to T); per-CTA counts are pushed to
+// every CTA; each kept index lands at position = number of kept tokens with a
+// lower index.  No sort, no global atomics, no global scratch.
 #include <algorithm>
 
 #include "dsa_internal.h"
@@ -141,15 +142,28 @@ __global__ void __launch_bounds__(kThreads, 1) topk_kernel(const TopkParams p) {
   uint32_t prefix = 0, pmask = 0;
   int krem = k;
   uint32_t *mine = priv + warp * kBins;
+  // contiguous run of this CTA's segment owned by warp w, in 32-key strips:
+  // index order is (CTA, warp, strip, lane)
+  const uint32_t lt_mask = (1u << lane) - 1u;
+  const int run = ((cnt + kWarps * 32 - 1) / (kWarps * 32)) * 32;
+  const int w_lo = min(cnt, warp * run), w_hi = min(cnt, w_lo + run);
+  int above_w = 0;  // keys of this lane above the 22-bit prefix (last pass)
 #pragma unroll 1
   for (int pass = 0; pass < 3; ++pass) {
     const int shift = (pass == 0) ? 21 : (pass == 1 ? 10 : 0);
     const uint32_t bmask = (pass < 2) ? 0x7FFu : 0x3FFu;
     uint32_t *mg = merged + (pass & 1) * kBins;
-    // warp-private counts of the keys that still match the prefix
-    for (int i = tid; i < cnt; i += kThreads) {
-      const uint32_t u = key_at(i);
-      if ((u & pmask) == prefix) atomicAdd(&mine[(u >> shift) & bmask], 1u);
+    // warp-private counts of the keys that still match the prefix; warp w
+    // walks its contiguous run, so in the last pass its histogram (plus the
+    // keys above the prefix) gives the warp's counts above / equal to T
+    for (int base = w_lo; base < w_hi; base += 32) {
+      const int i = base + lane;
+      if (i < w_hi) {
+        const uint32_t u = key_at(i);
+        const uint32_t hi = u & pmask;
+        if (hi == prefix) atomicAdd(&mine[(u >> shift) & bmask], 1u);
+        else if (pass == 2 && hi > prefix) ++above_w;
+      }
     }
     __syncthreads();
     // fold the warp histograms (thread t owns bins 4t .. 4t+3, clearing them
@@ -161,7 +175,7 @@ __global__ void __launch_bounds__(kThreads, 1) topk_kernel(const TopkParams p) {
         uint4 *ph = reinterpret_cast<uint4 *>(priv + w * kBins + 4 * tid);
         const uint4 x = *ph;
         v[0] += x.x; v[1] += x.y; v[2] += x.z; v[3] += x.w;
-        *ph = make_uint4(0, 0, 0, 0);
+        if (pass < 2) *ph = make_uint4(0, 0, 0, 0);  // the last pass's stay for the counts
       }
 #pragma unroll
       for (int q = 0; q < 4; ++q) {
@@ -198,19 +212,15 @@ __global__ void __launch_bounds__(kThreads, 1) topk_kernel(const TopkParams p) {
   const uint32_t T = prefix;   // the k-th largest key
   const int need_eq = krem;    // how many keys equal to T are kept
 
-  // Ordered compaction.  Warp w owns the contiguous run [w*run, (w+1)*run) of
-  // this CTA's segment and walks it in 32-key strips, so index order is
-  // (CTA, warp, strip, lane).
-  const uint32_t lt_mask = (1u << lane) - 1u;
-  const int run = ((cnt + kWarps * 32 - 1) / (kWarps * 32)) * 32;
-  const int w_lo = min(cnt, warp * run), w_hi = min(cnt, w_lo + run);
-  int gt_w = 0, eq_w = 0;
-  for (int base = w_lo; base < w_hi; base += 32) {
-    const int i = base + lane;
-    const uint32_t u = (i < w_hi) ? key_at(i) : 0u;
-    gt_w += __popc(__ballot_sync(0xffffffffu, i < w_hi && u > T));
-    eq_w += __popc(__ballot_sync(0xffffffffu, i < w_hi && u == T));
-  }
+  // Ordered compaction.  Per-warp counts of keys above / equal to T: keys
+  // above the 22-bit prefix, plus the last pass's warp histogram above /
+  // at T's low 10 bits.
+  const uint32_t b3 = T & 0x3FFu;
+  int gt_w = above_w, eq_w = 0;
+  for (uint32_t bin = b3 + 1 + lane; bin < 1024u; bin += 32) gt_w += static_cast<int>(mine[bin]);
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) gt_w += __shfl_xor_sync(0xffffffffu, gt_w, o);
+  eq_w = static_cast<int>(mine[b3]);
   int *wgt = warp_sums;  // [kWarps] per-warp counts, then exclusive prefixes
   int *weq = warp_sums + kWarps;
   if (lane == 0) { wgt[warp] = gt_w; weq[warp] = eq_w; }

@@ -81,10 +81,9 @@ def _no_device():
 
 def test_noalloc_size_check_host_only(L):
     _no_device()
-    # 18 rows of top-1,152 split 9 ways (more than an 8-CTA cluster): the
-    # partials need 18 x 9 x 64 x 512 x 4 B = 21.2 MB > the 16 MiB array
-    d = _dims(n_q=18, topk=1152)
-    c = _cache(num_seqs=18, max_pages=1024, num_pages=1024, max_seq_len=65536)
+    # 140 rows x 2 splits x 64 heads x 512 x 4 B = 36.7 MB > the 32 MiB array
+    d = _dims(n_q=140, topk=65536)
+    c = _cache(num_seqs=140, max_pages=1024, num_pages=1024, max_seq_len=65536)
     fake = ctypes.c_void_p(0x300000)
     st = L.dsa_sparse_mla_decode_noalloc(fake, fake, ctypes.byref(c), fake, ctypes.byref(d),
                                          fake, fake, None)
