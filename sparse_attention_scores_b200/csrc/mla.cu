@@ -506,14 +506,14 @@ __global__ void __launch_bounds__(kThreads, 1)
 // Merge the split partials of one (row, head):
 //   out = sum_s 2^(m_s - M) O_s / sum_s 2^(m_s - M) l_s,  lse = (M + log2 L) ln 2.
 // The first warp loads every split's (m, l) in parallel (nsplit <= 64) and
-// reduces them with shuffles; all threads then stream the partial rows.
+// reduces them with shuffles; then each thread owns four consecutive latent
+// columns and has all splits' 16-byte loads in flight at once.
 __global__ void __launch_bounds__(128) combine_kernel(const MlaParams p) {
   const int row = blockIdx.x, h = blockIdx.y;
   griddep_wait();
   griddep_launch_dependents();
   const float *ml = p.part_ml + static_cast<int64_t>(row) * p.nsplit * 2 * kHeads;
   __shared__ float wgt[64];
-  __shared__ float inv_l;
   if (threadIdx.x < 32) {
     const int lane = threadIdx.x;
     const int s0 = lane, s1 = lane + 32;
@@ -529,22 +529,38 @@ __global__ void __launch_bounds__(128) combine_kernel(const MlaParams p) {
     float L = w0 * l0 + w1 * l1;
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) L += __shfl_xor_sync(0xffffffffu, L, o);
-    wgt[s0] = w0;
-    wgt[s1] = w1;
-    if (lane == 0) {
-      inv_l = (L > 0.f) ? 1.f / L : 0.f;
+    const float il = (L > 0.f) ? 1.f / L : 0.f;
+    wgt[s0] = w0 * il;  // normalised merge weights
+    wgt[s1] = w1 * il;
+    if (lane == 0)
       p.lse[static_cast<int64_t>(row) * p.H + h] = (L > 0.f) ? (M + log2f(L)) * kLn2 : -INFINITY;
-    }
   }
   __syncthreads();
-  const float il = inv_l;
   const float *po = p.part_o + (static_cast<int64_t>(row) * p.nsplit * kHeads + h) * p.R;
   const int64_t sstride = static_cast<int64_t>(kHeads) * p.R;
-  for (int r = threadIdx.x; r < p.R; r += blockDim.x) {
-    float acc = 0.f;
-#pragma unroll 8
-    for (int s = 0; s < p.nsplit; ++s) acc += wgt[s] * po[s * sstride + r];
-    p.out[(static_cast<int64_t>(row) * p.H + h) * p.R + r] = acc * il;
+  float *dst = p.out + (static_cast<int64_t>(row) * p.H + h) * p.R;
+  for (int r = 4 * threadIdx.x; r < p.R; r += 4 * blockDim.x) {
+    float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+    int s = 0;
+    for (; s + 8 <= p.nsplit; s += 8) {
+      float4 v[8];
+#pragma unroll
+      for (int u = 0; u < 8; ++u) v[u] = *reinterpret_cast<const float4 *>(po + (s + u) * sstride + r);
+#pragma unroll
+      for (int u = 0; u < 8; ++u) {
+        const float w = wgt[s + u];
+        acc.x += w * v[u].x; acc.y += w * v[u].y; acc.z += w * v[u].z; acc.w += w * v[u].w;
+      }
+    }
+    for (; s < p.nsplit; ++s) {
+      const float4 v = *reinterpret_cast<const float4 *>(po + s * sstride + r);
+      const float w = wgt[s];
+      acc.x += w * v.x; acc.y += w * v.y; acc.z += w * v.z; acc.w += w * v.w;
+    }
+    dst[r] = acc.x;
+    dst[r + 1] = acc.y;
+    dst[r + 2] = acc.z;
+    dst[r + 3] = acc.w;
   }
 }
 

@@ -5,7 +5,7 @@
 // is right?": ties resolve as a stable argsort of -scores does, i.e. the lower
 // token index wins.)
 //
-// Design: one thread-block cluster of C <= 8 CTAs per row.  Each CTA owns a
+// Design: one thread-block cluster of C <= 16 CTAs per row.  Each CTA owns a
 // contiguous segment of the row, pulls it into shared memory with one bulk
 // copy and turns it into order-preserving 32-bit keys in place (segments too
 // large for shared memory are re-read from global memory).  Three radix passes
@@ -32,7 +32,7 @@ namespace {
 constexpr int kThreads = 512;
 constexpr int kWarps = kThreads / 32;
 constexpr int kBins = 2048;
-constexpr int kMaxC = 8;
+constexpr int kMaxC = 16;  // 16 needs the non-portable cluster size; 8 otherwise
 
 struct TopkParams {
   const float *scores;
@@ -265,17 +265,39 @@ __global__ void __launch_bounds__(kThreads, 1) topk_kernel(const TopkParams p) {
 
 }  // namespace
 
+// Largest cluster the device co-schedules for this kernel and shared memory
+// size: 16 where the non-portable size is available, else 8.  Queried once.
+int max_topk_cluster(size_t smem) {
+  static int cached[64];
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return 8;
+  if (cached[dev] == 0) {
+    int best = 8;
+    if (cudaFuncSetAttribute(topk_kernel, cudaFuncAttributeNonPortableClusterSizeAllowed, 1) ==
+        cudaSuccess) {
+      cudaLaunchConfig_t cfg = {};
+      cfg.gridDim = dim3(16, 1, 1);
+      cfg.blockDim = dim3(kThreads, 1, 1);
+      cfg.dynamicSmemBytes = smem;
+      cudaLaunchAttribute attr[1];
+      attr[0].id = cudaLaunchAttributeClusterDimension;
+      attr[0].val.clusterDim.x = 16;
+      attr[0].val.clusterDim.y = 1;
+      attr[0].val.clusterDim.z = 1;
+      cfg.attrs = attr;
+      cfg.numAttrs = 1;
+      int n = 0;
+      if (cudaOccupancyMaxActiveClusters(&n, topk_kernel, &cfg) == cudaSuccess && n > 0) best = 16;
+    }
+    cudaGetLastError();  // clear a rejected query
+    cached[dev] = best;
+  }
+  return cached[dev];
+}
+
 dsa_status_t launch_topk(const TopkLaunch &a, cudaStream_t stream) {
   const int max_len = std::max(1, a.max_len);
-  int C = (max_len + 4095) / 4096;
-  C = std::max(1, std::min(C, kMaxC));
-  const int seg = ((max_len + C - 1) / C + 3) & ~3;
-  const size_t fixed = 4 * ((kWarps + 2) * kBins + 2 * kWarps + 4 + 2 * kMaxC) + 16 + 64;
   const size_t max_smem = device_max_smem_optin();
-  const int cap_max = static_cast<int>((max_smem - fixed) / 4) & ~3;
-  const int seg_cap = std::min(seg, cap_max);
-  const size_t smem = fixed + 4 * static_cast<size_t>(seg_cap);
-
   static bool attr_set = false;
   if (!attr_set) {
     if (cudaFuncSetAttribute(topk_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
@@ -283,6 +305,13 @@ dsa_status_t launch_topk(const TopkLaunch &a, cudaStream_t stream) {
       return DSA_ERR_CUDA;
     attr_set = true;
   }
+  int C = (max_len + 4095) / 4096;
+  C = std::max(1, std::min(C, max_topk_cluster(max_smem)));
+  const int seg = ((max_len + C - 1) / C + 3) & ~3;
+  const size_t fixed = 4 * ((kWarps + 2) * kBins + 2 * kWarps + 4 + 2 * kMaxC) + 16 + 64;
+  const int cap_max = static_cast<int>((max_smem - fixed) / 4) & ~3;
+  const int seg_cap = std::min(seg, cap_max);
+  const size_t smem = fixed + 4 * static_cast<size_t>(seg_cap);
   TopkParams p;
   p.scores = a.scores;
   p.ld = a.ld;
