@@ -10,7 +10,8 @@
 // in Vx", "The model": one latent vector per token serves as key and value.)
 //
 // Design (sm_100a): a CTA of 8 warps owns one query row and a contiguous range
-// of 128-key chunks of its selection.  The 64-head absorbed query stays in
+// of 128-key chunks of its selection (64-key chunks, the upper half of each
+// tile masked, when few rows would leave SMs idle).  The 64-head absorbed query stays in
 // shared memory for the whole range.  Per chunk:
 //   gather   TMA tile::gather4 loads (four 128-byte row pieces per
 //            instruction) of the selected latent rows straight into a
@@ -60,6 +61,7 @@ struct MlaParams {
   float *part_ml;  // [n_q, nsplit, 2, 64]
   int n_q, H, R, W, topk, causal, q_pos0, max_pages, num_pages;
   int nsplit, chunks_per_split;
+  int kc;  // selected keys per chunk: 128, or 64 when few rows leave SMs idle
   float scale_log2;
   uint64_t wait_ns;
   int debug_stall;  // wait once on a barrier nothing arrives at (tests the time-out path)
@@ -173,7 +175,8 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int hh = warp >> 2;  // head half: heads 32*hh ..
   const int split = blockIdx.x, row = blockIdx.y;
   const int b = p.causal ? 0 : row;
-  const int nchunks = (p.topk + kChunk - 1) / kChunk;
+  const int kc = p.kc;
+  const int nchunks = (p.topk + kc - 1) / kc;
   const int c_begin = split * p.chunks_per_split;
   const int c_end = min(nchunks, c_begin + p.chunks_per_split);
   const int cpr = W / 8;  // 16-byte pieces per query row
@@ -235,8 +238,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     // resolve the 128 selected positions of this chunk to physical rows
     int valid = 0;
     if (tid < kChunk) {
-      const int slot = ch * kChunk + tid;
-      const int pos = (slot < p.topk) ? p.idx[static_cast<int64_t>(row) * p.topk + slot] : -1;
+      const int slot = ch * kc + tid;
+      const int pos = (tid < kc && slot < p.topk) ? p.idx[static_cast<int64_t>(row) * p.topk + slot] : -1;
       int phys = -1;
       if (pos >= 0) {
         if (pos >= limit) {
@@ -260,10 +263,12 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (lane == 0) {
       const int fb = static_cast<int>(misc[3]);
       for (int a = warp; a < nQ; a += kThreads / 32) {
-        mbar_arrive_expect_tx(&bar_atom[a], kAtomL);
+        // rows kc .. 127 of a 64-key chunk are never gathered: their keys are
+        // masked and the PV product stops at key kc
+        mbar_arrive_expect_tx(&bar_atom[a], static_cast<uint32_t>(kc) * 128u);
         uint8_t *dst = Ls + a * kAtomL;
 #pragma unroll 4
-        for (int g4 = 0; g4 < kChunk / 4; ++g4) {
+        for (int g4 = 0; g4 < kc / 4; ++g4) {
           int r[4];
 #pragma unroll
           for (int k = 0; k < 4; ++k) {
@@ -374,7 +379,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     // halves of 64 keys; each half multiplies by the hi and by the lo terms.
     // The 16 KB P region holds [hi | lo] for the 64 keys of one half.
     bool pv_failed = false;
-    for (int half = 0; half < 2; ++half) {
+    for (int half = 0; half < kc / 64; ++half) {
       if ((q4 >> 1) == half) {
         const int rk = 32 * (q4 & 1) + lane;
         const uint32_t base = smem_u32(Ps) + rk * 128;
@@ -576,11 +581,14 @@ size_t mla_smem_bytes(int R, int P) {
 }
 
 struct SplitPlan {
-  int nsplit, chunks_per_split, merge;
+  int nsplit, chunks_per_split, merge, kc;
 };
 
 SplitPlan plan_splits(int n_q, int topk) {
-  const int nchunks = (topk + kChunk - 1) / kChunk;
+  // with few rows, 64-key chunks put twice as many SMs on the gathers
+  const int kc = (static_cast<int64_t>(n_q) * ((topk + kChunk - 1) / kChunk) <
+                  device_sm_count() / 2) ? 64 : kChunk;
+  const int nchunks = (topk + kc - 1) / kc;
   int want = (device_sm_count() + n_q - 1) / std::max(1, n_q);
   want = std::max(1, std::min(want, std::min(nchunks, 64)));
   const int cps = (nchunks + want - 1) / want;
@@ -589,6 +597,7 @@ SplitPlan plan_splits(int n_q, int topk) {
   s.nsplit = ns;
   s.chunks_per_split = cps;
   s.merge = (ns == 1) ? kMergeNone : kMergeGlobal;
+  s.kc = kc;
   return s;
 }
 
@@ -648,6 +657,7 @@ dsa_status_t launch_mla(const MlaLaunch &a, cudaStream_t stream) {
   p.num_pages = a.num_pages;
   p.nsplit = sp.nsplit;
   p.chunks_per_split = sp.chunks_per_split;
+  p.kc = sp.kc;
   p.scale_log2 = static_cast<float>(static_cast<double>(a.scale) * 1.4426950408889634);
   p.wait_ns = wait_limit_ns();
   p.debug_stall = debug_stall() == kKernMla ? 1 : 0;

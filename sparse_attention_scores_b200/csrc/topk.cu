@@ -305,7 +305,9 @@ dsa_status_t launch_topk(const TopkLaunch &a, cudaStream_t stream) {
       return DSA_ERR_CUDA;
     attr_set = true;
   }
+  // about 4K keys per CTA, at most one wave of CTAs
   int C = (max_len + 4095) / 4096;
+  C = std::min(C, std::max(1, device_sm_count() / std::max(1, a.n_q)));
   C = std::max(1, std::min(C, max_topk_cluster(max_smem)));
   const int seg = ((max_len + C - 1) / C + 3) & ~3;
   const size_t fixed = 4 * ((kWarps + 2) * kBins + 2 * kWarps + 4 + 2 * kMaxC) + 16 + 64;
