@@ -96,6 +96,20 @@ bool make_map_2d(CUtensorMap *map, const void *base, uint64_t cols, uint64_t row
   return r == CUDA_SUCCESS;
 }
 
+size_t device_smem_per_sm() {
+  static size_t cached[kMaxDevices];
+  const int d = current_device();
+  if (d < 0) return 233472;
+  if (cached[d] == 0) {
+    int v = 0;
+    if (cudaDeviceGetAttribute(&v, cudaDevAttrMaxSharedMemoryPerMultiprocessor, d) != cudaSuccess ||
+        v <= 0)
+      return 233472;
+    cached[d] = static_cast<size_t>(v);
+  }
+  return cached[d];
+}
+
 namespace {
 
 constexpr size_t kStatusBytes = sizeof(DevStatus);

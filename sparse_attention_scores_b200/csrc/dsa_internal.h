@@ -60,6 +60,7 @@ cudaError_t launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t s
   return cudaLaunchKernelEx(&cfg, kernel, std::forward<Args>(args)...);
 }
 size_t device_max_smem_optin();
+size_t device_smem_per_sm();
 
 struct IndexerLaunch {
   const uint16_t *q_idx;

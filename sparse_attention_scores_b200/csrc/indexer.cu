@@ -16,9 +16,12 @@
 //              (two per tile) into a ring of shared-memory stages; the
 //              query tile when the row group changes
 //   warp 1     tcgen05.mma issuer (one thread), double-buffered accumulators
-//   warps 2-9  epilogue, two warpgroups taking alternate tiles: tcgen05.ld
-//              of a 128-lane accumulator, ReLU, head-weighted sum, coalesced
-//              fp32 stores; up to 8 accumulators let the MMA run ahead
+//   warps 2+   epilogue warpgroups taking alternate tiles: tcgen05.ld of a
+//              128-lane accumulator, ReLU, head-weighted sum, coalesced fp32
+//              stores; up to 8 accumulators let the MMA run ahead
+// Decode runs two CTAs per SM (one epilogue warpgroup each) so that one CTA's
+// pipeline bubbles are covered by the other; grouped prefill runs one CTA per
+// SM with two epilogue warpgroups.
 // Every wait is bounded in wall time; a time-out records an error in the
 // status block, drains what is in flight, frees tensor memory and returns.
 #include <algorithm>
@@ -28,7 +31,10 @@
 namespace dsa {
 namespace {
 
-constexpr int kThreads = 320;      // producer warp, MMA warp, two epilogue warpgroups
+// producer warp, MMA warp, NEG epilogue warpgroups (NEG = 2: one CTA per SM;
+// NEG = 1: two CTAs per SM, whose pipelines cover each other's bubbles)
+template <int NEG>
+__host__ __device__ constexpr int threads_of() { return 64 + 128 * NEG; }
 constexpr int kMaxAcc = 8;         // accumulator buffers in tensor memory
 constexpr int kTileKeys = 128;
 constexpr int kLookahead = 16;  // units whose page ids the producer fetches at once
@@ -43,6 +49,7 @@ struct IndexerParams {
   int max_pages, num_pages;
   int num_groups;
   int stages;
+  int q_buffers;   // 1 or 2 query tiles in shared memory
   uint64_t wait_ns;
   int debug_stall;  // the MMA issuer first waits on a barrier nothing arrives at
   DevStatus *status;
@@ -76,14 +83,16 @@ __device__ __forceinline__ int locate(const int *tile_start, int ng, int u) {
   return lo;
 }
 
-template <int G, int AW>
-__global__ void __launch_bounds__(kThreads, 1)
+template <int G, int AW, int NEG>
+__global__ void __launch_bounds__(threads_of<NEG>(), NEG == 1 ? 2 : 1)
     indexer_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmQ,
                    const IndexerParams p) {
+  constexpr int kThreads = threads_of<NEG>();
   extern __shared__ uint8_t smem_raw[];
   uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                               ~static_cast<uintptr_t>(1023));
   const int S = p.stages;
+  const int nqb = p.q_buffers;
   const int natoms = p.D_I * 2 / AW;            // swizzle atoms along K
   const int stage_bytes = kTileKeys * p.D_I * 2;
   const int ncols = G * p.H_I;                  // useful accumulator columns
@@ -98,7 +107,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   uint8_t *stage_base = smem;
   uint8_t *q_base = smem + S * stage_bytes;
-  uint64_t *bars = reinterpret_cast<uint64_t *>(q_base + 2 * q_bytes);
+  uint64_t *bars = reinterpret_cast<uint64_t *>(q_base + nqb * q_bytes);
   uint64_t *full = bars;
   uint64_t *empty = bars + S;
   uint64_t *qfull = bars + 2 * S;
@@ -164,28 +173,36 @@ __global__ void __launch_bounds__(kThreads, 1)
     uint32_t phase = 0, qphase = 0;
     uint32_t armed = 0, armed_par = 0;  // stages with loads in flight, their phase parity
     bool ok = true;
-    for (int ub = u0; ub < u1 && ok; ub += kLookahead) {
-      // lane-parallel lookahead: lane l fetches page (l & 1) of unit ub + l/2
-      const int my_u = ub + (lane >> 1);
-      int my_g = -1, my_id = -1;
+    // lane-parallel lookahead: lane l resolves page (l & 1) of unit ub + l/2;
+    // the next batch is fetched while the current one is issued
+    auto fetch = [&](int ub_, int &g_, int &id_) {
+      const int my_u = ub_ + (lane >> 1);
+      g_ = -1;
+      id_ = -1;
       if (my_u < u1) {
-        my_g = locate(tile_start, NG, my_u);
-        const int t = my_u - tile_start[my_g];
+        g_ = locate(tile_start, NG, my_u);
+        const int t = my_u - tile_start[g_];
         const int pg = 2 * t + (lane & 1);
-        if (pg * kPageSize < group_keys<G>(p, my_g)) {
-          const int b = p.causal ? 0 : my_g;
+        if (pg * kPageSize < group_keys<G>(p, g_)) {
+          const int b = p.causal ? 0 : g_;
           const int id = p.block_table[static_cast<int64_t>(b) * p.max_pages + pg];
           if (id < 0 || id >= p.num_pages)
             report(p.status, kErrBadPage, (kKernIndexer << 24) | (pg & 0xFFFF));
           else
-            my_id = id;
+            id_ = id;
         }
       }
+    };
+    int cur_g, cur_id;
+    fetch(u0, cur_g, cur_id);
+    for (int ub = u0; ub < u1 && ok; ub += kLookahead) {
+      int nxt_g, nxt_id;
+      fetch(ub + kLookahead, nxt_g, nxt_id);
       const int nb = min(kLookahead, u1 - ub);
       for (int i = 0; i < nb; ++i) {
-        const int g = __shfl_sync(0xffffffffu, my_g, 2 * i);
-        const int id0 = __shfl_sync(0xffffffffu, my_id, 2 * i);
-        const int id1 = __shfl_sync(0xffffffffu, my_id, 2 * i + 1);
+        const int g = __shfl_sync(0xffffffffu, cur_g, 2 * i);
+        const int id0 = __shfl_sync(0xffffffffu, cur_id, 2 * i);
+        const int id1 = __shfl_sync(0xffffffffu, cur_id, 2 * i + 1);
         int okl = 1;
         if (lane == 0) {
           if (*abort_flag) okl = 0;
@@ -225,11 +242,12 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (!okl) { ok = false; break; }
         if (g != cur) {
           cur = g;
-          qslot ^= 1;
-          if (qslot == 0) qphase ^= 1u;
+          if (++qslot == nqb) { qslot = 0; qphase ^= 1u; }
         }
         if (++stage == S) { stage = 0; phase ^= 1u; }
       }
+      cur_g = nxt_g;
+      cur_id = nxt_id;
     }
     if (lane == 0) {
       if (!ok && !*abort_flag) {
@@ -255,8 +273,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           if (!mbar_wait(&qfull[qslot], qphase, p.wait_ns)) { ok = false; break; }
           cur = g;
           cur_slot = qslot;
-          qslot ^= 1;
-          if (qslot == 0) qphase ^= 1u;
+          if (++qslot == nqb) { qslot = 0; qphase ^= 1u; }
         }
         // accumulator of the i-th unit of this CTA: i % nacc, its (i / nacc)-th use
         const int i_unit = u - u0;
@@ -301,7 +318,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     int wgroup = -1;
     bool ok = true;
     int g = (u0 < u1) ? locate(tile_start, NG, u0) : 0;
-    for (int u = u0 + eg; u < u1; u += 2) {
+    for (int u = u0 + eg; u < u1; u += NEG) {
       while (tile_start[g + 1] <= u) ++g;
       const int i_unit = u - u0;
       const int acc = i_unit % nacc;
@@ -385,8 +402,9 @@ __global__ void __launch_bounds__(kThreads, 1)
 // ---------------------------------------------------------------------------
 // host side
 // ---------------------------------------------------------------------------
-template <int G, int AW>
+template <int G, int AW, int NEG>
 dsa_status_t launch_impl(const IndexerLaunch &a, cudaStream_t stream) {
+  constexpr int kThreads = threads_of<NEG>();
   const int natoms = a.D_I * 2 / AW;
   const int ncols = G * a.H_I;
   const int n_mma = (ncols + 15) & ~15;
@@ -401,24 +419,30 @@ dsa_status_t launch_impl(const IndexerLaunch &a, cudaStream_t stream) {
 
   const size_t stage_bytes = static_cast<size_t>(kTileKeys) * a.D_I * 2;
   const size_t q_bytes = static_cast<size_t>(natoms) * n_mma * AW;
-  const size_t fixed = 1024 /*align*/ + 2 * q_bytes + 8 * (2 * 8 + 5 + 2 * kMaxAcc) + 16 + 4 * kThreads +
-                       4 * ((num_groups + 4) & ~3) + 64;
+  // two CTAs per SM share the SM's shared memory (one query tile each)
+  const int q_buffers = (NEG == 1) ? 1 : 2;
+  const size_t fixed = 1024 /*align*/ + q_buffers * q_bytes + 8 * (2 * 8 + 5 + 2 * kMaxAcc) + 16 +
+                       4 * kThreads + 4 * ((num_groups + 4) & ~3) + 64;
   const size_t max_smem = device_max_smem_optin();
-  int stages = static_cast<int>((max_smem - fixed) / stage_bytes);
+  const size_t budget = (NEG == 1) ? (device_smem_per_sm() / 2 - 1024) : max_smem;
+  int stages = static_cast<int>((std::min(budget, max_smem) - fixed) / stage_bytes);
   stages = std::min(stages, 8);
   if (stages < 2) return DSA_ERR_UNSUPPORTED;
   const size_t smem = fixed + stages * stage_bytes;
 
   static bool attr_set = false;  // per template instantiation
   if (!attr_set) {
-    if (cudaFuncSetAttribute(indexer_kernel<G, AW>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+    if (cudaFuncSetAttribute(indexer_kernel<G, AW, NEG>,
+                             cudaFuncAttributeMaxDynamicSharedMemorySize,
                              static_cast<int>(max_smem)) != cudaSuccess)
       return DSA_ERR_CUDA;
     attr_set = true;
   }
   const int64_t max_keys = a.causal ? static_cast<int64_t>(a.q_pos0) + a.n_q : a.max_seq_len;
   const int64_t max_units = static_cast<int64_t>(num_groups) * ((max_keys + kTileKeys - 1) / kTileKeys);
-  const int grid = static_cast<int>(std::max<int64_t>(1, std::min<int64_t>(device_sm_count(), max_units)));
+  const int per_sm = (NEG == 1) ? 2 : 1;
+  const int grid = static_cast<int>(
+      std::max<int64_t>(1, std::min<int64_t>(static_cast<int64_t>(per_sm) * device_sm_count(), max_units)));
 
   IndexerParams p;
   p.w = a.w;
@@ -435,11 +459,12 @@ dsa_status_t launch_impl(const IndexerLaunch &a, cudaStream_t stream) {
   p.num_pages = a.num_pages;
   p.num_groups = num_groups;
   p.stages = stages;
+  p.q_buffers = q_buffers;
   p.wait_ns = wait_limit_ns();
   p.debug_stall = debug_stall() == kKernIndexer ? 1 : 0;
   p.status = a.status;
-  if (launch_pdl(indexer_kernel<G, AW>, dim3(grid), dim3(kThreads), smem, stream, 1, tmK, tmQ, p) !=
-      cudaSuccess)
+  if (launch_pdl(indexer_kernel<G, AW, NEG>, dim3(grid), dim3(kThreads), smem, stream, 1, tmK, tmQ,
+                 p) != cudaSuccess)
     return DSA_ERR_CUDA;
   return DSA_OK;
 }
@@ -447,9 +472,11 @@ dsa_status_t launch_impl(const IndexerLaunch &a, cudaStream_t stream) {
 }  // namespace
 
 dsa_status_t launch_indexer(const IndexerLaunch &a, cudaStream_t stream) {
+  // causal prefill rows share keys: groups of 4 rows, one CTA per SM; decode
+  // rows: one row per unit, two CTAs per SM
   const bool grouped = a.causal && (a.H_I % 32 == 0) && (4 * a.H_I <= 256);
-  if (a.D_I == 32) return grouped ? launch_impl<4, 64>(a, stream) : launch_impl<1, 64>(a, stream);
-  return grouped ? launch_impl<4, 128>(a, stream) : launch_impl<1, 128>(a, stream);
+  if (a.D_I == 32) return grouped ? launch_impl<4, 64, 2>(a, stream) : launch_impl<1, 64, 1>(a, stream);
+  return grouped ? launch_impl<4, 128, 2>(a, stream) : launch_impl<1, 128, 1>(a, stream);
 }
 
 }  // namespace dsa
