@@ -142,15 +142,37 @@ class ClockSampler:
 
 
 # ---------------------------------------------------------------------------
+# replicas across ranks (weak scaling, no data-path collective)
+# ---------------------------------------------------------------------------
+
+def replica_workload(wl, rank: int):
+    """The workload rank `rank` runs: the same shapes, its own seeded batch."""
+    return wl if rank == 0 else di.replace(wl, seed=wl.seed + 1000 * rank)
+
+
+def max_over_ranks(x: float, dist, device) -> float:
+    """The largest of every rank's `x` (every rank must call this, in the same order)."""
+    if dist is None or not dist.is_initialized() or dist.get_world_size() == 1:
+        return float(x)
+    import torch
+    t = torch.tensor([float(x)], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def job_rows_per_s(rows_per_rank: int, world: int, ms_per_step: float) -> float:
+    """Whole-job throughput: the rows all ranks processed over the slowest rank's step."""
+    return rows_per_rank * world / (ms_per_step * 1e-3)
+
+
+# ---------------------------------------------------------------------------
 # GPU arm
 # ---------------------------------------------------------------------------
 
 class Case:
     """Device-resident inputs, outputs and workspace of one workload."""
 
-    def __init__(self, wl, torch, dsa, seed_offset=0):
-        if seed_offset:
-            wl = di.replace(wl, seed=wl.seed + seed_offset)
+    def __init__(self, wl, torch, dsa):
         self.wl = wl
         self.inp = di.make_inputs(wl)
         inp = self.inp
@@ -193,7 +215,8 @@ class Case:
         # (the same split rule as the library's launcher)
         n_q, topk = self.wl.n_q, self.wl.topk
         sms = self.torch.cuda.get_device_properties(0).multi_processor_count
-        nchunks = (topk + 127) // 128
+        kc = 64 if n_q * ((topk + 127) // 128) < sms // 2 else 128
+        nchunks = (topk + kc - 1) // kc
         want = max(1, min((sms + n_q - 1) // n_q, min(nchunks, 64)))
         cps = (nchunks + want - 1) // want
         nsplit = (nchunks + cps - 1) // cps
@@ -333,9 +356,10 @@ def run_ours(args):
 
     wl = di.CONFIGS[args.config]
     # weak scaling: every rank runs its own replica of the workload (its own batch)
-    case = Case(wl, torch, dsa, seed_offset=1000 * rank)
+    case = Case(replica_workload(wl, rank), torch, dsa)
     case.step()
     torch.cuda.synchronize()
+    pg = dist if world > 1 else None
 
     if world > 1:
         dist.barrier()
@@ -349,29 +373,20 @@ def run_ours(args):
         torch.cuda.synchronize()
     if world > 1:
         dist.barrier()
-    ms = head["us_per_step"] / 1e3
-    if world > 1:
-        tt = torch.tensor([ms], device="cuda")
-        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
-        ms = float(tt.item())
+    ms = max_over_ranks(head["us_per_step"] / 1e3, pg, "cuda")
     e2e = None if args.profile else measure_e2e(case, torch, args.steps, args.warmup)
-    if world > 1 and e2e is not None:
-        tt = torch.tensor([e2e["ms_per_step"]], device="cuda")
-        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
-        e2e["ms_per_step"] = float(tt.item())
-        e2e["value"] = wl.n_q * world / (e2e["ms_per_step"] * 1e-3)
+    if e2e is not None:
+        e2e["ms_per_step"] = max_over_ranks(e2e["ms_per_step"], pg, "cuda")
+        e2e["value"] = job_rows_per_s(wl.n_q, world, e2e["ms_per_step"])
 
     per_config = {}
     if not args.no_extra:
         for name in EXTRA:
-            c = Case(di.CONFIGS[name], torch, dsa, seed_offset=1000 * rank)
+            c = Case(replica_workload(di.CONFIGS[name], rank), torch, dsa)
             c.step()
             torch.cuda.synchronize()
             r = measure(c, torch, args.steps, args.warmup, flush_buf, peaks)
-            if world > 1:
-                tt = torch.tensor([r["us_per_step"]], device="cuda")
-                dist.all_reduce(tt, op=dist.ReduceOp.MAX)
-                r["us_per_step"] = float(tt.item())
+            r["us_per_step"] = max_over_ranks(r["us_per_step"], pg, "cuda")
             per_config[name] = r
             del c
             torch.cuda.empty_cache()
@@ -382,7 +397,7 @@ def run_ours(args):
         line = {
             "metric": "DSA attention decode tokens/s (one layer's DSA step: indexer, exact "
                       "top-2048, sparse absorbed MLA)",
-            "value": wl.n_q * world / (ms * 1e-3),
+            "value": job_rows_per_s(wl.n_q, world, ms),
             "unit": "tokens/s",
             "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
             "ms_per_step": ms, "us_per_step": ms * 1e3,

@@ -251,6 +251,24 @@ def test_sparse_attends_only_selected_rows():
 
 # ---------------------------------------------------------------- whole step
 
+def test_step_keeps_the_best_scored_tokens():
+    # the whole step: the kept set is the stable-argsort head of its own
+    # indexer scores, and the output is dense attention over exactly those rows
+    wl = di.small_decode([300, 97], H_I=3, D_I=16, topk=64, H=2, R=16, P=8, seed=14)
+    inp = di.make_inputs(wl)
+    res = orc.dsa_decode(inp)
+    for b, n in enumerate(wl.seq_lens):
+        r = res[b]
+        want = np.sort(np.argsort(-r["scores"], kind="stable")[:wl.topk]).tolist()
+        got = r["idx"][r["idx"] >= 0].tolist()
+        assert got == want
+        lat = orc.bf16_to_f64(orc.gather_paged_rows(inp["latent_pages"],
+                                                    inp["block_table"][b], want))
+        out, lse = orc.dense_mla_attention(orc.bf16_to_f64(inp["q"][b]), lat, wl.R, wl.scale)
+        np.testing.assert_allclose(r["out"], out, rtol=1e-10, atol=1e-12)
+        np.testing.assert_allclose(r["lse"], lse, rtol=1e-12)
+
+
 def test_prefill_row_equals_decode_at_same_position():
     # cached decode == full-prefix forward: prefill row t must equal a decode
     # query at position t over the same cache
