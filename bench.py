@@ -81,9 +81,14 @@ def algorithmic(wl):
     b_indexer = keys * (wl.D_I * 2 + 4) + wl.n_q * wl.H_I * (wl.D_I * 2 + 4)
     if wl.mode == "prefill":
         b_indexer = (wl.q_pos0 + wl.n_q) * wl.D_I * 2 + keys * 4
+    # top-k alone: every score read once, the index rows written
+    b_topk = keys * 4 + wl.n_q * wl.topk * 4
+    # sparse MLA + split merge: selected latent rows, q, idx in; out, lse out
+    b_mla = b_lat + wl.n_q * (wl.H * wl.W * 2 + wl.topk * 4 + wl.H * wl.R * 4 + wl.H * 4)
     return {"bytes": b_keys + b_lat + b_small, "bytes_keys": b_keys, "bytes_latent": b_lat,
             "flops": flops_idx + flops_mla, "flops_indexer": flops_idx, "flops_mla": flops_mla,
-            "bytes_indexer": b_indexer, "keys": keys, "selected": sel}
+            "bytes_indexer": b_indexer, "bytes_topk": b_topk, "bytes_mla": b_mla,
+            "keys": keys, "selected": sel}
 
 
 # ---------------------------------------------------------------------------
@@ -210,6 +215,22 @@ class Case:
         self.dsa.dsa_indexer_scores(t["q_idx"], t["w"], t["k_pages"], self.cache, self.dims,
                                     self.scores, self.ws)
 
+    def topk(self):
+        # the scores of the last indexer() call; decode rows end at their
+        # sequence length, prefill rows at q_pos0 + t
+        if self.wl.mode == "prefill":
+            self.dsa.dsa_topk(self.scores, None, self.wl.q_pos0, self.wl.topk, self.idx, self.ws)
+        else:
+            self.dsa.dsa_topk(self.scores, self.t["seq_lens"], 0, self.wl.topk, self.idx,
+                              self.ws)
+
+    def mla(self):
+        t = self.t
+        fn = (self.dsa.dsa_sparse_mla_prefill if self.wl.mode == "prefill"
+              else self.dsa.dsa_sparse_mla_decode)
+        fn(t["q"], t["latent_pages"], self.cache, self.idx, self.dims, self.out, self.lse,
+           self.ws)
+
     def launches_per_step(self):
         # indexer + top-k + MLA, plus the split combine when a row is split
         # (the same split rule as the library's launcher)
@@ -249,7 +270,13 @@ def measure(case, torch, steps, warmup, flush_buf, peaks):
     st, info = case.dsa.workspace_check(case.ws)
     if st != 0:
         raise RuntimeError(f"device status {st} ({info:#x}) on {wl.name}")
+    # each stage alone through its own entry point, L2 flushed before each
     ms_idx, _ = timed_events(torch, case.indexer, steps, warmup, flush_buf)
+    ms_topk, _ = timed_events(torch, case.topk, steps, warmup, flush_buf)
+    ms_mla, _ = timed_events(torch, case.mla, steps, warmup, flush_buf)
+    st, info = case.dsa.workspace_check(case.ws)
+    if st != 0:
+        raise RuntimeError(f"device status {st} ({info:#x}) in the stage timings of {wl.name}")
     s = ms * 1e-3
     res = {
         "workload": wl.name, "mode": wl.mode, "us_per_step": ms * 1e3,
@@ -264,8 +291,37 @@ def measure(case, torch, steps, warmup, flush_buf, peaks):
         "indexer_gbs": alg["bytes_indexer"] / (ms_idx * 1e-3) / 1e9,
         "indexer_frac_of_measured_hbm": alg["bytes_indexer"] / (ms_idx * 1e-3) / 1e9 / peaks["hbm_gbs"],
         "launches_per_step": case.launches_per_step(),
+        "stage_us": {"indexer": ms_idx * 1e3, "topk": ms_topk * 1e3, "mla": ms_mla * 1e3},
+        "stage_alg_bytes": {"indexer": alg["bytes_indexer"], "topk": alg["bytes_topk"],
+                            "mla": alg["bytes_mla"]},
     }
     return res
+
+
+STAGE_KERNELS = {"indexer": "indexer_kernel (tcgen05 + TMA)",
+                 "topk": "topk_kernel (cluster radix select)",
+                 "mla": "mla_kernel + combine_kernel (tcgen05 + TMA gather4, split merge)"}
+
+
+def roofline_of(res, wl, peaks):
+    """Roofline of the stage that takes the longest alone: algorithmic bytes
+    (or flops, for the tensor-bound prefill MLA) over its event time."""
+    stage = max(res["stage_us"], key=res["stage_us"].get)
+    us = res["stage_us"][stage]
+    if wl.mode == "prefill" and stage == "mla":
+        alg = algorithmic(wl)
+        achieved = alg["flops_mla"] / (us * 1e-6) / 1e12
+        return {"kernel": STAGE_KERNELS[stage], "stage": stage, "bound": "tensor",
+                "achieved": achieved, "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
+                "frac": achieved / peaks["bf16_tflops"], "traffic": None,
+                "peak_source": peaks["source"], "alg_flops_per_launch": alg["flops_mla"],
+                "launch_us": us}
+    b = res["stage_alg_bytes"][stage]
+    achieved = b / (us * 1e-6) / 1e9
+    return {"kernel": STAGE_KERNELS[stage], "stage": stage, "bound": "hbm",
+            "achieved": achieved, "peak": peaks["hbm_gbs"], "unit": "GB/s",
+            "frac": achieved / peaks["hbm_gbs"], "traffic": None,
+            "peak_source": peaks["source"], "alg_bytes_per_launch": b, "launch_us": us}
 
 
 def measure_e2e(case, torch, steps, warmup):
@@ -387,6 +443,7 @@ def run_ours(args):
             torch.cuda.synchronize()
             r = measure(c, torch, args.steps, args.warmup, flush_buf, peaks)
             r["us_per_step"] = max_over_ranks(r["us_per_step"], pg, "cuda")
+            r["roofline"] = roofline_of(r, c.wl, peaks)
             per_config[name] = r
             del c
             torch.cuda.empty_cache()
@@ -411,13 +468,8 @@ def run_ours(args):
                        "alg_bytes_per_step": alg["bytes"],
                        "achieved_gbs": alg["bytes"] / (ms * 1e-3) / 1e9,
                        "frac_of_8tbs": alg["bytes"] / (ms * 1e-3) / 1e9 / NOMINAL_HBM_GBS},
-            "roofline": {"kernel": "indexer (tcgen05 + TMA)", "bound": "hbm",
-                         "achieved": alg["bytes_indexer"] / idx_s / 1e9,
-                         "peak": peaks["hbm_gbs"], "unit": "GB/s",
-                         "frac": alg["bytes_indexer"] / idx_s / 1e9 / peaks["hbm_gbs"],
-                         "traffic": None, "peak_source": peaks["source"],
-                         "alg_bytes_per_launch": alg["bytes_indexer"],
-                         "launch_us": head["indexer_us"]},
+            "roofline": roofline_of(head, wl, peaks),
+            "stage_us": head["stage_us"],
             "e2e": e2e,
             "gpu_launches": head["launches_per_step"] * args.steps,
             "clocks": clk.summary(),

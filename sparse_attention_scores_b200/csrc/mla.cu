@@ -27,9 +27,10 @@
 //            P = hi + lo (two bf16 terms, near-fp32 weights), written over the
 //            rope atom, in two halves of 64 keys
 // A row split over several CTAs writes its partial (m, l, O) to global
-// scratch (O^T staged in shared memory, written with bulk asynchronous
-// stores); a merge kernel, launched dependent on this one, combines the
-// splits by log-sum-exp weights.
+// scratch: O goes through shared memory one 128-column block at a time, and
+// each block leaves with a bulk asynchronous store while the next is staged.
+// A merge kernel, launched dependent on this one, combines the splits by
+// log-sum-exp weights.
 #include <algorithm>
 #include <cuda_bf16.h>
 #include <math.h>
@@ -57,7 +58,7 @@ struct MlaParams {
   const int32_t *block_table;
   float *out;
   float *lse;
-  float *part_o;   // [n_q, nsplit, 64, R]   (kMergeGlobal)
+  float *part_o;   // [n_q, nsplit, R/128 blocks, 64 heads, 128]   (kMergeGlobal)
   float *part_ml;  // [n_q, nsplit, 2, 64]
   int n_q, H, R, W, topk, causal, q_pos0, max_pages, num_pages;
   int nsplit, chunks_per_split;
@@ -159,10 +160,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   float *mrun = red + 4 * kHeads;
   float *lrun = mrun + kHeads;
   float *alpha = lrun + kHeads;
-  float *fscale = alpha + kHeads;
-  float *Mfin = fscale + kHeads;
-  float *Lfin = Mfin + kHeads;
-  uint64_t *bar_atom = reinterpret_cast<uint64_t *>(Lfin + kHeads);  // [kMaxAtoms]
+  uint64_t *bar_atom = reinterpret_cast<uint64_t *>(alpha + kHeads);  // [kMaxAtoms]
   uint64_t *bar_s = bar_atom + kMaxAtoms;
   uint64_t *bar_o = bar_s + 1;
   uint64_t *bar_drain = bar_o + 1;
@@ -460,41 +458,38 @@ __global__ void __launch_bounds__(kThreads, 1)
           (l > 0.f) ? (mrun[tid] + log2f(l)) * kLn2 : -INFINITY;
     }
   } else {
-    // partial (m, l, O) of this split.  O^T goes through shared memory as
-    // [64 heads][R] fp32 (the latent tile is free now) and leaves with bulk
-    // asynchronous stores, which the load/store units do not throttle.
+    // partial (m, l, O) of this split.  O^T leaves one 128-column block at a
+    // time: staged as fp32 [64 heads][128] in shared memory (the latent tile
+    // is free now), then written by a bulk asynchronous store that runs while
+    // the next block is staged.
     float *Obuf = reinterpret_cast<float *>(Ls);
+    float *dst = p.part_o + (static_cast<int64_t>(row) * p.nsplit + split) * nmb * kHeads * 128;
+    if (tid < kHeads) {
+      float *ml = p.part_ml + (static_cast<int64_t>(row) * p.nsplit + split) * 2 * kHeads;
+      ml[tid] = mrun[tid];
+      ml[kHeads + tid] = lrun[tid];
+    }
     for (int mb = 0; mb < nmb; ++mb) {
       uint32_t v[32];
       if (have_o) {
         tmem_ld_32x32b_x32(tmem_o + lane_off + mb * kHeads + 32 * hh, v);
         tmem_ld_wait();
       }
-      const int r = mb * 128 + q4 * 32 + lane;
-      if (r < R) {
+      float *blk = Obuf + mb * kHeads * 128;
+      const int cc = q4 * 32 + lane;
 #pragma unroll
-        for (int i = 0; i < 32; ++i) Obuf[(32 * hh + i) * R + r] = have_o ? __uint_as_float(v[i]) : 0.f;
-      }
-    }
-    if (tid < kHeads) {
-      float *ml = p.part_ml + (static_cast<int64_t>(row) * p.nsplit + split) * 2 * kHeads;
-      ml[tid] = mrun[tid];
-      ml[kHeads + tid] = lrun[tid];
-    }
-    fence_proxy_async_smem();
-    __syncthreads();
-    if (tid == 0) {
-      uint8_t *dst = reinterpret_cast<uint8_t *>(
-          p.part_o + (static_cast<int64_t>(row) * p.nsplit + split) * kHeads * R);
-      const uint32_t total = static_cast<uint32_t>(kHeads * R * 4);
-      for (uint32_t off = 0; off < total; off += 32768u) {
-        const uint32_t n = min(32768u, total - off);
+      for (int i = 0; i < 32; ++i) blk[(32 * hh + i) * 128 + cc] = have_o ? __uint_as_float(v[i]) : 0.f;
+      fence_proxy_async_smem();
+      __syncthreads();
+      if (tid == 0) {
         asm volatile("cp.async.bulk.global.shared::cta.bulk_group [%0], [%1], %2;" ::"l"(
-                         reinterpret_cast<uint64_t>(dst + off)),
-                     "r"(smem_u32(reinterpret_cast<uint8_t *>(Obuf) + off)), "r"(n)
+                         reinterpret_cast<uint64_t>(dst + mb * kHeads * 128)),
+                     "r"(smem_u32(blk)), "r"(static_cast<uint32_t>(kHeads * 128 * 4))
                      : "memory");
+        asm volatile("cp.async.bulk.commit_group;" ::: "memory");
       }
-      asm volatile("cp.async.bulk.commit_group;" ::: "memory");
+    }
+    if (tid == 0) {
       // the shared memory must stay valid until the stores have read it
       asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory");
     }
@@ -508,64 +503,67 @@ __global__ void __launch_bounds__(kThreads, 1)
   }
 }
 
-// Merge the split partials of one (row, head):
+// Merge the split partials of one (row, head, 128-column block):
 //   out = sum_s 2^(m_s - M) O_s / sum_s 2^(m_s - M) l_s,  lse = (M + log2 L) ln 2.
-// The first warp loads every split's (m, l) in parallel (nsplit <= 64) and
-// reduces them with shuffles; then each thread owns four consecutive latent
-// columns and has all splits' 16-byte loads in flight at once.
-__global__ void __launch_bounds__(128) combine_kernel(const MlaParams p) {
-  const int row = blockIdx.x, h = blockIdx.y;
+// One warp per CTA; each lane owns four consecutive columns.  Its 16-byte
+// loads of up to 16 splits are issued before the merge weights are known,
+// while the same lanes load every split's (m, l) (nsplit <= 64), so both wait
+// on memory once; the weights reach every lane by shuffles.
+__global__ void __launch_bounds__(32) combine_kernel(const MlaParams p) {
+  constexpr int kBatch = 16;
+  const int row = blockIdx.x, h = blockIdx.y, mb = blockIdx.z, nmb = gridDim.z;
+  const int lane = threadIdx.x;
   griddep_wait();
   griddep_launch_dependents();
+  const int c = 4 * lane;
+  const int64_t sstride = static_cast<int64_t>(nmb) * kHeads * 128;  // floats per split
+  const float *po =
+      p.part_o + (static_cast<int64_t>(row) * p.nsplit * nmb + mb) * kHeads * 128 + h * 128 + c;
   const float *ml = p.part_ml + static_cast<int64_t>(row) * p.nsplit * 2 * kHeads;
-  __shared__ float wgt[64];
-  if (threadIdx.x < 32) {
-    const int lane = threadIdx.x;
-    const int s0 = lane, s1 = lane + 32;
-    const float m0 = (s0 < p.nsplit) ? ml[s0 * 2 * kHeads + h] : -INFINITY;
-    const float m1 = (s1 < p.nsplit) ? ml[s1 * 2 * kHeads + h] : -INFINITY;
-    const float l0 = (s0 < p.nsplit) ? ml[s0 * 2 * kHeads + kHeads + h] : 0.f;
-    const float l1 = (s1 < p.nsplit) ? ml[s1 * 2 * kHeads + kHeads + h] : 0.f;
-    float M = fmaxf(m0, m1);
+  float4 v[kBatch];
 #pragma unroll
-    for (int o = 16; o > 0; o >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, o));
-    const float w0 = (m0 == -INFINITY) ? 0.f : exp2f(m0 - M);
-    const float w1 = (m1 == -INFINITY) ? 0.f : exp2f(m1 - M);
-    float L = w0 * l0 + w1 * l1;
+  for (int u = 0; u < kBatch; ++u)
+    v[u] = (u < p.nsplit) ? *reinterpret_cast<const float4 *>(po + u * sstride)
+                          : make_float4(0.f, 0.f, 0.f, 0.f);
+  const int s0 = lane, s1 = lane + 32;
+  const float m0 = (s0 < p.nsplit) ? ml[s0 * 2 * kHeads + h] : -INFINITY;
+  const float m1 = (s1 < p.nsplit) ? ml[s1 * 2 * kHeads + h] : -INFINITY;
+  const float l0 = (s0 < p.nsplit) ? ml[s0 * 2 * kHeads + kHeads + h] : 0.f;
+  const float l1 = (s1 < p.nsplit) ? ml[s1 * 2 * kHeads + kHeads + h] : 0.f;
+  float M = fmaxf(m0, m1);
 #pragma unroll
-    for (int o = 16; o > 0; o >>= 1) L += __shfl_xor_sync(0xffffffffu, L, o);
-    const float il = (L > 0.f) ? 1.f / L : 0.f;
-    wgt[s0] = w0 * il;  // normalised merge weights
-    wgt[s1] = w1 * il;
-    if (lane == 0)
-      p.lse[static_cast<int64_t>(row) * p.H + h] = (L > 0.f) ? (M + log2f(L)) * kLn2 : -INFINITY;
+  for (int o = 16; o > 0; o >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, o));
+  const float e0 = (m0 == -INFINITY) ? 0.f : exp2f(m0 - M);
+  const float e1 = (m1 == -INFINITY) ? 0.f : exp2f(m1 - M);
+  float L = e0 * l0 + e1 * l1;
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) L += __shfl_xor_sync(0xffffffffu, L, o);
+  const float il = (L > 0.f) ? 1.f / L : 0.f;
+  const float w0 = e0 * il, w1 = e1 * il;  // normalised merge weights of splits lane, lane+32
+  if (lane == 0 && mb == 0)
+    p.lse[static_cast<int64_t>(row) * p.H + h] = (L > 0.f) ? (M + log2f(L)) * kLn2 : -INFINITY;
+  float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+  for (int s = 0; s < p.nsplit; s += kBatch) {
+    if (s > 0) {
+#pragma unroll
+      for (int u = 0; u < kBatch; ++u)
+        v[u] = (s + u < p.nsplit) ? *reinterpret_cast<const float4 *>(po + (s + u) * sstride)
+                                  : make_float4(0.f, 0.f, 0.f, 0.f);
+    }
+#pragma unroll
+    for (int u = 0; u < kBatch; ++u) {
+      const int su = s + u;  // warp-uniform
+      const float w = __shfl_sync(0xffffffffu, su < 32 ? w0 : w1, su & 31);
+      acc.x += w * v[u].x; acc.y += w * v[u].y; acc.z += w * v[u].z; acc.w += w * v[u].w;
+    }
   }
-  __syncthreads();
-  const float *po = p.part_o + (static_cast<int64_t>(row) * p.nsplit * kHeads + h) * p.R;
-  const int64_t sstride = static_cast<int64_t>(kHeads) * p.R;
-  float *dst = p.out + (static_cast<int64_t>(row) * p.H + h) * p.R;
-  for (int r = 4 * threadIdx.x; r < p.R; r += 4 * blockDim.x) {
-    float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-    int s = 0;
-    for (; s + 8 <= p.nsplit; s += 8) {
-      float4 v[8];
-#pragma unroll
-      for (int u = 0; u < 8; ++u) v[u] = *reinterpret_cast<const float4 *>(po + (s + u) * sstride + r);
-#pragma unroll
-      for (int u = 0; u < 8; ++u) {
-        const float w = wgt[s + u];
-        acc.x += w * v[u].x; acc.y += w * v[u].y; acc.z += w * v[u].z; acc.w += w * v[u].w;
-      }
-    }
-    for (; s < p.nsplit; ++s) {
-      const float4 v = *reinterpret_cast<const float4 *>(po + s * sstride + r);
-      const float w = wgt[s];
-      acc.x += w * v.x; acc.y += w * v.y; acc.z += w * v.z; acc.w += w * v.w;
-    }
-    dst[r] = acc.x;
-    dst[r + 1] = acc.y;
-    dst[r + 2] = acc.z;
-    dst[r + 3] = acc.w;
+  const int r = mb * 128 + c;
+  if (r < p.R) {
+    float *dst = p.out + (static_cast<int64_t>(row) * p.H + h) * p.R + r;  // 4-byte aligned only
+    dst[0] = acc.x;
+    dst[1] = acc.y;
+    dst[2] = acc.z;
+    dst[3] = acc.w;
   }
 }
 
@@ -576,7 +574,7 @@ size_t mla_smem_bytes(int R, int P) {
   const int nL = std::max(nQ, 2 * nmb);
   const bool p_overlays = nL > 2 * nmb;
   return 1024 + static_cast<size_t>(nL) * kAtomL + (p_overlays ? 0 : kAtomL) +
-         static_cast<size_t>(nQ) * kAtomQ + 4 * kChunk + 4 * (10 * kHeads) +
+         static_cast<size_t>(nQ) * kAtomQ + 4 * kChunk + 4 * (7 * kHeads) +
          8 * (kMaxAtoms + 4) + 16;
 }
 
@@ -608,7 +606,7 @@ int mla_num_splits(int n_q, int topk) { return plan_splits(n_q, topk).nsplit; }
 size_t mla_scratch_bytes(int n_q, int topk, int R) {
   const SplitPlan s = plan_splits(n_q, topk);
   if (s.merge != kMergeGlobal) return 0;
-  const size_t o = static_cast<size_t>(n_q) * s.nsplit * kHeads * R * 4;
+  const size_t o = static_cast<size_t>(n_q) * s.nsplit * ((R + 127) / 128) * kHeads * 128 * 4;
   const size_t ml = static_cast<size_t>(n_q) * s.nsplit * 2 * kHeads * 4;
   return ((o + 255) & ~static_cast<size_t>(255)) + ml;
 }
@@ -638,7 +636,8 @@ dsa_status_t launch_mla(const MlaLaunch &a, cudaStream_t stream) {
   p.part_o = nullptr;
   p.part_ml = nullptr;
   if (sp.merge == kMergeGlobal) {
-    const size_t o = static_cast<size_t>(a.n_q) * sp.nsplit * kHeads * a.R * 4;
+    const size_t o =
+        static_cast<size_t>(a.n_q) * sp.nsplit * ((a.R + 127) / 128) * kHeads * 128 * 4;
     const size_t need = ((o + 255) & ~static_cast<size_t>(255)) +
                         static_cast<size_t>(a.n_q) * sp.nsplit * 2 * kHeads * 4;
     if (a.scratch == nullptr || a.scratch_bytes < need) return DSA_ERR_WORKSPACE;
@@ -667,7 +666,8 @@ dsa_status_t launch_mla(const MlaLaunch &a, cudaStream_t stream) {
       cudaSuccess)
     return DSA_ERR_CUDA;
   if (sp.merge == kMergeGlobal) {
-    if (launch_pdl(combine_kernel, dim3(a.n_q, a.H), dim3(128), 0, stream, 1, p) != cudaSuccess)
+    if (launch_pdl(combine_kernel, dim3(a.n_q, a.H, (a.R + 127) / 128), dim3(32), 0, stream, 1,
+                   p) != cudaSuccess)
       return DSA_ERR_CUDA;
   }
   return DSA_OK;

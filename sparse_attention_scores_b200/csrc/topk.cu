@@ -8,20 +8,27 @@
 // Design: one thread-block cluster of C <= 16 CTAs per row.  Each CTA owns a
 // contiguous segment of the row, pulls it into shared memory with one bulk
 // copy and turns it into order-preserving 32-bit keys in place (segments too
-// large for shared memory are re-read from global memory).  Three radix passes
-// (11 + 11 + 10 bits) find the exact k-th largest key T:
-//   - every warp counts its keys into a private shared-memory histogram
-//     (no cross-warp contention, no match/vote aggregation);
-//   - each CTA folds the 16 warp histograms and pushes its non-zero bins into
-//     every CTA's merged histogram with remote reductions
-//     (red.shared::cluster.add): fire-and-forget, no remote loads;
-//   - after one cluster barrier every CTA scans the merged histogram itself.
+// large for shared memory are re-read from global memory).  The exact k-th
+// largest key T is found by radix select over the bits that vary in the row:
+//   - the cluster-wide AND and OR of the keys fix every bit that is the same
+//     in all keys (integer-valued scores leave long runs of those), so only
+//     the span from the highest to the lowest varying bit is searched, in
+//     11-bit digits (one to three passes);
+//   - per pass, warps count their keys into shared-memory histograms shared
+//     by a warp pair (the first digit spans the varying bits, so the keys
+//     spread over many bins and the atomics rarely collide);
+//   - the 2,048 bins form 16 coarse groups of 128, each owned by one CTA of
+//     the cluster.  Each CTA folds its histograms, adds every non-zero bin
+//     into the owner's merged histogram and its 16 coarse sums into every CTA
+//     (red.shared::cluster.add: fire-and-forget, one remote add per bin);
+//   - after one cluster barrier each CTA finds the coarse group holding the
+//     k-th key from its own coarse sums, then reads that group's 128 fine bins
+//     from the owner (one 16-byte remote load per lane of one warp).
 // The kept set is {key > T} plus the first (k - #{key > T}) keys equal to T in
 // index order.  Each warp walks a contiguous run of its CTA's segment in
-// 32-key strips (the histogram passes walk the same order, so the last pass
-// yields each warp's counts above / equal to T); per-CTA counts are pushed to
-// every CTA; each kept index lands at position = number of kept tokens with a
-// lower index.  No sort, no global atomics, no global scratch.
+// 32-key strips; per-warp and per-CTA counts of keys above / equal to T give
+// every kept index its output position (the number of kept tokens with a
+// lower index).  No sort, no global atomics, no global scratch.
 #include <algorithm>
 
 #include "dsa_internal.h"
@@ -31,8 +38,19 @@ namespace {
 
 constexpr int kThreads = 512;
 constexpr int kWarps = kThreads / 32;
-constexpr int kBins = 2048;
+constexpr int kBins = 2048;                  // one 11-bit digit
+constexpr int kDigitBits = 11;
+constexpr int kCoarse = 16;                  // coarse groups of bins
+constexpr int kCw = kBins / kCoarse;         // bins per coarse group (128)
+constexpr int kPairs = kWarps / 2;           // histograms, one per warp pair
+constexpr int kPrivWords = kPairs * kBins;
+constexpr int kMaxPasses = 3;                // 32 bits in 11-bit digits
+constexpr int kMergedWords = kMaxPasses * (kBins + kCoarse);
 constexpr int kMaxC = 16;  // 16 needs the non-portable cluster size; 8 otherwise
+// shared words before the key buffer: histograms, merged sets, warp AND/OR,
+// warp counts, broadcast slots, pushed CTA counts, this CTA's AND/OR (+pad)
+constexpr int kFixedWords =
+    kPrivWords + kMergedWords + 2 * kWarps + 2 * kWarps + 4 + 2 * kMaxC + 4;
 
 struct TopkParams {
   const float *scores;
@@ -47,41 +65,29 @@ struct TopkParams {
   DevStatus *status;
 };
 
-// exclusive suffix sum (sum over threads with a higher id)
-__device__ __forceinline__ int block_exclusive_suffix(int v, int *warp_sums) {
-  const int lane = lane_id(), warp = warp_id();
-  int x = v;
-#pragma unroll
-  for (int o = 1; o < 32; o <<= 1) {
-    const int y = __shfl_down_sync(0xffffffffu, x, o);
-    if (lane + o < 32) x += y;
-  }
-  if (lane == 0) warp_sums[warp] = x;
-  __syncthreads();
-  if (warp == 0) {
-    int s = (lane < kWarps) ? warp_sums[lane] : 0;
-#pragma unroll
-    for (int o = 1; o < 32; o <<= 1) {
-      const int y = __shfl_down_sync(0xffffffffu, s, o);
-      if (lane + o < 32) s += y;
-    }
-    if (lane < kWarps) warp_sums[lane] = s;
-  }
-  __syncthreads();
-  const int after = (warp + 1 < kWarps) ? warp_sums[warp + 1] : 0;
-  __syncthreads();
-  return after + x - v;
+// the 11-bit digit of key u whose top bit is bit `top` (bits below bit 0 read as 0)
+__device__ __forceinline__ uint32_t digit_of(uint32_t u, int shift) {
+  return (shift >= 0 ? (u >> shift) : (u << -shift)) & (kBins - 1);
+}
+__device__ __forceinline__ uint32_t digit_mask(int shift) {
+  return shift >= 0 ? (static_cast<uint32_t>(kBins - 1) << shift)
+                    : (static_cast<uint32_t>(kBins - 1) >> -shift);
+}
+__device__ __forceinline__ uint32_t digit_bits(uint32_t d, int shift) {
+  return shift >= 0 ? (d << shift) : (d >> -shift);
 }
 
 __global__ void __launch_bounds__(kThreads, 1) topk_kernel(const TopkParams p) {
   extern __shared__ __align__(16) uint32_t sm[];
-  uint32_t *priv = sm;                                         // [kWarps][kBins]
-  uint32_t *merged = priv + kWarps * kBins;                    // [2][kBins]
-  int *warp_sums = reinterpret_cast<int *>(merged + 2 * kBins);  // [2 * kWarps]
-  int *bcast = warp_sums + 2 * kWarps;                         // [4]
-  uint32_t *cnt_all = reinterpret_cast<uint32_t *>(bcast + 4);   // [kMaxC][2] pushed counts
-  uint64_t *bar = reinterpret_cast<uint64_t *>(cnt_all + 2 * kMaxC);
-  uint32_t *keys = reinterpret_cast<uint32_t *>(bar + 2);      // [seg_cap], 16-byte aligned
+  uint32_t *priv = sm;                                       // [kPairs][kBins]
+  uint32_t *merged = priv + kPrivWords;                      // [kMaxPasses][kBins + kCoarse]
+  uint32_t *wandor = merged + kMergedWords;                  // [2][kWarps] warp AND / OR
+  int *wcnt = reinterpret_cast<int *>(wandor + 2 * kWarps);  // [2][kWarps] warp counts
+  int *bcast = wcnt + 2 * kWarps;                            // [4]
+  uint32_t *cnt_all = reinterpret_cast<uint32_t *>(bcast + 4);  // [kMaxC][2] pushed counts
+  uint32_t *andor = cnt_all + 2 * kMaxC;                     // [2] this CTA's AND / OR, [2] pad
+  uint64_t *bar = reinterpret_cast<uint64_t *>(andor + 4);
+  uint32_t *keys = reinterpret_cast<uint32_t *>(bar + 2);    // [seg_cap], 16-byte aligned
 
   const int tid = threadIdx.x, warp = warp_id(), lane = lane_id();
   const uint32_t C = cluster_nctarank();
@@ -112,11 +118,14 @@ __global__ void __launch_bounds__(kThreads, 1) topk_kernel(const TopkParams p) {
   const int cnt = max(0, min(n, lo + seg) - lo);
   const bool cached = seg <= p.seg_cap;
 
-  // zero the histograms; merged[0] must be zero before any peer pushes into it
+  // zero the histograms; the merged ones must be zero before any peer adds into them
   {
     uint4 *z = reinterpret_cast<uint4 *>(priv);
-    for (int i = tid; i < (kWarps + 2) * kBins / 4; i += kThreads) z[i] = make_uint4(0, 0, 0, 0);
+    for (int i = tid; i < (kPrivWords + kMergedWords) / 4; i += kThreads)
+      z[i] = make_uint4(0, 0, 0, 0);
   }
+  // keys into shared memory; AND / OR of this CTA's keys
+  uint32_t k_and = 0xFFFFFFFFu, k_or = 0u;
   if (cached && cnt > 0) {
     const float *src = srow + lo;
     int done = 0;
@@ -132,98 +141,194 @@ __global__ void __launch_bounds__(kThreads, 1) topk_kernel(const TopkParams p) {
         }
       }
       __syncthreads();
-      for (int i = tid; i < done; i += kThreads) keys[i] = score_key(__uint_as_float(keys[i]));
+      for (int i = tid; i < done; i += kThreads) {
+        const uint32_t u = score_key(__uint_as_float(keys[i]));
+        keys[i] = u;
+        k_and &= u;
+        k_or |= u;
+      }
     }
-    for (int i = done + tid; i < cnt; i += kThreads) keys[i] = score_key(__ldg(src + i));
+    for (int i = done + tid; i < cnt; i += kThreads) {
+      const uint32_t u = score_key(__ldg(src + i));
+      keys[i] = u;
+      k_and &= u;
+      k_or |= u;
+    }
+  } else {
+    for (int i = tid; i < cnt; i += kThreads) {
+      const uint32_t u = score_key(srow[lo + i]);
+      k_and &= u;
+      k_or |= u;
+    }
   }
-  cluster_sync();  // histograms zeroed everywhere, keys in place
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) {
+    k_and &= __shfl_xor_sync(0xffffffffu, k_and, o);
+    k_or |= __shfl_xor_sync(0xffffffffu, k_or, o);
+  }
+  if (lane == 0) { wandor[warp] = k_and; wandor[kWarps + warp] = k_or; }
+  __syncthreads();
+  if (warp == 0) {
+    uint32_t a = (lane < kWarps) ? wandor[lane] : 0xFFFFFFFFu;
+    uint32_t o = (lane < kWarps) ? wandor[kWarps + lane] : 0u;
+#pragma unroll
+    for (int s = 16; s > 0; s >>= 1) {
+      a &= __shfl_xor_sync(0xffffffffu, a, s);
+      o |= __shfl_xor_sync(0xffffffffu, o, s);
+    }
+    if (lane == 0) { andor[0] = a; andor[1] = o; }
+  }
+  cluster_sync();  // histograms zeroed everywhere, keys in place, AND / OR published
   auto key_at = [&](int i) -> uint32_t { return cached ? keys[i] : score_key(srow[lo + i]); };
-
-  uint32_t prefix = 0, pmask = 0;
+  if (warp == 0) {
+    // the row's AND / OR from every CTA of the cluster
+    uint32_t a = 0xFFFFFFFFu, o = 0u;
+    if (static_cast<uint32_t>(lane) < C) {
+      if (static_cast<uint32_t>(lane) == c) {
+        a = andor[0];
+        o = andor[1];
+      } else {
+        a = ld_dsmem_u32(map_to_rank(smem_u32(&andor[0]), lane));
+        o = ld_dsmem_u32(map_to_rank(smem_u32(&andor[1]), lane));
+      }
+    }
+#pragma unroll
+    for (int s = 16; s > 0; s >>= 1) {
+      a &= __shfl_xor_sync(0xffffffffu, a, s);
+      o |= __shfl_xor_sync(0xffffffffu, o, s);
+    }
+    if (lane == 0) { bcast[2] = static_cast<int>(a); bcast[3] = static_cast<int>(o); }
+  }
+  __syncthreads();
+  const uint32_t g_and = static_cast<uint32_t>(bcast[2]);
+  const uint32_t vary = g_and ^ static_cast<uint32_t>(bcast[3]);
+  // bits that never vary are part of T already
+  uint32_t pmask = ~vary, prefix = g_and & ~vary;
+  const int hb = vary ? 31 - __clz(vary) : -1;
+  const int lb = vary ? __ffs(vary) - 1 : 0;
+  const int npass = vary ? (hb - lb + kDigitBits) / kDigitBits : 0;
   int krem = k;
-  uint32_t *mine = priv + warp * kBins;
+
   // contiguous run of this CTA's segment owned by warp w, in 32-key strips:
   // index order is (CTA, warp, strip, lane)
   const uint32_t lt_mask = (1u << lane) - 1u;
   const int run = ((cnt + kWarps * 32 - 1) / (kWarps * 32)) * 32;
   const int w_lo = min(cnt, warp * run), w_hi = min(cnt, w_lo + run);
-  int above_w = 0;  // keys of this lane above the 22-bit prefix (last pass)
+  uint32_t *mine = priv + (warp >> 1) * kBins;
 #pragma unroll 1
-  for (int pass = 0; pass < 3; ++pass) {
-    const int shift = (pass == 0) ? 21 : (pass == 1 ? 10 : 0);
-    const uint32_t bmask = (pass < 2) ? 0x7FFu : 0x3FFu;
-    uint32_t *mg = merged + (pass & 1) * kBins;
-    // warp-private counts of the keys that still match the prefix; warp w
-    // walks its contiguous run, so in the last pass its histogram (plus the
-    // keys above the prefix) gives the warp's counts above / equal to T
-    for (int base = w_lo; base < w_hi; base += 32) {
-      const int i = base + lane;
-      if (i < w_hi) {
-        const uint32_t u = key_at(i);
-        const uint32_t hi = u & pmask;
-        if (hi == prefix) atomicAdd(&mine[(u >> shift) & bmask], 1u);
-        else if (pass == 2 && hi > prefix) ++above_w;
+  for (int pass = 0; pass < npass; ++pass) {
+    const int shift = hb - kDigitBits * pass - (kDigitBits - 1);  // may be negative
+    uint32_t *mfine = merged + pass * (kBins + kCoarse);
+    uint32_t *mcoarse = mfine + kBins;
+    // histogram of the keys that match the prefix, four strips in flight
+    for (int base = w_lo; base < w_hi; base += 128) {
+      uint32_t bins[4];
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        const int i = base + 32 * j + lane;
+        uint32_t b = 0xFFFFFFFFu;  // no bin: past the run, or outside the prefix
+        if (i < w_hi) {
+          const uint32_t u = key_at(i);
+          if ((u & pmask) == prefix) b = digit_of(u, shift);
+        }
+        bins[j] = b;
       }
+#pragma unroll
+      for (int j = 0; j < 4; ++j)
+        if (bins[j] != 0xFFFFFFFFu) atomicAdd(&mine[bins[j]], 1u);
     }
     __syncthreads();
-    // fold the warp histograms (thread t owns bins 4t .. 4t+3, clearing them
-    // for the next pass) and push non-zero bins into every CTA's merged one
+    // fold: thread t owns bins 4t .. 4t+3, clearing the pair histograms for
+    // the next pass; each non-zero bin goes to its coarse group's owner, the
+    // coarse sums (one group per warp) to every CTA
     {
       uint32_t v[4] = {0u, 0u, 0u, 0u};
 #pragma unroll
-      for (int w = 0; w < kWarps; ++w) {
-        uint4 *ph = reinterpret_cast<uint4 *>(priv + w * kBins + 4 * tid);
+      for (int h = 0; h < kPairs; ++h) {
+        uint4 *ph = reinterpret_cast<uint4 *>(priv + h * kBins + 4 * tid);
         const uint4 x = *ph;
         v[0] += x.x; v[1] += x.y; v[2] += x.z; v[3] += x.w;
-        if (pass < 2) *ph = make_uint4(0, 0, 0, 0);  // the last pass's stay for the counts
+        *ph = make_uint4(0, 0, 0, 0);
       }
+      const uint32_t owner = static_cast<uint32_t>(warp) % C;  // group = warp (kCw / 4 = 32)
 #pragma unroll
-      for (int q = 0; q < 4; ++q) {
-        if (v[q] == 0u) continue;
-        const uint32_t addr = smem_u32(&mg[4 * tid + q]);
-        for (uint32_t r = 0; r < C; ++r) red_dsmem_add_u32(map_to_rank(addr, r), v[q]);
+      for (int q = 0; q < 4; ++q)
+        if (v[q] != 0u) red_dsmem_add_u32(map_to_rank(smem_u32(&mfine[4 * tid + q]), owner), v[q]);
+      uint32_t cs = v[0] + v[1] + v[2] + v[3];
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) cs += __shfl_xor_sync(0xffffffffu, cs, o);
+      if (lane == 0 && cs != 0u) {
+        const uint32_t addr = smem_u32(&mcoarse[warp]);
+        for (uint32_t r = 0; r < C; ++r) red_dsmem_add_u32(map_to_rank(addr, r), cs);
       }
-      // the other buffer is next pass's target: clear it before the barrier
-      // (its last reader, the scan of the previous pass, is behind us)
-      uint32_t *nx = merged + ((pass + 1) & 1) * kBins;
-      *reinterpret_cast<uint4 *>(&nx[4 * tid]) = make_uint4(0, 0, 0, 0);
     }
-    cluster_sync();  // every CTA's counts are in every merged histogram
-    uint32_t gh[4];
-    {
-      const uint4 x = *reinterpret_cast<const uint4 *>(&mg[4 * tid]);
-      gh[0] = x.x; gh[1] = x.y; gh[2] = x.z; gh[3] = x.w;
-    }
-    int above = block_exclusive_suffix(static_cast<int>(gh[0] + gh[1] + gh[2] + gh[3]), warp_sums);
-    // the bin where the running count from the top reaches krem
+    cluster_sync();  // every CTA's counts are in the owners' and everyone's coarse sums
+    if (warp == 0) {
+      // coarse group holding the krem-th key from the top
+      const uint32_t cc = (lane < kCoarse) ? mcoarse[lane] : 0u;
+      int after = static_cast<int>(cc);  // inclusive suffix sum over lanes >= this one
 #pragma unroll
-    for (int q = 3; q >= 0; --q) {
-      const int h = static_cast<int>(gh[q]);
-      if (above < krem && krem <= above + h) { bcast[0] = 4 * tid + q; bcast[1] = krem - above; }
-      above += h;
+      for (int o = 1; o < 32; o <<= 1) {
+        const int y = __shfl_down_sync(0xffffffffu, after, o);
+        if (lane + o < 32) after += y;
+      }
+      after -= static_cast<int>(cc);  // keys in higher groups
+      const bool hit = lane < kCoarse && after < krem && krem <= after + static_cast<int>(cc);
+      const uint32_t hm = __ballot_sync(0xffffffffu, hit);
+      const int gsel = hm ? __ffs(hm) - 1 : 0;  // exactly one group qualifies
+      const int k1 = krem - __shfl_sync(0xffffffffu, after, gsel);
+      // its 128 fine bins, four per lane, from the owner
+      const uint32_t owner = static_cast<uint32_t>(gsel) % C;
+      const uint32_t *fsrc = &mfine[gsel * kCw + 4 * lane];
+      const uint4 f = (owner == c) ? *reinterpret_cast<const uint4 *>(fsrc)
+                                   : ld_dsmem_v4(map_to_rank(smem_u32(fsrc), owner));
+      const int tot = static_cast<int>(f.x + f.y + f.z + f.w);
+      int above = tot;  // inclusive suffix sum, then keys in higher lanes' bins
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        const int y = __shfl_down_sync(0xffffffffu, above, o);
+        if (lane + o < 32) above += y;
+      }
+      above -= tot;
+      const int fv[4] = {static_cast<int>(f.x), static_cast<int>(f.y), static_cast<int>(f.z),
+                         static_cast<int>(f.w)};
+#pragma unroll
+      for (int q = 3; q >= 0; --q) {
+        if (above < k1 && k1 <= above + fv[q]) {
+          bcast[0] = gsel * kCw + 4 * lane + q;
+          bcast[1] = k1 - above;
+        }
+        above += fv[q];
+      }
     }
     __syncthreads();
     const uint32_t sel = static_cast<uint32_t>(bcast[0]);
     krem = bcast[1];
-    prefix |= sel << shift;
-    pmask |= bmask << shift;
+    prefix |= digit_bits(sel, shift);
+    pmask |= digit_mask(shift);
     __syncthreads();  // bcast is rewritten by the next pass
   }
-  const uint32_t T = prefix;   // the k-th largest key
-  const int need_eq = krem;    // how many keys equal to T are kept
+  const uint32_t T = prefix;  // the k-th largest key (every bit is fixed now)
+  const int need_eq = krem;   // how many keys equal to T are kept
 
-  // Ordered compaction.  Per-warp counts of keys above / equal to T: keys
-  // above the 22-bit prefix, plus the last pass's warp histogram above /
-  // at T's low 10 bits.
-  const uint32_t b3 = T & 0x3FFu;
-  int gt_w = above_w, eq_w = 0;
-  for (uint32_t bin = b3 + 1 + lane; bin < 1024u; bin += 32) gt_w += static_cast<int>(mine[bin]);
+  // Ordered compaction: per-warp counts of keys above / equal to T, their
+  // prefixes over warps and CTAs, then ballots place every kept key.
+  {
+    int gt = 0, eq = 0;
+    for (int i = w_lo + lane; i < w_hi; i += 32) {
+      const uint32_t u = key_at(i);
+      gt += u > T;
+      eq += u == T;
+    }
 #pragma unroll
-  for (int o = 16; o > 0; o >>= 1) gt_w += __shfl_xor_sync(0xffffffffu, gt_w, o);
-  eq_w = static_cast<int>(mine[b3]);
-  int *wgt = warp_sums;  // [kWarps] per-warp counts, then exclusive prefixes
-  int *weq = warp_sums + kWarps;
-  if (lane == 0) { wgt[warp] = gt_w; weq[warp] = eq_w; }
+    for (int o = 16; o > 0; o >>= 1) {
+      gt += __shfl_xor_sync(0xffffffffu, gt, o);
+      eq += __shfl_xor_sync(0xffffffffu, eq, o);
+    }
+    if (lane == 0) { wcnt[warp] = gt; wcnt[kWarps + warp] = eq; }
+  }
+  int *wgt = wcnt;  // [kWarps] per-warp counts, then exclusive prefixes
+  int *weq = wcnt + kWarps;
   __syncthreads();
   if (tid == 0) {
     int g = 0, e = 0;
@@ -310,7 +415,7 @@ dsa_status_t launch_topk(const TopkLaunch &a, cudaStream_t stream) {
   C = std::min(C, std::max(1, device_sm_count() / std::max(1, a.n_q)));
   C = std::max(1, std::min(C, max_topk_cluster(max_smem)));
   const int seg = ((max_len + C - 1) / C + 3) & ~3;
-  const size_t fixed = 4 * ((kWarps + 2) * kBins + 2 * kWarps + 4 + 2 * kMaxC) + 16 + 64;
+  const size_t fixed = 4 * static_cast<size_t>(kFixedWords) + 16 + 64;
   const int cap_max = static_cast<int>((max_smem - fixed) / 4) & ~3;
   const int seg_cap = std::min(seg, cap_max);
   const size_t smem = fixed + 4 * static_cast<size_t>(seg_cap);
