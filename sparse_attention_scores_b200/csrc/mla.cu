@@ -13,10 +13,9 @@
 // of 128-key chunks of its selection (64-key chunks, the upper half of each
 // tile masked, when few rows would leave SMs idle).  The 64-head absorbed query stays in
 // shared memory for the whole range.  Per chunk:
-//   gather   TMA tile::gather4 loads (four 128-byte row pieces per
-//            instruction) of the selected latent rows straight into a
-//            128B-swizzled K-major tile, one mbarrier per 64-column atom, so
-//            the first MMAs start while the last atoms are in flight
+//   gather   16-byte cp.async pieces of the selected latent rows straight
+//            into a 128B-swizzled K-major tile (all threads, zero-fill for
+//            unused slots)
 //   S^T      tcgen05.mma, M = 128 keys, N = 64 heads, K = R + P, into TMEM
 //   softmax  warp w reads keys 32*(w%4).. and heads 32*(w/4).. of S^T; per-head
 //            max and sum over the 128 keys by a transposing butterfly of warp
@@ -45,7 +44,6 @@ constexpr int kChunk = 128;           // keys per chunk = MMA M
 constexpr int kHeads = 64;            // head columns of every tile = MMA N
 constexpr int kAtomL = kChunk * 128;  // bytes of one 64-column atom of the latent tile
 constexpr int kAtomQ = kHeads * 128;  // bytes of one 64-column atom of the query tile
-constexpr int kMaxAtoms = 9;          // R + P <= 576
 constexpr float kRescaleLog2 = 8.0f;
 constexpr float kLn2 = 0.69314718055994531f;
 
@@ -53,6 +51,7 @@ enum : int { kMergeNone = 0, kMergeGlobal = 1 };
 
 struct MlaParams {
   const uint16_t *q;
+  const uint16_t *latent;  // paged latent rows [num_pages * 64][W]
   const int32_t *idx;
   const int32_t *seq_lens;
   const int32_t *block_table;
@@ -85,18 +84,6 @@ __device__ __forceinline__ void tmem_st_32x32b_x32(uint32_t taddr, const uint32_
 }
 __device__ __forceinline__ void tmem_st_wait() {
   asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
-}
-
-// TMA gather of four rows (one 64-column atom piece of each) into consecutive
-// 128-byte rows of shared memory; the tensor map's box is one row high.
-__device__ __forceinline__ void tma_gather4(void *dst, const CUtensorMap *map, int x, int r0,
-                                            int r1, int r2, int r3, uint64_t *bar) {
-  asm volatile(
-      "cp.async.bulk.tensor.2d.shared::cluster.global.tile::gather4.mbarrier::complete_tx::bytes"
-      " [%0], [%1, {%2, %3, %4, %5, %6}], [%7];" ::"r"(smem_u32(dst)),
-      "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(r0), "r"(r1), "r"(r2), "r"(r3),
-      "r"(smem_u32(bar))
-      : "memory");
 }
 
 // Reduce 32 per-key values over the 32 keys (lanes) of a warp, for 32 heads at
@@ -142,7 +129,7 @@ __device__ __forceinline__ float butterfly32(Get v) {
 }
 
 __global__ void __launch_bounds__(kThreads, 1)
-    mla_kernel(const __grid_constant__ CUtensorMap tmL, const MlaParams p) {
+    mla_kernel(const MlaParams p) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                               ~static_cast<uintptr_t>(1023));
@@ -160,12 +147,11 @@ __global__ void __launch_bounds__(kThreads, 1)
   float *mrun = red + 4 * kHeads;
   float *lrun = mrun + kHeads;
   float *alpha = lrun + kHeads;
-  uint64_t *bar_atom = reinterpret_cast<uint64_t *>(alpha + kHeads);  // [kMaxAtoms]
-  uint64_t *bar_s = bar_atom + kMaxAtoms;
+  uint64_t *bar_s = reinterpret_cast<uint64_t *>(alpha + kHeads);
   uint64_t *bar_o = bar_s + 1;
   uint64_t *bar_drain = bar_o + 1;
   uint64_t *bar_stall = bar_drain + 1;
-  // [0] tmem base, [1] rescale flag, [2] failed, [3] fallback row
+  // [0] tmem base, [1] rescale flag, [2] failed
   uint32_t *misc = reinterpret_cast<uint32_t *>(bar_stall + 1);
 
   const int tid = threadIdx.x, warp = warp_id(), lane = lane_id();
@@ -182,7 +168,6 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint32_t tmem_cols = 32;
   while (tmem_cols < static_cast<uint32_t>(kHeads + nmb * kHeads)) tmem_cols <<= 1;
   if (tid == 0) {
-    for (int a = 0; a < kMaxAtoms; ++a) mbar_init(&bar_atom[a], 1);
     mbar_init(bar_s, 1);
     mbar_init(bar_o, 1);
     mbar_init(bar_drain, 1);
@@ -190,7 +175,6 @@ __global__ void __launch_bounds__(kThreads, 1)
     misc[1] = 0u;
     misc[2] = 0u;
     fence_barrier_init();
-    tma_prefetch_desc(&tmL);
   }
   if (tid < kHeads) { mrun[tid] = -INFINITY; lrun[tid] = 0.f; }
   if (warp == 0) { tmem_alloc(&misc[0], tmem_cols); tmem_relinquish(); }
@@ -223,7 +207,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   const uint32_t lane_off = static_cast<uint32_t>(q4 * 32) << 16;
   const uint32_t idesc_s = idesc_bf16_f32(kChunk, kHeads, 0, 0);
   const uint32_t idesc_pv = idesc_bf16_f32(kChunk, kHeads, 1, 1);
-  uint32_t g_phase = 0, s_phase = 0, o_phase = 0;
+  uint32_t s_phase = 0, o_phase = 0;
   bool have_o = false;
   bool failed = false;
 
@@ -252,54 +236,47 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       rowi[tid] = phys;
       valid = phys >= 0;
-      if (valid) misc[3] = static_cast<uint32_t>(phys);  // any valid row stands in for unused slots
       if (tid == 0) misc[1] = 0u;
     }
     if (__syncthreads_count(valid) == 0) continue;  // nothing to attend in this chunk
-    // gather: lane 0 of warp w loads atoms w, w + 8; unused slots repeat a
-    // valid row (their probabilities are zero)
-    if (lane == 0) {
-      const int fb = static_cast<int>(misc[3]);
-      for (int a = warp; a < nQ; a += kThreads / 32) {
-        // rows kc .. 127 of a 64-key chunk are never gathered: their keys are
-        // masked and the PV product stops at key kc
-        mbar_arrive_expect_tx(&bar_atom[a], static_cast<uint32_t>(kc) * 128u);
-        uint8_t *dst = Ls + a * kAtomL;
-#pragma unroll 4
-        for (int g4 = 0; g4 < kc / 4; ++g4) {
-          int r[4];
-#pragma unroll
-          for (int k = 0; k < 4; ++k) {
-            const int v = rowi[4 * g4 + k];
-            r[k] = v >= 0 ? v : fb;
-          }
-          tma_gather4(dst + g4 * 512, &tmL, a * 64, r[0], r[1], r[2], r[3], &bar_atom[a]);
-        }
+    // gather: the selected latent rows into the 128B-swizzled K-major tile,
+    // 16 bytes per cp.async, consecutive threads on consecutive pieces of a
+    // row; unused rows are zero-filled.  (TMA row gathers were measured to be
+    // issue-bound at 15-19 GB/s per SM, whether the rows were in L2 or not.)
+    // Rows kc .. 127 of a 64-key chunk are never written: their keys are
+    // masked and the PV product stops at key kc.
+    {
+      const uint32_t ls = smem_u32(Ls);
+      const int npieces = kc * cpr;
+      int r = tid / cpr, cc = tid - (tid / cpr) * cpr;
+      for (int pc = tid; pc < npieces; pc += kThreads) {
+        const int phys = rowi[r];
+        const uint16_t *src = phys >= 0 ? p.latent + static_cast<int64_t>(phys) * W + cc * 8 : p.latent;
+        cp_async_16(ls + (cc >> 3) * kAtomL + r * 128 + (((cc & 7) ^ (r & 7)) << 4), src,
+                    phys >= 0 ? 16u : 0u);
+        r += kThreads / cpr;  // the piece kThreads further on (cpr pieces per row)
+        cc += kThreads % cpr;
+        if (cc >= cpr) { cc -= cpr; ++r; }
       }
+      cp_async_commit();
     }
-    if (ch == c_begin) cp_async_wait_all();  // the query tile
+    cp_async_wait_all();  // this thread's pieces (and, first time round, the query tile)
     fence_proxy_async_smem();
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
-    // S^T = L . Q^T  (M = 128 keys, N = 64 heads, K = W), atom by atom as they land
+    // S^T = L . Q^T  (M = 128 keys, N = 64 heads, K = W)
     if (tid == 0) {
       const uint32_t ls = smem_u32(Ls), qs = smem_u32(Qs);
-      bool ok = true;
-      for (int a = 0; a < nQ && ok; ++a) {
-        if (!mbar_wait(&bar_atom[a], g_phase, p.wait_ns)) { ok = false; break; }
-        tc_fence_after();
+      for (int a = 0; a < nQ; ++a)
         for (int kk = 0; kk < 4; ++kk) {
           if (a * 64 + kk * 16 >= W) break;
           mma_bf16(misc[0], smem_desc(ls + a * kAtomL + kk * 32, 16, 1024, kLayoutSW128),
                    smem_desc(qs + a * kAtomQ + kk * 32, 16, 1024, kLayoutSW128), idesc_s,
                    (a | kk) != 0 ? 1u : 0u);
         }
-      }
-      if (!ok) misc[2] = 1u;
       mma_commit(bar_s);
     }
-    g_phase ^= 1u;
     if (!mbar_wait(bar_s, s_phase, p.wait_ns)) misc[2] = 1u;
     s_phase ^= 1u;
     tc_fence_after();
@@ -424,8 +401,6 @@ __global__ void __launch_bounds__(kThreads, 1)
       report(p.status, kErrTimeout, (kKernMla << 24) | 1u);
       mma_commit(bar_drain);  // fires once every MMA issued above has completed
       mbar_wait(bar_drain, 0u, kDrainLimitNs);
-      // let gathers still in flight land before the shared memory is reused
-      for (int a = 0; a < nQ; ++a) mbar_wait(&bar_atom[a], g_phase ^ 1u, kDrainLimitNs);
     }
     if (tid < kHeads) { mrun[tid] = -INFINITY; lrun[tid] = 0.f; }
     have_o = false;
@@ -575,7 +550,7 @@ size_t mla_smem_bytes(int R, int P) {
   const bool p_overlays = nL > 2 * nmb;
   return 1024 + static_cast<size_t>(nL) * kAtomL + (p_overlays ? 0 : kAtomL) +
          static_cast<size_t>(nQ) * kAtomQ + 4 * kChunk + 4 * (7 * kHeads) +
-         8 * (kMaxAtoms + 4) + 16;
+         8 * 4 + 16;
 }
 
 struct SplitPlan {
@@ -623,11 +598,9 @@ dsa_status_t launch_mla(const MlaLaunch &a, cudaStream_t stream) {
     attr_set = true;
   }
   const SplitPlan sp = plan_splits(a.n_q, a.topk);
-  CUtensorMap tmL;
-  if (!make_map_2d(&tmL, a.latent, W, static_cast<uint64_t>(a.num_pages) * kPageSize, 64, 1, 128))
-    return DSA_ERR_CUDA;
   MlaParams p;
   p.q = a.q;
+  p.latent = a.latent;
   p.idx = a.idx;
   p.seq_lens = a.seq_lens;
   p.block_table = a.block_table;
@@ -662,7 +635,7 @@ dsa_status_t launch_mla(const MlaLaunch &a, cudaStream_t stream) {
   p.debug_stall = debug_stall() == kKernMla ? 1 : 0;
   p.early_q = a.early_q;
   p.status = a.status;
-  if (launch_pdl(mla_kernel, dim3(sp.nsplit, a.n_q), dim3(kThreads), smem, stream, 1, tmL, p) !=
+  if (launch_pdl(mla_kernel, dim3(sp.nsplit, a.n_q), dim3(kThreads), smem, stream, 1, p) !=
       cudaSuccess)
     return DSA_ERR_CUDA;
   if (sp.merge == kMergeGlobal) {
