@@ -298,6 +298,40 @@ def measure(case, torch, steps, warmup, flush_buf, peaks):
     return res
 
 
+# DRAM traffic per launch (dram__bytes_read.sum + dram__bytes_write.sum) of
+# each stage's kernels from one ncu capture (profiles/<kernel>_<workload>.md),
+# with a digest of the sources the capture was taken on: the bench reports
+# the figure only while those sources are unchanged.
+TRAFFIC_SOURCES = {"indexer": ["indexer.cu"], "topk": ["topk.cu"], "mla": ["mla.cu"]}
+TRAFFIC_COMMON = ["dsa_common.cuh", "dsa_internal.h"]
+TRAFFIC = {
+    # (stage, workload): (bytes per launch, digest of the stage's sources)
+    ("indexer", "glm5_decode_8k"): (2164480, "ee2f6041a779d556"),
+    ("indexer", "glm5_decode_4x128k"): (134359040 + 4805120, "ee2f6041a779d556"),
+    ("topk", "glm5_decode_8k"): (70912, "5efcabd2a44e59af"),
+    ("topk", "glm5_decode_4x128k"): (2135808, "5efcabd2a44e59af"),
+    # mla_kernel + combine_kernel (the merge reads the split partials)
+    ("mla", "glm5_decode_8k"): (2513920 + 4226304, "a69f3b783441a492"),
+    ("mla", "glm5_decode_4x128k"): (9870592 + 16858624, "a69f3b783441a492"),
+}
+
+
+def source_digest(stage):
+    import hashlib
+    h = hashlib.sha256()
+    for f in TRAFFIC_SOURCES[stage] + TRAFFIC_COMMON:
+        with open(os.path.join(ROOT, "sparse_attention_scores_b200", "csrc", f), "rb") as fh:
+            h.update(fh.read())
+    return h.hexdigest()[:16]
+
+
+def traffic_of(stage, workload):
+    t = TRAFFIC.get((stage, workload))
+    if t is None or t[1] != source_digest(stage):
+        return None
+    return t[0]
+
+
 STAGE_KERNELS = {"indexer": "indexer_kernel (tcgen05 + TMA)",
                  "topk": "topk_kernel (cluster radix select)",
                  "mla": "mla_kernel + combine_kernel (tcgen05 + TMA gather4, split merge)"}
@@ -313,14 +347,14 @@ def roofline_of(res, wl, peaks):
         achieved = alg["flops_mla"] / (us * 1e-6) / 1e12
         return {"kernel": STAGE_KERNELS[stage], "stage": stage, "bound": "tensor",
                 "achieved": achieved, "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
-                "frac": achieved / peaks["bf16_tflops"], "traffic": None,
+                "frac": achieved / peaks["bf16_tflops"], "traffic": traffic_of(stage, wl.name),
                 "peak_source": peaks["source"], "alg_flops_per_launch": alg["flops_mla"],
                 "launch_us": us}
     b = res["stage_alg_bytes"][stage]
     achieved = b / (us * 1e-6) / 1e9
     return {"kernel": STAGE_KERNELS[stage], "stage": stage, "bound": "hbm",
             "achieved": achieved, "peak": peaks["hbm_gbs"], "unit": "GB/s",
-            "frac": achieved / peaks["hbm_gbs"], "traffic": None,
+            "frac": achieved / peaks["hbm_gbs"], "traffic": traffic_of(stage, wl.name),
             "peak_source": peaks["source"], "alg_bytes_per_launch": b, "launch_us": us}
 
 
