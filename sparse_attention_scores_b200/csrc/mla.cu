@@ -196,7 +196,22 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     cp_async_commit();
   }
-  if (p.early_q) griddep_wait();
+  // In the fused forward the block table predates this step too: stage the
+  // row's page ids in the (still unused) latent tile, so the first chunk
+  // resolves its rows without a second dependent global load.
+  int staged_pages = 0;
+  const int *tbl = reinterpret_cast<const int *>(Ls);
+  if (p.early_q) {
+    const int len = p.causal ? p.q_pos0 + row + 1 : p.seq_lens[b];
+    const int npg = min(p.max_pages, (max(len, 0) + kPageSize - 1) / kPageSize);
+    if (npg <= (nL * kAtomL) / 4) {
+      staged_pages = npg;
+      int *t = reinterpret_cast<int *>(Ls);
+      for (int i = tid; i < npg; i += kThreads)
+        t[i] = p.block_table[static_cast<int64_t>(b) * p.max_pages + i];
+    }
+    griddep_wait();
+  }
   griddep_launch_dependents();
   const int limit = min(p.causal ? p.q_pos0 + row + 1 : p.seq_lens[b], p.max_pages * kPageSize);
   tc_fence_before();
@@ -227,7 +242,9 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (pos >= limit) {
           report(p.status, kErrBadIndex, (kKernMla << 24) | (slot & 0xFFFF));
         } else {
-          const int page = p.block_table[static_cast<int64_t>(b) * p.max_pages + pos / kPageSize];
+          const int page = (ch == c_begin && pos / kPageSize < staged_pages)
+                               ? tbl[pos / kPageSize]
+                               : p.block_table[static_cast<int64_t>(b) * p.max_pages + pos / kPageSize];
           if (page < 0 || page >= p.num_pages)
             report(p.status, kErrBadPage, (kKernMla << 24) | (slot & 0xFFFF));
           else
@@ -240,24 +257,22 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     if (__syncthreads_count(valid) == 0) continue;  // nothing to attend in this chunk
     // gather: the selected latent rows into the 128B-swizzled K-major tile,
-    // 16 bytes per cp.async, consecutive threads on consecutive pieces of a
-    // row; unused rows are zero-filled.  (TMA row gathers were measured to be
-    // issue-bound at 15-19 GB/s per SM, whether the rows were in L2 or not.)
-    // Rows kc .. 127 of a 64-key chunk are never written: their keys are
-    // masked and the PV product stops at key kc.
+    // 16 bytes per cp.async, eight threads per 128-byte atom row; unused rows
+    // are zero-filled.  (TMA row gathers were measured to be issue-bound at
+    // 15-19 GB/s per SM, whether the rows were in L2 or not.)  Rows kc .. 127
+    // of a 64-key chunk are never written: their keys are masked and the PV
+    // product stops at key kc.
     {
       const uint32_t ls = smem_u32(Ls);
-      const int npieces = kc * cpr;
-      int r = tid / cpr, cc = tid - (tid / cpr) * cpr;
-      for (int pc = tid; pc < npieces; pc += kThreads) {
-        const int phys = rowi[r];
-        const uint16_t *src = phys >= 0 ? p.latent + static_cast<int64_t>(phys) * W + cc * 8 : p.latent;
-        cp_async_16(ls + (cc >> 3) * kAtomL + r * 128 + (((cc & 7) ^ (r & 7)) << 4), src,
-                    phys >= 0 ? 16u : 0u);
-        r += kThreads / cpr;  // the piece kThreads further on (cpr pieces per row)
-        cc += kThreads % cpr;
-        if (cc >= cpr) { cc -= cpr; ++r; }
-      }
+      const int per_atom = kc * 8;  // pieces of one atom: 8 per row
+      for (int a = 0; a < nQ; ++a)
+        for (int pc = tid; pc < per_atom; pc += kThreads) {
+          const int r = pc >> 3, j = pc & 7, cc = a * 8 + j;
+          const int phys = rowi[r];
+          const bool ok = phys >= 0 && cc < cpr;
+          const uint16_t *src = ok ? p.latent + static_cast<int64_t>(phys) * W + cc * 8 : p.latent;
+          cp_async_16(ls + a * kAtomL + r * 128 + ((j ^ (r & 7)) << 4), src, ok ? 16u : 0u);
+        }
       cp_async_commit();
     }
     cp_async_wait_all();  // this thread's pieces (and, first time round, the query tile)

@@ -10,8 +10,9 @@
 // copy and turns it into order-preserving 32-bit keys in place (segments too
 // large for shared memory are re-read from global memory).  The exact k-th
 // largest key T is found by radix select over the bits that vary in the row:
-//   - the cluster-wide AND and OR of the keys fix every bit that is the same
-//     in all keys (integer-valued scores leave long runs of those), so only
+//   - the cluster-wide AND and OR of the keys (every CTA adds its own into all
+//     CTAs' slots between the two halves of the first cluster barrier) fix
+//     every bit that is the same in all keys (integer-valued scores leave long runs of those), so only
 //     the span from the highest to the lowest varying bit is searched, in
 //     11-bit digits (one to three passes);
 //   - per pass, warps count their keys into shared-memory histograms shared
@@ -85,7 +86,7 @@ __global__ void __launch_bounds__(kThreads, 1) topk_kernel(const TopkParams p) {
   int *wcnt = reinterpret_cast<int *>(wandor + 2 * kWarps);  // [2][kWarps] warp counts
   int *bcast = wcnt + 2 * kWarps;                            // [4]
   uint32_t *cnt_all = reinterpret_cast<uint32_t *>(bcast + 4);  // [kMaxC][2] pushed counts
-  uint32_t *andor = cnt_all + 2 * kMaxC;                     // [2] this CTA's AND / OR, [2] pad
+  uint32_t *andor = cnt_all + 2 * kMaxC;  // [2] the row's ~AND / OR from every CTA, [2] pad
   uint64_t *bar = reinterpret_cast<uint64_t *>(andor + 4);
   uint32_t *keys = reinterpret_cast<uint32_t *>(bar + 2);    // [seg_cap], 16-byte aligned
 
@@ -118,12 +119,15 @@ __global__ void __launch_bounds__(kThreads, 1) topk_kernel(const TopkParams p) {
   const int cnt = max(0, min(n, lo + seg) - lo);
   const bool cached = seg <= p.seg_cap;
 
-  // zero the histograms; the merged ones must be zero before any peer adds into them
+  // zero the histograms and the AND / OR slots: the merged histograms and the
+  // slots must be zero before any peer adds into them (first cluster arrive)
   {
     uint4 *z = reinterpret_cast<uint4 *>(priv);
     for (int i = tid; i < (kPrivWords + kMergedWords) / 4; i += kThreads)
       z[i] = make_uint4(0, 0, 0, 0);
+    if (tid < 2) andor[tid] = 0u;
   }
+  cluster_arrive();
   // keys into shared memory; AND / OR of this CTA's keys
   uint32_t k_and = 0xFFFFFFFFu, k_or = 0u;
   if (cached && cnt > 0) {
@@ -168,6 +172,7 @@ __global__ void __launch_bounds__(kThreads, 1) topk_kernel(const TopkParams p) {
   }
   if (lane == 0) { wandor[warp] = k_and; wandor[kWarps + warp] = k_or; }
   __syncthreads();
+  cluster_wait();  // every CTA's slots are zero: add this CTA's AND / OR into all of them
   if (warp == 0) {
     uint32_t a = (lane < kWarps) ? wandor[lane] : 0xFFFFFFFFu;
     uint32_t o = (lane < kWarps) ? wandor[kWarps + lane] : 0u;
@@ -176,32 +181,16 @@ __global__ void __launch_bounds__(kThreads, 1) topk_kernel(const TopkParams p) {
       a &= __shfl_xor_sync(0xffffffffu, a, s);
       o |= __shfl_xor_sync(0xffffffffu, o, s);
     }
-    if (lane == 0) { andor[0] = a; andor[1] = o; }
-  }
-  cluster_sync();  // histograms zeroed everywhere, keys in place, AND / OR published
-  auto key_at = [&](int i) -> uint32_t { return cached ? keys[i] : score_key(srow[lo + i]); };
-  if (warp == 0) {
-    // the row's AND / OR from every CTA of the cluster
-    uint32_t a = 0xFFFFFFFFu, o = 0u;
+    // slot 0 collects the OR of the complements (the complement of the AND)
     if (static_cast<uint32_t>(lane) < C) {
-      if (static_cast<uint32_t>(lane) == c) {
-        a = andor[0];
-        o = andor[1];
-      } else {
-        a = ld_dsmem_u32(map_to_rank(smem_u32(&andor[0]), lane));
-        o = ld_dsmem_u32(map_to_rank(smem_u32(&andor[1]), lane));
-      }
+      red_dsmem_or_u32(map_to_rank(smem_u32(&andor[0]), lane), ~a);
+      red_dsmem_or_u32(map_to_rank(smem_u32(&andor[1]), lane), o);
     }
-#pragma unroll
-    for (int s = 16; s > 0; s >>= 1) {
-      a &= __shfl_xor_sync(0xffffffffu, a, s);
-      o |= __shfl_xor_sync(0xffffffffu, o, s);
-    }
-    if (lane == 0) { bcast[2] = static_cast<int>(a); bcast[3] = static_cast<int>(o); }
   }
-  __syncthreads();
-  const uint32_t g_and = static_cast<uint32_t>(bcast[2]);
-  const uint32_t vary = g_and ^ static_cast<uint32_t>(bcast[3]);
+  cluster_sync();  // histograms zeroed everywhere, keys in place, the row's AND / OR local
+  auto key_at = [&](int i) -> uint32_t { return cached ? keys[i] : score_key(srow[lo + i]); };
+  const uint32_t g_and = ~andor[0];
+  const uint32_t vary = g_and ^ andor[1];
   // bits that never vary are part of T already
   uint32_t pmask = ~vary, prefix = g_and & ~vary;
   const int hb = vary ? 31 - __clz(vary) : -1;
