@@ -85,7 +85,10 @@ def algorithmic(wl):
     b_topk = keys * 4 + wl.n_q * wl.topk * 4
     # sparse MLA + split merge: selected latent rows, q, idx in; out, lse out
     b_mla = b_lat + wl.n_q * (wl.H * wl.W * 2 + wl.topk * 4 + wl.H * wl.R * 4 + wl.H * 4)
+    # cache append: each new row read once and written once (key + latent)
+    b_append = 2 * wl.n_q * (wl.D_I * 2 + wl.W * 2)
     return {"bytes": b_keys + b_lat + b_small, "bytes_keys": b_keys, "bytes_latent": b_lat,
+            "bytes_append": b_append,
             "flops": flops_idx + flops_mla, "flops_indexer": flops_idx, "flops_mla": flops_mla,
             "bytes_indexer": b_indexer, "bytes_topk": b_topk, "bytes_mla": b_mla,
             "keys": keys, "selected": sel}
@@ -202,6 +205,14 @@ class Case:
         self.ws = dsa.workspace(dsa.OP_ATTENTION_FORWARD, self.dims, self.cache)
         ld = max(4, (max(row_lengths(wl)) + 3) // 4 * 4)
         self.scores = torch.empty((wl.n_q, ld), dtype=torch.float32, device=dev)
+        # the current tokens' own rows, to time the cache append without
+        # changing the caches (appending them again is idempotent)
+        lens = np.asarray(row_lengths(wl), dtype=np.int64)
+        seqs = np.zeros_like(lens) if wl.mode == "prefill" else np.arange(wl.n_q)
+        pos = lens - 1
+        phys = inp["block_table"][seqs, pos // 64].astype(np.int64) * 64 + pos % 64
+        self.k_new = bf(inp["k_pages"].reshape(-1, wl.D_I)[phys])
+        self.l_new = bf(inp["latent_pages"].reshape(-1, wl.W)[phys])
         self.dsa = dsa
         self.torch = torch
 
@@ -214,6 +225,11 @@ class Case:
         t = self.t
         self.dsa.dsa_indexer_scores(t["q_idx"], t["w"], t["k_pages"], self.cache, self.dims,
                                     self.scores, self.ws)
+
+    def append(self):
+        t = self.t
+        self.dsa.dsa_cache_append(self.k_new, self.l_new, t["k_pages"], t["latent_pages"],
+                                  self.cache, self.dims, self.ws)
 
     def topk(self):
         # the scores of the last indexer() call; decode rows end at their
@@ -274,6 +290,8 @@ def measure(case, torch, steps, warmup, flush_buf, peaks):
     ms_idx, _ = timed_events(torch, case.indexer, steps, warmup, flush_buf)
     ms_topk, _ = timed_events(torch, case.topk, steps, warmup, flush_buf)
     ms_mla, _ = timed_events(torch, case.mla, steps, warmup, flush_buf)
+    # the cache append in front of the step (a separate entry point, not in the step)
+    ms_app, _ = timed_events(torch, case.append, steps, warmup, flush_buf)
     st, info = case.dsa.workspace_check(case.ws)
     if st != 0:
         raise RuntimeError(f"device status {st} ({info:#x}) in the stage timings of {wl.name}")
@@ -294,6 +312,9 @@ def measure(case, torch, steps, warmup, flush_buf, peaks):
         "stage_us": {"indexer": ms_idx * 1e3, "topk": ms_topk * 1e3, "mla": ms_mla * 1e3},
         "stage_alg_bytes": {"indexer": alg["bytes_indexer"], "topk": alg["bytes_topk"],
                             "mla": alg["bytes_mla"]},
+        "append_us": ms_app * 1e3,
+        "append_alg_bytes": alg["bytes_append"],
+        "append_gbs": alg["bytes_append"] / (ms_app * 1e-3) / 1e9,
     }
     return res
 

@@ -113,7 +113,8 @@ typedef enum {
   DSA_OP_TOPK = 1,
   DSA_OP_SPARSE_MLA_DECODE = 2,
   DSA_OP_SPARSE_MLA_PREFILL = 3,
-  DSA_OP_ATTENTION_FORWARD = 4
+  DSA_OP_ATTENTION_FORWARD = 4,
+  DSA_OP_CACHE_APPEND = 5
 } dsa_op_t;
 
 /* Library version (major * 10000 + minor * 100 + patch). */
@@ -194,6 +195,28 @@ DSA_API dsa_status_t dsa_attention_forward(const uint16_t *q_idx, const float *w
                                    const dsa_dims_t *dims, int32_t *idx_out, float *out,
                                    float *lse, void *ws, size_t ws_bytes, dsa_stream_t stream);
 
+/* Cache append: write the new tokens' index keys and latent rows into the
+ * paged caches, the step in front of the indexer ("Self-contained GLM-5
+ * serving stack ...", file list: absorbed MLA decode over compressed
+ * request-local KV, which the engine grows by one compressed row per token).
+ *   k_idx_new    [n_q, D_I]    bf16 index key of each new token
+ *   latent_new   [n_q, R + P]  bf16 latent row ([c_kv | k_rope]) of each new token
+ *   k_idx_pages, latent_pages  the page pools, written in place
+ * Row r goes to the position the step gives its query: decode row b to
+ * position seq_lens[b] - 1 of sequence b (seq_lens already counts it);
+ * prefill row t (dims.causal = 1) to position q_pos0 + t of sequence 0.
+ * Position s of a sequence lives in page block_table[seq][s / 64], slot
+ * s % 64.  A page id outside [0, num_pages) or a position outside the block
+ * table skips that row and is reported as DSA_ERR_DEVICE_CHECK by the next
+ * dsa_workspace_check.  Distinct rows must target distinct slots.  Only
+ * dims.n_q, D_I, R, P, causal and q_pos0 are used.  Launched with
+ * programmatic dependent launch, so a following dsa_attention_forward on the
+ * same stream starts its prologue while the append finishes. */
+DSA_API dsa_status_t dsa_cache_append(const uint16_t *k_idx_new, const uint16_t *latent_new,
+                              uint16_t *k_idx_pages, uint16_t *latent_pages,
+                              const dsa_cache_t *cache, const dsa_dims_t *dims, void *ws,
+                              size_t ws_bytes, dsa_stream_t stream);
+
 /* Sparse MLA decode for callers that cannot allocate device memory.
  *
  * The pages have no counterpart of this entry point: it exists for callers
@@ -207,7 +230,8 @@ DSA_API dsa_status_t dsa_attention_forward(const uint16_t *q_idx, const float *w
  *
  *   Arguments as for dsa_sparse_mla_decode, without ws / ws_bytes.
  *   Returns DSA_ERR_WORKSPACE, before launching anything, when the partial
- *   results of this call (n_q * splits * 64 * R * 4 bytes; rows are split
+ *   results of this call (n_q * splits * 64 * R' * 4 bytes, R' = R rounded up
+ *   to a multiple of 128; rows are split
  *   when there are fewer rows than SMs) would not fit in the 32 MiB array:
  *   a batch of 32 at R = 512 and top-2,048 (16.8 MB) fits; 140 rows of
  *   top-65,536 (two splits each, 36.7 MB) are rejected.

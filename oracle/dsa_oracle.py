@@ -7,7 +7,8 @@ nothing from the product.  It shares no code, tables or constants with the CUDA
 kernels: inputs arrive as NumPy arrays (bf16 values as raw uint16 bits) and
 every step is written out in float64.
 
-What it computes (one query row):
+What it computes (one query row), after the new tokens' rows have been
+appended to the paged caches (cache_append):
 
 1. Indexer scores.  "GLM on an A100, in Vx", section "The model": a separate
    indexer scores every earlier token; section "How do we know it is right?":
@@ -75,6 +76,43 @@ def gather_paged_rows(pages: np.ndarray, block_table_row: np.ndarray,
     pos = np.asarray(positions, dtype=np.int64).reshape(-1)
     phys = np.asarray(block_table_row, dtype=np.int64)[pos // PAGE_SIZE]
     return pages[phys, pos % PAGE_SIZE]
+
+
+# --------------------------------------------------------------------------
+# the step in front of the indexer: appending the new tokens to the caches
+# --------------------------------------------------------------------------
+
+def append_positions(inp: dict) -> list:
+    """(sequence, position) that each new row of the step is written to.
+
+    Decode row b is the query at position seq_lens[b] - 1 of sequence b (its
+    own token is part of the context it scores); prefill row t sits at
+    position q_pos0 + t of sequence 0.
+    """
+    if inp.get("mode") == "prefill":
+        return [(0, int(inp["q_pos0"]) + t) for t in range(inp["q_idx"].shape[0])]
+    return [(b, int(n) - 1) for b, n in enumerate(inp["seq_lens"])]
+
+
+def cache_append(k_pages, latent_pages, block_table, positions, k_new, latent_new):
+    """The page pools after writing row i of k_new / latent_new at (seq, pos) =
+    positions[i].  "Self-contained GLM-5 serving stack ...", file list: the
+    decode runs over compressed request-local KV, one compressed row per token,
+    plus the indexer's key for that token.  Returns new arrays (the inputs are
+    not modified); raises on a position outside the block table or an invalid
+    page id.
+    """
+    k_out = np.array(k_pages, copy=True)
+    l_out = np.array(latent_pages, copy=True)
+    for i, (seq, pos) in enumerate(positions):
+        if pos < 0 or pos // PAGE_SIZE >= block_table.shape[1]:
+            raise ValueError(f"row {i}: position {pos} outside the block table")
+        page = int(block_table[seq, pos // PAGE_SIZE])
+        if page < 0 or page >= k_out.shape[0]:
+            raise ValueError(f"row {i}: page id {page} outside the pool")
+        k_out[page, pos % PAGE_SIZE] = k_new[i]
+        l_out[page, pos % PAGE_SIZE] = latent_new[i]
+    return k_out, l_out
 
 
 # --------------------------------------------------------------------------

@@ -27,6 +27,7 @@ OP_TOPK = 1
 OP_SPARSE_MLA_DECODE = 2
 OP_SPARSE_MLA_PREFILL = 3
 OP_ATTENTION_FORWARD = 4
+OP_CACHE_APPEND = 5
 
 STATUS_NAMES = {0: "DSA_OK", 1: "DSA_ERR_INVALID_ARG", 2: "DSA_ERR_UNSUPPORTED",
                 3: "DSA_ERR_CUDA", 4: "DSA_ERR_WORKSPACE", 5: "DSA_ERR_TIMEOUT",
@@ -34,7 +35,8 @@ STATUS_NAMES = {0: "DSA_OK", 1: "DSA_ERR_INVALID_ARG", 2: "DSA_ERR_UNSUPPORTED",
 
 EXPORTED = ["dsa_version", "dsa_status_string", "dsa_workspace_bytes", "dsa_workspace_init",
             "dsa_workspace_check", "dsa_indexer_scores", "dsa_topk", "dsa_sparse_mla_decode",
-            "dsa_sparse_mla_prefill", "dsa_attention_forward", "dsa_sparse_mla_decode_noalloc"]
+            "dsa_sparse_mla_prefill", "dsa_attention_forward", "dsa_sparse_mla_decode_noalloc",
+            "dsa_cache_append"]
 
 
 class DsaError(RuntimeError):
@@ -84,6 +86,7 @@ def lib() -> ctypes.CDLL:
             "dsa_attention_forward": ([vp, vp, vp, vp, vp, pc, pd, vp, vp, vp, vp, sz, vp],
                                       ctypes.c_int),
             "dsa_sparse_mla_decode_noalloc": ([vp, vp, pc, vp, pd, vp, vp, vp], ctypes.c_int),
+            "dsa_cache_append": ([vp, vp, vp, vp, pc, pd, vp, sz, vp], ctypes.c_int),
         }
         for name, (args, res) in sigs.items():
             fn = getattr(L, name)
@@ -214,3 +217,14 @@ def dsa_attention_forward(q_idx, w, k_idx_pages, q, latent_pages, cache: PagedCa
                                        ctypes.byref(dims.struct()), _ptr(idx_out), _ptr(out),
                                        _ptr(lse), _ptr(ws), ws.numel(), _stream(stream)),
            "dsa_attention_forward")
+
+
+def dsa_cache_append(k_idx_new, latent_new, k_idx_pages, latent_pages, cache: PagedCache,
+                     dims: Dims, ws, stream=None) -> None:
+    """Write the new tokens' index keys [n_q, D_I] and latent rows [n_q, R + P]
+    into the page pools at the positions of the step's query rows (decode row b:
+    seq_lens[b] - 1 of sequence b; prefill row t: q_pos0 + t of sequence 0)."""
+    _check(lib().dsa_cache_append(_ptr(k_idx_new), _ptr(latent_new), _ptr(k_idx_pages),
+                                  _ptr(latent_pages), ctypes.byref(cache.struct()),
+                                  ctypes.byref(dims.struct()), _ptr(ws), ws.numel(),
+                                  _stream(stream)), "dsa_cache_append")

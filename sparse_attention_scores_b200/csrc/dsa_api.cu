@@ -192,6 +192,7 @@ size_t ws_bytes_for(dsa_op_t op, const dsa_dims_t &d, const dsa_cache_t &c) {
   switch (op) {
     case DSA_OP_INDEXER_SCORES:
     case DSA_OP_TOPK:
+    case DSA_OP_CACHE_APPEND:
       return kStatusBytes;
     case DSA_OP_SPARSE_MLA_DECODE:
     case DSA_OP_SPARSE_MLA_PREFILL:
@@ -319,7 +320,8 @@ const char *dsa_status_string(dsa_status_t s) {
 
 size_t dsa_workspace_bytes(dsa_op_t op, const dsa_dims_t *dims, const dsa_cache_t *cache) {
   if (check_dims_common(dims) != DSA_OK) return 0;
-  if (op == DSA_OP_INDEXER_SCORES || op == DSA_OP_TOPK) return kStatusBytes;
+  if (op == DSA_OP_INDEXER_SCORES || op == DSA_OP_TOPK || op == DSA_OP_CACHE_APPEND)
+    return kStatusBytes;
   if (check_mla_dims(*dims) != DSA_OK) return 0;
   if (op == DSA_OP_ATTENTION_FORWARD && (cache == nullptr || check_cache(cache, *dims) != DSA_OK))
     return 0;
@@ -431,6 +433,42 @@ dsa_status_t dsa_attention_forward(const uint16_t *q_idx, const float *w,
                    static_cast<int>(max_keys(d, c)), st, s));
   return run_mla(q, latent_pages, c, idx, d, out, lse, scratch, scratch_bytes, st, s,
                  /*early_q=*/1);
+}
+
+dsa_status_t dsa_cache_append(const uint16_t *k_idx_new, const uint16_t *latent_new,
+                              uint16_t *k_idx_pages, uint16_t *latent_pages,
+                              const dsa_cache_t *cache, const dsa_dims_t *dims, void *ws,
+                              size_t ws_bytes, dsa_stream_t stream) {
+  DSA_TRY(check_dims_common(dims));
+  const dsa_dims_t &d = *dims;
+  if (d.D_I != 32 && d.D_I != 64 && d.D_I != 128) return DSA_ERR_UNSUPPORTED;
+  if (d.R < 64 || d.R > 512 || d.R % 64 != 0) return DSA_ERR_UNSUPPORTED;
+  if (d.P < 0 || d.P % 16 != 0 || d.R + d.P > 576) return DSA_ERR_UNSUPPORTED;
+  DSA_TRY(check_cache(cache, d));
+  if (k_idx_new == nullptr || latent_new == nullptr || k_idx_pages == nullptr ||
+      latent_pages == nullptr)
+    return DSA_ERR_INVALID_ARG;
+  if (!aligned16(k_idx_new) || !aligned16(latent_new) || !aligned16(k_idx_pages) ||
+      !aligned16(latent_pages))
+    return DSA_ERR_INVALID_ARG;
+  DSA_TRY(check_ws(ws, ws_bytes, kStatusBytes));
+  if (d.n_q == 0) return DSA_OK;
+  AppendLaunch a;
+  a.k_new = k_idx_new;
+  a.lat_new = latent_new;
+  a.k_pages = k_idx_pages;
+  a.lat_pages = latent_pages;
+  a.seq_lens = cache->seq_lens;
+  a.block_table = cache->block_table;
+  a.n_q = d.n_q;
+  a.D_I = d.D_I;
+  a.W = d.R + d.P;
+  a.causal = d.causal;
+  a.q_pos0 = d.q_pos0;
+  a.max_pages = cache->max_pages;
+  a.num_pages = cache->num_pages;
+  a.status = status_of(ws);
+  return launch_append(a, as_stream(stream));
 }
 
 }  // extern "C"

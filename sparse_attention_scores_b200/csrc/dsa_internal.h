@@ -89,6 +89,18 @@ struct TopkLaunch {
 };
 dsa_status_t launch_topk(const TopkLaunch &a, cudaStream_t stream);
 
+struct AppendLaunch {
+  const uint16_t *k_new;
+  const uint16_t *lat_new;
+  uint16_t *k_pages;
+  uint16_t *lat_pages;
+  const int32_t *seq_lens;
+  const int32_t *block_table;
+  int n_q, D_I, W, causal, q_pos0, max_pages, num_pages;
+  DevStatus *status;
+};
+dsa_status_t launch_append(const AppendLaunch &a, cudaStream_t stream);
+
 struct MlaLaunch {
   const uint16_t *q;
   const uint16_t *latent;

@@ -27,7 +27,7 @@ def _declared_symbols():
 
 def test_every_declared_symbol_is_exported(L):
     declared = _declared_symbols()
-    assert len(declared) == 11
+    assert len(declared) == 12
     assert sorted(declared) == sorted(dsa.EXPORTED)
     out = subprocess.run(["nm", "-D", "--defined-only", dsa.LIB_PATH], capture_output=True,
                          text=True, check=True).stdout
@@ -136,3 +136,19 @@ def test_host_validation_rejects_without_launch(L):
     st = L.dsa_indexer_scores(fake, fake, fake, ctypes.byref(_cache(max_seq_len=128 * 64 + 1)),
                               ctypes.byref(d), fake, 8196, ws, 1 << 30, None)
     assert st == 1
+    # cache append: null / misaligned pointers, unsupported widths, no workspace
+    st = L.dsa_cache_append(None, fake, fake, fake, ctypes.byref(c), ctypes.byref(d), ws,
+                            1 << 20, None)
+    assert st == 1
+    st = L.dsa_cache_append(ctypes.c_void_p(0x300008), fake, fake, fake, ctypes.byref(c),
+                            ctypes.byref(d), ws, 1 << 20, None)
+    assert st == 1
+    st = L.dsa_cache_append(fake, fake, fake, fake, ctypes.byref(c), ctypes.byref(_dims(D_I=48)),
+                            ws, 1 << 20, None)
+    assert st == 2
+    st = L.dsa_cache_append(fake, fake, fake, fake, ctypes.byref(c), ctypes.byref(_dims(P=8)),
+                            ws, 1 << 20, None)
+    assert st == 2
+    st = L.dsa_cache_append(fake, fake, fake, fake, ctypes.byref(c), ctypes.byref(d), ws, 16,
+                            None)
+    assert st == 4

@@ -161,6 +161,19 @@ def _absorb_without_transpose(q_nope, q_rope, W_UK):
     return np.concatenate([q_lat, q_rope], axis=1)
 
 
+def _append_one_slot_late(k_pages, latent_pages, block_table, positions, k_new, latent_new):
+    shifted = [(seq, pos + 1) for seq, pos in positions]
+    return _ORIG_APPEND(k_pages, latent_pages, block_table, shifted, k_new, latent_new)
+
+
+def _append_positions_of_the_next_token(inp):
+    return [(seq, pos + 1) for seq, pos in _ORIG_POSITIONS(inp)]
+
+
+_ORIG_APPEND = orc.cache_append
+_ORIG_POSITIONS = orc.append_positions
+
+
 MUTANTS = {
     "indexer: ReLU dropped": ("indexer_scores", _indexer_no_relu),
     "indexer: ReLU after the head sum": ("indexer_scores", _indexer_relu_after_sum),
@@ -187,6 +200,8 @@ MUTANTS = {
     "decode: last token not visible": ("dsa_decode", _decode_sees_one_less),
     "step: selection skipped": ("dsa_query", _query_skips_topk),
     "absorption: W_UK not transposed": ("absorb_query", _absorb_without_transpose),
+    "append: written one slot late": ("cache_append", _append_one_slot_late),
+    "append: the next token's position": ("append_positions", _append_positions_of_the_next_token),
 }
 
 

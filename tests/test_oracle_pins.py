@@ -249,6 +249,79 @@ def test_sparse_attends_only_selected_rows():
         assert (not np.array_equal(r["out"], base["out"])) == changes
 
 
+# ---------------------------------------------------------------- cache append
+
+def _new_rows(n, width, seed):
+    rng = np.random.default_rng(seed)
+    return di.f32_to_bf16_bits(rng.standard_normal((n, width)).astype(np.float32))
+
+
+def test_append_reads_back_through_the_block_table():
+    wl = di.small_decode([300, 129, 64, 1000], H_I=2, D_I=16, topk=32, H=2, R=16, P=8, seed=3,
+                         shuffle_pages=True)
+    inp = di.make_inputs(wl)
+    pos = orc.append_positions(inp)
+    assert pos == [(b, n - 1) for b, n in enumerate(wl.seq_lens)]
+    k_new, l_new = _new_rows(4, wl.D_I, 1), _new_rows(4, wl.W, 2)
+    kp, lp = orc.cache_append(inp["k_pages"], inp["latent_pages"], inp["block_table"], pos,
+                              k_new, l_new)
+    for b, n in enumerate(wl.seq_lens):
+        old = orc.gather_paged_rows(inp["latent_pages"], inp["block_table"][b], range(n))
+        new = orc.gather_paged_rows(lp, inp["block_table"][b], range(n))
+        assert np.array_equal(new[:n - 1], old[:n - 1])   # earlier tokens untouched
+        assert np.array_equal(new[n - 1], l_new[b])       # the new token at its position
+        newk = orc.gather_paged_rows(kp, inp["block_table"][b], [n - 1])
+        assert np.array_equal(newk[0], k_new[b])
+    # exactly one row per appended token changed in each pool
+    assert (kp != inp["k_pages"]).any(axis=2).sum() == 4
+    assert (lp != inp["latent_pages"]).any(axis=2).sum() == 4
+
+
+def test_append_round_trip_restores_the_step():
+    # blank the current tokens' rows, append them again: the pools and the
+    # step's result are what they were
+    wl = di.small_decode([200, 65], H_I=2, D_I=16, topk=16, H=2, R=16, P=8, seed=5,
+                         shuffle_pages=True)
+    inp = di.make_inputs(wl)
+    pos = orc.append_positions(inp)
+    k_cur = np.stack([orc.gather_paged_rows(inp["k_pages"], inp["block_table"][b], [p])[0]
+                      for b, p in pos])
+    l_cur = np.stack([orc.gather_paged_rows(inp["latent_pages"], inp["block_table"][b], [p])[0]
+                      for b, p in pos])
+    blank = dict(inp)
+    blank["k_pages"], blank["latent_pages"] = orc.cache_append(
+        inp["k_pages"], inp["latent_pages"], inp["block_table"], pos,
+        np.zeros_like(k_cur), np.zeros_like(l_cur))
+    kp, lp = orc.cache_append(blank["k_pages"], blank["latent_pages"], inp["block_table"], pos,
+                              k_cur, l_cur)
+    assert np.array_equal(kp, inp["k_pages"]) and np.array_equal(lp, inp["latent_pages"])
+    again = dict(inp, k_pages=kp, latent_pages=lp)
+    r0, r1 = orc.dsa_decode(inp), orc.dsa_decode(again)
+    for b in r0:
+        assert np.array_equal(r0[b]["idx"], r1[b]["idx"])
+        np.testing.assert_array_equal(r0[b]["out"], r1[b]["out"])
+
+
+def test_append_prefill_positions_and_checks():
+    wl = di.small_prefill(70, q_pos0=10, H_I=2, D_I=16, topk=16, H=2, R=16, P=8, seed=2)
+    inp = di.make_inputs(wl)
+    pos = orc.append_positions(inp)
+    assert pos == [(0, 10 + t) for t in range(70)]
+    k_new, l_new = _new_rows(70, wl.D_I, 3), _new_rows(70, wl.W, 4)
+    kp, lp = orc.cache_append(inp["k_pages"], inp["latent_pages"], inp["block_table"], pos,
+                              k_new, l_new)
+    got = orc.gather_paged_rows(lp, inp["block_table"][0], range(10, 80))
+    assert np.array_equal(got, l_new)
+    with pytest.raises(ValueError):
+        orc.cache_append(inp["k_pages"], inp["latent_pages"], inp["block_table"],
+                         [(0, inp["block_table"].shape[1] * 64)], k_new[:1], l_new[:1])
+    bad = inp["block_table"].copy()
+    bad[0, 0] = inp["k_pages"].shape[0]
+    with pytest.raises(ValueError):
+        orc.cache_append(inp["k_pages"], inp["latent_pages"], bad, [(0, 0)], k_new[:1],
+                         l_new[:1])
+
+
 # ---------------------------------------------------------------- whole step
 
 def test_step_keeps_the_best_scored_tokens():
