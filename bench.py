@@ -213,6 +213,18 @@ class Case:
         phys = inp["block_table"][seqs, pos // 64].astype(np.int64) * 64 + pos % 64
         self.k_new = bf(inp["k_pages"].reshape(-1, wl.D_I)[phys])
         self.l_new = bf(inp["latent_pages"].reshape(-1, wl.W)[phys])
+        # the absorption GEMMs around the step (GLM-5 head dims: q_nope 128, v 128)
+        g = torch.Generator(device="cpu").manual_seed(wl.seed + 77)
+        self.d_nope, self.d_v = 128, 128
+        H, R, P = wl.H, wl.R, wl.P
+        self.q_nope = torch.randn((wl.n_q, H, self.d_nope), generator=g).to(torch.bfloat16).to(dev)
+        self.q_rope = torch.randn((wl.n_q, H, P), generator=g).to(torch.bfloat16).to(dev)
+        self.w_uk = (torch.randn((H, self.d_nope, R), generator=g) / self.d_nope ** 0.5).to(
+            torch.bfloat16).to(dev)
+        self.w_uv = (torch.randn((H, R, self.d_v), generator=g) / R ** 0.5).to(torch.bfloat16).to(dev)
+        self.q_abs = torch.empty((wl.n_q, H, R + P), dtype=torch.bfloat16, device=dev)
+        self.v_out = torch.empty((wl.n_q, H, self.d_v), dtype=torch.float32, device=dev)
+        self.sws = dsa.status_workspace()
         self.dsa = dsa
         self.torch = torch
 
@@ -230,6 +242,18 @@ class Case:
         t = self.t
         self.dsa.dsa_cache_append(self.k_new, self.l_new, t["k_pages"], t["latent_pages"],
                                   self.cache, self.dims, self.ws)
+
+    def absorb(self):
+        self.dsa.dsa_absorb_query(self.q_nope, self.q_rope, self.w_uk, self.q_abs, self.sws)
+
+    def project(self):
+        self.dsa.dsa_project_values(self.out, self.w_uv, self.v_out, self.sws)
+
+    def absorb_bytes_flops(self):
+        wl, n, H = self.wl, self.wl.n_q, self.wl.H
+        a_bytes = H * self.d_nope * wl.R * 2 + n * H * (self.d_nope + wl.P + wl.R + wl.P) * 2
+        p_bytes = H * wl.R * self.d_v * 2 + n * H * (wl.R + self.d_v) * 4
+        return (a_bytes, 2 * n * H * self.d_nope * wl.R, p_bytes, 2 * n * H * wl.R * self.d_v)
 
     def topk(self):
         # the scores of the last indexer() call; decode rows end at their
@@ -290,8 +314,15 @@ def measure(case, torch, steps, warmup, flush_buf, peaks):
     ms_idx, _ = timed_events(torch, case.indexer, steps, warmup, flush_buf)
     ms_topk, _ = timed_events(torch, case.topk, steps, warmup, flush_buf)
     ms_mla, _ = timed_events(torch, case.mla, steps, warmup, flush_buf)
-    # the cache append in front of the step (a separate entry point, not in the step)
+    # the cache append in front of the step and the absorption GEMMs around it
+    # (separate entry points, not in the step)
     ms_app, _ = timed_events(torch, case.append, steps, warmup, flush_buf)
+    ms_abs, _ = timed_events(torch, case.absorb, steps, warmup, flush_buf)
+    ms_prj, _ = timed_events(torch, case.project, steps, warmup, flush_buf)
+    st, info = case.dsa.workspace_check(case.sws)
+    if st != 0:
+        raise RuntimeError(f"device status {st} ({info:#x}) in the absorption GEMMs of {wl.name}")
+    ab, af, pb, pf = case.absorb_bytes_flops()
     st, info = case.dsa.workspace_check(case.ws)
     if st != 0:
         raise RuntimeError(f"device status {st} ({info:#x}) in the stage timings of {wl.name}")
@@ -315,6 +346,10 @@ def measure(case, torch, steps, warmup, flush_buf, peaks):
         "append_us": ms_app * 1e3,
         "append_alg_bytes": alg["bytes_append"],
         "append_gbs": alg["bytes_append"] / (ms_app * 1e-3) / 1e9,
+        "absorb_query": {"us": ms_abs * 1e3, "alg_bytes": ab, "gbs": ab / (ms_abs * 1e-3) / 1e9,
+                         "tflops": af / (ms_abs * 1e-3) / 1e12},
+        "project_values": {"us": ms_prj * 1e3, "alg_bytes": pb, "gbs": pb / (ms_prj * 1e-3) / 1e9,
+                           "tflops": pf / (ms_prj * 1e-3) / 1e12},
     }
     return res
 

@@ -217,6 +217,40 @@ DSA_API dsa_status_t dsa_cache_append(const uint16_t *k_idx_new, const uint16_t 
                               const dsa_cache_t *cache, const dsa_dims_t *dims, void *ws,
                               size_t ws_bytes, dsa_stream_t stream);
 
+/* Workspace of the entry points that need only the status block
+ * (dsa_absorb_query, dsa_project_values; also what dsa_workspace_bytes returns
+ * for DSA_OP_INDEXER_SCORES, DSA_OP_TOPK and DSA_OP_CACHE_APPEND). */
+#define DSA_STATUS_WORKSPACE_BYTES 256
+
+/* Query absorption, the product in front of the logits: the per-head key
+ * up-projection folded into the query, so the step scores queries against the
+ * compressed latent rows directly ("Self-contained GLM-5 serving stack ...",
+ * file list: absorbed MLA decode over compressed request-local KV).
+ *   q_nope  [n_q, H, d_nope] bf16, q_rope [n_q, H, P] bf16 (may be NULL when P = 0)
+ *   w_uk    [H, d_nope, R] bf16 (row d of head h maps q_nope[., h, d] onto the R latent columns)
+ *   q_abs   [n_q, H, R + P] bf16 output, the step's q:
+ *           q_abs[b, h, 0:R] = bf16(sum_d q_nope[b, h, d] * w_uk[h, d, :]) (fp32 accumulate,
+ *           round to nearest even), q_abs[b, h, R:] = q_rope[b, h, :]
+ * d_nope: multiple of 64, <= 512; R: multiple of 64, <= 512; P: multiple of 16,
+ * R + P <= 576; H <= 128.  All pointers 16-byte aligned.  tcgen05 tensor cores
+ * (D^T = W^T . q^T per head, the weight tile as the MN-major A operand). */
+DSA_API dsa_status_t dsa_absorb_query(const uint16_t *q_nope, const uint16_t *q_rope,
+                              const uint16_t *w_uk, uint16_t *q_abs, int32_t n_q, int32_t H,
+                              int32_t d_nope, int32_t R, int32_t P, void *ws, size_t ws_bytes,
+                              dsa_stream_t stream);
+
+/* Value projection, the product after the split merge: the per-head value
+ * up-projection applied to the latent-space output (same pages as above).
+ *   o_lat   [n_q, H, R] fp32 (the `out` of the step), 16-byte aligned
+ *   w_uv    [H, R, d_v] bf16, 16-byte aligned
+ *   v_out   [n_q, H, d_v] fp32 output: v_out[b, h, :] = sum_r o_lat[b, h, r] * w_uv[h, r, :]
+ * o_lat enters the tensor cores as two bf16 terms (hi + lo), so its precision
+ * is kept to about 2^-17 relative.  R: multiple of 64, <= 512; d_v: multiple of
+ * 64, <= 512; H <= 128. */
+DSA_API dsa_status_t dsa_project_values(const float *o_lat, const uint16_t *w_uv, float *v_out,
+                                int32_t n_q, int32_t H, int32_t R, int32_t d_v, void *ws,
+                                size_t ws_bytes, dsa_stream_t stream);
+
 /* Sparse MLA decode for callers that cannot allocate device memory.
  *
  * The pages have no counterpart of this entry point: it exists for callers

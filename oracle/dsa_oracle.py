@@ -238,6 +238,13 @@ def absorb_query(q_nope, q_rope, W_UK):
     return np.concatenate([q_lat, q_rope], axis=1)
 
 
+def project_values(o_lat, W_UV):
+    """Per-head value up-projection of the latent-space output:
+    v[h] = W_UV[h]^T o_lat[h].  o_lat [H, R], W_UV [H, R, d_v] -> [H, d_v]."""
+    H = o_lat.shape[0]
+    return np.stack([W_UV[h].T @ o_lat[h] for h in range(H)])
+
+
 # --------------------------------------------------------------------------
 # the whole step
 # --------------------------------------------------------------------------

@@ -36,7 +36,7 @@ STATUS_NAMES = {0: "DSA_OK", 1: "DSA_ERR_INVALID_ARG", 2: "DSA_ERR_UNSUPPORTED",
 EXPORTED = ["dsa_version", "dsa_status_string", "dsa_workspace_bytes", "dsa_workspace_init",
             "dsa_workspace_check", "dsa_indexer_scores", "dsa_topk", "dsa_sparse_mla_decode",
             "dsa_sparse_mla_prefill", "dsa_attention_forward", "dsa_sparse_mla_decode_noalloc",
-            "dsa_cache_append"]
+            "dsa_cache_append", "dsa_absorb_query", "dsa_project_values"]
 
 
 class DsaError(RuntimeError):
@@ -87,6 +87,9 @@ def lib() -> ctypes.CDLL:
                                       ctypes.c_int),
             "dsa_sparse_mla_decode_noalloc": ([vp, vp, pc, vp, pd, vp, vp, vp], ctypes.c_int),
             "dsa_cache_append": ([vp, vp, vp, vp, pc, pd, vp, sz, vp], ctypes.c_int),
+            "dsa_absorb_query": ([vp, vp, vp, vp, i32, i32, i32, i32, i32, vp, sz, vp],
+                                 ctypes.c_int),
+            "dsa_project_values": ([vp, vp, vp, i32, i32, i32, i32, vp, sz, vp], ctypes.c_int),
         }
         for name, (args, res) in sigs.items():
             fn = getattr(L, name)
@@ -162,6 +165,18 @@ def workspace(op: int, dims: Dims, cache: PagedCache | None, device="cuda", stre
     return ws
 
 
+STATUS_WORKSPACE_BYTES = 256  # DSA_STATUS_WORKSPACE_BYTES
+
+
+def status_workspace(device="cuda", stream=None):
+    """Workspace of the entry points that need only the status block."""
+    import torch
+    ws = torch.empty(STATUS_WORKSPACE_BYTES, dtype=torch.uint8, device=device)
+    _check(lib().dsa_workspace_init(_ptr(ws), STATUS_WORKSPACE_BYTES, _stream(stream)),
+           "dsa_workspace_init")
+    return ws
+
+
 def workspace_check(ws, stream=None) -> tuple[int, int]:
     info = ctypes.c_uint32(0)
     st = lib().dsa_workspace_check(_ptr(ws), _stream(stream), ctypes.byref(info))
@@ -228,3 +243,22 @@ def dsa_cache_append(k_idx_new, latent_new, k_idx_pages, latent_pages, cache: Pa
                                   _ptr(latent_pages), ctypes.byref(cache.struct()),
                                   ctypes.byref(dims.struct()), _ptr(ws), ws.numel(),
                                   _stream(stream)), "dsa_cache_append")
+
+
+def dsa_absorb_query(q_nope, q_rope, w_uk, q_abs, ws, stream=None) -> None:
+    """q_abs [n, H, R + P] = [q_nope [n, H, d_nope] . w_uk [H, d_nope, R] | q_rope [n, H, P]]."""
+    n, H, d_nope = (int(x) for x in q_nope.shape)
+    R = int(w_uk.shape[2])
+    P = int(q_rope.shape[2]) if q_rope is not None else 0
+    _check(lib().dsa_absorb_query(_ptr(q_nope), _ptr(q_rope), _ptr(w_uk), _ptr(q_abs), n, H,
+                                  d_nope, R, P, _ptr(ws), ws.numel(), _stream(stream)),
+           "dsa_absorb_query")
+
+
+def dsa_project_values(o_lat, w_uv, v_out, ws, stream=None) -> None:
+    """v_out [n, H, d_v] = o_lat [n, H, R] (fp32) . w_uv [H, R, d_v]."""
+    n, H, R = (int(x) for x in o_lat.shape)
+    d_v = int(w_uv.shape[2])
+    _check(lib().dsa_project_values(_ptr(o_lat), _ptr(w_uv), _ptr(v_out), n, H, R, d_v,
+                                    _ptr(ws), ws.numel(), _stream(stream)),
+           "dsa_project_values")

@@ -113,6 +113,7 @@ size_t device_smem_per_sm() {
 namespace {
 
 constexpr size_t kStatusBytes = sizeof(DevStatus);
+static_assert(kStatusBytes == DSA_STATUS_WORKSPACE_BYTES, "status block size in the header");
 
 size_t align256(size_t x) { return (x + 255) & ~static_cast<size_t>(255); }
 bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
@@ -469,6 +470,59 @@ dsa_status_t dsa_cache_append(const uint16_t *k_idx_new, const uint16_t *latent_
   a.num_pages = cache->num_pages;
   a.status = status_of(ws);
   return launch_append(a, as_stream(stream));
+}
+
+dsa_status_t dsa_absorb_query(const uint16_t *q_nope, const uint16_t *q_rope, const uint16_t *w_uk,
+                              uint16_t *q_abs, int32_t n_q, int32_t H, int32_t d_nope, int32_t R,
+                              int32_t P, void *ws, size_t ws_bytes, dsa_stream_t stream) {
+  if (n_q < 0 || H < 1 || H > 128) return DSA_ERR_INVALID_ARG;
+  if (d_nope < 64 || d_nope > 512 || d_nope % 64 != 0) return DSA_ERR_UNSUPPORTED;
+  if (R < 64 || R > 512 || R % 64 != 0) return DSA_ERR_UNSUPPORTED;
+  if (P < 0 || P % 16 != 0 || R + P > 576) return DSA_ERR_UNSUPPORTED;
+  if (q_nope == nullptr || w_uk == nullptr || q_abs == nullptr || (P > 0 && q_rope == nullptr))
+    return DSA_ERR_INVALID_ARG;
+  if (!aligned16(q_nope) || !aligned16(w_uk) || !aligned16(q_abs) ||
+      (P > 0 && !aligned16(q_rope)))
+    return DSA_ERR_INVALID_ARG;
+  DSA_TRY(check_ws(ws, ws_bytes, kStatusBytes));
+  if (n_q == 0) return DSA_OK;
+  AbsorbLaunch a = {};
+  a.project = false;
+  a.x = q_nope;
+  a.rope = q_rope;
+  a.w = w_uk;
+  a.out_bf16 = q_abs;
+  a.n = n_q;
+  a.H = H;
+  a.K = d_nope;
+  a.M = R;
+  a.P = P;
+  a.status = status_of(ws);
+  return launch_absorb(a, as_stream(stream));
+}
+
+dsa_status_t dsa_project_values(const float *o_lat, const uint16_t *w_uv, float *v_out,
+                                int32_t n_q, int32_t H, int32_t R, int32_t d_v, void *ws,
+                                size_t ws_bytes, dsa_stream_t stream) {
+  if (n_q < 0 || H < 1 || H > 128) return DSA_ERR_INVALID_ARG;
+  if (R < 64 || R > 512 || R % 64 != 0) return DSA_ERR_UNSUPPORTED;
+  if (d_v < 64 || d_v > 512 || d_v % 64 != 0) return DSA_ERR_UNSUPPORTED;
+  if (o_lat == nullptr || w_uv == nullptr || v_out == nullptr) return DSA_ERR_INVALID_ARG;
+  if (!aligned16(o_lat) || !aligned16(w_uv) || !aligned4(v_out)) return DSA_ERR_INVALID_ARG;
+  DSA_TRY(check_ws(ws, ws_bytes, kStatusBytes));
+  if (n_q == 0) return DSA_OK;
+  AbsorbLaunch a = {};
+  a.project = true;
+  a.xf = o_lat;
+  a.w = w_uv;
+  a.out_f32 = v_out;
+  a.n = n_q;
+  a.H = H;
+  a.K = R;
+  a.M = d_v;
+  a.P = 0;
+  a.status = status_of(ws);
+  return launch_absorb(a, as_stream(stream));
 }
 
 }  // extern "C"

@@ -37,7 +37,8 @@ enum : unsigned int {
   kErrBadPage = 2u,    // block-table entry outside [0, num_pages)
   kErrBadIndex = 4u,   // selected token position outside the row's context
 };
-enum : unsigned int { kKernIndexer = 1u, kKernTopk = 2u, kKernMla = 3u, kKernCombine = 4u, kKernAppend = 5u };
+enum : unsigned int { kKernIndexer = 1u, kKernTopk = 2u, kKernMla = 3u, kKernCombine = 4u, kKernAppend = 5u,
+                      kKernAbsorb = 6u };
 
 __device__ __forceinline__ void report(DevStatus *st, unsigned int bit, unsigned int code) {
   if (st == nullptr) return;

@@ -101,6 +101,19 @@ struct AppendLaunch {
 };
 dsa_status_t launch_append(const AppendLaunch &a, cudaStream_t stream);
 
+struct AbsorbLaunch {
+  bool project;          // false: q_abs = q_nope . W_UK (+ rope); true: v_out = o_lat . W_UV
+  const uint16_t *x;     // q_nope [n, H, K] bf16 (absorb)
+  const float *xf;       // o_lat  [n, H, K] fp32 (project)
+  const uint16_t *rope;  // q_rope [n, H, P] (absorb, may be null when P == 0)
+  const uint16_t *w;     // W_UK [H, K, M] or W_UV [H, K, M] bf16
+  uint16_t *out_bf16;    // q_abs [n, H, M + P]
+  float *out_f32;        // v_out [n, H, M]
+  int n, H, K, M, P;
+  DevStatus *status;
+};
+dsa_status_t launch_absorb(const AbsorbLaunch &a, cudaStream_t stream);
+
 struct MlaLaunch {
   const uint16_t *q;
   const uint16_t *latent;

@@ -170,6 +170,12 @@ def _append_positions_of_the_next_token(inp):
     return [(seq, pos + 1) for seq, pos in _ORIG_POSITIONS(inp)]
 
 
+def _project_without_transpose(o_lat, W_UV):
+    H = o_lat.shape[0]
+    return np.stack([np.resize(W_UV[h] @ np.resize(o_lat[h], W_UV.shape[2]), W_UV.shape[2])
+                     for h in range(H)])
+
+
 _ORIG_APPEND = orc.cache_append
 _ORIG_POSITIONS = orc.append_positions
 
@@ -201,6 +207,7 @@ MUTANTS = {
     "step: selection skipped": ("dsa_query", _query_skips_topk),
     "absorption: W_UK not transposed": ("absorb_query", _absorb_without_transpose),
     "append: written one slot late": ("cache_append", _append_one_slot_late),
+    "projection: W_UV not transposed": ("project_values", _project_without_transpose),
     "append: the next token's position": ("append_positions", _append_positions_of_the_next_token),
 }
 

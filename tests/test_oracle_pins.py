@@ -224,7 +224,7 @@ def test_absorbed_equals_nonabsorbed():
                                                      W_UK, W_UV, scale)
     q_abs = orc.absorb_query(q_nope, q_rope, W_UK)
     lat_out, lse, _ = orc.mla_attention(q_abs, np.concatenate([c_kv, k_rope], 1), R, scale)
-    out = np.stack([lat_out[h] @ W_UV[h] for h in range(H)])
+    out = orc.project_values(lat_out, W_UV)
     np.testing.assert_allclose(out, ref_out, rtol=1e-10, atol=1e-12)
     np.testing.assert_allclose(lse, ref_lse, rtol=1e-12)
 
