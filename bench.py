@@ -36,6 +36,8 @@ import dsa_inputs as di  # noqa: E402
 
 HEADLINE = "glm5_decode_8k"
 EXTRA = ["tiny_decode", "glm5_decode_b32_ragged", "glm5_prefill_2300", "glm5_decode_4x128k"]
+# the same workloads with the index keys held as E4M3 bytes + one scale per token
+EXTRA_K8 = ["glm5_decode_8k", "glm5_decode_b32_ragged", "glm5_decode_4x128k"]
 NOMINAL_HBM_GBS = 8000.0
 FLUSH_BYTES = 512 << 20
 
@@ -63,24 +65,26 @@ def row_lengths(wl):
     return list(wl.seq_lens)
 
 
-def algorithmic(wl):
-    """Must-move bytes and flops of one step (scores and page tables excluded)."""
+def algorithmic(wl, k8=False):
+    """Must-move bytes and flops of one step (scores and page tables excluded).
+    k8: the index keys as E4M3 bytes plus a 4-byte scale per token."""
     lens = row_lengths(wl)
     keys = sum(lens)
     sel = sum(min(wl.topk, n) for n in lens)
-    b_keys = keys * wl.D_I * 2
+    key_bytes = (wl.D_I + 4) if k8 else wl.D_I * 2
+    b_keys = keys * key_bytes
     b_lat = sel * wl.W * 2
     b_small = wl.n_q * (wl.H * wl.W * 2 + wl.H_I * wl.D_I * 2 + wl.H_I * 4 + wl.H * wl.R * 4
                         + wl.H * 4)
     if wl.mode == "prefill":   # every row reads the same (L2-resident) cache
-        b_keys = (wl.q_pos0 + wl.n_q) * wl.D_I * 2
+        b_keys = (wl.q_pos0 + wl.n_q) * key_bytes
         b_lat = (wl.q_pos0 + wl.n_q) * wl.W * 2
     flops_idx = 2 * wl.H_I * wl.D_I * keys
     flops_mla = sel * wl.H * 2 * (wl.W + wl.R)
     # indexer kernel alone: key rows read + fp32 score per key written
-    b_indexer = keys * (wl.D_I * 2 + 4) + wl.n_q * wl.H_I * (wl.D_I * 2 + 4)
+    b_indexer = keys * (key_bytes + 4) + wl.n_q * wl.H_I * (wl.D_I * 2 + 4)
     if wl.mode == "prefill":
-        b_indexer = (wl.q_pos0 + wl.n_q) * wl.D_I * 2 + keys * 4
+        b_indexer = (wl.q_pos0 + wl.n_q) * key_bytes + keys * 4
     # top-k alone: every score read once, the index rows written
     b_topk = keys * 4 + wl.n_q * wl.topk * 4
     # sparse MLA + split merge: selected latent rows, q, idx in; out, lse out
@@ -180,8 +184,9 @@ def job_rows_per_s(rows_per_rank: int, world: int, ms_per_step: float) -> float:
 class Case:
     """Device-resident inputs, outputs and workspace of one workload."""
 
-    def __init__(self, wl, torch, dsa):
+    def __init__(self, wl, torch, dsa, k8=False):
         self.wl = wl
+        self.k8 = k8
         self.inp = di.make_inputs(wl)
         inp = self.inp
         dev = "cuda"
@@ -193,6 +198,11 @@ class Case:
                   "latent_pages": bf(inp["latent_pages"]), "w": torch.from_numpy(inp["w"]).to(dev),
                   "block_table": torch.from_numpy(inp["block_table"]).to(dev),
                   "seq_lens": torch.from_numpy(inp["seq_lens"]).to(dev)}
+        if k8:   # the index keys as E4M3 bytes with one scale per token
+            k8in = di.with_fp8_keys(inp, seed=wl.seed)
+            self.t["k8_pages"] = torch.from_numpy(k8in["k8_pages"]).to(dev)
+            self.t["k_scale"] = torch.from_numpy(k8in["k_scale"]).to(dev)
+            del self.t["k_pages"]
         self.cache = dsa.PagedCache(self.t["seq_lens"], self.t["block_table"],
                                     num_pages=int(inp["k_pages"].shape[0]),
                                     max_seq_len=int(inp["seq_lens"].max()))
@@ -202,7 +212,8 @@ class Case:
         self.idx = torch.empty((wl.n_q, wl.topk), dtype=torch.int32, device=dev)
         self.out = torch.empty((wl.n_q, wl.H, wl.R), dtype=torch.float32, device=dev)
         self.lse = torch.empty((wl.n_q, wl.H), dtype=torch.float32, device=dev)
-        self.ws = dsa.workspace(dsa.OP_ATTENTION_FORWARD, self.dims, self.cache)
+        self.ws = dsa.workspace(dsa.OP_ATTENTION_FORWARD_K8 if k8 else dsa.OP_ATTENTION_FORWARD,
+                                self.dims, self.cache)
         ld = max(4, (max(row_lengths(wl)) + 3) // 4 * 4)
         self.scores = torch.empty((wl.n_q, ld), dtype=torch.float32, device=dev)
         # the current tokens' own rows, to time the cache append without
@@ -230,13 +241,23 @@ class Case:
 
     def step(self):
         t = self.t
-        self.dsa.dsa_attention_forward(t["q_idx"], t["w"], t["k_pages"], t["q"], t["latent_pages"],
-                                       self.cache, self.dims, self.idx, self.out, self.lse, self.ws)
+        if self.k8:
+            self.dsa.dsa_attention_forward_k8(t["q_idx"], t["w"], t["k8_pages"], t["k_scale"],
+                                              t["q"], t["latent_pages"], self.cache, self.dims,
+                                              self.idx, self.out, self.lse, self.ws)
+        else:
+            self.dsa.dsa_attention_forward(t["q_idx"], t["w"], t["k_pages"], t["q"],
+                                           t["latent_pages"], self.cache, self.dims, self.idx,
+                                           self.out, self.lse, self.ws)
 
     def indexer(self):
         t = self.t
-        self.dsa.dsa_indexer_scores(t["q_idx"], t["w"], t["k_pages"], self.cache, self.dims,
-                                    self.scores, self.ws)
+        if self.k8:
+            self.dsa.dsa_indexer_scores_k8(t["q_idx"], t["w"], t["k8_pages"], t["k_scale"],
+                                           self.cache, self.dims, self.scores, self.ws)
+        else:
+            self.dsa.dsa_indexer_scores(t["q_idx"], t["w"], t["k_pages"], self.cache, self.dims,
+                                        self.scores, self.ws)
 
     def append(self):
         t = self.t
@@ -303,9 +324,9 @@ def timed_events(torch, fn, steps, warmup, flush_buf):
     return sum(times) / len(times), times
 
 
-def measure(case, torch, steps, warmup, flush_buf, peaks):
+def measure(case, torch, steps, warmup, flush_buf, peaks, extras=True):
     wl = case.wl
-    alg = algorithmic(wl)
+    alg = algorithmic(wl, case.k8)
     ms, _ = timed_events(torch, case.step, steps, warmup, flush_buf)
     st, info = case.dsa.workspace_check(case.ws)
     if st != 0:
@@ -314,21 +335,13 @@ def measure(case, torch, steps, warmup, flush_buf, peaks):
     ms_idx, _ = timed_events(torch, case.indexer, steps, warmup, flush_buf)
     ms_topk, _ = timed_events(torch, case.topk, steps, warmup, flush_buf)
     ms_mla, _ = timed_events(torch, case.mla, steps, warmup, flush_buf)
-    # the cache append in front of the step and the absorption GEMMs around it
-    # (separate entry points, not in the step)
-    ms_app, _ = timed_events(torch, case.append, steps, warmup, flush_buf)
-    ms_abs, _ = timed_events(torch, case.absorb, steps, warmup, flush_buf)
-    ms_prj, _ = timed_events(torch, case.project, steps, warmup, flush_buf)
-    st, info = case.dsa.workspace_check(case.sws)
-    if st != 0:
-        raise RuntimeError(f"device status {st} ({info:#x}) in the absorption GEMMs of {wl.name}")
-    ab, af, pb, pf = case.absorb_bytes_flops()
     st, info = case.dsa.workspace_check(case.ws)
     if st != 0:
         raise RuntimeError(f"device status {st} ({info:#x}) in the stage timings of {wl.name}")
     s = ms * 1e-3
     res = {
-        "workload": wl.name, "mode": wl.mode, "us_per_step": ms * 1e3,
+        "workload": wl.name, "mode": wl.mode, "index_keys": "e4m3+scale" if case.k8 else "bf16",
+        "us_per_step": ms * 1e3,
         "tokens_per_s": wl.n_q / s,
         "alg_bytes": alg["bytes"], "alg_gbs": alg["bytes"] / s / 1e9,
         "frac_of_8tbs": alg["bytes"] / s / 1e9 / NOMINAL_HBM_GBS,
@@ -343,6 +356,19 @@ def measure(case, torch, steps, warmup, flush_buf, peaks):
         "stage_us": {"indexer": ms_idx * 1e3, "topk": ms_topk * 1e3, "mla": ms_mla * 1e3},
         "stage_alg_bytes": {"indexer": alg["bytes_indexer"], "topk": alg["bytes_topk"],
                             "mla": alg["bytes_mla"]},
+    }
+    if not extras:
+        return res
+    # the cache append in front of the step and the absorption GEMMs around it
+    # (separate entry points, not in the step)
+    ms_app, _ = timed_events(torch, case.append, steps, warmup, flush_buf)
+    ms_abs, _ = timed_events(torch, case.absorb, steps, warmup, flush_buf)
+    ms_prj, _ = timed_events(torch, case.project, steps, warmup, flush_buf)
+    st, info = case.dsa.workspace_check(case.sws)
+    if st != 0:
+        raise RuntimeError(f"device status {st} ({info:#x}) in the absorption GEMMs of {wl.name}")
+    ab, af, pb, pf = case.absorb_bytes_flops()
+    res.update({
         "append_us": ms_app * 1e3,
         "append_alg_bytes": alg["bytes_append"],
         "append_gbs": alg["bytes_append"] / (ms_app * 1e-3) / 1e9,
@@ -350,7 +376,7 @@ def measure(case, torch, steps, warmup, flush_buf, peaks):
                          "tflops": af / (ms_abs * 1e-3) / 1e12},
         "project_values": {"us": ms_prj * 1e3, "alg_bytes": pb, "gbs": pb / (ms_prj * 1e-3) / 1e9,
                            "tflops": pf / (ms_prj * 1e-3) / 1e12},
-    }
+    })
     return res
 
 
@@ -393,7 +419,7 @@ STAGE_KERNELS = {"indexer": "indexer_kernel (tcgen05 + TMA)",
                  "mla": "mla_kernel + combine_kernel (tcgen05 + TMA gather4, split merge)"}
 
 
-def roofline_of(res, wl, peaks):
+def roofline_of(res, wl, peaks, k8=False):
     """Roofline of the stage that takes the longest alone: algorithmic bytes
     (or flops, for the tensor-bound prefill MLA) over its event time."""
     stage = max(res["stage_us"], key=res["stage_us"].get)
@@ -403,14 +429,16 @@ def roofline_of(res, wl, peaks):
         achieved = alg["flops_mla"] / (us * 1e-6) / 1e12
         return {"kernel": STAGE_KERNELS[stage], "stage": stage, "bound": "tensor",
                 "achieved": achieved, "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
-                "frac": achieved / peaks["bf16_tflops"], "traffic": traffic_of(stage, wl.name),
+                "frac": achieved / peaks["bf16_tflops"],
+                "traffic": None if k8 else traffic_of(stage, wl.name),
                 "peak_source": peaks["source"], "alg_flops_per_launch": alg["flops_mla"],
                 "launch_us": us}
     b = res["stage_alg_bytes"][stage]
     achieved = b / (us * 1e-6) / 1e9
     return {"kernel": STAGE_KERNELS[stage], "stage": stage, "bound": "hbm",
             "achieved": achieved, "peak": peaks["hbm_gbs"], "unit": "GB/s",
-            "frac": achieved / peaks["hbm_gbs"], "traffic": traffic_of(stage, wl.name),
+            "frac": achieved / peaks["hbm_gbs"],
+            "traffic": None if k8 else traffic_of(stage, wl.name),
             "peak_source": peaks["source"], "alg_bytes_per_launch": b, "launch_us": us}
 
 
@@ -535,6 +563,16 @@ def run_ours(args):
             r["us_per_step"] = max_over_ranks(r["us_per_step"], pg, "cuda")
             r["roofline"] = roofline_of(r, c.wl, peaks)
             per_config[name] = r
+            del c
+            torch.cuda.empty_cache()
+        for name in EXTRA_K8:
+            c = Case(replica_workload(di.CONFIGS[name], rank), torch, dsa, k8=True)
+            c.step()
+            torch.cuda.synchronize()
+            r = measure(c, torch, args.steps, args.warmup, flush_buf, peaks, extras=False)
+            r["us_per_step"] = max_over_ranks(r["us_per_step"], pg, "cuda")
+            r["roofline"] = roofline_of(r, c.wl, peaks, k8=True)
+            per_config[name + "+fp8_keys"] = r
             del c
             torch.cuda.empty_cache()
 

@@ -181,3 +181,23 @@ def small_prefill(T, *, q_pos0=0, H_I=4, D_I=32, topk=64, H=8, R=64, P=16, seed=
 __all__ = ["Workload", "CONFIGS", "CONFIG_ORDER", "make_inputs", "f32_to_bf16_bits",
            "small_decode", "small_prefill", "ragged_lengths", "pages_needed", "PAGE_SIZE",
            "replace", "field"]
+
+
+def with_fp8_keys(inp: dict, seed: int = 0, max_shift: int = 7) -> dict:
+    """The same inputs with the index-key cache held as E4M3 bytes plus one
+    fp32 scale per token: each token's integer key k is stored as the codes of
+    k * 2^j and the scale 2^-j, j drawn per token in [0, max_shift] (seeded),
+    so the keys the codes stand for are the original ones exactly.  The codes
+    come from torch's float8_e4m3fn conversion (exact for these values)."""
+    import torch
+    k = (inp["k_pages"].astype(np.uint32) << 16).view(np.float32)   # bf16 -> f32, exact
+    if not np.array_equal(k, np.round(k)) or np.abs(k).max() * 2 ** max_shift > 448:
+        raise ValueError("FP8 key inputs need integer keys within E4M3 range")
+    rng = np.random.default_rng(np.random.PCG64([seed, 0xF8]))
+    j = rng.integers(0, max_shift + 1, k.shape[:2])                # one shift per token
+    scaled = k * np.exp2(j)[..., None].astype(np.float32)
+    codes = torch.from_numpy(np.ascontiguousarray(scaled)).to(torch.float8_e4m3fn).view(torch.uint8)
+    out = dict(inp)
+    out["k8_pages"] = codes.numpy()
+    out["k_scale"] = np.exp2(-j).astype(np.float32).reshape(-1)
+    return out

@@ -114,7 +114,9 @@ typedef enum {
   DSA_OP_SPARSE_MLA_DECODE = 2,
   DSA_OP_SPARSE_MLA_PREFILL = 3,
   DSA_OP_ATTENTION_FORWARD = 4,
-  DSA_OP_CACHE_APPEND = 5
+  DSA_OP_CACHE_APPEND = 5,
+  DSA_OP_INDEXER_SCORES_K8 = 6,   /* dsa_indexer_scores_k8 */
+  DSA_OP_ATTENTION_FORWARD_K8 = 7 /* dsa_attention_forward_k8 */
 } dsa_op_t;
 
 /* Library version (major * 10000 + minor * 100 + patch). */
@@ -194,6 +196,37 @@ DSA_API dsa_status_t dsa_attention_forward(const uint16_t *q_idx, const float *w
                                    const uint16_t *latent_pages, const dsa_cache_t *cache,
                                    const dsa_dims_t *dims, int32_t *idx_out, float *out,
                                    float *lse, void *ws, size_t ws_bytes, dsa_stream_t stream);
+
+/* FP8 index keys: the indexer, and the whole step, over an index-key cache
+ * held as E4M3 bytes with one fp32 scale per token ("GLM on an A100, in Vx",
+ * section "INT4, FP8 and BF16": E4M3 bytes with a float32 scale per block;
+ * here a block is one token's key).  Key s of a page is dequantized as
+ * k_scale[row] * e4m3(k8_pages[row, :]) with row = page * 64 + slot, so
+ *   score[r, s] = k_scale[row(s)] * sum_h w[r, h] * max(0, q_idx[r, h] . e4m3(k8[row(s)]))
+ * (the scale is taken out of the ReLU and the head sum; a scale must be > 0).
+ *   k8_pages  [num_pages, 64, D_I] uint8 E4M3 codes (sign, 4 exponent bits with
+ *             bias 7, 3 mantissa bits; 0x7F / 0xFF are NaN), 16-byte aligned
+ *   k_scale   [num_pages * 64] fp32
+ * Everything else as dsa_indexer_scores / dsa_attention_forward; workspaces
+ * from dsa_workspace_bytes(DSA_OP_INDEXER_SCORES_K8 / _ATTENTION_FORWARD_K8).
+ * D_I must be 128.  The tensor cores multiply the keys as E4M3 (half the
+ * bytes and MMA time of bf16 keys); the query enters as two E4M3 terms,
+ * q * 2^s = hi + lo, s a power-of-two scale per (row, head) folded into w, so
+ * a query element is carried exactly unless it is nonzero and below about
+ * 2^-11 of its head's largest magnitude (then to a multiple of 2^(-9 - s)).
+ * Scores are exact whenever the bf16 path's would be, the query elements are
+ * so carried and every key scale is a power of two. */
+DSA_API dsa_status_t dsa_indexer_scores_k8(const uint16_t *q_idx, const float *w,
+                                   const uint8_t *k8_pages, const float *k_scale,
+                                   const dsa_cache_t *cache, const dsa_dims_t *dims,
+                                   float *scores, int64_t ld, void *ws, size_t ws_bytes,
+                                   dsa_stream_t stream);
+DSA_API dsa_status_t dsa_attention_forward_k8(const uint16_t *q_idx, const float *w,
+                                      const uint8_t *k8_pages, const float *k_scale,
+                                      const uint16_t *q, const uint16_t *latent_pages,
+                                      const dsa_cache_t *cache, const dsa_dims_t *dims,
+                                      int32_t *idx_out, float *out, float *lse, void *ws,
+                                      size_t ws_bytes, dsa_stream_t stream);
 
 /* Cache append: write the new tokens' index keys and latent rows into the
  * paged caches, the step in front of the indexer ("Self-contained GLM-5

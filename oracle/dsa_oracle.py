@@ -61,6 +61,28 @@ def bf16_to_f64(bits: np.ndarray) -> np.ndarray:
     return (bits.astype(np.uint32) << 16).view(np.float32).astype(np.float64)
 
 
+def e4m3_to_f64(codes: np.ndarray) -> np.ndarray:
+    """Widen E4M3 bytes to float64 exactly ("GLM on an A100, in Vx", section
+    "INT4, FP8 and BF16": E4M3 bytes).  Bit 7 is the sign, bits 6..3 the
+    exponent with bias 7, bits 2..0 the mantissa; exponent 0 holds subnormals
+    (m / 8 * 2^-6); exponent 15 with mantissa 7 is NaN (there is no infinity).
+    """
+    c = np.asarray(codes, dtype=np.uint8).astype(np.int64)
+    sign = np.where(c & 0x80, -1.0, 1.0)
+    e = (c >> 3) & 0xF
+    m = (c & 0x7).astype(np.float64)
+    normal = (1.0 + m / 8.0) * np.exp2(e - 7.0)
+    sub = (m / 8.0) * 2.0 ** -6
+    v = sign * np.where(e == 0, sub, normal)
+    return np.where((e == 15) & ((c & 0x7) == 7), np.nan, v)
+
+
+def dequantize_keys(k8_rows: np.ndarray, scale_rows: np.ndarray) -> np.ndarray:
+    """Index keys from E4M3 codes [n, D_I] and one fp32 scale per token [n]:
+    the FP8 format the pages describe, with a block of one token's key."""
+    return np.asarray(scale_rows, np.float64).reshape(-1, 1) * e4m3_to_f64(k8_rows)
+
+
 # --------------------------------------------------------------------------
 # paged cache lookup
 # --------------------------------------------------------------------------
@@ -264,7 +286,13 @@ def dsa_query(q_idx, w, k_rows, q, latent_of, k: int, R: int, scale: float):
 
 
 def _query_row(inp, r, table_row, n):
-    k_rows = bf16_to_f64(gather_paged_rows(inp["k_pages"], table_row, np.arange(n)))
+    if "k8_pages" in inp:   # FP8 index keys with one scale per token
+        codes = gather_paged_rows(inp["k8_pages"], table_row, np.arange(n))
+        scales = gather_paged_rows(np.asarray(inp["k_scale"]).reshape(-1, PAGE_SIZE, 1), table_row,
+                                   np.arange(n))
+        k_rows = dequantize_keys(codes, scales)
+    else:
+        k_rows = bf16_to_f64(gather_paged_rows(inp["k_pages"], table_row, np.arange(n)))
 
     def latent_of(sel):
         return bf16_to_f64(gather_paged_rows(inp["latent_pages"], table_row, sel))

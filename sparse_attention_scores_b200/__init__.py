@@ -28,6 +28,8 @@ OP_SPARSE_MLA_DECODE = 2
 OP_SPARSE_MLA_PREFILL = 3
 OP_ATTENTION_FORWARD = 4
 OP_CACHE_APPEND = 5
+OP_INDEXER_SCORES_K8 = 6
+OP_ATTENTION_FORWARD_K8 = 7
 
 STATUS_NAMES = {0: "DSA_OK", 1: "DSA_ERR_INVALID_ARG", 2: "DSA_ERR_UNSUPPORTED",
                 3: "DSA_ERR_CUDA", 4: "DSA_ERR_WORKSPACE", 5: "DSA_ERR_TIMEOUT",
@@ -36,7 +38,8 @@ STATUS_NAMES = {0: "DSA_OK", 1: "DSA_ERR_INVALID_ARG", 2: "DSA_ERR_UNSUPPORTED",
 EXPORTED = ["dsa_version", "dsa_status_string", "dsa_workspace_bytes", "dsa_workspace_init",
             "dsa_workspace_check", "dsa_indexer_scores", "dsa_topk", "dsa_sparse_mla_decode",
             "dsa_sparse_mla_prefill", "dsa_attention_forward", "dsa_sparse_mla_decode_noalloc",
-            "dsa_cache_append", "dsa_absorb_query", "dsa_project_values"]
+            "dsa_cache_append", "dsa_absorb_query", "dsa_project_values",
+            "dsa_indexer_scores_k8", "dsa_attention_forward_k8"]
 
 
 class DsaError(RuntimeError):
@@ -90,6 +93,9 @@ def lib() -> ctypes.CDLL:
             "dsa_absorb_query": ([vp, vp, vp, vp, i32, i32, i32, i32, i32, vp, sz, vp],
                                  ctypes.c_int),
             "dsa_project_values": ([vp, vp, vp, i32, i32, i32, i32, vp, sz, vp], ctypes.c_int),
+            "dsa_indexer_scores_k8": ([vp, vp, vp, vp, pc, pd, vp, i64, vp, sz, vp], ctypes.c_int),
+            "dsa_attention_forward_k8": ([vp, vp, vp, vp, vp, vp, pc, pd, vp, vp, vp, vp, sz, vp],
+                                         ctypes.c_int),
         }
         for name, (args, res) in sigs.items():
             fn = getattr(L, name)
@@ -262,3 +268,23 @@ def dsa_project_values(o_lat, w_uv, v_out, ws, stream=None) -> None:
     _check(lib().dsa_project_values(_ptr(o_lat), _ptr(w_uv), _ptr(v_out), n, H, R, d_v,
                                     _ptr(ws), ws.numel(), _stream(stream)),
            "dsa_project_values")
+
+
+def dsa_indexer_scores_k8(q_idx, w, k8_pages, k_scale, cache: PagedCache, dims: Dims, scores, ws,
+                          stream=None) -> None:
+    """dsa_indexer_scores over E4M3 index keys [pages, 64, D_I] (uint8) with one
+    fp32 scale per key row [pages * 64]."""
+    _check(lib().dsa_indexer_scores_k8(_ptr(q_idx), _ptr(w), _ptr(k8_pages), _ptr(k_scale),
+                                       ctypes.byref(cache.struct()), ctypes.byref(dims.struct()),
+                                       _ptr(scores), int(scores.stride(0)), _ptr(ws), ws.numel(),
+                                       _stream(stream)), "dsa_indexer_scores_k8")
+
+
+def dsa_attention_forward_k8(q_idx, w, k8_pages, k_scale, q, latent_pages, cache: PagedCache,
+                             dims: Dims, idx_out, out, lse, ws, stream=None) -> None:
+    """dsa_attention_forward with the index-key cache as E4M3 bytes plus scales."""
+    _check(lib().dsa_attention_forward_k8(_ptr(q_idx), _ptr(w), _ptr(k8_pages), _ptr(k_scale),
+                                          _ptr(q), _ptr(latent_pages), ctypes.byref(cache.struct()),
+                                          ctypes.byref(dims.struct()), _ptr(idx_out), _ptr(out),
+                                          _ptr(lse), _ptr(ws), ws.numel(), _stream(stream)),
+           "dsa_attention_forward_k8")

@@ -96,6 +96,22 @@ bool make_map_2d(CUtensorMap *map, const void *base, uint64_t cols, uint64_t row
   return r == CUDA_SUCCESS;
 }
 
+// bytes (the FP8 index keys and query terms); aw = swizzle width, 128 or 64
+bool make_map_2d_u8(CUtensorMap *map, const void *base, uint64_t cols, uint64_t rows,
+                    uint32_t box_cols, uint32_t box_rows, int aw) {
+  auto encode = get_encode_fn();
+  if (encode == nullptr) return false;
+  cuuint64_t dims[2] = {cols, rows};
+  cuuint64_t strides[1] = {cols};
+  cuuint32_t box[2] = {box_cols, box_rows};
+  cuuint32_t estr[2] = {1, 1};
+  CUresult r = encode(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void *>(base), dims,
+                      strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                      aw == 128 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_64B,
+                      CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
 size_t device_smem_per_sm() {
   static size_t cached[kMaxDevices];
   const int d = current_device();
@@ -189,12 +205,25 @@ dsa_status_t check_ws(void *ws, size_t ws_bytes, size_t need) {
     if (st__ != DSA_OK) return st__;         \
   } while (0)
 
+// FP8-key indexer region after the status block: the E4M3 query terms
+// [2][n_q][H_I][D_I] bytes, then the scaled head weights [n_q][H_I] fp32
+size_t k8_q_bytes(const dsa_dims_t &d) {
+  return align256(2 * static_cast<size_t>(d.n_q) * d.H_I * d.D_I);
+}
+size_t k8_region_bytes(const dsa_dims_t &d) {
+  return k8_q_bytes(d) + align256(static_cast<size_t>(d.n_q) * d.H_I * 4);
+}
+
 size_t ws_bytes_for(dsa_op_t op, const dsa_dims_t &d, const dsa_cache_t &c) {
   switch (op) {
     case DSA_OP_INDEXER_SCORES:
     case DSA_OP_TOPK:
     case DSA_OP_CACHE_APPEND:
       return kStatusBytes;
+    case DSA_OP_INDEXER_SCORES_K8:
+      return kStatusBytes + k8_region_bytes(d);
+    case DSA_OP_ATTENTION_FORWARD_K8:
+      return k8_region_bytes(d) + ws_bytes_for(DSA_OP_ATTENTION_FORWARD, d, c);
     case DSA_OP_SPARSE_MLA_DECODE:
     case DSA_OP_SPARSE_MLA_PREFILL:
       return kStatusBytes + align256(mla_scratch_bytes(d.n_q, d.topk, d.R));
@@ -208,13 +237,26 @@ size_t ws_bytes_for(dsa_op_t op, const dsa_dims_t &d, const dsa_cache_t &c) {
   return 0;
 }
 
+// k8_pages != nullptr: E4M3 index keys with one fp32 scale per key row
+// (k_scale); k8_region (k8_region_bytes) receives the E4M3 query terms and the
+// scaled head weights
 dsa_status_t run_indexer(const uint16_t *q_idx, const float *w, const uint16_t *k_pages,
                          const dsa_cache_t &c, const dsa_dims_t &d, float *scores, int64_t ld,
-                         DevStatus *st, cudaStream_t s) {
+                         DevStatus *st, cudaStream_t s, const uint8_t *k8_pages = nullptr,
+                         const float *k_scale = nullptr, uint8_t *k8_region = nullptr) {
   IndexerLaunch a;
   a.q_idx = q_idx;
   a.w = w;
   a.k_pages = k_pages;
+  a.k8_pages = k8_pages;
+  a.k_scale = k_scale;
+  if (k8_pages != nullptr) {
+    uint8_t *q8 = k8_region;
+    float *w8 = reinterpret_cast<float *>(k8_region + k8_q_bytes(d));
+    DSA_TRY(launch_q8_prep(q_idx, w, q8, w8, d.n_q, d.H_I, d.D_I, s));
+    a.q8 = q8;
+    a.w = w8;
+  }
   a.seq_lens = c.seq_lens;
   a.block_table = c.block_table;
   a.scores = scores;
@@ -297,6 +339,16 @@ dsa_status_t mla_entry(const uint16_t *q, const uint16_t *latent_pages, const ds
                  as_stream(stream));
 }
 
+dsa_status_t indexer_entry(const uint16_t *q_idx, const float *w, const uint16_t *k_idx_pages,
+                           const uint8_t *k8_pages, const float *k_scale, const dsa_cache_t *cache,
+                           const dsa_dims_t *dims, float *scores, int64_t ld, void *ws,
+                           size_t ws_bytes, dsa_stream_t stream);
+dsa_status_t forward_entry(const uint16_t *q_idx, const float *w, const uint16_t *k_idx_pages,
+                           const uint8_t *k8_pages, const float *k_scale, const uint16_t *q,
+                           const uint16_t *latent_pages, const dsa_cache_t *cache,
+                           const dsa_dims_t *dims, int32_t *idx_out, float *out, float *lse,
+                           void *ws, size_t ws_bytes, dsa_stream_t stream);
+
 }  // namespace
 }  // namespace dsa
 
@@ -323,8 +375,10 @@ size_t dsa_workspace_bytes(dsa_op_t op, const dsa_dims_t *dims, const dsa_cache_
   if (check_dims_common(dims) != DSA_OK) return 0;
   if (op == DSA_OP_INDEXER_SCORES || op == DSA_OP_TOPK || op == DSA_OP_CACHE_APPEND)
     return kStatusBytes;
+  if (op == DSA_OP_INDEXER_SCORES_K8) return ws_bytes_for(op, *dims, dsa_cache_t{});
   if (check_mla_dims(*dims) != DSA_OK) return 0;
-  if (op == DSA_OP_ATTENTION_FORWARD && (cache == nullptr || check_cache(cache, *dims) != DSA_OK))
+  if ((op == DSA_OP_ATTENTION_FORWARD || op == DSA_OP_ATTENTION_FORWARD_K8) &&
+      (cache == nullptr || check_cache(cache, *dims) != DSA_OK))
     return 0;
   dsa_cache_t empty = {};
   return ws_bytes_for(op, *dims, cache ? *cache : empty);
@@ -352,18 +406,17 @@ dsa_status_t dsa_workspace_check(const void *ws, dsa_stream_t stream, uint32_t *
 dsa_status_t dsa_indexer_scores(const uint16_t *q_idx, const float *w, const uint16_t *k_idx_pages,
                                 const dsa_cache_t *cache, const dsa_dims_t *dims, float *scores,
                                 int64_t ld, void *ws, size_t ws_bytes, dsa_stream_t stream) {
-  DSA_TRY(check_dims_common(dims));
-  DSA_TRY(check_indexer_dims(*dims));
-  DSA_TRY(check_cache(cache, *dims));
-  if (q_idx == nullptr || w == nullptr || k_idx_pages == nullptr || scores == nullptr)
-    return DSA_ERR_INVALID_ARG;
-  if (!aligned16(q_idx) || !aligned16(k_idx_pages) || !aligned16(scores) || !aligned4(w))
-    return DSA_ERR_INVALID_ARG;
-  if (ld < max_keys(*dims, *cache) || ld % 4 != 0 || ld <= 0) return DSA_ERR_INVALID_ARG;
-  DSA_TRY(check_ws(ws, ws_bytes, kStatusBytes));
-  if (dims->n_q == 0) return DSA_OK;
-  return run_indexer(q_idx, w, k_idx_pages, *cache, *dims, scores, ld, status_of(ws),
-                     as_stream(stream));
+  return indexer_entry(q_idx, w, k_idx_pages, nullptr, nullptr, cache, dims, scores, ld, ws,
+                       ws_bytes, stream);
+}
+
+dsa_status_t dsa_indexer_scores_k8(const uint16_t *q_idx, const float *w, const uint8_t *k8_pages,
+                                   const float *k_scale, const dsa_cache_t *cache,
+                                   const dsa_dims_t *dims, float *scores, int64_t ld, void *ws,
+                                   size_t ws_bytes, dsa_stream_t stream) {
+  if (k8_pages == nullptr || k_scale == nullptr) return DSA_ERR_INVALID_ARG;
+  return indexer_entry(q_idx, w, nullptr, k8_pages, k_scale, cache, dims, scores, ld, ws,
+                       ws_bytes, stream);
 }
 
 dsa_status_t dsa_topk(const float *scores, int64_t ld, int32_t n_q, const int32_t *valid_len,
@@ -403,38 +456,100 @@ dsa_status_t dsa_attention_forward(const uint16_t *q_idx, const float *w,
                                    const uint16_t *latent_pages, const dsa_cache_t *cache,
                                    const dsa_dims_t *dims, int32_t *idx_out, float *out,
                                    float *lse, void *ws, size_t ws_bytes, dsa_stream_t stream) {
+  return forward_entry(q_idx, w, k_idx_pages, nullptr, nullptr, q, latent_pages, cache, dims,
+                       idx_out, out, lse, ws, ws_bytes, stream);
+}
+
+dsa_status_t dsa_attention_forward_k8(const uint16_t *q_idx, const float *w,
+                                      const uint8_t *k8_pages, const float *k_scale,
+                                      const uint16_t *q, const uint16_t *latent_pages,
+                                      const dsa_cache_t *cache, const dsa_dims_t *dims,
+                                      int32_t *idx_out, float *out, float *lse, void *ws,
+                                      size_t ws_bytes, dsa_stream_t stream) {
+  if (k8_pages == nullptr || k_scale == nullptr) return DSA_ERR_INVALID_ARG;
+  return forward_entry(q_idx, w, nullptr, k8_pages, k_scale, q, latent_pages, cache, dims,
+                       idx_out, out, lse, ws, ws_bytes, stream);
+}
+
+}  // extern "C"
+
+namespace dsa {
+namespace {
+
+// the indexer entry for bf16 keys (k_idx_pages) or E4M3 keys (k8_pages + k_scale)
+dsa_status_t indexer_entry(const uint16_t *q_idx, const float *w, const uint16_t *k_idx_pages,
+                           const uint8_t *k8_pages, const float *k_scale, const dsa_cache_t *cache,
+                           const dsa_dims_t *dims, float *scores, int64_t ld, void *ws,
+                           size_t ws_bytes, dsa_stream_t stream) {
+  DSA_TRY(check_dims_common(dims));
+  DSA_TRY(check_indexer_dims(*dims));
+  DSA_TRY(check_cache(cache, *dims));
+  const void *keys = k8_pages ? static_cast<const void *>(k8_pages) : k_idx_pages;
+  if (q_idx == nullptr || w == nullptr || keys == nullptr || scores == nullptr)
+    return DSA_ERR_INVALID_ARG;
+  if (!aligned16(q_idx) || !aligned16(keys) || !aligned16(scores) || !aligned4(w) ||
+      (k_scale && !aligned4(k_scale)))
+    return DSA_ERR_INVALID_ARG;
+  if (k8_pages && dims->D_I != 128) return DSA_ERR_UNSUPPORTED;
+  if (ld < max_keys(*dims, *cache) || ld % 4 != 0 || ld <= 0) return DSA_ERR_INVALID_ARG;
+  DSA_TRY(check_ws(ws, ws_bytes,
+                   k8_pages ? ws_bytes_for(DSA_OP_INDEXER_SCORES_K8, *dims, *cache) : kStatusBytes));
+  if (dims->n_q == 0) return DSA_OK;
+  return run_indexer(q_idx, w, k_idx_pages, *cache, *dims, scores, ld, status_of(ws),
+                     as_stream(stream), k8_pages, k_scale, static_cast<uint8_t *>(ws) + kStatusBytes);
+}
+
+// the whole step for bf16 keys (k_idx_pages) or E4M3 keys (k8_pages + k_scale)
+dsa_status_t forward_entry(const uint16_t *q_idx, const float *w, const uint16_t *k_idx_pages,
+                           const uint8_t *k8_pages, const float *k_scale, const uint16_t *q,
+                           const uint16_t *latent_pages, const dsa_cache_t *cache,
+                           const dsa_dims_t *dims, int32_t *idx_out, float *out, float *lse,
+                           void *ws, size_t ws_bytes, dsa_stream_t stream) {
   DSA_TRY(check_dims_common(dims));
   DSA_TRY(check_indexer_dims(*dims));
   DSA_TRY(check_mla_dims(*dims));
   DSA_TRY(check_cache(cache, *dims));
-  if (q_idx == nullptr || w == nullptr || k_idx_pages == nullptr || q == nullptr ||
+  const void *keys = k8_pages ? static_cast<const void *>(k8_pages) : k_idx_pages;
+  if (q_idx == nullptr || w == nullptr || keys == nullptr || q == nullptr ||
       latent_pages == nullptr || out == nullptr || lse == nullptr)
     return DSA_ERR_INVALID_ARG;
-  if (!aligned16(q_idx) || !aligned16(k_idx_pages) || !aligned16(q) || !aligned16(latent_pages) ||
-      !aligned4(w) || !aligned4(out) || !aligned4(lse) || (idx_out && !aligned4(idx_out)))
+  if (!aligned16(q_idx) || !aligned16(keys) || !aligned16(q) || !aligned16(latent_pages) ||
+      !aligned4(w) || !aligned4(out) || !aligned4(lse) || (idx_out && !aligned4(idx_out)) ||
+      (k_scale && !aligned4(k_scale)))
     return DSA_ERR_INVALID_ARG;
+  if (k8_pages && dims->D_I != 128) return DSA_ERR_UNSUPPORTED;
   const dsa_dims_t &d = *dims;
   const dsa_cache_t &c = *cache;
-  DSA_TRY(check_ws(ws, ws_bytes, ws_bytes_for(DSA_OP_ATTENTION_FORWARD, d, c)));
+  DSA_TRY(check_ws(ws, ws_bytes,
+                   ws_bytes_for(k8_pages ? DSA_OP_ATTENTION_FORWARD_K8 : DSA_OP_ATTENTION_FORWARD,
+                                d, c)));
   if (d.n_q == 0) return DSA_OK;
 
-  uint8_t *base = static_cast<uint8_t *>(ws);
+  // FP8 keys: the query terms right after the status block, the rest shifted
+  uint8_t *k8_region = static_cast<uint8_t *>(ws) + kStatusBytes;
+  uint8_t *base = static_cast<uint8_t *>(ws) + (k8_pages ? k8_region_bytes(d) : 0);
   DevStatus *st = status_of(ws);
   const int64_t ld = scores_ld(d, c);
   float *scores = reinterpret_cast<float *>(base + kStatusBytes);
   int32_t *idx_ws = reinterpret_cast<int32_t *>(
       base + kStatusBytes + align256(static_cast<size_t>(d.n_q) * ld * 4));
   uint8_t *scratch = reinterpret_cast<uint8_t *>(idx_ws) + align256(static_cast<size_t>(d.n_q) * d.topk * 4);
-  const size_t scratch_bytes = ws_bytes - static_cast<size_t>(scratch - base);
+  const size_t scratch_bytes = ws_bytes - static_cast<size_t>(scratch - static_cast<uint8_t *>(ws));
   int32_t *idx = idx_out ? idx_out : idx_ws;
   cudaStream_t s = as_stream(stream);
 
-  DSA_TRY(run_indexer(q_idx, w, k_idx_pages, c, d, scores, ld, st, s));
+  DSA_TRY(run_indexer(q_idx, w, k_idx_pages, c, d, scores, ld, st, s, k8_pages, k_scale,
+                      k8_region));
   DSA_TRY(run_topk(scores, ld, d.n_q, d.causal ? nullptr : c.seq_lens, d.q_pos0, d.topk, idx,
                    static_cast<int>(max_keys(d, c)), st, s));
   return run_mla(q, latent_pages, c, idx, d, out, lse, scratch, scratch_bytes, st, s,
                  /*early_q=*/1);
 }
+
+}  // namespace
+}  // namespace dsa
+
+extern "C" {
 
 dsa_status_t dsa_cache_append(const uint16_t *k_idx_new, const uint16_t *latent_new,
                               uint16_t *k_idx_pages, uint16_t *latent_pages,

@@ -29,6 +29,8 @@ int device_sm_count();
 // bytes) with a box of box_cols x box_rows and a 128- (aw = 128) or 64-byte
 // (aw = 64) swizzle.  Returns false when the driver entry point is missing or
 // rejects the request.
+bool make_map_2d_u8(CUtensorMap *map, const void *base, uint64_t cols, uint64_t rows,
+                    uint32_t box_cols, uint32_t box_rows, int aw);
 bool make_map_2d(CUtensorMap *map, const void *base, uint64_t cols, uint64_t rows,
                  uint32_t box_cols, uint32_t box_rows, int aw);
 
@@ -66,6 +68,9 @@ struct IndexerLaunch {
   const uint16_t *q_idx;
   const float *w;
   const uint16_t *k_pages;
+  const uint8_t *k8_pages = nullptr;  // E4M3 keys instead of k_pages (with k_scale)
+  const float *k_scale = nullptr;     // per physical key row
+  const uint8_t *q8 = nullptr;        // K8: E4M3 query terms [2][n_q][H_I][D_I] (w = scaled weights)
   const int32_t *seq_lens;
   const int32_t *block_table;
   float *scores;
@@ -75,6 +80,9 @@ struct IndexerLaunch {
   DevStatus *status;
 };
 dsa_status_t launch_indexer(const IndexerLaunch &a, cudaStream_t stream);
+// the E4M3 query terms [2][n_q][H_I][D_I] and scaled weights [n_q][H_I] of the FP8-key indexer
+dsa_status_t launch_q8_prep(const uint16_t *q_idx, const float *w, uint8_t *q8, float *w8,
+                            int n_q, int H_I, int D_I, cudaStream_t stream);
 
 struct TopkLaunch {
   const float *scores;

@@ -22,9 +22,26 @@
 // Decode runs two CTAs per SM (one epilogue warpgroup each) so that one CTA's
 // pipeline bubbles are covered by the other; grouped prefill runs one CTA per
 // SM with two epilogue warpgroups.
+//
+// FP8 index keys (K8): the cache holds each key as E4M3 bytes with one fp32
+// scale per token ("GLM on an A100, in Vx", "INT4, FP8 and BF16": E4M3 bytes
+// with a float32 scale per block; here a block is one token's key).  The byte
+// pages go by TMA straight into the MMA's swizzled K-major layout and the
+// tensor cores multiply them as E4M3 (kind::f8f6f4, half the bytes and half
+// the MMA time of bf16 keys).  The bf16 queries enter as two E4M3 terms,
+// q * 2^s = hi + lo with a power-of-two scale s per head (a small kernel
+// before the indexer writes them, and folds 2^-s into the head weights); the
+// two terms accumulate into one fp32 accumulator.  hi + lo holds all eight
+// significant bits of a bf16 element unless the element is below about 2^-11
+// of its head's largest one.  The epilogue multiplies a key's score by its
+// scale, which commutes with the ReLU and the head sum because the scale is
+// positive.
 // Every wait is bounded in wall time; a time-out records an error in the
 // status block, drains what is in flight, frees tensor memory and returns.
 #include <algorithm>
+
+#include <cuda_fp16.h>
+#include <cuda_fp8.h>
 
 #include "dsa_internal.h"
 
@@ -35,6 +52,7 @@ namespace {
 // NEG = 1: two CTAs per SM, whose pipelines cover each other's bubbles)
 template <int NEG>
 __host__ __device__ constexpr int threads_of() { return 64 + 128 * NEG; }
+constexpr int kMaxStages = 8;
 constexpr int kMaxAcc = 8;         // accumulator buffers in tensor memory
 constexpr int kTileKeys = 128;
 constexpr int kLookahead = 16;  // units whose page ids the producer fetches at once
@@ -52,6 +70,7 @@ struct IndexerParams {
   int q_buffers;   // 1 or 2 query tiles in shared memory
   uint64_t wait_ns;
   int debug_stall;  // the MMA issuer first waits on a barrier nothing arrives at
+  const float *k_scale;  // K8: per physical key row [num_pages * 64]
   DevStatus *status;
 };
 
@@ -83,7 +102,7 @@ __device__ __forceinline__ int locate(const int *tile_start, int ng, int u) {
   return lo;
 }
 
-template <int G, int AW, int NEG>
+template <int G, int AW, int NEG, bool K8>
 __global__ void __launch_bounds__(threads_of<NEG>(), NEG == 1 ? 2 : 1)
     indexer_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmQ,
                    const IndexerParams p) {
@@ -93,11 +112,13 @@ __global__ void __launch_bounds__(threads_of<NEG>(), NEG == 1 ? 2 : 1)
                                               ~static_cast<uintptr_t>(1023));
   const int S = p.stages;
   const int nqb = p.q_buffers;
-  const int natoms = p.D_I * 2 / AW;            // swizzle atoms along K
-  const int stage_bytes = kTileKeys * p.D_I * 2;
+  constexpr int kEB = K8 ? 1 : 2;                // key / query bytes per element
+  const int natoms = p.D_I * kEB / AW;          // swizzle atoms along K
+  const int stage_bytes = kTileKeys * p.D_I * kEB;
   const int ncols = G * p.H_I;                  // useful accumulator columns
   const int n_mma = (ncols + 15) & ~15;         // MMA N (multiple of 16)
-  const int q_bytes = natoms * n_mma * AW;
+  // K8: the hi and lo query terms, each [n_mma rows][D_I bytes]
+  const int q_bytes = (K8 ? 2 : 1) * natoms * n_mma * AW;
   const uint32_t acc_stride = (n_mma + 31) & ~31;
   // as many accumulators as fit 512 columns (<= 8): the MMA warp runs that
   // many tiles ahead of the epilogue
@@ -108,9 +129,9 @@ __global__ void __launch_bounds__(threads_of<NEG>(), NEG == 1 ? 2 : 1)
   uint8_t *stage_base = smem;
   uint8_t *q_base = smem + S * stage_bytes;
   uint64_t *bars = reinterpret_cast<uint64_t *>(q_base + nqb * q_bytes);
-  uint64_t *full = bars;
-  uint64_t *empty = bars + S;
-  uint64_t *qfull = bars + 2 * S;
+  uint64_t *full = bars;                   // [S] key tile landed
+  uint64_t *empty = bars + kMaxStages;     // [S] key tile consumed by the MMA
+  uint64_t *qfull = bars + 2 * kMaxStages;
   uint64_t *qempty = qfull + 2;
   uint64_t *tfull = qempty + 2;
   uint64_t *tempty = tfull + kMaxAcc;
@@ -210,27 +231,36 @@ __global__ void __launch_bounds__(threads_of<NEG>(), NEG == 1 ? 2 : 1)
             if (!mbar_wait(&qempty[qslot], qphase ^ 1u, p.wait_ns)) {
               okl = 0;
             } else {
-              mbar_arrive_expect_tx(&qfull[qslot], static_cast<uint32_t>(natoms * ncols * AW));
-              for (int a = 0; a < natoms; ++a)
-                tma_load_2d(q_base + qslot * q_bytes + a * n_mma * AW, &tmQ, a * (AW / 2),
-                            g * ncols, &qfull[qslot]);
+              mbar_arrive_expect_tx(&qfull[qslot],
+                                    static_cast<uint32_t>((K8 ? 2 : 1) * natoms * ncols * AW));
+              if (K8) {
+                // hi plane rows [g * ncols, ...), lo plane rows n_q * H_I further on
+                uint8_t *qd = q_base + qslot * q_bytes;
+                tma_load_2d(qd, &tmQ, 0, g * ncols, &qfull[qslot]);
+                tma_load_2d(qd + n_mma * AW, &tmQ, 0, p.n_q * p.H_I + g * ncols, &qfull[qslot]);
+              } else {
+                for (int a = 0; a < natoms; ++a)
+                  tma_load_2d(q_base + qslot * q_bytes + a * n_mma * AW, &tmQ, a * (AW / 2),
+                              g * ncols, &qfull[qslot]);
+              }
             }
           }
           if (okl && !mbar_wait(&empty[stage], phase ^ 1u, p.wait_ns)) okl = 0;
           if (okl) {
-            const uint32_t page_bytes = kPageSize * p.D_I * 2;
+            const uint32_t page_bytes = kPageSize * p.D_I * kEB;
             const uint32_t bytes = ((id0 >= 0) + (id1 >= 0)) * page_bytes;
             uint8_t *dst = stage_base + stage * stage_bytes;
             if (bytes == 0) {
               mbar_arrive(&full[stage]);
             } else {
               mbar_arrive_expect_tx(&full[stage], bytes);
+              // an atom is AW bytes of a key row: AW / 2 bf16 or AW E4M3 elements
               for (int a = 0; a < natoms; ++a) {
                 if (id0 >= 0)
-                  tma_load_2d(dst + a * kTileKeys * AW, &tmK, a * (AW / 2), id0 * kPageSize,
+                  tma_load_2d(dst + a * kTileKeys * AW, &tmK, a * (AW / kEB), id0 * kPageSize,
                               &full[stage]);
                 if (id1 >= 0)
-                  tma_load_2d(dst + a * kTileKeys * AW + kPageSize * AW, &tmK, a * (AW / 2),
+                  tma_load_2d(dst + a * kTileKeys * AW + kPageSize * AW, &tmK, a * (AW / kEB),
                               id1 * kPageSize, &full[stage]);
               }
               armed |= 1u << stage;
@@ -260,7 +290,8 @@ __global__ void __launch_bounds__(threads_of<NEG>(), NEG == 1 ? 2 : 1)
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issuer
     if (lane == 0) {
-      const uint32_t idesc = idesc_bf16_f32(kTileKeys, n_mma, 0, 0);
+      const uint32_t idesc =
+          K8 ? idesc_e4m3_f32(kTileKeys, n_mma) : idesc_bf16_f32(kTileKeys, n_mma, 0, 0);
       int stage = 0, qslot = 0, cur = -1, cur_slot = 0;
       uint32_t phase = 0, qphase = 0;
       bool ok = true;
@@ -285,11 +316,24 @@ __global__ void __launch_bounds__(threads_of<NEG>(), NEG == 1 ? 2 : 1)
         const uint32_t d = tmem_base + acc * acc_stride;
         const uint32_t a_base = smem_u32(stage_base + stage * stage_bytes);
         const uint32_t b_base = smem_u32(q_base + cur_slot * q_bytes);
-        for (int a = 0; a < natoms; ++a) {
-          for (int kk = 0; kk < AW / 32; ++kk) {
-            const uint64_t adesc = smem_desc(a_base + a * kTileKeys * AW + kk * 32, 16, 8 * AW, layout);
-            const uint64_t bdesc = smem_desc(b_base + a * n_mma * AW + kk * 32, 16, 8 * AW, layout);
-            mma_bf16(d, adesc, bdesc, idesc, (a | kk) != 0 ? 1u : 0u);
+        if (K8) {
+          // E4M3 keys x (hi + lo) E4M3 query terms, 32 elements (32 bytes) per MMA
+          for (int term = 0; term < 2; ++term)
+            for (int a = 0; a < natoms; ++a)
+              for (int kk = 0; kk < AW / 32; ++kk) {
+                const uint64_t adesc =
+                    smem_desc(a_base + a * kTileKeys * AW + kk * 32, 16, 8 * AW, layout);
+                const uint64_t bdesc = smem_desc(
+                    b_base + term * natoms * n_mma * AW + a * n_mma * AW + kk * 32, 16, 8 * AW, layout);
+                mma_e4m3(d, adesc, bdesc, idesc, (term | a | kk) != 0 ? 1u : 0u);
+              }
+        } else {
+          for (int a = 0; a < natoms; ++a) {
+            for (int kk = 0; kk < AW / 32; ++kk) {
+              const uint64_t adesc = smem_desc(a_base + a * kTileKeys * AW + kk * 32, 16, 8 * AW, layout);
+              const uint64_t bdesc = smem_desc(b_base + a * n_mma * AW + kk * 32, 16, 8 * AW, layout);
+              mma_bf16(d, adesc, bdesc, idesc, (a | kk) != 0 ? 1u : 0u);
+            }
           }
         }
         mma_commit(&empty[stage]);
@@ -328,6 +372,19 @@ __global__ void __launch_bounds__(threads_of<NEG>(), NEG == 1 ? 2 : 1)
         for (int i = 0; i < 32; ++i)
           wreg[i] = (i < p.H_I) ? __ldg(p.w + static_cast<int64_t>(g) * p.H_I + i) : 0.f;
         wgroup = g;
+      }
+      // K8: this key's scale (its page id, then the scale), in flight while
+      // the accumulator is waited for
+      float kscale = 1.f;
+      if (K8) {
+        const int tt = u - tile_start[g];
+        const int pg = 2 * tt + (key_in_tile >> 6);
+        const int b = p.causal ? 0 : g;
+        if (pg < p.max_pages && pg * kPageSize < group_keys<G>(p, g)) {
+          const int id = __ldg(p.block_table + static_cast<int64_t>(b) * p.max_pages + pg);
+          if (id >= 0 && id < p.num_pages)
+            kscale = __ldg(p.k_scale + static_cast<int64_t>(id) * kPageSize + (key_in_tile & 63));
+        }
       }
       if (__any_sync(0xffffffffu, *abort_flag != 0u)) { ok = false; break; }
       if (!__all_sync(0xffffffffu, mbar_wait(&tfull[acc], aphase, p.wait_ns))) { ok = false; break; }
@@ -381,7 +438,8 @@ __global__ void __launch_bounds__(threads_of<NEG>(), NEG == 1 ? 2 : 1)
 #pragma unroll
       for (int j = 0; j < G; ++j) {
         const int r = p.causal ? g * G + j : g;
-        if (r < p.n_q && key < row_keys(p, r)) p.scores[static_cast<int64_t>(r) * p.ld + key] = s[j];
+        if (r < p.n_q && key < row_keys(p, r))
+          p.scores[static_cast<int64_t>(r) * p.ld + key] = K8 ? s[j] * kscale : s[j];
       }
     }
     if (!ok && lane == 0 && !*abort_flag) {
@@ -399,40 +457,102 @@ __global__ void __launch_bounds__(threads_of<NEG>(), NEG == 1 ? 2 : 1)
   }
 }
 
+// The E4M3 query terms of the FP8-key indexer: per (row, head), the power-of-
+// two scale 2^s that brings the largest |q| to at most 448 (the largest E4M3
+// value), q * 2^s = hi + lo with hi = E4M3(q * 2^s) and lo = E4M3 of the
+// remainder (both rounded to nearest even), and the head weight times 2^-s.
+// One warp per (row, head); D_I / 32 elements per lane.
+__global__ void __launch_bounds__(256) q8_prep_kernel(const uint16_t *q_idx, const float *w,
+                                                       uint8_t *q8, float *w8, int n_q, int H_I,
+                                                       int D_I) {
+  griddep_wait();
+  griddep_launch_dependents();
+  const int wid = blockIdx.x * 8 + (threadIdx.x >> 5), lane = threadIdx.x & 31;
+  if (wid >= n_q * H_I) return;
+  const int per = D_I / 32;  // 1, 2 or 4
+  const uint16_t *src = q_idx + static_cast<int64_t>(wid) * D_I + lane * per;
+  float v[4];
+  float m = 0.f;
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    v[i] = (i < per) ? __uint_as_float(static_cast<uint32_t>(src[i]) << 16) : 0.f;
+    m = fmaxf(m, fabsf(v[i]));
+  }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
+  // m = f * 2^e, f in [0.5, 1): 2^s with s = 9 - e keeps m * 2^s = f * 512 <= 448
+  // when f <= 0.875, else one power less
+  int s = 0;
+  if (m > 0.f) {
+    int e;
+    const float f = frexpf(m, &e);
+    s = (f <= 0.875f) ? 9 - e : 8 - e;
+  }
+  uint32_t hi4 = 0u, lo4 = 0u;
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    if (i >= per) break;
+    const float x = ldexpf(v[i], s);
+    const __nv_fp8_storage_t h = __nv_cvt_float_to_fp8(x, __NV_SATFINITE, __NV_E4M3);
+    const float hv = __half2float(__half(__nv_cvt_fp8_to_halfraw(h, __NV_E4M3)));
+    const __nv_fp8_storage_t l = __nv_cvt_float_to_fp8(x - hv, __NV_SATFINITE, __NV_E4M3);
+    hi4 |= static_cast<uint32_t>(h) << (8 * i);
+    lo4 |= static_cast<uint32_t>(l) << (8 * i);
+  }
+  uint8_t *dh = q8 + static_cast<int64_t>(wid) * D_I + lane * per;
+  uint8_t *dl = dh + static_cast<int64_t>(n_q) * H_I * D_I;
+  for (int i = 0; i < per; ++i) {
+    dh[i] = static_cast<uint8_t>(hi4 >> (8 * i));
+    dl[i] = static_cast<uint8_t>(lo4 >> (8 * i));
+  }
+  if (lane == 0) w8[wid] = ldexpf(w[wid], -s);
+}
+
 // ---------------------------------------------------------------------------
 // host side
 // ---------------------------------------------------------------------------
-template <int G, int AW, int NEG>
+template <int G, int AW, int NEG, bool K8 = false>
 dsa_status_t launch_impl(const IndexerLaunch &a, cudaStream_t stream) {
   constexpr int kThreads = threads_of<NEG>();
-  const int natoms = a.D_I * 2 / AW;
+  constexpr int kEB = K8 ? 1 : 2;
+  const int natoms = a.D_I * kEB / AW;
   const int ncols = G * a.H_I;
   const int n_mma = (ncols + 15) & ~15;
   const int num_groups = a.causal ? (a.n_q + G - 1) / G : a.n_q;
   CUtensorMap tmK, tmQ;
-  if (!make_map_2d(&tmK, a.k_pages, a.D_I, static_cast<uint64_t>(a.num_pages) * kPageSize, AW / 2,
-                   kPageSize, AW))
-    return DSA_ERR_CUDA;
-  if (!make_map_2d(&tmQ, a.q_idx, a.D_I, static_cast<uint64_t>(a.n_q) * a.H_I, AW / 2, ncols, AW))
-    return DSA_ERR_CUDA;
+  if (K8) {
+    // byte keys [pages * 64 rows][D_I]; the query terms [2 * n_q * H_I rows][D_I]
+    if (!make_map_2d_u8(&tmK, a.k8_pages, a.D_I, static_cast<uint64_t>(a.num_pages) * kPageSize,
+                        AW, kPageSize, AW))
+      return DSA_ERR_CUDA;
+    if (!make_map_2d_u8(&tmQ, a.q8, a.D_I, 2ull * a.n_q * a.H_I, AW, ncols, AW))
+      return DSA_ERR_CUDA;
+  } else {
+    if (!make_map_2d(&tmK, a.k_pages, a.D_I, static_cast<uint64_t>(a.num_pages) * kPageSize,
+                     AW / 2, kPageSize, AW))
+      return DSA_ERR_CUDA;
+    if (!make_map_2d(&tmQ, a.q_idx, a.D_I, static_cast<uint64_t>(a.n_q) * a.H_I, AW / 2, ncols, AW))
+      return DSA_ERR_CUDA;
+  }
   (void)natoms;
 
-  const size_t stage_bytes = static_cast<size_t>(kTileKeys) * a.D_I * 2;
-  const size_t q_bytes = static_cast<size_t>(natoms) * n_mma * AW;
+  const size_t stage_bytes = static_cast<size_t>(kTileKeys) * a.D_I * kEB;
+  const size_t q_bytes = static_cast<size_t>(K8 ? 2 : 1) * natoms * n_mma * AW;
   // two CTAs per SM share the SM's shared memory (one query tile each)
   const int q_buffers = (NEG == 1) ? 1 : 2;
-  const size_t fixed = 1024 /*align*/ + q_buffers * q_bytes + 8 * (2 * 8 + 5 + 2 * kMaxAcc) + 16 +
-                       4 * kThreads + 4 * ((num_groups + 4) & ~3) + 64;
+  const size_t fixed = 1024 /*align*/ + q_buffers * q_bytes +
+                       8 * (2 * kMaxStages + 4 + 2 * kMaxAcc + 1) + 16 + 4 * kThreads +
+                       4 * ((num_groups + 4) & ~3) + 64;
   const size_t max_smem = device_max_smem_optin();
-  const size_t budget = (NEG == 1) ? (device_smem_per_sm() / 2 - 1024) : max_smem;
-  int stages = static_cast<int>((std::min(budget, max_smem) - fixed) / stage_bytes);
-  stages = std::min(stages, 8);
+  const size_t budget = std::min((NEG == 1) ? (device_smem_per_sm() / 2 - 1024) : max_smem, max_smem);
+  if (budget <= fixed) return DSA_ERR_UNSUPPORTED;
+  const int stages = static_cast<int>(std::min<size_t>(kMaxStages, (budget - fixed) / stage_bytes));
   if (stages < 2) return DSA_ERR_UNSUPPORTED;
   const size_t smem = fixed + stages * stage_bytes;
 
   static bool attr_set = false;  // per template instantiation
   if (!attr_set) {
-    if (cudaFuncSetAttribute(indexer_kernel<G, AW, NEG>,
+    if (cudaFuncSetAttribute(indexer_kernel<G, AW, NEG, K8>,
                              cudaFuncAttributeMaxDynamicSharedMemorySize,
                              static_cast<int>(max_smem)) != cudaSuccess)
       return DSA_ERR_CUDA;
@@ -462,8 +582,9 @@ dsa_status_t launch_impl(const IndexerLaunch &a, cudaStream_t stream) {
   p.q_buffers = q_buffers;
   p.wait_ns = wait_limit_ns();
   p.debug_stall = debug_stall() == kKernIndexer ? 1 : 0;
+  p.k_scale = a.k_scale;
   p.status = a.status;
-  if (launch_pdl(indexer_kernel<G, AW, NEG>, dim3(grid), dim3(kThreads), smem, stream, 1, tmK, tmQ,
+  if (launch_pdl(indexer_kernel<G, AW, NEG, K8>, dim3(grid), dim3(kThreads), smem, stream, 1, tmK, tmQ,
                  p) != cudaSuccess)
     return DSA_ERR_CUDA;
   return DSA_OK;
@@ -471,10 +592,24 @@ dsa_status_t launch_impl(const IndexerLaunch &a, cudaStream_t stream) {
 
 }  // namespace
 
+dsa_status_t launch_q8_prep(const uint16_t *q_idx, const float *w, uint8_t *q8, float *w8,
+                            int n_q, int H_I, int D_I, cudaStream_t stream) {
+  const unsigned grid = static_cast<unsigned>((static_cast<int64_t>(n_q) * H_I + 7) / 8);
+  if (launch_pdl(q8_prep_kernel, dim3(grid), dim3(256), 0, stream, 1, q_idx, w, q8, w8, n_q, H_I,
+                 D_I) != cudaSuccess)
+    return DSA_ERR_CUDA;
+  return DSA_OK;
+}
+
 dsa_status_t launch_indexer(const IndexerLaunch &a, cudaStream_t stream) {
   // causal prefill rows share keys: groups of 4 rows, one CTA per SM; decode
   // rows: one row per unit, two CTAs per SM
   const bool grouped = a.causal && (a.H_I % 32 == 0) && (4 * a.H_I <= 256);
+  if (a.k8_pages != nullptr) {
+    // E4M3 keys: 128-byte key rows (D_I = 128), the same CTA shapes as bf16
+    if (a.D_I != 128) return DSA_ERR_UNSUPPORTED;
+    return grouped ? launch_impl<4, 128, 2, true>(a, stream) : launch_impl<1, 128, 1, true>(a, stream);
+  }
   if (a.D_I == 32) return grouped ? launch_impl<4, 64, 2>(a, stream) : launch_impl<1, 64, 1>(a, stream);
   return grouped ? launch_impl<4, 128, 2>(a, stream) : launch_impl<1, 128, 1>(a, stream);
 }

@@ -27,7 +27,7 @@ def _declared_symbols():
 
 def test_every_declared_symbol_is_exported(L):
     declared = _declared_symbols()
-    assert len(declared) == 14
+    assert len(declared) == 16
     assert sorted(declared) == sorted(dsa.EXPORTED)
     out = subprocess.run(["nm", "-D", "--defined-only", dsa.LIB_PATH], capture_output=True,
                          text=True, check=True).stdout
@@ -135,6 +135,20 @@ def test_host_validation_rejects_without_launch(L):
     # max_seq_len beyond what the block table can address
     st = L.dsa_indexer_scores(fake, fake, fake, ctypes.byref(_cache(max_seq_len=128 * 64 + 1)),
                               ctypes.byref(d), fake, 8196, ws, 1 << 30, None)
+    assert st == 1
+    # FP8 keys: missing scales, D_I = 32
+    st = L.dsa_indexer_scores_k8(fake, fake, fake, None, ctypes.byref(c), ctypes.byref(d), fake,
+                                 8192, ws, 1 << 30, None)
+    assert st == 1
+    st = L.dsa_indexer_scores_k8(fake, fake, fake, fake, ctypes.byref(c),
+                                 ctypes.byref(_dims(D_I=64)), fake, 8192, ws, 1 << 30, None)
+    assert st == 2
+    # the FP8-key indexer needs room for its query terms
+    st = L.dsa_indexer_scores_k8(fake, fake, fake, fake, ctypes.byref(c), ctypes.byref(d), fake,
+                                 8192, ws, 256, None)
+    assert st == 4
+    st = L.dsa_attention_forward_k8(fake, fake, None, fake, fake, fake, ctypes.byref(c),
+                                    ctypes.byref(d), None, fake, fake, ws, 1 << 30, None)
     assert st == 1
     # absorption GEMMs: shapes outside the tiles, misaligned pointers, no workspace
     st = L.dsa_absorb_query(fake, fake, fake, fake, 4, 64, 128, 160, 64, ws, 256, None)

@@ -176,6 +176,17 @@ def _project_without_transpose(o_lat, W_UV):
                      for h in range(H)])
 
 
+def _e4m3_bias_8(codes):
+    c = np.asarray(codes, dtype=np.uint8).astype(np.int64)
+    e, m = (c >> 3) & 0xF, (c & 0x7).astype(np.float64)
+    v = np.where(e == 0, m / 8 * 2.0 ** -7, (1 + m / 8) * np.exp2(e - 8.0))
+    return np.where(c & 0x80, -v, v)
+
+
+def _dequantize_scale_ignored(k8_rows, scale_rows):
+    return orc.e4m3_to_f64(k8_rows)
+
+
 _ORIG_APPEND = orc.cache_append
 _ORIG_POSITIONS = orc.append_positions
 
@@ -208,6 +219,8 @@ MUTANTS = {
     "absorption: W_UK not transposed": ("absorb_query", _absorb_without_transpose),
     "append: written one slot late": ("cache_append", _append_one_slot_late),
     "projection: W_UV not transposed": ("project_values", _project_without_transpose),
+    "e4m3: exponent bias 8": ("e4m3_to_f64", _e4m3_bias_8),
+    "fp8 keys: scale ignored": ("dequantize_keys", _dequantize_scale_ignored),
     "append: the next token's position": ("append_positions", _append_positions_of_the_next_token),
 }
 

@@ -402,3 +402,46 @@ def test_bf16_widening_all_encodings():
     ok = ~np.isnan(ref)
     np.testing.assert_array_equal(mine[ok], ref[ok])
     np.testing.assert_array_equal(np.signbit(mine[ok]), np.signbit(ref[ok]))
+
+
+# ---------------------------------------------------------------- FP8 index keys
+
+def test_e4m3_decoding_all_encodings():
+    codes = np.arange(256, dtype=np.uint8)
+    mine = orc.e4m3_to_f64(codes)
+    ref = torch.from_numpy(codes).view(torch.float8_e4m3fn).to(torch.float64).numpy()
+    np.testing.assert_array_equal(np.isnan(mine), np.isnan(ref))
+    ok = ~np.isnan(ref)
+    np.testing.assert_array_equal(mine[ok], ref[ok])
+    np.testing.assert_array_equal(np.signbit(mine[ok]), np.signbit(ref[ok]))
+    # a few by hand: 1.0, -2.0, 448 (largest), 2^-9 (smallest subnormal)
+    assert orc.e4m3_to_f64(np.array([0x38, 0xC0, 0x7E, 0x01], np.uint8)).tolist() == \
+        [1.0, -2.0, 448.0, 2.0 ** -9]
+
+
+def test_fp8_keys_stand_for_the_same_keys_and_scores():
+    wl = di.small_decode([300, 129], H_I=4, D_I=64, topk=32, H=2, R=16, P=8, seed=31,
+                         shuffle_pages=True)
+    inp = di.make_inputs(wl)
+    k8 = di.with_fp8_keys(inp, seed=3)
+    assert k8["k8_pages"].dtype == np.uint8 and k8["k_scale"].shape == (inp["k_pages"].shape[0] * 64,)
+    assert len(set(k8["k_scale"].tolist())) > 1          # the scales vary per token
+    deq = orc.dequantize_keys(k8["k8_pages"].reshape(-1, wl.D_I), k8["k_scale"])
+    np.testing.assert_array_equal(deq, orc.bf16_to_f64(inp["k_pages"]).reshape(-1, wl.D_I))
+    r_bf, r_k8 = orc.dsa_decode(inp), orc.dsa_decode(k8)
+    for b in r_bf:
+        np.testing.assert_array_equal(r_bf[b]["scores"], r_k8[b]["scores"])
+        assert np.array_equal(r_bf[b]["idx"], r_k8[b]["idx"])
+
+
+def test_fp8_key_scale_is_a_factor_of_the_score():
+    # a positive per-token scale comes out of the ReLU and the head sum
+    rng = np.random.default_rng(41)
+    q = rng.standard_normal((3, 16))
+    w = rng.uniform(0, 2, 3)
+    codes = rng.integers(0, 256, (20, 16)).astype(np.uint8)
+    codes[(codes & 0x7F) == 0x7F] = 0                      # no NaN codes
+    scale = rng.uniform(0.1, 4.0, 20)
+    s1 = orc.indexer_scores(q, w, orc.dequantize_keys(codes, np.ones(20)))
+    s2 = orc.indexer_scores(q, w, orc.dequantize_keys(codes, scale))
+    np.testing.assert_allclose(s2, scale * s1, rtol=1e-12)
