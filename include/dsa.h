@@ -206,7 +206,7 @@ DSA_API dsa_status_t dsa_attention_forward(const uint16_t *q_idx, const float *w
  * (the scale is taken out of the ReLU and the head sum; a scale must be > 0).
  *   k8_pages  [num_pages, 64, D_I] uint8 E4M3 codes (sign, 4 exponent bits with
  *             bias 7, 3 mantissa bits; 0x7F / 0xFF are NaN), 16-byte aligned
- *   k_scale   [num_pages * 64] fp32
+ *   k_scale   [num_pages * 64] fp32, 16-byte aligned
  * Everything else as dsa_indexer_scores / dsa_attention_forward; workspaces
  * from dsa_workspace_bytes(DSA_OP_INDEXER_SCORES_K8 / _ATTENTION_FORWARD_K8).
  * D_I must be 128.  The tensor cores multiply the keys as E4M3 (half the

@@ -488,7 +488,7 @@ dsa_status_t indexer_entry(const uint16_t *q_idx, const float *w, const uint16_t
   if (q_idx == nullptr || w == nullptr || keys == nullptr || scores == nullptr)
     return DSA_ERR_INVALID_ARG;
   if (!aligned16(q_idx) || !aligned16(keys) || !aligned16(scores) || !aligned4(w) ||
-      (k_scale && !aligned4(k_scale)))
+      (k_scale && !aligned16(k_scale)))
     return DSA_ERR_INVALID_ARG;
   if (k8_pages && dims->D_I != 128) return DSA_ERR_UNSUPPORTED;
   if (ld < max_keys(*dims, *cache) || ld % 4 != 0 || ld <= 0) return DSA_ERR_INVALID_ARG;
@@ -515,7 +515,7 @@ dsa_status_t forward_entry(const uint16_t *q_idx, const float *w, const uint16_t
     return DSA_ERR_INVALID_ARG;
   if (!aligned16(q_idx) || !aligned16(keys) || !aligned16(q) || !aligned16(latent_pages) ||
       !aligned4(w) || !aligned4(out) || !aligned4(lse) || (idx_out && !aligned4(idx_out)) ||
-      (k_scale && !aligned4(k_scale)))
+      (k_scale && !aligned16(k_scale)))
     return DSA_ERR_INVALID_ARG;
   if (k8_pages && dims->D_I != 128) return DSA_ERR_UNSUPPORTED;
   const dsa_dims_t &d = *dims;

@@ -114,7 +114,9 @@ __global__ void __launch_bounds__(threads_of<NEG>(), NEG == 1 ? 2 : 1)
   const int nqb = p.q_buffers;
   constexpr int kEB = K8 ? 1 : 2;                // key / query bytes per element
   const int natoms = p.D_I * kEB / AW;          // swizzle atoms along K
-  const int stage_bytes = kTileKeys * p.D_I * kEB;
+  // K8: the tile's 128 key scales follow its key bytes (1 KB keeps stages aligned)
+  const int kStageScales = kTileKeys * p.D_I * kEB;
+  const int stage_bytes = kStageScales + (K8 ? 1024 : 0);
   const int ncols = G * p.H_I;                  // useful accumulator columns
   const int n_mma = (ncols + 15) & ~15;         // MMA N (multiple of 16)
   // K8: the hi and lo query terms, each [n_mma rows][D_I bytes]
@@ -137,14 +139,16 @@ __global__ void __launch_bounds__(threads_of<NEG>(), NEG == 1 ? 2 : 1)
   uint64_t *tempty = tfull + kMaxAcc;
   uint64_t *drain = tempty + kMaxAcc;
   uint32_t *misc = reinterpret_cast<uint32_t *>(drain + 1);  // [0] tmem base, [1] abort
-  int *scan_tmp = reinterpret_cast<int *>(misc + 4);          // [kThreads]
-  int *tile_start = scan_tmp + kThreads;                      // [num_groups + 1]
+  int *scan_tmp = reinterpret_cast<int *>(misc + 4);          // [kThreads + 32]
+  int *tile_start = scan_tmp + kThreads + 32;                 // [num_groups + 1]
 
   const int warp = warp_id(), lane = lane_id();
   const int NG = p.num_groups;
 
   if (threadIdx.x == 0) {
-    for (int i = 0; i < S; ++i) { mbar_init(&full[i], 1); mbar_init(&empty[i], 1); }
+    // K8: a stage is free once the MMA has run and the four epilogue warps that
+    // take its unit have read their scales
+    for (int i = 0; i < S; ++i) { mbar_init(&full[i], 1); mbar_init(&empty[i], K8 ? 5 : 1); }
     for (int i = 0; i < 2; ++i) { mbar_init(&qfull[i], 1); mbar_init(&qempty[i], 1); }
     for (int i = 0; i < kMaxAcc; ++i) { mbar_init(&tfull[i], 1); mbar_init(&tempty[i], 4); }
     mbar_init(drain, 1);
@@ -163,15 +167,29 @@ __global__ void __launch_bounds__(threads_of<NEG>(), NEG == 1 ? 2 : 1)
     const int g0 = min(NG, static_cast<int>(threadIdx.x) * per), g1 = min(NG, g0 + per);
     int local = 0;
     for (int g = g0; g < g1; ++g) local += (group_keys<G>(p, g) + kTileKeys - 1) / kTileKeys;
-    scan_tmp[threadIdx.x] = local;
+    // exclusive scan of `local` over the block: within warps by shuffles, then
+    // over the warp totals (kThreads / 32 <= 32 of them) by the first warp
+    int incl = local;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int y = __shfl_up_sync(0xffffffffu, incl, o);
+      if (lane >= o) incl += y;
+    }
+    if (lane == 31) scan_tmp[warp] = incl;
     __syncthreads();
-    if (threadIdx.x == 0) {
-      int run = 0;
-      for (int i = 0; i < kThreads; ++i) { const int v = scan_tmp[i]; scan_tmp[i] = run; run += v; }
-      tile_start[NG] = run;
+    if (warp == 0) {
+      const int v = (lane < kThreads / 32) ? scan_tmp[lane] : 0;
+      int wi = v;
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        const int y = __shfl_up_sync(0xffffffffu, wi, o);
+        if (lane >= o) wi += y;
+      }
+      if (lane < kThreads / 32) scan_tmp[kThreads + lane] = wi - v;  // warps before
+      if (lane == kThreads / 32 - 1) tile_start[NG] = wi;
     }
     __syncthreads();
-    int run = scan_tmp[threadIdx.x];
+    int run = scan_tmp[kThreads + warp] + incl - local;
     for (int g = g0; g < g1; ++g) {
       tile_start[g] = run;
       run += (group_keys<G>(p, g) + kTileKeys - 1) / kTileKeys;
@@ -247,7 +265,8 @@ __global__ void __launch_bounds__(threads_of<NEG>(), NEG == 1 ? 2 : 1)
           }
           if (okl && !mbar_wait(&empty[stage], phase ^ 1u, p.wait_ns)) okl = 0;
           if (okl) {
-            const uint32_t page_bytes = kPageSize * p.D_I * kEB;
+            // K8: each page also brings its 64 scales (256 bytes) into the stage
+            const uint32_t page_bytes = kPageSize * p.D_I * kEB + (K8 ? kPageSize * 4 : 0);
             const uint32_t bytes = ((id0 >= 0) + (id1 >= 0)) * page_bytes;
             uint8_t *dst = stage_base + stage * stage_bytes;
             if (bytes == 0) {
@@ -262,6 +281,15 @@ __global__ void __launch_bounds__(threads_of<NEG>(), NEG == 1 ? 2 : 1)
                 if (id1 >= 0)
                   tma_load_2d(dst + a * kTileKeys * AW + kPageSize * AW, &tmK, a * (AW / kEB),
                               id1 * kPageSize, &full[stage]);
+              }
+              if (K8) {
+                uint8_t *sc = dst + kStageScales;
+                if (id0 >= 0)
+                  bulk_load(sc, p.k_scale + static_cast<int64_t>(id0) * kPageSize, kPageSize * 4,
+                            &full[stage]);
+                if (id1 >= 0)
+                  bulk_load(sc + kPageSize * 4, p.k_scale + static_cast<int64_t>(id1) * kPageSize,
+                            kPageSize * 4, &full[stage]);
               }
               armed |= 1u << stage;
               armed_par = (armed_par & ~(1u << stage)) | (phase << stage);
@@ -373,18 +401,17 @@ __global__ void __launch_bounds__(threads_of<NEG>(), NEG == 1 ? 2 : 1)
           wreg[i] = (i < p.H_I) ? __ldg(p.w + static_cast<int64_t>(g) * p.H_I + i) : 0.f;
         wgroup = g;
       }
-      // K8: this key's scale (its page id, then the scale), in flight while
-      // the accumulator is waited for
+      // K8: this key's scale, which the producer copied into the unit's stage
+      // with its key bytes; the stage is released once the MMA has run and
+      // every epilogue warp has read its scales
       float kscale = 1.f;
       if (K8) {
-        const int tt = u - tile_start[g];
-        const int pg = 2 * tt + (key_in_tile >> 6);
-        const int b = p.causal ? 0 : g;
-        if (pg < p.max_pages && pg * kPageSize < group_keys<G>(p, g)) {
-          const int id = __ldg(p.block_table + static_cast<int64_t>(b) * p.max_pages + pg);
-          if (id >= 0 && id < p.num_pages)
-            kscale = __ldg(p.k_scale + static_cast<int64_t>(id) * kPageSize + (key_in_tile & 63));
-        }
+        const int su = i_unit % S;
+        const uint32_t sph = static_cast<uint32_t>(i_unit / S) & 1u;
+        if (!__all_sync(0xffffffffu, mbar_wait(&full[su], sph, p.wait_ns))) { ok = false; break; }
+        kscale = reinterpret_cast<const float *>(stage_base + su * stage_bytes + kStageScales)[key_in_tile];
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&empty[su]);
       }
       if (__any_sync(0xffffffffu, *abort_flag != 0u)) { ok = false; break; }
       if (!__all_sync(0xffffffffu, mbar_wait(&tfull[acc], aphase, p.wait_ns))) { ok = false; break; }
@@ -536,12 +563,12 @@ dsa_status_t launch_impl(const IndexerLaunch &a, cudaStream_t stream) {
   }
   (void)natoms;
 
-  const size_t stage_bytes = static_cast<size_t>(kTileKeys) * a.D_I * kEB;
+  const size_t stage_bytes = static_cast<size_t>(kTileKeys) * a.D_I * kEB + (K8 ? 1024 : 0);
   const size_t q_bytes = static_cast<size_t>(K8 ? 2 : 1) * natoms * n_mma * AW;
   // two CTAs per SM share the SM's shared memory (one query tile each)
   const int q_buffers = (NEG == 1) ? 1 : 2;
   const size_t fixed = 1024 /*align*/ + q_buffers * q_bytes +
-                       8 * (2 * kMaxStages + 4 + 2 * kMaxAcc + 1) + 16 + 4 * kThreads +
+                       8 * (2 * kMaxStages + 4 + 2 * kMaxAcc + 1) + 16 + 4 * (kThreads + 32) +
                        4 * ((num_groups + 4) & ~3) + 64;
   const size_t max_smem = device_max_smem_optin();
   const size_t budget = std::min((NEG == 1) ? (device_smem_per_sm() / 2 - 1024) : max_smem, max_smem);
