@@ -476,6 +476,58 @@ def measure_e2e(case, torch, steps, warmup):
             "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h)}
 
 
+def measure_cp(wl, ranks, torch, dsa, steps, warmup, flush_buf):
+    """Context-parallel decode of `wl` split `ranks` ways, emulated on this GPU:
+    each step of rank 0 (its local scores/top-k/candidates, the global select,
+    its attention, the merge) timed with events; the two all-gathers between
+    them cannot be timed on one GPU and are reported as bytes."""
+    from sparse_attention_scores_b200.context_parallel import RankShard, cuda_ops
+    inp = di.make_inputs(wl)
+    dims = dsa.Dims(n_q=wl.n_q, H_I=wl.H_I, D_I=wl.D_I, topk=wl.topk, H=wl.H, R=wl.R, P=wl.P,
+                    causal=0, q_pos0=0, scale=wl.scale)
+    ops = cuda_ops(dims)
+
+    def bf(x):
+        return torch.from_numpy(np.ascontiguousarray(x).view(np.int16)).view(torch.bfloat16).cuda()
+
+    shards = []
+    for r in range(ranks):
+        lo = np.array([di.shard_bounds(n, ranks)[r] for n in wl.seq_lens])
+        hi = np.array([di.shard_bounds(n, ranks)[r + 1] for n in wl.seq_lens])
+        sh = di.shard_inputs(inp, lo, hi)
+        t = {"q_idx": bf(sh["q_idx"]), "w": torch.from_numpy(sh["w"]).cuda(),
+             "k_pages": bf(sh["k_pages"]), "q": bf(sh["q"]),
+             "latent_pages": bf(sh["latent_pages"])}
+        seq_lens = torch.from_numpy(sh["seq_lens"]).cuda()
+        t["cache"] = dsa.PagedCache(seq_lens, torch.from_numpy(sh["block_table"]).cuda(),
+                                    num_pages=int(sh["k_pages"].shape[0]),
+                                    max_seq_len=int(sh["seq_lens"].max()))
+        shards.append(RankShard(offsets=torch.from_numpy(sh["offsets"]).cuda(), lens=seq_lens,
+                                local=t))
+    cand = [ops.candidates(*ops.local_topk(s, wl.topk), s.offsets) for s in shards]
+    all_s, all_i = torch.stack([c[0] for c in cand]), torch.stack([c[1] for c in cand])
+    gidx, own = ops.select(all_s, all_i, shards[0].offsets, shards[0].lens)
+    part = [ops.attend(s, ops.select(all_s, all_i, s.offsets, s.lens)[1]) for s in shards]
+    outs, lses = torch.stack([p[0] for p in part]), torch.stack([p[1] for p in part])
+    torch.cuda.synchronize()
+    s0 = shards[0]
+    t_local, _ = timed_events(torch, lambda: ops.candidates(*ops.local_topk(s0, wl.topk), s0.offsets),
+                              steps, warmup, flush_buf)
+    t_sel, _ = timed_events(torch, lambda: ops.select(all_s, all_i, s0.offsets, s0.lens), steps,
+                            warmup, flush_buf)
+    t_att, _ = timed_events(torch, lambda: ops.attend(s0, own), steps, warmup, flush_buf)
+    t_mrg, _ = timed_events(torch, lambda: ops.merge(outs, lses), steps, warmup, flush_buf)
+    cand_bytes = ranks * wl.n_q * wl.topk * 8
+    part_bytes = ranks * wl.n_q * wl.H * (wl.R + 1) * 4
+    return {"workload": wl.name, "ranks": ranks, "emulated_on_one_gpu": True,
+            "keys_per_rank_per_row": int(max(wl.seq_lens)) // ranks,
+            "rank_local_us": t_local * 1e3, "select_us": t_sel * 1e3,
+            "attend_us": t_att * 1e3, "merge_us": t_mrg * 1e3,
+            "per_rank_compute_us": (t_local + t_sel + t_att + t_mrg) * 1e3,
+            "all_gather_bytes": {"candidates": cand_bytes, "partials": part_bytes},
+            "all_gather_us_at_770_gbs_modelled": (cand_bytes + part_bytes) / 770e9 * 1e6}
+
+
 def oracle_rows_per_s(wl, budget_s: float):
     """Time the float64 oracle on whole query rows of `wl` for ~budget_s."""
     from oracle import dsa_oracle as orc
@@ -565,6 +617,10 @@ def run_ours(args):
             per_config[name] = r
             del c
             torch.cuda.empty_cache()
+        # context-parallel decode of the 4 x 131,072 rows over 8 ranks, emulated here
+        per_config["glm5_decode_4x128k/context_parallel_8"] = measure_cp(
+            di.CONFIGS["glm5_decode_4x128k"], 8, torch, dsa, args.steps, args.warmup, flush_buf)
+        torch.cuda.empty_cache()
         for name in EXTRA_K8:
             c = Case(replica_workload(di.CONFIGS[name], rank), torch, dsa, k8=True)
             c.step()

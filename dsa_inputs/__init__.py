@@ -201,3 +201,41 @@ def with_fp8_keys(inp: dict, seed: int = 0, max_shift: int = 7) -> dict:
     out["k8_pages"] = codes.numpy()
     out["k_scale"] = np.exp2(-j).astype(np.float32).reshape(-1)
     return out
+
+
+def shard_bounds(n: int, ranks: int) -> np.ndarray:
+    """Key-range boundaries of n keys split over ranks: [bounds[i], bounds[i+1])."""
+    return np.linspace(0, n, ranks + 1).astype(np.int64)
+
+
+def shard_inputs(inp: dict, lo, hi) -> dict:
+    """The keys [lo[b], hi[b]) of every sequence b (index keys and latent rows)
+    as inputs of their own, re-paged from local position 0 with an identity
+    block table; "offsets" holds lo.  Queries and weights are unchanged."""
+    lo, hi = np.asarray(lo, np.int64), np.asarray(hi, np.int64)
+    lens = (hi - lo).astype(np.int32)
+    B = len(lens)
+    maxp = max(1, max(pages_needed(int(n)) for n in lens))
+    D, Wd = inp["k_pages"].shape[2], inp["latent_pages"].shape[2]
+    kp, lp = [], []
+    bt = np.full((B, maxp), -1, dtype=np.int32)
+    for b in range(B):
+        pos = np.arange(lo[b], hi[b])
+        phys = inp["block_table"][b][pos // 64].astype(np.int64) * 64 + pos % 64
+        k_rows = inp["k_pages"].reshape(-1, D)[phys]
+        l_rows = inp["latent_pages"].reshape(-1, Wd)[phys]
+        for j in range(pages_needed(int(lens[b]))):
+            kpg = np.zeros((64, D), dtype=np.uint16)
+            lpg = np.zeros((64, Wd), dtype=np.uint16)
+            kpg[:len(k_rows[64 * j:64 * j + 64])] = k_rows[64 * j:64 * j + 64]
+            lpg[:len(l_rows[64 * j:64 * j + 64])] = l_rows[64 * j:64 * j + 64]
+            bt[b, j] = len(kp)
+            kp.append(kpg)
+            lp.append(lpg)
+    if not kp:
+        kp.append(np.zeros((64, D), np.uint16))
+        lp.append(np.zeros((64, Wd), np.uint16))
+    out = dict(inp)
+    out.update(k_pages=np.stack(kp), latent_pages=np.stack(lp), block_table=bt, seq_lens=lens,
+               offsets=lo.astype(np.int32))
+    return out

@@ -284,6 +284,41 @@ DSA_API dsa_status_t dsa_project_values(const float *o_lat, const uint16_t *w_uv
                                 int32_t n_q, int32_t H, int32_t R, int32_t d_v, void *ws,
                                 size_t ws_bytes, dsa_stream_t stream);
 
+/* Context-parallel decode of one long sequence whose keys are split over
+ * ranks (GPUs), the key range of rank i before that of rank i + 1 ("GLM on an
+ * A100, in Vx", "The model": contexts of up to 1,048,576 tokens, each query
+ * keeping its 2,048 best-scoring earlier tokens).  Each rank runs
+ * dsa_indexer_scores and dsa_topk over its own keys (local positions); then
+ *   1. dsa_cp_candidates: its kept local positions idx_local [n_q, k] become
+ *      (score, global index) pairs cand_scores / cand_idx [n_q, k] (pads:
+ *      -inf, -1); offsets [n_q] = the global position of the rank's first key;
+ *   2. the caller all-gathers the pairs, rank by rank: all_scores / all_idx
+ *      [ranks, n_q, k];
+ *   3. dsa_cp_select: the exact global top-k of the pairs (the lower global
+ *      index wins ties, as in dsa_topk) into gidx [n_q, k] (ascending, -1
+ *      padded), and in own_idx [n_q, k] the same slots as this rank's local
+ *      positions (-1 for tokens of other ranks); my_offsets / my_lens [n_q]
+ *      give this rank's key range.  Workspace: dsa_cp_workspace_bytes;
+ *   4. dsa_sparse_mla_decode with own_idx over the rank's latent rows, then
+ *      the caller all-gathers (out, lse): outs [ranks, n_q, H, dv], lses
+ *      [ranks, n_q, H];
+ *   5. dsa_cp_merge: out = sum_r exp(lse_r - L) out_r, L = log sum_r
+ *      exp(lse_r) (natural log; a rank with no kept token has lse = -inf).
+ * The global top-k lies within the union of the local top-ks, so the result
+ * is the one-device step's.  Pointers 4-byte aligned; ranks <= 1024. */
+DSA_API size_t dsa_cp_workspace_bytes(int32_t ranks, int32_t n_q, int32_t k);
+DSA_API dsa_status_t dsa_cp_candidates(const float *scores, int64_t ld, int32_t n_q,
+                               const int32_t *idx_local, int32_t k, const int32_t *offsets,
+                               float *cand_scores, int32_t *cand_idx, void *ws, size_t ws_bytes,
+                               dsa_stream_t stream);
+DSA_API dsa_status_t dsa_cp_select(const float *all_scores, const int32_t *all_idx,
+                           int32_t ranks, int32_t n_q, int32_t k, const int32_t *my_offsets,
+                           const int32_t *my_lens, int32_t *gidx, int32_t *own_idx, void *ws,
+                           size_t ws_bytes, dsa_stream_t stream);
+DSA_API dsa_status_t dsa_cp_merge(const float *outs, const float *lses, int32_t ranks,
+                          int32_t n_q, int32_t H, int32_t dv, float *out, float *lse, void *ws,
+                          size_t ws_bytes, dsa_stream_t stream);
+
 /* Sparse MLA decode for callers that cannot allocate device memory.
  *
  * The pages have no counterpart of this entry point: it exists for callers

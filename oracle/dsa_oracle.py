@@ -329,3 +329,50 @@ def dsa_prefill(inp: dict, rows=None) -> dict:
     q_pos0 = int(inp.get("q_pos0", 0))
     return {int(t): _query_row(inp, t, inp["block_table"][0], q_pos0 + int(t) + 1)
             for t in rows}
+
+
+# --------------------------------------------------------------------------
+# context-parallel decode of one long sequence (key range split over ranks)
+# --------------------------------------------------------------------------
+
+def cp_local_candidates(scores_local: np.ndarray, k: int, offset: int):
+    """One rank's candidates: its exact top-k over its own key range, as
+    (score, global index) pairs in ascending index order, padded with
+    (-inf, -1).  "GLM on an A100, in Vx", "The model": a context of up to
+    1,048,576 tokens; each query keeps the k best-scoring earlier tokens."""
+    sel = topk_select(scores_local, k)
+    cand_s = np.full(k, -np.inf)
+    cand_i = np.full(k, -1, dtype=np.int64)
+    m = sel >= 0
+    cand_s[m] = np.asarray(scores_local, np.float64)[sel[m]]
+    cand_i[m] = offset + sel[m]
+    return cand_s, cand_i
+
+
+def cp_merge_candidates(cand_s: np.ndarray, cand_i: np.ndarray, k: int) -> np.ndarray:
+    """The global top-k from every rank's candidates ([R, k] each, ranks in
+    key-range order): the best k valid pairs by (-score, global index),
+    ascending, padded with -1.  A token of the global top-k is in its own
+    rank's local top-k, so nothing is lost."""
+    s = np.asarray(cand_s, np.float64).reshape(-1)
+    i = np.asarray(cand_i, np.int64).reshape(-1)
+    valid = i >= 0
+    pairs = sorted(zip(-s[valid], i[valid]))[:k]
+    out = np.full(k, -1, dtype=np.int64)
+    out[:len(pairs)] = sorted(int(g) for _, g in pairs)
+    return out
+
+
+def cp_merge_partials(outs, lses):
+    """Attention over the union of disjoint key sets from each set's own
+    normalised output and log-sum-exp: out = sum_r exp(lse_r - L) out_r with
+    L = log sum_r exp(lse_r); a set with no key has lse = -inf."""
+    lses = np.asarray(lses, np.float64)          # [R, H]
+    outs = np.asarray(outs, np.float64)          # [R, H, dv]
+    top = np.max(lses, axis=0)
+    fin = np.isfinite(top)
+    wts = np.where(np.isfinite(lses), np.exp(lses - np.where(fin, top, 0.0)), 0.0)
+    tot = wts.sum(axis=0)
+    out = np.einsum("rh,rhd->hd", wts, outs) / np.where(tot > 0, tot, 1.0)[:, None]
+    lse = np.where(tot > 0, top + np.log(np.where(tot > 0, tot, 1.0)), -np.inf)
+    return out, lse

@@ -39,7 +39,8 @@ EXPORTED = ["dsa_version", "dsa_status_string", "dsa_workspace_bytes", "dsa_work
             "dsa_workspace_check", "dsa_indexer_scores", "dsa_topk", "dsa_sparse_mla_decode",
             "dsa_sparse_mla_prefill", "dsa_attention_forward", "dsa_sparse_mla_decode_noalloc",
             "dsa_cache_append", "dsa_absorb_query", "dsa_project_values",
-            "dsa_indexer_scores_k8", "dsa_attention_forward_k8"]
+            "dsa_indexer_scores_k8", "dsa_attention_forward_k8", "dsa_cp_workspace_bytes",
+            "dsa_cp_candidates", "dsa_cp_select", "dsa_cp_merge"]
 
 
 class DsaError(RuntimeError):
@@ -96,6 +97,10 @@ def lib() -> ctypes.CDLL:
             "dsa_indexer_scores_k8": ([vp, vp, vp, vp, pc, pd, vp, i64, vp, sz, vp], ctypes.c_int),
             "dsa_attention_forward_k8": ([vp, vp, vp, vp, vp, vp, pc, pd, vp, vp, vp, vp, sz, vp],
                                          ctypes.c_int),
+            "dsa_cp_workspace_bytes": ([i32, i32, i32], sz),
+            "dsa_cp_candidates": ([vp, i64, i32, vp, i32, vp, vp, vp, vp, sz, vp], ctypes.c_int),
+            "dsa_cp_select": ([vp, vp, i32, i32, i32, vp, vp, vp, vp, vp, sz, vp], ctypes.c_int),
+            "dsa_cp_merge": ([vp, vp, i32, i32, i32, i32, vp, vp, vp, sz, vp], ctypes.c_int),
         }
         for name, (args, res) in sigs.items():
             fn = getattr(L, name)
@@ -288,3 +293,34 @@ def dsa_attention_forward_k8(q_idx, w, k8_pages, k_scale, q, latent_pages, cache
                                           ctypes.byref(dims.struct()), _ptr(idx_out), _ptr(out),
                                           _ptr(lse), _ptr(ws), ws.numel(), _stream(stream)),
            "dsa_attention_forward_k8")
+
+
+def cp_workspace(ranks: int, n_q: int, k: int, device="cuda", stream=None):
+    """Workspace of dsa_cp_select."""
+    import torch
+    n = int(lib().dsa_cp_workspace_bytes(ranks, n_q, k))
+    if n == 0:
+        raise DsaError(1, "dsa_cp_workspace_bytes")
+    ws = torch.empty(n, dtype=torch.uint8, device=device)
+    _check(lib().dsa_workspace_init(_ptr(ws), n, _stream(stream)), "dsa_workspace_init")
+    return ws
+
+
+def dsa_cp_candidates(scores, idx_local, offsets, cand_scores, cand_idx, ws, stream=None) -> None:
+    n_q, k = (int(x) for x in idx_local.shape)
+    _check(lib().dsa_cp_candidates(_ptr(scores), int(scores.stride(0)), n_q, _ptr(idx_local), k,
+                                   _ptr(offsets), _ptr(cand_scores), _ptr(cand_idx), _ptr(ws),
+                                   ws.numel(), _stream(stream)), "dsa_cp_candidates")
+
+
+def dsa_cp_select(all_scores, all_idx, my_offsets, my_lens, gidx, own_idx, ws, stream=None) -> None:
+    ranks, n_q, k = (int(x) for x in all_scores.shape)
+    _check(lib().dsa_cp_select(_ptr(all_scores), _ptr(all_idx), ranks, n_q, k, _ptr(my_offsets),
+                               _ptr(my_lens), _ptr(gidx), _ptr(own_idx), _ptr(ws), ws.numel(),
+                               _stream(stream)), "dsa_cp_select")
+
+
+def dsa_cp_merge(outs, lses, out, lse, ws, stream=None) -> None:
+    ranks, n_q, H, dv = (int(x) for x in outs.shape)
+    _check(lib().dsa_cp_merge(_ptr(outs), _ptr(lses), ranks, n_q, H, dv, _ptr(out), _ptr(lse),
+                              _ptr(ws), ws.numel(), _stream(stream)), "dsa_cp_merge")

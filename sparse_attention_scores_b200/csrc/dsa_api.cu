@@ -471,6 +471,69 @@ dsa_status_t dsa_attention_forward_k8(const uint16_t *q_idx, const float *w,
                        idx_out, out, lse, ws, ws_bytes, stream);
 }
 
+size_t dsa_cp_workspace_bytes(int32_t ranks, int32_t n_q, int32_t k) {
+  if (ranks < 1 || n_q < 0 || k < 1) return 0;
+  const int64_t ld = (static_cast<int64_t>(ranks) * k + 3) & ~static_cast<int64_t>(3);
+  return kStatusBytes + align256(static_cast<size_t>(n_q) * ld * 4) +
+         align256(static_cast<size_t>(n_q) * k * 4) + align256(static_cast<size_t>(n_q) * 4);
+}
+
+dsa_status_t dsa_cp_candidates(const float *scores, int64_t ld, int32_t n_q, const int32_t *idx_local,
+                               int32_t k, const int32_t *offsets, float *cand_scores,
+                               int32_t *cand_idx, void *ws, size_t ws_bytes, dsa_stream_t stream) {
+  if (n_q < 0 || k < 1 || ld < 1) return DSA_ERR_INVALID_ARG;
+  if (scores == nullptr || idx_local == nullptr || offsets == nullptr || cand_scores == nullptr ||
+      cand_idx == nullptr)
+    return DSA_ERR_INVALID_ARG;
+  if (!aligned4(scores) || !aligned4(idx_local) || !aligned4(offsets) || !aligned4(cand_scores) ||
+      !aligned4(cand_idx))
+    return DSA_ERR_INVALID_ARG;
+  DSA_TRY(check_ws(ws, ws_bytes, kStatusBytes));
+  if (n_q == 0) return DSA_OK;
+  return launch_cp_candidates(scores, ld, n_q, idx_local, k, offsets, cand_scores, cand_idx,
+                              as_stream(stream));
+}
+
+dsa_status_t dsa_cp_select(const float *all_scores, const int32_t *all_idx, int32_t ranks,
+                           int32_t n_q, int32_t k, const int32_t *my_offsets,
+                           const int32_t *my_lens, int32_t *gidx, int32_t *own_idx, void *ws,
+                           size_t ws_bytes, dsa_stream_t stream) {
+  if (ranks < 1 || n_q < 0 || k < 1 || k > 65536) return DSA_ERR_INVALID_ARG;
+  if (static_cast<int64_t>(ranks) * k > (1 << 24)) return DSA_ERR_UNSUPPORTED;
+  if (all_scores == nullptr || all_idx == nullptr || my_offsets == nullptr || my_lens == nullptr ||
+      gidx == nullptr || own_idx == nullptr)
+    return DSA_ERR_INVALID_ARG;
+  if (!aligned4(all_scores) || !aligned4(all_idx) || !aligned4(my_offsets) || !aligned4(my_lens) ||
+      !aligned4(gidx) || !aligned4(own_idx))
+    return DSA_ERR_INVALID_ARG;
+  DSA_TRY(check_ws(ws, ws_bytes, dsa_cp_workspace_bytes(ranks, n_q, k)));
+  if (n_q == 0) return DSA_OK;
+  const int64_t ld = (static_cast<int64_t>(ranks) * k + 3) & ~static_cast<int64_t>(3);
+  uint8_t *base = static_cast<uint8_t *>(ws) + kStatusBytes;
+  float *packed = reinterpret_cast<float *>(base);
+  int32_t *pos = reinterpret_cast<int32_t *>(base + align256(static_cast<size_t>(n_q) * ld * 4));
+  int32_t *vlen = reinterpret_cast<int32_t *>(reinterpret_cast<uint8_t *>(pos) +
+                                              align256(static_cast<size_t>(n_q) * k * 4));
+  cudaStream_t s = as_stream(stream);
+  DSA_TRY(launch_cp_pack(all_scores, ranks, n_q, k, ld, packed, vlen, s));
+  DSA_TRY(run_topk(packed, ld, n_q, vlen, 0, k, pos, static_cast<int>(ranks * k), status_of(ws), s));
+  return launch_cp_select(pos, all_idx, ranks, n_q, k, my_offsets, my_lens, gidx, own_idx, s);
+}
+
+dsa_status_t dsa_cp_merge(const float *outs, const float *lses, int32_t ranks, int32_t n_q,
+                          int32_t H, int32_t dv, float *out, float *lse, void *ws, size_t ws_bytes,
+                          dsa_stream_t stream) {
+  if (ranks < 1 || n_q < 0 || H < 1 || H > 65535 || dv < 1) return DSA_ERR_INVALID_ARG;
+  if (ranks > 1024) return DSA_ERR_UNSUPPORTED;
+  if (outs == nullptr || lses == nullptr || out == nullptr || lse == nullptr)
+    return DSA_ERR_INVALID_ARG;
+  if (!aligned4(outs) || !aligned4(lses) || !aligned4(out) || !aligned4(lse))
+    return DSA_ERR_INVALID_ARG;
+  DSA_TRY(check_ws(ws, ws_bytes, kStatusBytes));
+  if (n_q == 0) return DSA_OK;
+  return launch_cp_merge(outs, lses, ranks, n_q, H, dv, out, lse, as_stream(stream));
+}
+
 }  // extern "C"
 
 namespace dsa {

@@ -122,6 +122,18 @@ struct AbsorbLaunch {
 };
 dsa_status_t launch_absorb(const AbsorbLaunch &a, cudaStream_t stream);
 
+// context-parallel decode (cp.cu)
+dsa_status_t launch_cp_candidates(const float *scores, int64_t ld, int n_q, const int32_t *idx_local,
+                                  int k, const int32_t *offsets, float *cand_s, int32_t *cand_i,
+                                  cudaStream_t s);
+dsa_status_t launch_cp_pack(const float *all_s, int R, int n_q, int k, int64_t ld, float *packed,
+                            int32_t *vlen, cudaStream_t s);
+dsa_status_t launch_cp_select(const int32_t *pos, const int32_t *all_i, int R, int n_q, int k,
+                              const int32_t *my_off, const int32_t *my_len, int32_t *gidx,
+                              int32_t *own, cudaStream_t s);
+dsa_status_t launch_cp_merge(const float *outs, const float *lses, int R, int n_q, int H, int dv,
+                             float *out, float *lse, cudaStream_t s);
+
 struct MlaLaunch {
   const uint16_t *q;
   const uint16_t *latent;

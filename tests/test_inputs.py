@@ -36,3 +36,23 @@ def test_ragged_config_lengths():
     assert len(wl.seq_lens) == 32
     assert min(wl.seq_lens) >= 2048 and max(wl.seq_lens) <= 65536
     assert wl.seq_lens == di.ragged_lengths(32, 2048, 65536, 1)
+
+
+def test_shards_hold_the_sequence_keys():
+    wl = di.small_decode([300, 65], H_I=2, D_I=16, topk=8, H=2, R=16, P=8, seed=5,
+                         shuffle_pages=True)
+    inp = di.make_inputs(wl)
+    for ranks in (2, 3):
+        rows_k = [[] for _ in wl.seq_lens]
+        for r in range(ranks):
+            lo = np.array([di.shard_bounds(n, ranks)[r] for n in wl.seq_lens])
+            hi = np.array([di.shard_bounds(n, ranks)[r + 1] for n in wl.seq_lens])
+            sh = di.shard_inputs(inp, lo, hi)
+            assert np.array_equal(sh["offsets"], lo) and np.array_equal(sh["seq_lens"], hi - lo)
+            for b in range(len(wl.seq_lens)):
+                for p in range(int(hi[b] - lo[b])):
+                    pg = sh["block_table"][b][p // 64]
+                    rows_k[b].append(sh["k_pages"][pg, p % 64])
+        for b, n in enumerate(wl.seq_lens):
+            want = [inp["k_pages"][inp["block_table"][b][p // 64], p % 64] for p in range(n)]
+            assert np.array_equal(np.stack(rows_k[b]), np.stack(want))

@@ -25,9 +25,14 @@ def _pin_calls(golden_dir):
         if not (name.startswith("test_") and inspect.isfunction(fn)):
             continue
         params = inspect.signature(fn).parameters
-        if "seed" in params:
-            for seed in range(8):
-                calls.append((f"{name}[{seed}]", lambda fn=fn, seed=seed: fn(seed=seed)))
+        marks = [m for m in getattr(fn, "pytestmark", []) if m.name == "parametrize"]
+        if marks:
+            # the first eight parameter sets of the (single) parametrize mark
+            argnames, argvalues = marks[0].args[0], marks[0].args[1]
+            names = [a.strip() for a in argnames.split(",")] if isinstance(argnames, str) else list(argnames)
+            for j, vals in enumerate(list(argvalues)[:8]):
+                kw = dict(zip(names, vals if len(names) > 1 else (vals,)))
+                calls.append((f"{name}[{j}]", lambda fn=fn, kw=kw: fn(**kw)))
         elif "golden_dir" in params:
             calls.append((name, lambda fn=fn: fn(golden_dir=golden_dir)))
         else:
@@ -187,6 +192,21 @@ def _dequantize_scale_ignored(k8_rows, scale_rows):
     return orc.e4m3_to_f64(k8_rows)
 
 
+def _cp_merge_ties_to_higher_index(cand_s, cand_i, k):
+    s = np.asarray(cand_s, np.float64).reshape(-1)
+    i = np.asarray(cand_i, np.int64).reshape(-1)
+    valid = i >= 0
+    pairs = sorted(zip(-s[valid], -i[valid]))[:k]
+    out = np.full(k, -1, dtype=np.int64)
+    out[:len(pairs)] = sorted(-int(g) for _, g in pairs)
+    return out
+
+
+def _cp_merge_partials_unweighted(outs, lses):
+    outs = np.asarray(outs, np.float64)
+    return outs.mean(axis=0), np.max(np.asarray(lses, np.float64), axis=0)
+
+
 _ORIG_APPEND = orc.cache_append
 _ORIG_POSITIONS = orc.append_positions
 
@@ -220,6 +240,8 @@ MUTANTS = {
     "append: written one slot late": ("cache_append", _append_one_slot_late),
     "projection: W_UV not transposed": ("project_values", _project_without_transpose),
     "e4m3: exponent bias 8": ("e4m3_to_f64", _e4m3_bias_8),
+    "cp: candidate ties to the higher index": ("cp_merge_candidates", _cp_merge_ties_to_higher_index),
+    "cp: partials averaged without LSE weights": ("cp_merge_partials", _cp_merge_partials_unweighted),
     "fp8 keys: scale ignored": ("dequantize_keys", _dequantize_scale_ignored),
     "append: the next token's position": ("append_positions", _append_positions_of_the_next_token),
 }

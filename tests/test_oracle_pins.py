@@ -445,3 +445,49 @@ def test_fp8_key_scale_is_a_factor_of_the_score():
     s1 = orc.indexer_scores(q, w, orc.dequantize_keys(codes, np.ones(20)))
     s2 = orc.indexer_scores(q, w, orc.dequantize_keys(codes, scale))
     np.testing.assert_allclose(s2, scale * s1, rtol=1e-12)
+
+
+# ---------------------------------------------------------------- context-parallel decode
+
+@pytest.mark.parametrize("ranks", [2, 3, 5])
+def test_context_parallel_equals_one_gpu_decode(ranks):
+    # split one sequence's keys over ranks: local top-k, global merge of the
+    # candidates, each rank's attention over its own kept keys, LSE merge ==
+    # the one-device step (indices exactly)
+    wl = di.small_decode([1500], H_I=4, D_I=32, topk=200, H=3, R=16, P=8, seed=61)
+    inp = di.make_inputs(wl)
+    ref = orc.dsa_decode(inp)[0]
+    n = wl.seq_lens[0]
+    bounds = np.linspace(0, n, ranks + 1).astype(int)
+    cs, ci = [], []
+    for r in range(ranks):
+        s_r, i_r = orc.cp_local_candidates(ref["scores"][bounds[r]:bounds[r + 1]], wl.topk,
+                                           int(bounds[r]))
+        cs.append(s_r)
+        ci.append(i_r)
+    gidx = orc.cp_merge_candidates(np.stack(cs), np.stack(ci), wl.topk)
+    assert np.array_equal(gidx, ref["idx"])
+    q = orc.bf16_to_f64(inp["q"][0])
+    outs, lses = [], []
+    for r in range(ranks):
+        own = gidx[(gidx >= bounds[r]) & (gidx < bounds[r + 1])]
+        if len(own) == 0:
+            outs.append(np.zeros((wl.H, wl.R)))
+            lses.append(np.full(wl.H, -np.inf))
+            continue
+        rows = orc.bf16_to_f64(orc.gather_paged_rows(inp["latent_pages"], inp["block_table"][0], own))
+        o, l, _ = orc.mla_attention(q, rows, wl.R, wl.scale)
+        outs.append(o)
+        lses.append(l)
+    out, lse = orc.cp_merge_partials(outs, lses)
+    np.testing.assert_allclose(out, ref["out"], rtol=1e-10, atol=1e-12)
+    np.testing.assert_allclose(lse, ref["lse"], rtol=1e-12)
+
+
+def test_cp_merge_candidates_tie_rule_across_ranks():
+    # equal scores on two ranks: the lower global index (the earlier rank) wins
+    s = np.array([[5.0, 3.0, -np.inf], [5.0, 3.0, 3.0]])
+    i = np.array([[2, 7, -1], [10, 11, 12]])
+    assert orc.cp_merge_candidates(s, i, 3).tolist() == [2, 7, 10]
+    assert orc.cp_merge_candidates(s, i, 4).tolist() == [2, 7, 10, 11]
+    assert orc.cp_merge_candidates(s, i, 9).tolist() == [2, 7, 10, 11, 12, -1, -1, -1, -1]
