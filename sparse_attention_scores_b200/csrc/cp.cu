@@ -142,11 +142,48 @@ __global__ void __launch_bounds__(128) cp_merge_kernel(const float *outs, const 
     if (lane == 0) lse[static_cast<int64_t>(r) * H + h] = (tot > 0.f) ? m + logf(tot) : -INFINITY;
   }
   __syncthreads();
-  for (int c = threadIdx.x; c < dv; c += blockDim.x) {
-    float acc = 0.f;
-    for (int q = 0; q < R; ++q)
-      if (wts[q] != 0.f) acc += wts[q] * outs[((static_cast<int64_t>(q) * n_q + r) * H + h) * dv + c];
-    out[(static_cast<int64_t>(r) * H + h) * dv + c] = acc;
+  // every rank's row of this (query, head) is read in groups of eight ranks,
+  // all loads of a group in flight before the sums; a rank with no weight
+  // (nothing selected there) adds nothing, whatever its row holds
+  const int64_t rstride = static_cast<int64_t>(n_q) * H * dv;  // floats between ranks
+  const float *src = outs + (static_cast<int64_t>(r) * H + h) * dv;
+  float *dst = out + (static_cast<int64_t>(r) * H + h) * dv;
+  const bool vec = (dv % 4) == 0 && (reinterpret_cast<uintptr_t>(outs) & 15u) == 0 &&
+                   (reinterpret_cast<uintptr_t>(out) & 15u) == 0;
+  if (vec) {
+    for (int c = 4 * threadIdx.x; c < dv; c += 4 * blockDim.x) {
+      float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+      for (int q0 = 0; q0 < R; q0 += 8) {
+        float4 v[8];
+#pragma unroll
+        for (int u = 0; u < 8; ++u)
+          v[u] = (q0 + u < R) ? __ldg(reinterpret_cast<const float4 *>(src + (q0 + u) * rstride + c))
+                              : make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+        for (int u = 0; u < 8; ++u) {
+          const float w = (q0 + u < R) ? wts[q0 + u] : 0.f;
+          if (w != 0.f) {
+            acc.x += w * v[u].x; acc.y += w * v[u].y; acc.z += w * v[u].z; acc.w += w * v[u].w;
+          }
+        }
+      }
+      *reinterpret_cast<float4 *>(dst + c) = acc;
+    }
+  } else {
+    for (int c = threadIdx.x; c < dv; c += blockDim.x) {
+      float acc = 0.f;
+      for (int q0 = 0; q0 < R; q0 += 8) {
+        float v[8];
+#pragma unroll
+        for (int u = 0; u < 8; ++u) v[u] = (q0 + u < R) ? __ldg(src + (q0 + u) * rstride + c) : 0.f;
+#pragma unroll
+        for (int u = 0; u < 8; ++u) {
+          const float w = (q0 + u < R) ? wts[q0 + u] : 0.f;
+          if (w != 0.f) acc += w * v[u];
+        }
+      }
+      dst[c] = acc;
+    }
   }
 }
 

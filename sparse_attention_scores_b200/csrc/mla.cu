@@ -61,7 +61,8 @@ struct MlaParams {
   float *part_ml;  // [n_q, nsplit, 2, 64]
   int n_q, H, R, W, topk, causal, q_pos0, max_pages, num_pages;
   int nsplit, chunks_per_split;
-  int kc;  // selected keys per chunk: 128, or 64 when few rows leave SMs idle
+  int kc;   // selected keys per chunk: 128, or 64 when few rows leave SMs idle
+  int ncb;  // CTAs per (row, split): 1, or one per 128-column block of the output
   float scale_log2;
   uint64_t wait_ns;
   int debug_stall;  // wait once on a barrier nothing arrives at (tests the time-out path)
@@ -158,6 +159,10 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int q4 = warp & 3;   // tensor-memory lane quadrant: keys / rows 32*q4 ..
   const int hh = warp >> 2;  // head half: heads 32*hh ..
   const int split = blockIdx.x, row = blockIdx.y;
+  // with few rows the 128-column blocks of the output go to separate CTAs
+  // (each computes the chunk's logits and softmax, and its block of PV)
+  const int mb0 = p.ncb > 1 ? static_cast<int>(blockIdx.z) : 0;
+  const int nmb_l = p.ncb > 1 ? 1 : nmb;  // O^T blocks accumulated here
   const int b = p.causal ? 0 : row;
   const int kc = p.kc;
   const int nchunks = (p.topk + kc - 1) / kc;
@@ -166,7 +171,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int cpr = W / 8;  // 16-byte pieces per query row
 
   uint32_t tmem_cols = 32;
-  while (tmem_cols < static_cast<uint32_t>(kHeads + nmb * kHeads)) tmem_cols <<= 1;
+  while (tmem_cols < static_cast<uint32_t>(kHeads + nmb_l * kHeads)) tmem_cols <<= 1;
   if (tid == 0) {
     mbar_init(bar_s, 1);
     mbar_init(bar_o, 1);
@@ -231,20 +236,35 @@ __global__ void __launch_bounds__(kThreads, 1)
     __syncthreads();
     if (misc[2]) failed = true;
   }
+  // Selected position of this thread's slot (threads 0..127) in the chunk
+  // resolved next; the next chunk's position is loaded at the top of each
+  // chunk and its page id before the PV product, so a chunk's rows resolve
+  // without a dependent global load (the first chunk's come from the staged
+  // table in the fused forward).
+  auto slot_pos = [&](int ch) -> int {
+    const int slot = ch * kc + tid;
+    return (tid < kc && ch < c_end && slot < p.topk)
+               ? p.idx[static_cast<int64_t>(row) * p.topk + slot]
+               : -1;
+  };
+  int pos_n = slot_pos(c_begin);
+  int page_n = -2;  // page id of pos_n when prefetched, -2 when not
   for (int ch = c_begin; ch < c_end && !failed; ++ch) {
     // resolve the 128 selected positions of this chunk to physical rows
     int valid = 0;
     if (tid < kChunk) {
       const int slot = ch * kc + tid;
-      const int pos = (tid < kc && slot < p.topk) ? p.idx[static_cast<int64_t>(row) * p.topk + slot] : -1;
+      const int pos = pos_n;
       int phys = -1;
       if (pos >= 0) {
         if (pos >= limit) {
           report(p.status, kErrBadIndex, (kKernMla << 24) | (slot & 0xFFFF));
         } else {
-          const int page = (ch == c_begin && pos / kPageSize < staged_pages)
-                               ? tbl[pos / kPageSize]
-                               : p.block_table[static_cast<int64_t>(b) * p.max_pages + pos / kPageSize];
+          const int pg = pos / kPageSize;
+          const int page = (page_n != -2) ? page_n
+                           : (ch == c_begin && pg < staged_pages)
+                               ? tbl[pg]
+                               : p.block_table[static_cast<int64_t>(b) * p.max_pages + pg];
           if (page < 0 || page >= p.num_pages)
             report(p.status, kErrBadPage, (kKernMla << 24) | (slot & 0xFFFF));
           else
@@ -255,13 +275,16 @@ __global__ void __launch_bounds__(kThreads, 1)
       valid = phys >= 0;
       if (tid == 0) misc[1] = 0u;
     }
+    pos_n = slot_pos(ch + 1);
+    page_n = -2;
     if (__syncthreads_count(valid) == 0) continue;  // nothing to attend in this chunk
     // gather: the selected latent rows into the 128B-swizzled K-major tile,
     // 16 bytes per cp.async, eight threads per 128-byte atom row; unused rows
     // are zero-filled.  (TMA row gathers were measured to be issue-bound at
-    // 15-19 GB/s per SM, whether the rows were in L2 or not.)  Rows kc .. 127
-    // of a 64-key chunk are never written: their keys are masked and the PV
-    // product stops at key kc.
+    // 15-19 GB/s per SM, whether the rows were in L2 or not; waiting and
+    // issuing the logits product atom by atom was slower than one wait.)
+    // Rows kc .. 127 of a 64-key chunk are never written: their keys are
+    // masked and the PV product stops at key kc.
     {
       const uint32_t ls = smem_u32(Ls);
       const int per_atom = kc * 8;  // pieces of one atom: 8 per row
@@ -353,8 +376,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     // rescale the O accumulator when some head's running max moved
     if (misc[1]) {
-      for (int mb = 0; mb < nmb; ++mb) {
-        const uint32_t ta = tmem_o + lane_off + mb * kHeads + 32 * hh;
+      for (int mi = 0; mi < nmb_l; ++mi) {
+        const uint32_t ta = tmem_o + lane_off + mi * kHeads + 32 * hh;
         uint32_t v[32];
         tmem_ld_32x32b_x32(ta, v);
         tmem_ld_wait();
@@ -365,6 +388,9 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       tmem_st_wait();
     }
+    // the next chunk's page ids, from its positions loaded at the top
+    if (tid < kChunk && pos_n >= 0 && pos_n < limit)
+      page_n = p.block_table[static_cast<int64_t>(b) * p.max_pages + pos_n / kPageSize];
     // O^T += L^T . P^T  (M = 128 latent columns per block, N = 64 heads), in two
     // halves of 64 keys; each half multiplies by the hi and by the lo terms.
     // The 16 KB P region holds [hi | lo] for the 64 keys of one half.
@@ -390,11 +416,11 @@ __global__ void __launch_bounds__(kThreads, 1)
       tc_fence_after();
       if (tid == 0) {
         const uint32_t ls = smem_u32(Ls), ps = smem_u32(Ps);
-        for (int mb = 0; mb < nmb; ++mb)
+        for (int mi = 0; mi < nmb_l; ++mi)
           for (int part = 0; part < 2; ++part)
             for (int ks = 0; ks < 4; ++ks)
-              mma_bf16(tmem_o + mb * kHeads,
-                       smem_desc(ls + 2 * mb * kAtomL + (half * 4 + ks) * 2048, kAtomL, 1024,
+              mma_bf16(tmem_o + mi * kHeads,
+                       smem_desc(ls + 2 * (mb0 + mi) * kAtomL + (half * 4 + ks) * 2048, kAtomL, 1024,
                                  kLayoutSW128),
                        smem_desc(ps + part * 8192 + ks * 2048, kAtomQ, 1024, kLayoutSW128),
                        idesc_pv, (have_o || half || part || ks) ? 1u : 0u);
@@ -424,13 +450,13 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   if (p.nsplit == 1) {
     // the whole selection ran here: normalise and write the output
-    for (int mb = 0; mb < nmb; ++mb) {
+    for (int mi = 0; mi < nmb_l; ++mi) {
       uint32_t v[32];
       if (have_o) {
-        tmem_ld_32x32b_x32(tmem_o + lane_off + mb * kHeads + 32 * hh, v);
+        tmem_ld_32x32b_x32(tmem_o + lane_off + mi * kHeads + 32 * hh, v);
         tmem_ld_wait();
       }
-      const int r = mb * 128 + q4 * 32 + lane;
+      const int r = (mb0 + mi) * 128 + q4 * 32 + lane;
       if (r < R) {
 #pragma unroll
         for (int i = 0; i < 32; ++i) {
@@ -442,7 +468,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
       }
     }
-    if (tid < p.H) {
+    if (tid < p.H && mb0 == 0) {
       const float l = lrun[tid];
       p.lse[static_cast<int64_t>(row) * p.H + tid] =
           (l > 0.f) ? (mrun[tid] + log2f(l)) * kLn2 : -INFINITY;
@@ -454,18 +480,18 @@ __global__ void __launch_bounds__(kThreads, 1)
     // the next block is staged.
     float *Obuf = reinterpret_cast<float *>(Ls);
     float *dst = p.part_o + (static_cast<int64_t>(row) * p.nsplit + split) * nmb * kHeads * 128;
-    if (tid < kHeads) {
+    if (tid < kHeads && mb0 == 0) {
       float *ml = p.part_ml + (static_cast<int64_t>(row) * p.nsplit + split) * 2 * kHeads;
       ml[tid] = mrun[tid];
       ml[kHeads + tid] = lrun[tid];
     }
-    for (int mb = 0; mb < nmb; ++mb) {
+    for (int mi = 0; mi < nmb_l; ++mi) {
       uint32_t v[32];
       if (have_o) {
-        tmem_ld_32x32b_x32(tmem_o + lane_off + mb * kHeads + 32 * hh, v);
+        tmem_ld_32x32b_x32(tmem_o + lane_off + mi * kHeads + 32 * hh, v);
         tmem_ld_wait();
       }
-      float *blk = Obuf + mb * kHeads * 128;
+      float *blk = Obuf + mi * kHeads * 128;
       const int cc = q4 * 32 + lane;
 #pragma unroll
       for (int i = 0; i < 32; ++i) blk[(32 * hh + i) * 128 + cc] = have_o ? __uint_as_float(v[i]) : 0.f;
@@ -473,7 +499,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       __syncthreads();
       if (tid == 0) {
         asm volatile("cp.async.bulk.global.shared::cta.bulk_group [%0], [%1], %2;" ::"l"(
-                         reinterpret_cast<uint64_t>(dst + mb * kHeads * 128)),
+                         reinterpret_cast<uint64_t>(dst + (mb0 + mi) * kHeads * 128)),
                      "r"(smem_u32(blk)), "r"(static_cast<uint32_t>(kHeads * 128 * 4))
                      : "memory");
         asm volatile("cp.async.bulk.commit_group;" ::: "memory");
@@ -650,7 +676,10 @@ dsa_status_t launch_mla(const MlaLaunch &a, cudaStream_t stream) {
   p.debug_stall = debug_stall() == kKernMla ? 1 : 0;
   p.early_q = a.early_q;
   p.status = a.status;
-  if (launch_pdl(mla_kernel, dim3(sp.nsplit, a.n_q), dim3(kThreads), smem, stream, 1, p) !=
+  // few CTAs: one per 128-column block of the output as well, when that still fits one wave
+  const int nmb = (a.R + 127) / 128;
+  p.ncb = (nmb > 1 && static_cast<int64_t>(a.n_q) * sp.nsplit * nmb <= device_sm_count()) ? nmb : 1;
+  if (launch_pdl(mla_kernel, dim3(sp.nsplit, a.n_q, p.ncb), dim3(kThreads), smem, stream, 1, p) !=
       cudaSuccess)
     return DSA_ERR_CUDA;
   if (sp.merge == kMergeGlobal) {

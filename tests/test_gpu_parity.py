@@ -147,6 +147,33 @@ def test_topk_long_rows(n):
         assert np.array_equal(got[r].astype(np.int64), want)
 
 
+@pytest.mark.parametrize("kind", ["ints", "normal"])
+@pytest.mark.parametrize("lengths", [
+    [4096, 3000, 300],                 # one CTA per row, 4 keys per thread
+    [8192, 8191, 2049],                # one CTA per row, 8 keys per thread
+    [16384, 9001, 12345],              # one CTA per row, 16 keys per thread
+    [16388, 16001],                    # clusters, 4 keys per thread
+    [131072, 70001],                   # clusters of 16, 8 keys per thread
+    [65536] * 24 + [40000] * 8,        # 32 rows: clusters of 4, 16 keys per thread
+], ids=["small4", "small8", "small16", "cluster4", "cluster8", "cluster16"])
+def test_topk_kernel_paths(kind, lengths):
+    # each row set lands on one of the top-k kernels (chosen by the row count
+    # and the longest row); the ragged rows of a launch share it
+    k = 2048
+    s = _topk_rows(lengths, k, seed=len(lengths) + lengths[0], kind=kind)
+    scores = torch.from_numpy(s).cuda()
+    vl = torch.tensor(lengths, dtype=torch.int32, device="cuda")
+    idx = torch.full((len(lengths), k), -7, dtype=torch.int32, device="cuda")
+    ws = dsa.workspace(dsa.OP_TOPK, dsa.Dims(len(lengths), 1, 32, k, 1, 64, 0), None)
+    dsa.dsa_topk(scores, vl, 0, k, idx, ws)
+    got = idx.cpu().numpy()
+    for r, m in enumerate(lengths):
+        want = np.full(k, -1, np.int64)
+        sel = np.sort(np.argsort(-s[r, :m].astype(np.float64), kind="stable")[:k])
+        want[:len(sel)] = sel
+        assert np.array_equal(got[r].astype(np.int64), want), (r, m)
+
+
 # ---------------------------------------------------------------- step 3
 
 def _random_selection(rng, lengths, k):
