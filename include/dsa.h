@@ -116,7 +116,8 @@ typedef enum {
   DSA_OP_ATTENTION_FORWARD = 4,
   DSA_OP_CACHE_APPEND = 5,
   DSA_OP_INDEXER_SCORES_K8 = 6,   /* dsa_indexer_scores_k8 */
-  DSA_OP_ATTENTION_FORWARD_K8 = 7 /* dsa_attention_forward_k8 */
+  DSA_OP_ATTENTION_FORWARD_K8 = 7, /* dsa_attention_forward_k8 */
+  DSA_OP_ATTENTION_FORWARD_HOST = 8 /* dsa_attention_forward_host */
 } dsa_op_t;
 
 /* Library version (major * 10000 + minor * 100 + patch). */
@@ -196,6 +197,34 @@ DSA_API dsa_status_t dsa_attention_forward(const uint16_t *q_idx, const float *w
                                    const uint16_t *latent_pages, const dsa_cache_t *cache,
                                    const dsa_dims_t *dims, int32_t *idx_out, float *out,
                                    float *lse, void *ws, size_t ws_bytes, dsa_stream_t stream);
+
+/* The whole step with host buffers, for callers whose per-step inputs and
+ * results live in host memory.  On `stream`, in order: the inputs are copied
+ * into the workspace, the step runs (as dsa_attention_forward), the results are
+ * copied back to host memory.  Host buffers the device can address (page-locked
+ * and mapped, as pinned allocations are under unified addressing) are moved by
+ * one small kernel each way, the SMs reading and writing them over the host
+ * link (a copy-engine transfer costs microseconds of latency per buffer);
+ * any other host buffer by its own cudaMemcpyAsync, which for pageable memory
+ * waits for the host.  The call returns once everything is queued: the host
+ * results are valid after the stream has passed it (e.g. cudaStreamSynchronize).
+ *   q_idx_h [n_q, H_I, D_I] bf16, w_h [n_q, H_I] fp32, q_h [n_q, H, R + P] bf16:
+ *             host copies of dsa_attention_forward's inputs (any alignment)
+ *   cache_h   as dsa_cache_t, except that seq_lens and block_table point to
+ *             HOST memory (4-byte aligned); they are copied with the inputs
+ *   k_idx_pages, latent_pages: the device page pools, as dsa_attention_forward
+ *   idx_h [n_q, topk] i32 (may be NULL), out_h [n_q, H, R] fp32, lse_h [n_q, H]
+ *             fp32: host results
+ *   ws        device workspace of dsa_workspace_bytes(DSA_OP_ATTENTION_FORWARD_HOST):
+ *             the step's workspace, then the staged inputs and results
+ * Errors as dsa_attention_forward; a failed host check copies nothing, and a
+ * failed copy returns DSA_ERR_CUDA. */
+DSA_API dsa_status_t dsa_attention_forward_host(const uint16_t *q_idx_h, const float *w_h,
+                                        const uint16_t *k_idx_pages, const uint16_t *q_h,
+                                        const uint16_t *latent_pages, const dsa_cache_t *cache_h,
+                                        const dsa_dims_t *dims, int32_t *idx_h, float *out_h,
+                                        float *lse_h, void *ws, size_t ws_bytes,
+                                        dsa_stream_t stream);
 
 /* FP8 index keys: the indexer, and the whole step, over an index-key cache
  * held as E4M3 bytes with one fp32 scale per token ("GLM on an A100, in Vx",

@@ -30,6 +30,7 @@ OP_ATTENTION_FORWARD = 4
 OP_CACHE_APPEND = 5
 OP_INDEXER_SCORES_K8 = 6
 OP_ATTENTION_FORWARD_K8 = 7
+OP_ATTENTION_FORWARD_HOST = 8
 
 STATUS_NAMES = {0: "DSA_OK", 1: "DSA_ERR_INVALID_ARG", 2: "DSA_ERR_UNSUPPORTED",
                 3: "DSA_ERR_CUDA", 4: "DSA_ERR_WORKSPACE", 5: "DSA_ERR_TIMEOUT",
@@ -40,7 +41,8 @@ EXPORTED = ["dsa_version", "dsa_status_string", "dsa_workspace_bytes", "dsa_work
             "dsa_sparse_mla_prefill", "dsa_attention_forward", "dsa_sparse_mla_decode_noalloc",
             "dsa_cache_append", "dsa_absorb_query", "dsa_project_values",
             "dsa_indexer_scores_k8", "dsa_attention_forward_k8", "dsa_cp_workspace_bytes",
-            "dsa_cp_candidates", "dsa_cp_select", "dsa_cp_merge"]
+            "dsa_cp_candidates", "dsa_cp_select", "dsa_cp_merge",
+            "dsa_attention_forward_host"]
 
 
 class DsaError(RuntimeError):
@@ -101,6 +103,8 @@ def lib() -> ctypes.CDLL:
             "dsa_cp_candidates": ([vp, i64, i32, vp, i32, vp, vp, vp, vp, sz, vp], ctypes.c_int),
             "dsa_cp_select": ([vp, vp, i32, i32, i32, vp, vp, vp, vp, vp, sz, vp], ctypes.c_int),
             "dsa_cp_merge": ([vp, vp, i32, i32, i32, i32, vp, vp, vp, sz, vp], ctypes.c_int),
+            "dsa_attention_forward_host": ([vp, vp, vp, vp, vp, pc, pd, vp, vp, vp, vp, sz, vp],
+                                           ctypes.c_int),
         }
         for name, (args, res) in sigs.items():
             fn = getattr(L, name)
@@ -243,6 +247,21 @@ def dsa_attention_forward(q_idx, w, k_idx_pages, q, latent_pages, cache: PagedCa
                                        ctypes.byref(dims.struct()), _ptr(idx_out), _ptr(out),
                                        _ptr(lse), _ptr(ws), ws.numel(), _stream(stream)),
            "dsa_attention_forward")
+
+
+def dsa_attention_forward_host(q_idx_h, w_h, k_idx_pages, q_h, latent_pages,
+                               cache_h: PagedCache, dims: Dims, idx_h, out_h, lse_h, ws,
+                               stream=None) -> None:
+    """The whole step with host buffers: q_idx_h, w_h, q_h, cache_h.seq_lens,
+    cache_h.block_table, idx_h (may be None), out_h and lse_h are CPU tensors
+    (pinned for an asynchronous call); the page pools and ws are CUDA tensors.
+    The host results are valid once the stream has reached the call."""
+    _check(lib().dsa_attention_forward_host(_ptr(q_idx_h), _ptr(w_h), _ptr(k_idx_pages),
+                                            _ptr(q_h), _ptr(latent_pages),
+                                            ctypes.byref(cache_h.struct()),
+                                            ctypes.byref(dims.struct()), _ptr(idx_h), _ptr(out_h),
+                                            _ptr(lse_h), _ptr(ws), ws.numel(), _stream(stream)),
+           "dsa_attention_forward_host")
 
 
 def dsa_cache_append(k_idx_new, latent_new, k_idx_pages, latent_pages, cache: PagedCache,

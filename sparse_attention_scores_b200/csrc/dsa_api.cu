@@ -214,6 +214,41 @@ size_t k8_region_bytes(const dsa_dims_t &d) {
   return k8_q_bytes(d) + align256(static_cast<size_t>(d.n_q) * d.H_I * 4);
 }
 
+// device staging of dsa_attention_forward_host, after the step's workspace:
+// q_idx, w, q, seq_lens, block_table, then idx, out, lse, each 256-aligned
+struct HostStage {
+  size_t q_idx, w, q, seq_lens, block_table, idx, out, lse;
+};
+HostStage host_stage_sizes(const dsa_dims_t &d, const dsa_cache_t &c) {
+  const size_t n = static_cast<size_t>(d.n_q);
+  HostStage h;
+  h.q_idx = n * d.H_I * d.D_I * 2;
+  h.w = n * d.H_I * 4;
+  h.q = n * d.H * (d.R + d.P) * 2;
+  h.seq_lens = static_cast<size_t>(c.num_seqs) * 4;
+  h.block_table = static_cast<size_t>(c.num_seqs) * c.max_pages * 4;
+  h.idx = n * d.topk * 4;
+  h.out = n * d.H * d.R * 4;
+  h.lse = n * d.H * 4;
+  return h;
+}
+// the device address of a pinned, mapped host buffer, or nullptr for memory
+// the device cannot address (pageable host memory, or not host memory at all)
+void *mapped_host(const void *p) {
+  cudaPointerAttributes at;
+  if (cudaPointerGetAttributes(&at, p) != cudaSuccess) {
+    cudaGetLastError();
+    return nullptr;
+  }
+  return (at.type == cudaMemoryTypeHost) ? at.devicePointer : nullptr;
+}
+
+size_t host_stage_bytes(const dsa_dims_t &d, const dsa_cache_t &c) {
+  const HostStage h = host_stage_sizes(d, c);
+  return align256(h.q_idx) + align256(h.w) + align256(h.q) + align256(h.seq_lens) +
+         align256(h.block_table) + align256(h.idx) + align256(h.out) + align256(h.lse);
+}
+
 size_t ws_bytes_for(dsa_op_t op, const dsa_dims_t &d, const dsa_cache_t &c) {
   switch (op) {
     case DSA_OP_INDEXER_SCORES:
@@ -233,6 +268,8 @@ size_t ws_bytes_for(dsa_op_t op, const dsa_dims_t &d, const dsa_cache_t &c) {
       return kStatusBytes + align256(scores) + align256(idx) +
              align256(mla_scratch_bytes(d.n_q, d.topk, d.R));
     }
+    case DSA_OP_ATTENTION_FORWARD_HOST:
+      return ws_bytes_for(DSA_OP_ATTENTION_FORWARD, d, c) + host_stage_bytes(d, c);
   }
   return 0;
 }
@@ -377,7 +414,8 @@ size_t dsa_workspace_bytes(dsa_op_t op, const dsa_dims_t *dims, const dsa_cache_
     return kStatusBytes;
   if (op == DSA_OP_INDEXER_SCORES_K8) return ws_bytes_for(op, *dims, dsa_cache_t{});
   if (check_mla_dims(*dims) != DSA_OK) return 0;
-  if ((op == DSA_OP_ATTENTION_FORWARD || op == DSA_OP_ATTENTION_FORWARD_K8) &&
+  if ((op == DSA_OP_ATTENTION_FORWARD || op == DSA_OP_ATTENTION_FORWARD_K8 ||
+       op == DSA_OP_ATTENTION_FORWARD_HOST) &&
       (cache == nullptr || check_cache(cache, *dims) != DSA_OK))
     return 0;
   dsa_cache_t empty = {};
@@ -458,6 +496,78 @@ dsa_status_t dsa_attention_forward(const uint16_t *q_idx, const float *w,
                                    float *lse, void *ws, size_t ws_bytes, dsa_stream_t stream) {
   return forward_entry(q_idx, w, k_idx_pages, nullptr, nullptr, q, latent_pages, cache, dims,
                        idx_out, out, lse, ws, ws_bytes, stream);
+}
+
+dsa_status_t dsa_attention_forward_host(const uint16_t *q_idx_h, const float *w_h,
+                                        const uint16_t *k_idx_pages, const uint16_t *q_h,
+                                        const uint16_t *latent_pages, const dsa_cache_t *cache_h,
+                                        const dsa_dims_t *dims, int32_t *idx_h, float *out_h,
+                                        float *lse_h, void *ws, size_t ws_bytes,
+                                        dsa_stream_t stream) {
+  DSA_TRY(check_dims_common(dims));
+  DSA_TRY(check_indexer_dims(*dims));
+  DSA_TRY(check_mla_dims(*dims));
+  DSA_TRY(check_cache(cache_h, *dims));
+  if (q_idx_h == nullptr || w_h == nullptr || k_idx_pages == nullptr || q_h == nullptr ||
+      latent_pages == nullptr || out_h == nullptr || lse_h == nullptr)
+    return DSA_ERR_INVALID_ARG;
+  if (!aligned16(k_idx_pages) || !aligned16(latent_pages)) return DSA_ERR_INVALID_ARG;
+  const dsa_dims_t &d = *dims;
+  const dsa_cache_t &ch = *cache_h;
+  const size_t fwd = ws_bytes_for(DSA_OP_ATTENTION_FORWARD, d, ch);  // a multiple of 256
+  DSA_TRY(check_ws(ws, ws_bytes, fwd + host_stage_bytes(d, ch)));
+  if (d.n_q == 0) return DSA_OK;
+  const HostStage h = host_stage_sizes(d, ch);
+  uint8_t *p = static_cast<uint8_t *>(ws) + fwd;
+  auto take = [&p](size_t bytes) {
+    uint8_t *r = p;
+    p += align256(bytes);
+    return r;
+  };
+  uint16_t *q_idx = reinterpret_cast<uint16_t *>(take(h.q_idx));
+  float *w = reinterpret_cast<float *>(take(h.w));
+  uint16_t *q = reinterpret_cast<uint16_t *>(take(h.q));
+  int32_t *seq_lens = reinterpret_cast<int32_t *>(take(h.seq_lens));
+  int32_t *block_table = reinterpret_cast<int32_t *>(take(h.block_table));
+  int32_t *idx = reinterpret_cast<int32_t *>(take(h.idx));
+  float *out = reinterpret_cast<float *>(take(h.out));
+  float *lse = reinterpret_cast<float *>(take(h.lse));
+  cudaStream_t s = as_stream(stream);
+  // Host buffers the device can address (pinned and mapped) move with one
+  // kernel each way; any other buffer with its own cudaMemcpyAsync.
+  CopyList in{}, out_l{};
+  bool ok = true;
+  auto add = [&](CopyList &l, const void *src, void *dst, size_t bytes, const void *host,
+                 bool to_device) {
+    void *mapped = mapped_host(host);
+    if (mapped != nullptr) {
+      CopyPiece &pc = l.piece[l.n++];
+      pc.src = to_device ? mapped : src;
+      pc.dst = to_device ? dst : mapped;
+      pc.bytes = bytes;
+    } else if (cudaMemcpyAsync(dst, src, bytes,
+                               to_device ? cudaMemcpyHostToDevice : cudaMemcpyDeviceToHost,
+                               s) != cudaSuccess) {
+      ok = false;
+    }
+  };
+  add(in, q_idx_h, q_idx, h.q_idx, q_idx_h, true);
+  add(in, w_h, w, h.w, w_h, true);
+  add(in, q_h, q, h.q, q_h, true);
+  add(in, ch.seq_lens, seq_lens, h.seq_lens, ch.seq_lens, true);
+  add(in, ch.block_table, block_table, h.block_table, ch.block_table, true);
+  if (!ok) return DSA_ERR_CUDA;
+  DSA_TRY(launch_copy_pieces(in, s));
+  dsa_cache_t cd = ch;
+  cd.seq_lens = seq_lens;
+  cd.block_table = block_table;
+  DSA_TRY(forward_entry(q_idx, w, k_idx_pages, nullptr, nullptr, q, latent_pages, &cd, dims,
+                        idx_h ? idx : nullptr, out, lse, ws, fwd, stream));
+  if (idx_h) add(out_l, idx, idx_h, h.idx, idx_h, false);
+  add(out_l, out, out_h, h.out, out_h, false);
+  add(out_l, lse, lse_h, h.lse, lse_h, false);
+  if (!ok) return DSA_ERR_CUDA;
+  return launch_copy_pieces(out_l, s);
 }
 
 dsa_status_t dsa_attention_forward_k8(const uint16_t *q_idx, const float *w,

@@ -97,6 +97,19 @@ struct TopkLaunch {
 };
 dsa_status_t launch_topk(const TopkLaunch &a, cudaStream_t stream);
 
+// several device-addressable buffers copied by one kernel (host-buffer step)
+constexpr int kMaxCopyPieces = 8;
+struct CopyPiece {
+  const void *src;
+  void *dst;
+  uint64_t bytes;
+};
+struct CopyList {
+  CopyPiece piece[kMaxCopyPieces];
+  int n;
+};
+dsa_status_t launch_copy_pieces(const CopyList &l, cudaStream_t stream);
+
 struct AppendLaunch {
   const uint16_t *k_new;
   const uint16_t *lat_new;

@@ -27,7 +27,7 @@ def _declared_symbols():
 
 def test_every_declared_symbol_is_exported(L):
     declared = _declared_symbols()
-    assert len(declared) == 20
+    assert len(declared) == 21
     assert sorted(declared) == sorted(dsa.EXPORTED)
     out = subprocess.run(["nm", "-D", "--defined-only", dsa.LIB_PATH], capture_output=True,
                          text=True, check=True).stdout
@@ -66,6 +66,12 @@ def test_workspace_bytes_host_only(L):
     assert n_fwd >= 256 + 8192 * 4 + 2048 * 4
     bad = _dims(R=100)
     assert L.dsa_workspace_bytes(dsa.OP_ATTENTION_FORWARD, ctypes.byref(bad), ctypes.byref(c)) == 0
+    # host-buffer step: the step's workspace, then the staged inputs and results
+    # (q_idx 8 KiB, w 128 B, q 72 KiB, seq_lens, block_table 512 B, idx 8 KiB,
+    # out 128 KiB, lse 256 B, each rounded up to 256 bytes)
+    n_host = L.dsa_workspace_bytes(dsa.OP_ATTENTION_FORWARD_HOST, ctypes.byref(d), ctypes.byref(c))
+    assert n_host == n_fwd + 8192 + 256 + 73728 + 256 + 512 + 8192 + 131072 + 256
+    assert L.dsa_workspace_bytes(dsa.OP_ATTENTION_FORWARD_HOST, ctypes.byref(d), None) == 0
 
 
 def _no_device():
@@ -180,3 +186,18 @@ def test_host_validation_rejects_without_launch(L):
     st = L.dsa_cache_append(fake, fake, fake, fake, ctypes.byref(c), ctypes.byref(d), ws, 16,
                             None)
     assert st == 4
+    # host-buffer step: missing host buffers, misaligned device pools, shapes,
+    # a workspace without room for the staging
+    hb = ctypes.c_void_p(0x500004)  # host buffers need no alignment
+    n_host = L.dsa_workspace_bytes(dsa.OP_ATTENTION_FORWARD_HOST, ctypes.byref(d), ctypes.byref(c))
+    n_fwd = L.dsa_workspace_bytes(dsa.OP_ATTENTION_FORWARD, ctypes.byref(d), ctypes.byref(c))
+    args = lambda **kw: dict(dict(qi=hb, w=hb, kp=fake, q=hb, lp=fake, c=ctypes.byref(c),
+                                  d=ctypes.byref(d), idx=hb, out=hb, lse=hb, ws=ws, n=n_host), **kw)
+    call = lambda a: L.dsa_attention_forward_host(a["qi"], a["w"], a["kp"], a["q"], a["lp"], a["c"],
+                                                  a["d"], a["idx"], a["out"], a["lse"], a["ws"],
+                                                  a["n"], None)
+    assert call(args(q=None)) == 1
+    assert call(args(out=None)) == 1
+    assert call(args(kp=ctypes.c_void_p(0x300008))) == 1
+    assert call(args(d=ctypes.byref(_dims(R=100)))) == 2
+    assert call(args(n=n_fwd)) == 4
