@@ -63,6 +63,7 @@ struct MlaParams {
   int nsplit, chunks_per_split;
   int kc;   // selected keys per chunk: 128, or 64 when few rows leave SMs idle
   int ncb;  // CTAs per (row, split): 1, or one per 128-column block of the output
+  int comb_ws;  // merge: warps per 128-column block (1, 2 or 4)
   float scale_log2;
   uint64_t wait_ns;
   int debug_stall;  // wait once on a barrier nothing arrives at (tests the time-out path)
@@ -519,62 +520,79 @@ __global__ void __launch_bounds__(kThreads, 1)
   }
 }
 
-// Merge the split partials of one (row, head, 128-column block):
+// Merge the split partials of (row, head) over 128-column blocks:
 //   out = sum_s 2^(m_s - M) O_s / sum_s 2^(m_s - M) l_s,  lse = (M + log2 L) ln 2.
-// One warp per CTA; each lane owns four consecutive columns.  Its 16-byte
-// loads of up to 16 splits are issued before the merge weights are known,
-// while the same lanes load every split's (m, l) (nsplit <= 64), so both wait
-// on memory once; the weights reach every lane by shuffles.
-__global__ void __launch_bounds__(32) combine_kernel(const MlaParams p) {
+// Four warps per CTA: ws = p.comb_ws warps share one column block (warp
+// taking every ws-th split) and the CTA covers 4 / ws blocks, so few splits
+// give fat CTAs and many splits give short load chains.  Each lane owns four
+// consecutive columns.  A warp issues the 16-byte loads of all its splits (at
+// most 16) before it computes the merge weights, while its lanes load every
+// split's (m, l) (nsplit <= 64), so it waits on memory once; the partial sums
+// of a block's warps meet in shared memory.
+constexpr int kCombineWarps = 4;
+__global__ void __launch_bounds__(32 * kCombineWarps) combine_kernel(const MlaParams p) {
   constexpr int kBatch = 16;
-  const int row = blockIdx.x, h = blockIdx.y, mb = blockIdx.z, nmb = gridDim.z;
-  const int lane = threadIdx.x;
+  __shared__ float4 part[kCombineWarps][32];
+  const int row = blockIdx.x, h = blockIdx.y;
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const int ws = p.comb_ws, sub = warp % ws;
+  const int mb = blockIdx.z * (kCombineWarps / ws) + warp / ws;
+  const int nmb = (p.R + 127) / 128;
   griddep_wait();
   griddep_launch_dependents();
+  const bool active = mb < nmb;  // warp-uniform
   const int c = 4 * lane;
-  const int64_t sstride = static_cast<int64_t>(nmb) * kHeads * 128;  // floats per split
-  const float *po =
-      p.part_o + (static_cast<int64_t>(row) * p.nsplit * nmb + mb) * kHeads * 128 + h * 128 + c;
-  const float *ml = p.part_ml + static_cast<int64_t>(row) * p.nsplit * 2 * kHeads;
-  float4 v[kBatch];
-#pragma unroll
-  for (int u = 0; u < kBatch; ++u)
-    v[u] = (u < p.nsplit) ? *reinterpret_cast<const float4 *>(po + u * sstride)
-                          : make_float4(0.f, 0.f, 0.f, 0.f);
-  const int s0 = lane, s1 = lane + 32;
-  const float m0 = (s0 < p.nsplit) ? ml[s0 * 2 * kHeads + h] : -INFINITY;
-  const float m1 = (s1 < p.nsplit) ? ml[s1 * 2 * kHeads + h] : -INFINITY;
-  const float l0 = (s0 < p.nsplit) ? ml[s0 * 2 * kHeads + kHeads + h] : 0.f;
-  const float l1 = (s1 < p.nsplit) ? ml[s1 * 2 * kHeads + kHeads + h] : 0.f;
-  float M = fmaxf(m0, m1);
-#pragma unroll
-  for (int o = 16; o > 0; o >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, o));
-  const float e0 = (m0 == -INFINITY) ? 0.f : exp2f(m0 - M);
-  const float e1 = (m1 == -INFINITY) ? 0.f : exp2f(m1 - M);
-  float L = e0 * l0 + e1 * l1;
-#pragma unroll
-  for (int o = 16; o > 0; o >>= 1) L += __shfl_xor_sync(0xffffffffu, L, o);
-  const float il = (L > 0.f) ? 1.f / L : 0.f;
-  const float w0 = e0 * il, w1 = e1 * il;  // normalised merge weights of splits lane, lane+32
-  if (lane == 0 && mb == 0)
-    p.lse[static_cast<int64_t>(row) * p.H + h] = (L > 0.f) ? (M + log2f(L)) * kLn2 : -INFINITY;
   float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-  for (int s = 0; s < p.nsplit; s += kBatch) {
-    if (s > 0) {
-#pragma unroll
-      for (int u = 0; u < kBatch; ++u)
-        v[u] = (s + u < p.nsplit) ? *reinterpret_cast<const float4 *>(po + (s + u) * sstride)
-                                  : make_float4(0.f, 0.f, 0.f, 0.f);
-    }
+  if (active) {
+    const int64_t sstride = static_cast<int64_t>(nmb) * kHeads * 128;  // floats per split
+    const float *po =
+        p.part_o + (static_cast<int64_t>(row) * p.nsplit * nmb + mb) * kHeads * 128 + h * 128 + c;
+    const float *ml = p.part_ml + static_cast<int64_t>(row) * p.nsplit * 2 * kHeads;
+    float4 v[kBatch];
 #pragma unroll
     for (int u = 0; u < kBatch; ++u) {
-      const int su = s + u;  // warp-uniform
-      const float w = __shfl_sync(0xffffffffu, su < 32 ? w0 : w1, su & 31);
-      acc.x += w * v[u].x; acc.y += w * v[u].y; acc.z += w * v[u].z; acc.w += w * v[u].w;
+      const int su = sub + ws * u;
+      v[u] = (su < p.nsplit) ? *reinterpret_cast<const float4 *>(po + su * sstride)
+                             : make_float4(0.f, 0.f, 0.f, 0.f);
+    }
+    const int s0 = lane, s1 = lane + 32;
+    const float m0 = (s0 < p.nsplit) ? ml[s0 * 2 * kHeads + h] : -INFINITY;
+    const float m1 = (s1 < p.nsplit) ? ml[s1 * 2 * kHeads + h] : -INFINITY;
+    const float l0 = (s0 < p.nsplit) ? ml[s0 * 2 * kHeads + kHeads + h] : 0.f;
+    const float l1 = (s1 < p.nsplit) ? ml[s1 * 2 * kHeads + kHeads + h] : 0.f;
+    float M = fmaxf(m0, m1);
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, o));
+    const float e0 = (m0 == -INFINITY) ? 0.f : exp2f(m0 - M);
+    const float e1 = (m1 == -INFINITY) ? 0.f : exp2f(m1 - M);
+    float L = e0 * l0 + e1 * l1;
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) L += __shfl_xor_sync(0xffffffffu, L, o);
+    const float il = (L > 0.f) ? 1.f / L : 0.f;
+    const float w0 = e0 * il, w1 = e1 * il;  // normalised merge weights of splits lane, lane+32
+    if (sub == 0 && lane == 0 && mb == 0)
+      p.lse[static_cast<int64_t>(row) * p.H + h] = (L > 0.f) ? (M + log2f(L)) * kLn2 : -INFINITY;
+#pragma unroll
+    for (int u = 0; u < kBatch; ++u) {
+      const int su = sub + ws * u;  // warp-uniform
+      if (su < p.nsplit) {
+        const float w = __shfl_sync(0xffffffffu, su < 32 ? w0 : w1, su & 31);
+        acc.x += w * v[u].x; acc.y += w * v[u].y; acc.z += w * v[u].z; acc.w += w * v[u].w;
+      }
+    }
+  }
+  if (ws > 1) {
+    part[warp][lane] = acc;
+    __syncthreads();
+    if (sub == 0) {
+      for (int q = 1; q < ws; ++q) {
+        const float4 b = part[warp + q][lane];
+        acc.x += b.x; acc.y += b.y; acc.z += b.z; acc.w += b.w;
+      }
     }
   }
   const int r = mb * 128 + c;
-  if (r < p.R) {
+  if (active && sub == 0 && r < p.R) {
     float *dst = p.out + (static_cast<int64_t>(row) * p.H + h) * p.R + r;  // 4-byte aligned only
     dst[0] = acc.x;
     dst[1] = acc.y;
@@ -679,12 +697,17 @@ dsa_status_t launch_mla(const MlaLaunch &a, cudaStream_t stream) {
   // few CTAs: one per 128-column block of the output as well, when that still fits one wave
   const int nmb = (a.R + 127) / 128;
   p.ncb = (nmb > 1 && static_cast<int64_t>(a.n_q) * sp.nsplit * nmb <= device_sm_count()) ? nmb : 1;
+  p.comb_ws = 1;
   if (launch_pdl(mla_kernel, dim3(sp.nsplit, a.n_q, p.ncb), dim3(kThreads), smem, stream, 1, p) !=
       cudaSuccess)
     return DSA_ERR_CUDA;
   if (sp.merge == kMergeGlobal) {
-    if (launch_pdl(combine_kernel, dim3(a.n_q, a.H, (a.R + 127) / 128), dim3(32), 0, stream, 1,
-                   p) != cudaSuccess)
+    // warps per column block: enough that each loads at most eight splits
+    p.comb_ws = sp.nsplit > 16 ? 4 : (sp.nsplit > 8 ? 2 : 1);
+    const int blocks_per_cta = kCombineWarps / p.comb_ws;
+    if (launch_pdl(combine_kernel,
+                   dim3(a.n_q, a.H, (nmb + blocks_per_cta - 1) / blocks_per_cta),
+                   dim3(32 * kCombineWarps), 0, stream, 1, p) != cudaSuccess)
       return DSA_ERR_CUDA;
   }
   return DSA_OK;
