@@ -388,13 +388,14 @@ TRAFFIC_SOURCES = {"indexer": ["indexer.cu"], "topk": ["topk.cu"], "mla": ["mla.
 TRAFFIC_COMMON = ["dsa_common.cuh", "dsa_internal.h"]
 TRAFFIC = {
     # (stage, workload): (bytes per launch, digest of the stage's sources)
-    ("indexer", "glm5_decode_8k"): (2164480, "ee2f6041a779d556"),
-    ("indexer", "glm5_decode_4x128k"): (134359040 + 4805120, "ee2f6041a779d556"),
-    ("topk", "glm5_decode_8k"): (70912, "5efcabd2a44e59af"),
-    ("topk", "glm5_decode_4x128k"): (2135808, "5efcabd2a44e59af"),
+    ("indexer", "glm5_decode_8k"): (2156800, "47b644e2cca64cae"),
+    ("indexer", "glm5_decode_4x128k"): (139531776, "47b644e2cca64cae"),
+    # topk_small_kernel at 8,192 keys, topk_creg_kernel at 4 x 131,072
+    ("topk", "glm5_decode_8k"): (52224, "731efc00e61e528a"),
+    ("topk", "glm5_decode_4x128k"): (2122240, "731efc00e61e528a"),
     # mla_kernel + combine_kernel (the merge reads the split partials)
-    ("mla", "glm5_decode_8k"): (2513920 + 4226304, "a69f3b783441a492"),
-    ("mla", "glm5_decode_4x128k"): (9870592 + 16858624, "a69f3b783441a492"),
+    ("mla", "glm5_decode_8k"): (2509824 + 4232448, "a1ef539e4d9cea7f"),
+    ("mla", "glm5_decode_4x128k"): (9864960 + 16864256, "a1ef539e4d9cea7f"),
 }
 
 
@@ -415,8 +416,8 @@ def traffic_of(stage, workload):
 
 
 STAGE_KERNELS = {"indexer": "indexer_kernel (tcgen05 + TMA)",
-                 "topk": "topk_kernel (cluster radix select)",
-                 "mla": "mla_kernel + combine_kernel (tcgen05 + TMA gather4, split merge)"}
+                 "topk": "topk_small_kernel / topk_creg_kernel (radix select, keys in registers)",
+                 "mla": "mla_kernel + combine_kernel (tcgen05, cp.async gather, split merge)"}
 
 
 def roofline_of(res, wl, peaks, k8=False):
