@@ -357,15 +357,17 @@ __global__ void __launch_bounds__(kThreads, 1) topk_kernel(const TopkParams p) {
   }
 }
 
-// Short rows (at most 16 x 1,024 keys): one CTA of 1,024 threads per row with
+// Short rows (at most 8 x 1,024 keys): one CTA of 1,024 threads per row with
 // the keys in registers, thread t holding keys [E*t, E*t + E), so thread order
 // is index order.  The same radix select over the varying bits and the same
 // kept set and output order as the cluster kernel, with block barriers in
 // place of cluster barriers and a block scan in place of the ordered walk.
 constexpr int kSmallThreads = 1024;
 constexpr int kSmallWarps = kSmallThreads / 32;
-constexpr int kSmallCopies = 8;  // private histograms, one per four warps
-constexpr int kSmallMaxLen = 16 * kSmallThreads;
+constexpr int kSmallCopies = 4;  // private histograms, one per eight warps
+constexpr int kWarpsPerCopy = kSmallWarps / kSmallCopies;
+// longer rows go to clusters: at 16K keys two CTAs beat one, at 8K one wins
+constexpr int kSmallMaxLen = 8 * kSmallThreads;
 constexpr size_t kSmallSmem = (static_cast<size_t>(kSmallCopies) * kBins + 2 * kSmallWarps + 4) * 4;
 
 template <int E>
@@ -442,7 +444,7 @@ __global__ void __launch_bounds__(kSmallThreads, 1) topk_small_kernel(const Topk
   const int lb = vary ? __ffs(vary) - 1 : 0;
   const int npass = vary ? (hb - lb + kDigitBits) / kDigitBits : 0;
   int krem = k;
-  uint32_t *mine = hist + (warp >> 2) * kBins;
+  uint32_t *mine = hist + (warp / kWarpsPerCopy) * kBins;
 #pragma unroll 1
   for (int pass = 0; pass < npass; ++pass) {
     const int shift = hb - kDigitBits * pass - (kDigitBits - 1);  // may be negative
@@ -634,7 +636,7 @@ __global__ void __launch_bounds__(kSmallThreads, 1) topk_creg_kernel(const TopkP
   const int lb = vary ? __ffs(vary) - 1 : 0;
   const int npass = vary ? (hb - lb + kDigitBits) / kDigitBits : 0;
   int krem = k;
-  uint32_t *mine = priv + (warp >> 2) * kBins;
+  uint32_t *mine = priv + (warp / kWarpsPerCopy) * kBins;
 #pragma unroll 1
   for (int pass = 0; pass < npass; ++pass) {
     const int shift = hb - kDigitBits * pass - (kDigitBits - 1);  // may be negative
@@ -833,15 +835,12 @@ dsa_status_t launch_topk(const TopkLaunch &a, cudaStream_t stream) {
       if (cudaFuncSetAttribute(topk_small_kernel<4>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                static_cast<int>(kSmallSmem)) != cudaSuccess ||
           cudaFuncSetAttribute(topk_small_kernel<8>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                               static_cast<int>(kSmallSmem)) != cudaSuccess ||
-          cudaFuncSetAttribute(topk_small_kernel<16>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                static_cast<int>(kSmallSmem)) != cudaSuccess)
         return DSA_ERR_CUDA;
       small_attr = true;
     }
-    void (*kern)(const TopkParams) = max_len <= 4 * kSmallThreads   ? topk_small_kernel<4>
-                                     : max_len <= 8 * kSmallThreads ? topk_small_kernel<8>
-                                                                    : topk_small_kernel<16>;
+    void (*kern)(const TopkParams) =
+        max_len <= 4 * kSmallThreads ? topk_small_kernel<4> : topk_small_kernel<8>;
     if (launch_pdl(kern, dim3(static_cast<unsigned>(a.n_q)), dim3(kSmallThreads), kSmallSmem, stream,
                    1u, p) != cudaSuccess)
       return DSA_ERR_CUDA;

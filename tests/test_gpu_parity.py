@@ -151,11 +151,11 @@ def test_topk_long_rows(n):
 @pytest.mark.parametrize("lengths", [
     [4096, 3000, 300],                 # one CTA per row, 4 keys per thread
     [8192, 8191, 2049],                # one CTA per row, 8 keys per thread
-    [16384, 9001, 12345],              # one CTA per row, 16 keys per thread
-    [16388, 16001],                    # clusters, 4 keys per thread
+    [16384, 9001, 12345],              # clusters of 4, 4 keys per thread
+    [16388, 16001],                    # clusters of 5, 4 keys per thread
     [131072, 70001],                   # clusters of 16, 8 keys per thread
     [65536] * 24 + [40000] * 8,        # 32 rows: clusters of 4, 16 keys per thread
-], ids=["small4", "small8", "small16", "cluster4", "cluster8", "cluster16"])
+], ids=["small4", "small8", "cluster4x4", "cluster5x4", "cluster16x8", "cluster4x16"])
 def test_topk_kernel_paths(kind, lengths):
     # each row set lands on one of the top-k kernels (chosen by the row count
     # and the longest row); the ragged rows of a launch share it
