@@ -45,6 +45,7 @@ constexpr int kHeads = 64;            // head columns of every tile = MMA N
 constexpr int kAtomL = kChunk * 128;  // bytes of one 64-column atom of the latent tile
 constexpr int kAtomQ = kHeads * 128;  // bytes of one 64-column atom of the query tile
 constexpr float kRescaleLog2 = 8.0f;
+constexpr int kMaxMergeCluster = 8;  // splits merged inside one cluster
 constexpr float kLn2 = 0.69314718055994531f;
 
 enum : int { kMergeNone = 0, kMergeGlobal = 1 };
@@ -64,6 +65,7 @@ struct MlaParams {
   int kc;   // selected keys per chunk: 128, or 64 when few rows leave SMs idle
   int ncb;  // CTAs per (row, split): 1, or one per 128-column block of the output
   int comb_ws;  // merge: warps per 128-column block (1, 2 or 4)
+  int cluster_merge;  // the row's splits form one cluster and merge through DSMEM
   float scale_log2;
   uint64_t wait_ns;
   int debug_stall;  // wait once on a barrier nothing arrives at (tests the time-out path)
@@ -130,8 +132,95 @@ __device__ __forceinline__ float butterfly32(Get v) {
   return op(up ? d[1] : d[0], __shfl_xor_sync(0xffffffffu, up ? d[0] : d[1], 1));
 }
 
-__global__ void __launch_bounds__(kThreads, 1)
-    mla_kernel(const MlaParams p) {
+// The split merge of a row whose splits are the CTAs of one cluster (only the
+// cluster instantiation of the kernel contains it).
+// The row's splits are the CTAs of this cluster.  Each one sends its (m, l) to
+// every CTA, then its O^T, scaled to the common maximum, in 32-column units
+// (32 latent columns x 64 heads, 8 KB) to the unit's owner CTA (unit u =
+// 4 mb + quadrant, owner u % C), into the owner's latent tile, which every CTA
+// has finished with at the first barrier.  An owner sums its units over the C
+// senders and writes the output.
+__device__ __forceinline__ void cluster_merge_epilogue(const MlaParams &p, uint8_t *Ls, float *ml_all,
+                                                    const float *mrun, const float *lrun,
+                                                    float *alpha, float *red, uint32_t tmem_ol,
+                                                    bool have_o, int row, int nmb) {
+  const int tid = threadIdx.x, warp = warp_id(), lane = lane_id();
+  const int q4 = warp & 3, hh = warp >> 2;
+  const int R = p.R;
+  const uint32_t C = cluster_nctarank(), me = cluster_ctarank();
+  if (tid < 2 * kHeads) {
+    const int h = tid & (kHeads - 1);
+    const float v = (tid < kHeads) ? mrun[h] : lrun[h];
+    const uint32_t a = smem_u32(&ml_all[(me * 2 + (tid >> 6)) * kHeads + h]);
+    for (uint32_t r = 0; r < C; ++r) st_dsmem_u32(map_to_rank(a, r), __float_as_uint(v));
+  }
+  cluster_sync();  // every split's loop is done and its (m, l) is everywhere
+  if (tid < kHeads) {
+    float M = -INFINITY;
+    for (uint32_t r = 0; r < C; ++r) M = fmaxf(M, ml_all[(r * 2) * kHeads + tid]);
+    float L = 0.f;
+    for (uint32_t r = 0; r < C; ++r) {
+      const float m = ml_all[(r * 2) * kHeads + tid];
+      if (m != -INFINITY) L += exp2f(m - M) * ml_all[(r * 2 + 1) * kHeads + tid];
+    }
+    alpha[tid] = (mrun[tid] == -INFINITY) ? 0.f : exp2f(mrun[tid] - M);  // this split's weight
+    red[tid] = (L > 0.f) ? 1.f / L : 0.f;
+    if (me == 0 && tid < p.H)
+      p.lse[static_cast<int64_t>(row) * p.H + tid] = (L > 0.f) ? (M + log2f(L)) * kLn2 : -INFINITY;
+  }
+  __syncthreads();
+  const uint32_t recv = smem_u32(Ls);  // [units / C][C senders][32 columns][64 heads]
+  for (int mb = 0; mb < nmb; ++mb) {
+    uint32_t v[32];
+    if (have_o) {
+      tmem_ld_32x32b_x32(tmem_ol + mb * kHeads + 32 * hh, v);
+      tmem_ld_wait();
+    }
+#pragma unroll
+    for (int i = 0; i < 32; ++i)
+      v[i] = have_o ? __float_as_uint(__uint_as_float(v[i]) * alpha[32 * hh + i]) : 0u;
+    const uint32_t u = static_cast<uint32_t>(mb * 4 + q4);
+    const uint32_t owner = u % C, slot = (u / C) * C + me;
+    // column `lane`, heads 32 hh + 4 jj .. +3, at lane * 64 + (h ^ 4 (lane & 7))
+    const uint32_t base = recv + (slot * 2048u + lane * 64u) * 4u;
+#pragma unroll
+    for (int jj = 0; jj < 8; ++jj) {
+      const uint32_t hsw = static_cast<uint32_t>((32 * hh + 4 * jj) ^ ((lane & 7) << 2));
+      st_dsmem_v4(map_to_rank(base + hsw * 4u, owner), v[4 * jj], v[4 * jj + 1], v[4 * jj + 2],
+                  v[4 * jj + 3]);
+    }
+  }
+  cluster_sync();  // every unit is in its owner's buffer; no remote access follows
+  const float *rbuf = reinterpret_cast<const float *>(Ls);
+  const uint32_t nunits = static_cast<uint32_t>(nmb * 4);
+  for (uint32_t j = 0; j * C + me < nunits; ++j) {
+    const uint32_t u = j * C + me;
+    const int col0 = static_cast<int>(u >> 2) * 128 + static_cast<int>(u & 3) * 32;
+    const int c = lane;
+#pragma unroll
+    for (int k = 0; k < 2; ++k) {
+      const int g = warp + 8 * k;  // heads 4g .. 4g+3
+      const int hsw = (4 * g) ^ ((c & 7) << 2);
+      float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+      for (uint32_t src = 0; src < C; ++src) {
+        const float4 x =
+            *reinterpret_cast<const float4 *>(rbuf + ((j * C + src) * 2048u + c * 64 + hsw));
+        acc.x += x.x; acc.y += x.y; acc.z += x.z; acc.w += x.w;
+      }
+      const float a4[4] = {acc.x, acc.y, acc.z, acc.w};
+      const int col = col0 + c;
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        const int h = 4 * g + i;
+        if (h < p.H && col < R)
+          p.out[(static_cast<int64_t>(row) * p.H + h) * R + col] = a4[i] * red[h];
+      }
+    }
+  }
+}
+
+template <bool kClusterMerge>
+__global__ void __launch_bounds__(kThreads, 1) mla_kernel(const MlaParams p) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                               ~static_cast<uintptr_t>(1023));
@@ -153,8 +242,10 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint64_t *bar_o = bar_s + 1;
   uint64_t *bar_drain = bar_o + 1;
   uint64_t *bar_stall = bar_drain + 1;
-  // [0] tmem base, [1] rescale flag, [2] failed
+  // [0] tmem base, [1] rescale flag, [2] failed, [3] pad
   uint32_t *misc = reinterpret_cast<uint32_t *>(bar_stall + 1);
+  // cluster merge: every split's (m, l) per head, [kMaxMergeCluster][2][64]
+  float *ml_all = reinterpret_cast<float *>(misc + 4);
 
   const int tid = threadIdx.x, warp = warp_id(), lane = lane_id();
   const int q4 = warp & 3;   // tensor-memory lane quadrant: keys / rows 32*q4 ..
@@ -449,7 +540,10 @@ __global__ void __launch_bounds__(kThreads, 1)
     __syncthreads();
   }
 
-  if (p.nsplit == 1) {
+  if constexpr (kClusterMerge) {
+    cluster_merge_epilogue(p, Ls, ml_all, mrun, lrun, alpha, red, tmem_o + lane_off, have_o, row,
+                           nmb);
+  } else if (p.nsplit == 1) {
     // the whole selection ran here: normalise and write the output
     for (int mi = 0; mi < nmb_l; ++mi) {
       uint32_t v[32];
@@ -609,7 +703,7 @@ size_t mla_smem_bytes(int R, int P) {
   const bool p_overlays = nL > 2 * nmb;
   return 1024 + static_cast<size_t>(nL) * kAtomL + (p_overlays ? 0 : kAtomL) +
          static_cast<size_t>(nQ) * kAtomQ + 4 * kChunk + 4 * (7 * kHeads) +
-         8 * 4 + 16;
+         8 * 4 + 16 + 4 * (kMaxMergeCluster * 2 * kHeads);
 }
 
 struct SplitPlan {
@@ -645,13 +739,44 @@ size_t mla_scratch_bytes(int n_q, int topk, int R) {
   return ((o + 255) & ~static_cast<size_t>(255)) + ml;
 }
 
+// whether clusters of `size` MLA CTAs with `smem` bytes each can be co-scheduled
+// (queried once per size and device)
+bool mla_cluster_ok(int size, size_t smem) {
+  static int cached[64][kMaxMergeCluster + 1];
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64 || size < 2 ||
+      size > kMaxMergeCluster)
+    return false;
+  if (cached[dev][size] == 0) {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(size, 1, 1);
+    cfg.blockDim = dim3(kThreads, 1, 1);
+    cfg.dynamicSmemBytes = smem;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = size;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    int n = 0;
+    const bool ok =
+        cudaOccupancyMaxActiveClusters(&n, mla_kernel<true>, &cfg) == cudaSuccess && n > 0;
+    cudaGetLastError();  // clear a rejected query
+    cached[dev][size] = ok ? 1 : -1;
+  }
+  return cached[dev][size] > 0;
+}
+
 dsa_status_t launch_mla(const MlaLaunch &a, cudaStream_t stream) {
   const int W = a.R + a.P;
   const size_t smem = mla_smem_bytes(a.R, a.P);
   if (smem > device_max_smem_optin()) return DSA_ERR_UNSUPPORTED;
   static bool attr_set = false;
   if (!attr_set) {
-    if (cudaFuncSetAttribute(mla_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+    if (cudaFuncSetAttribute(mla_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             static_cast<int>(device_max_smem_optin())) != cudaSuccess ||
+        cudaFuncSetAttribute(mla_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              static_cast<int>(device_max_smem_optin())) != cudaSuccess)
       return DSA_ERR_CUDA;
     attr_set = true;
@@ -698,10 +823,19 @@ dsa_status_t launch_mla(const MlaLaunch &a, cudaStream_t stream) {
   const int nmb = (a.R + 127) / 128;
   p.ncb = (nmb > 1 && static_cast<int64_t>(a.n_q) * sp.nsplit * nmb <= device_sm_count()) ? nmb : 1;
   p.comb_ws = 1;
-  if (launch_pdl(mla_kernel, dim3(sp.nsplit, a.n_q, p.ncb), dim3(kThreads), smem, stream, 1, p) !=
-      cudaSuccess)
-    return DSA_ERR_CUDA;
-  if (sp.merge == kMergeGlobal) {
+  // a row split over 2..8 CTAs that divide its 32-column units merges inside
+  // one cluster, when the device co-schedules such clusters
+  p.cluster_merge = (sp.merge == kMergeGlobal && p.ncb == 1 && sp.nsplit <= kMaxMergeCluster &&
+                     (nmb * 4) % sp.nsplit == 0 && mla_cluster_ok(sp.nsplit, smem))
+                        ? 1 : 0;
+  const cudaError_t le =
+      p.cluster_merge
+          ? launch_pdl(mla_kernel<true>, dim3(sp.nsplit, a.n_q, p.ncb), dim3(kThreads), smem,
+                       stream, static_cast<unsigned>(sp.nsplit), p)
+          : launch_pdl(mla_kernel<false>, dim3(sp.nsplit, a.n_q, p.ncb), dim3(kThreads), smem,
+                       stream, 1u, p);
+  if (le != cudaSuccess) return DSA_ERR_CUDA;
+  if (sp.merge == kMergeGlobal && !p.cluster_merge) {
     // warps per column block: enough that each loads at most eight splits
     p.comb_ws = sp.nsplit > 16 ? 4 : (sp.nsplit > 8 ? 2 : 1);
     const int blocks_per_cta = kCombineWarps / p.comb_ws;

@@ -198,7 +198,20 @@ def test_sparse_mla_decode_many_splits(batch):
     _mla_decode_case(dict(H=64, R=512, P=64, k=8192), batch)
 
 
-def _mla_decode_case(shape, batch):
+@pytest.mark.parametrize("shape,batch", [
+    (dict(H=64, R=512, P=64, k=2048), 10),   # 8 splits per row, merged in a cluster of 8
+    (dict(H=64, R=512, P=64, k=2048), 32),   # clusters of 4
+    (dict(H=64, R=512, P=64, k=2048), 74),   # clusters of 2
+    (dict(H=4, R=64, P=16, k=256), 40),      # one 128-column block, clusters of 2
+    (dict(H=16, R=192, P=32, k=2048), 10),   # a ragged last column block, clusters of 8
+], ids=["c8", "c4", "c2", "tiny_c2", "r192_c8"])
+def test_sparse_mla_cluster_merge(shape, batch):
+    # rows split over 2..8 CTAs merge their partials through distributed shared
+    # memory; short rows leave some splits empty and one row selects nothing
+    _mla_decode_case(shape, batch, every_row=True, empty_row=batch // 2)
+
+
+def _mla_decode_case(shape, batch, every_row=False, empty_row=None):
     rng = np.random.default_rng(batch * 7 + shape["k"])
     lengths = rng.integers(1, 3 * shape["k"], size=batch).tolist()
     wl = di.small_decode(lengths, H_I=4, D_I=32, topk=shape["k"], H=shape["H"], R=shape["R"],
@@ -207,14 +220,20 @@ def _mla_decode_case(shape, batch):
     t = upload(inp)
     cache, dims = cache_of(inp, t), dims_of(inp)
     sel = _random_selection(rng, lengths, shape["k"])
+    if empty_row is not None:
+        sel[empty_row, :] = -1
     idx = torch.from_numpy(sel).cuda()
-    out = torch.empty((batch, wl.H, wl.R), device="cuda")
-    lse = torch.empty((batch, wl.H), device="cuda")
+    out = torch.full((batch, wl.H, wl.R), float("nan"), device="cuda")
+    lse = torch.full((batch, wl.H), float("nan"), device="cuda")
     ws = dsa.workspace(dsa.OP_SPARSE_MLA_DECODE, dims, cache)
     dsa.dsa_sparse_mla_decode(t["q"], t["latent_pages"], cache, idx, dims, out, lse, ws)
     assert dsa.workspace_check(ws)[0] == 0
     out, lse = out.cpu().numpy(), lse.cpu().numpy()
-    for b in range(0, batch, max(1, batch // 12)):
+    if empty_row is not None:
+        assert (out[empty_row] == 0).all() and np.isneginf(lse[empty_row]).all()
+    for b in range(0, batch, 1 if every_row else max(1, batch // 12)):
+        if b == empty_row:
+            continue
         s = sel[b][sel[b] >= 0]
         rows = orc.bf16_to_f64(orc.gather_paged_rows(inp["latent_pages"], inp["block_table"][b], s))
         ref_out, ref_lse, _ = orc.mla_attention(orc.bf16_to_f64(inp["q"][b]), rows, wl.R, wl.scale)
