@@ -808,7 +808,10 @@ int max_topk_cluster(size_t smem) {
 }
 
 dsa_status_t launch_topk(const TopkLaunch &a, cudaStream_t stream) {
-  const int max_len = std::max(1, a.max_len);
+  // rounded up to a multiple of 4 like the rows' stride, so that every row's
+  // segment (at most the stride) fits the per-thread key count chosen here
+  const int max_len = static_cast<int>(
+      std::min<int64_t>(INT32_MAX & ~3, (std::max<int64_t>(1, a.max_len) + 3) & ~int64_t{3}));
   const size_t max_smem = device_max_smem_optin();
   static bool attr_set = false;
   if (!attr_set) {
