@@ -266,6 +266,31 @@ def test_sparse_mla_prefill_and_empty_rows():
         assert np.max(np.abs(lse[r] - ref_lse)) <= LSE_TOL
 
 
+@pytest.mark.parametrize("T,q_pos0,k,R,P,H", [(40, 0, 256, 64, 16, 4), (12, 3000, 2048, 512, 64, 64)],
+                         ids=["short_c2", "long_context_c8"])
+def test_sparse_mla_prefill_cluster_merge(T, q_pos0, k, R, P, H):
+    # a short prefill chunk splits its rows over 2..8 CTAs, which merge in a cluster
+    wl = di.small_prefill(T, q_pos0=q_pos0, H_I=4, D_I=32, topk=k, H=H, R=R, P=P, seed=T + 1)
+    inp = di.make_inputs(wl)
+    t = upload(inp)
+    cache, dims = cache_of(inp, t), dims_of(inp)
+    rng = np.random.default_rng(T)
+    sel = _random_selection(rng, [q_pos0 + r + 1 for r in range(T)], k)
+    idx = torch.from_numpy(sel).cuda()
+    out = torch.full((T, wl.H, wl.R), float("nan"), device="cuda")
+    lse = torch.full((T, wl.H), float("nan"), device="cuda")
+    ws = dsa.workspace(dsa.OP_SPARSE_MLA_PREFILL, dims, cache)
+    dsa.dsa_sparse_mla_prefill(t["q"], t["latent_pages"], cache, idx, dims, out, lse, ws)
+    assert dsa.workspace_check(ws)[0] == 0
+    out, lse = out.cpu().numpy(), lse.cpu().numpy()
+    for r in range(T):
+        s = sel[r][sel[r] >= 0]
+        rows = orc.bf16_to_f64(orc.gather_paged_rows(inp["latent_pages"], inp["block_table"][0], s))
+        ref_out, ref_lse, _ = orc.mla_attention(orc.bf16_to_f64(inp["q"][r]), rows, wl.R, wl.scale)
+        assert norm_err(out[r], ref_out) <= OUT_TOL, r
+        assert np.max(np.abs(lse[r] - ref_lse)) <= LSE_TOL, r
+
+
 # ---------------------------------------------------------------- whole step
 
 FORWARD_CASES = [
