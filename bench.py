@@ -6,11 +6,13 @@
 
 One step = one dsa_attention_forward call (indexer scores -> exact top-k ->
 sparse MLA -> split combine) over one batch of synthetic GLM-5-shaped input
-already resident in HBM.  The headline workload is the GLM-5-width decode
-(batch 1, context 8,192); every other workload is measured too and reported
-under "per_config".  L2 is flushed (a 512 MB read) before every timed step;
-each step is timed with CUDA events on the launching stream; multi-GPU runs
-are independent replicas (weak scaling) timed as the max over ranks.
+already resident in HBM.  The headline workload is the batched GLM-5-width
+decode (32 sequences, contexts 2,048-65,536, ragged paged caches), the largest
+workload that is a decode on one GPU; every other workload is measured too and
+reported under "per_config".  L2 is flushed (a 512 MB read) before every timed
+step; each step is timed with CUDA events on the launching stream; the same
+step with L2 left warm is reported as "hot".  Multi-GPU runs are independent
+replicas (weak scaling) timed as the max over ranks.
 
 `--impl reference` times the float64 CPU oracle on this host's cores on the
 same workload (bounded samples), with the same JSON keys.
@@ -34,8 +36,8 @@ sys.path.insert(0, ROOT)
 
 import dsa_inputs as di  # noqa: E402
 
-HEADLINE = "glm5_decode_8k"
-EXTRA = ["tiny_decode", "glm5_decode_b32_ragged", "glm5_prefill_2300", "glm5_decode_4x128k"]
+HEADLINE = "glm5_decode_b32_ragged"
+EXTRA = ["tiny_decode", "glm5_decode_8k", "glm5_prefill_2300", "glm5_decode_4x128k"]
 # the same workloads with the index keys held as E4M3 bytes + one scale per token
 EXTRA_K8 = ["glm5_decode_8k", "glm5_decode_b32_ragged", "glm5_decode_4x128k"]
 NOMINAL_HBM_GBS = 8000.0
@@ -293,16 +295,12 @@ class Case:
            self.ws)
 
     def launches_per_step(self):
-        # indexer + top-k + MLA, plus the split combine when a row is split
-        # (the same split rule as the library's launcher)
-        n_q, topk = self.wl.n_q, self.wl.topk
-        sms = self.torch.cuda.get_device_properties(0).multi_processor_count
-        kc = 64 if n_q * ((topk + 127) // 128) < sms // 2 else 128
-        nchunks = (topk + kc - 1) // kc
-        want = max(1, min((sms + n_q - 1) // n_q, min(nchunks, 64)))
-        cps = (nchunks + want - 1) // want
-        nsplit = (nchunks + cps - 1) // cps
-        return 3 + (1 if nsplit > 1 else 0)
+        # the library's own launch plan for these shapes on this device
+        op = self.dsa.OP_ATTENTION_FORWARD_K8 if self.k8 else self.dsa.OP_ATTENTION_FORWARD
+        n = self.dsa.forward_launches(op, self.dims, self.cache)
+        if n <= 0:
+            raise RuntimeError(f"no launch plan for {self.wl.name}")
+        return n
 
 
 def timed_events(torch, fn, steps, warmup, flush_buf):
@@ -324,10 +322,25 @@ def timed_events(torch, fn, steps, warmup, flush_buf):
     return sum(times) / len(times), times
 
 
+def timed_hot(torch, fn, steps, warmup):
+    """Mean ms of fn over `steps` back-to-back runs (L2 left warm)."""
+    for _ in range(warmup):
+        fn()
+    torch.cuda.synchronize()
+    ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    ev0.record()
+    for _ in range(steps):
+        fn()
+    ev1.record()
+    torch.cuda.synchronize()
+    return ev0.elapsed_time(ev1) / steps
+
+
 def measure(case, torch, steps, warmup, flush_buf, peaks, extras=True):
     wl = case.wl
     alg = algorithmic(wl, case.k8)
     ms, _ = timed_events(torch, case.step, steps, warmup, flush_buf)
+    ms_hot = timed_hot(torch, case.step, steps, warmup)
     st, info = case.dsa.workspace_check(case.ws)
     if st != 0:
         raise RuntimeError(f"device status {st} ({info:#x}) on {wl.name}")
@@ -346,6 +359,8 @@ def measure(case, torch, steps, warmup, flush_buf, peaks, extras=True):
         "alg_bytes": alg["bytes"], "alg_gbs": alg["bytes"] / s / 1e9,
         "frac_of_8tbs": alg["bytes"] / s / 1e9 / NOMINAL_HBM_GBS,
         "frac_of_measured_hbm": alg["bytes"] / s / 1e9 / peaks["hbm_gbs"],
+        "hot_us_per_step": ms_hot * 1e3,
+        "hot_tokens_per_s": wl.n_q / (ms_hot * 1e-3),
         "tflops": alg["flops"] / s / 1e12,
         "frac_of_bf16_peak": alg["flops"] / s / 1e12 / peaks["bf16_tflops"],
         "indexer_us": ms_idx * 1e3,
@@ -381,7 +396,7 @@ def measure(case, torch, steps, warmup, flush_buf, peaks, extras=True):
 
 
 # DRAM traffic per launch (dram__bytes_read.sum + dram__bytes_write.sum) of
-# each stage's kernels from one ncu capture (profiles/<kernel>_<workload>.md),
+# each stage's kernels from one ncu capture of that kernel on that workload,
 # with a digest of the sources the capture was taken on: the bench reports
 # the figure only while those sources are unchanged.
 TRAFFIC_SOURCES = {"indexer": ["indexer.cu"], "topk": ["topk.cu"], "mla": ["mla.cu"]}
@@ -445,11 +460,12 @@ def roofline_of(res, wl, peaks, k8=False):
             "peak_source": peaks["source"], "alg_bytes_per_launch": b, "launch_us": us}
 
 
-def measure_e2e(case, torch, steps, warmup):
+def measure_e2e(case, torch, steps, warmup, flush_buf):
     """Same metric through the C ABI's host-buffer entry point
     (dsa_attention_forward_host): every step copies its inputs in from pinned
     host memory and its results back, inside the timed region; the paged
-    caches stay resident in HBM."""
+    caches stay resident in HBM, and L2 is flushed before every step (outside
+    the timed region) as for the device-timed step."""
     dsa, t = case.dsa, case.t
     names_in = ["q_idx", "w", "q", "seq_lens", "block_table"]
     host_in = {k: t[k].cpu().pin_memory() for k in names_in}
@@ -467,22 +483,14 @@ def measure_e2e(case, torch, steps, warmup):
                                        t["latent_pages"], cache_h, case.dims, host_out["idx"],
                                        host_out["out"], host_out["lse"], hws)
 
-    for _ in range(warmup):
-        one()
-    torch.cuda.synchronize()
-    ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    ev0.record()
-    for _ in range(steps):
-        one()
-    ev1.record()
-    torch.cuda.synchronize()
+    ms, _ = timed_events(torch, one, steps, warmup, flush_buf)
     st, info = dsa.workspace_check(hws)
     if st != 0:
         raise RuntimeError(f"device status {st} ({info:#x}) in the host-buffer step")
-    ms = ev0.elapsed_time(ev1) / steps
     return {"value": case.wl.n_q / (ms * 1e-3), "unit": "tokens/s", "ms_per_step": ms,
             "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h),
-            "api": "dsa_attention_forward_host"}
+            "api": "dsa_attention_forward_host", "workload": case.wl.name,
+            "l2": "flushed (512 MB read) before every step, outside the timed region"}
 
 
 def measure_cp(wl, ranks, torch, dsa, steps, warmup, flush_buf):
@@ -565,11 +573,34 @@ def blas_threads():
         return os.cpu_count() or 1
 
 
+def cpu_model():
+    try:
+        with open("/proc/cpuinfo") as f:
+            for line in f:
+                if line.startswith("model name"):
+                    return line.split(":", 1)[1].strip()
+    except OSError:
+        pass
+    import platform
+    return platform.processor() or "unknown"
+
+
 def cpu_baseline(wl, budget_s=10.0):
+    """The oracle as it stands on this host: all BLAS threads, then one."""
     rate, n, el = oracle_rows_per_s(wl, budget_s)
-    return {"value": rate, "unit": "tokens/s", "cores": blas_threads(), "kind": "oracle",
-            "sample": f"{n} query rows of {wl.name} through the float64 oracle in {el:.1f} s "
-                      f"(host: {os.cpu_count()} logical cores)"}
+    res = {"value": rate, "unit": "tokens/s", "cores": blas_threads(), "kind": "oracle",
+           "sample": f"{n} query rows of {wl.name} through the float64 oracle in {el:.1f} s "
+                     f"(host: {os.cpu_count()} logical cores)",
+           "cpu_model": cpu_model(), "logical_cores": os.cpu_count()}
+    try:
+        from threadpoolctl import threadpool_limits
+        with threadpool_limits(limits=1):
+            r1, n1, el1 = oracle_rows_per_s(wl, budget_s / 2)
+        res["one_thread"] = {"value": r1, "unit": "tokens/s", "cores": 1,
+                             "sample": f"{n1} query rows in {el1:.1f} s with one BLAS thread"}
+    except Exception as e:   # threadpoolctl missing: report why
+        res["one_thread"] = {"unavailable": str(e)}
+    return res
 
 
 def run_ours(args):
@@ -612,7 +643,8 @@ def run_ours(args):
         dist.barrier()
     ms = max_over_ranks(head["us_per_step"] / 1e3, pg, "cuda")
     # the host-buffer entry point serves bf16 index keys
-    e2e = None if (args.profile or args.fp8_keys) else measure_e2e(case, torch, args.steps, args.warmup)
+    e2e = None if (args.profile or args.fp8_keys) else measure_e2e(case, torch, args.steps,
+                                                                    args.warmup, flush_buf)
     if e2e is not None:
         e2e["ms_per_step"] = max_over_ranks(e2e["ms_per_step"], pg, "cuda")
         e2e["value"] = job_rows_per_s(wl.n_q, world, e2e["ms_per_step"])
@@ -663,7 +695,12 @@ def run_ours(args):
                        "l2": "flushed (512 MB read) before every timed step",
                        "alg_bytes_per_step": alg["bytes"],
                        "achieved_gbs": alg["bytes"] / (ms * 1e-3) / 1e9,
+                       "frac_of_measured_hbm": alg["bytes"] / (ms * 1e-3) / 1e9 / peaks["hbm_gbs"],
+                       "hbm_peak_gbs": peaks["hbm_gbs"], "hbm_peak_source": peaks["source"],
                        "frac_of_8tbs": alg["bytes"] / (ms * 1e-3) / 1e9 / NOMINAL_HBM_GBS},
+            "hot": {"us_per_step": head["hot_us_per_step"],
+                    "tokens_per_s": head["hot_tokens_per_s"],
+                    "l2": "warm: steps back to back, no flush"},
             "roofline": roofline_of(head, wl, peaks, k8=args.fp8_keys),
             "stage_us": head["stage_us"],
             "e2e": e2e,

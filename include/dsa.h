@@ -131,6 +131,15 @@ DSA_API const char *dsa_status_string(dsa_status_t status);
  * contents are undefined between calls.  Returns 0 for invalid input. */
 DSA_API size_t dsa_workspace_bytes(dsa_op_t op, const dsa_dims_t *dims, const dsa_cache_t *cache);
 
+/* Number of kernels one dsa_attention_forward (op = DSA_OP_ATTENTION_FORWARD)
+ * or dsa_attention_forward_k8 (DSA_OP_ATTENTION_FORWARD_K8) call launches for
+ * these dims and cache on the current device: the indexer (plus the E4M3
+ * query split for FP8 keys), the top-k, the sparse MLA, and the split merge
+ * when a row's partial results meet in global memory.  A query of the launch
+ * plan with no counterpart on the pages; launches nothing.  Returns -1 for
+ * invalid input. */
+DSA_API int32_t dsa_forward_launches(dsa_op_t op, const dsa_dims_t *dims, const dsa_cache_t *cache);
+
 /* Clear the status block of a workspace (asynchronous on `stream`).  Call it
  * once after allocating a workspace and after reading an error. */
 DSA_API dsa_status_t dsa_workspace_init(void *ws, size_t ws_bytes, dsa_stream_t stream);
@@ -372,15 +381,24 @@ DSA_API dsa_status_t dsa_cp_merge(const float *outs, const float *lses, int32_t 
  * capture.  All calls on a device share the one array, and it keeps the last
  * call's contents: calls whose executions overlap on the GPU (different
  * streams, or different host threads) race on it and must be ordered by the
- * caller.  Device-side range-check events of this call are recorded in the
- * array's status block, which is cleared at the start of every call and is
- * not reported back; validate indices on the host, or use
- * dsa_sparse_mla_decode with a workspace when that check is needed.
+ * caller.  Device-side range-check events (a token index or page id out of
+ * range) and bounded-wait time-outs of this call are recorded in the array's
+ * status block, which is cleared at the start of every call; read it back
+ * with dsa_noalloc_status() after the call.
  * Allocates nothing: no cudaMalloc, no cudaFree, no allocating library call. */
 DSA_API dsa_status_t dsa_sparse_mla_decode_noalloc(const uint16_t *q, const uint16_t *latent_pages,
                                            const dsa_cache_t *cache, const int32_t *idx,
                                            const dsa_dims_t *dims, float *out, float *lse,
                                            dsa_stream_t stream);
+
+/* The device-side status of the last dsa_sparse_mla_decode_noalloc call on the
+ * current device (the status block of its built-in array), read on `stream`:
+ * synchronises `stream`, then returns DSA_OK, DSA_ERR_DEVICE_CHECK (an index
+ * or page id was out of range and skipped) or DSA_ERR_TIMEOUT (a bounded wait
+ * gave up), with the first event's code in *info when info is not NULL.
+ * Like the entry point it has no counterpart on the pages, and allocates
+ * nothing (one 256-byte device-to-host copy into the caller's stack). */
+DSA_API dsa_status_t dsa_noalloc_status(dsa_stream_t stream, uint32_t *info);
 
 #ifdef __cplusplus
 }

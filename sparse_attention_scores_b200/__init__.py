@@ -42,7 +42,7 @@ EXPORTED = ["dsa_version", "dsa_status_string", "dsa_workspace_bytes", "dsa_work
             "dsa_cache_append", "dsa_absorb_query", "dsa_project_values",
             "dsa_indexer_scores_k8", "dsa_attention_forward_k8", "dsa_cp_workspace_bytes",
             "dsa_cp_candidates", "dsa_cp_select", "dsa_cp_merge",
-            "dsa_attention_forward_host"]
+            "dsa_attention_forward_host", "dsa_noalloc_status", "dsa_forward_launches"]
 
 
 class DsaError(RuntimeError):
@@ -92,6 +92,8 @@ def lib() -> ctypes.CDLL:
             "dsa_attention_forward": ([vp, vp, vp, vp, vp, pc, pd, vp, vp, vp, vp, sz, vp],
                                       ctypes.c_int),
             "dsa_sparse_mla_decode_noalloc": ([vp, vp, pc, vp, pd, vp, vp, vp], ctypes.c_int),
+            "dsa_noalloc_status": ([vp, ctypes.POINTER(ctypes.c_uint32)], ctypes.c_int),
+            "dsa_forward_launches": ([ctypes.c_int, pd, pc], i32),
             "dsa_cache_append": ([vp, vp, vp, vp, pc, pd, vp, sz, vp], ctypes.c_int),
             "dsa_absorb_query": ([vp, vp, vp, vp, i32, i32, i32, i32, i32, vp, sz, vp],
                                  ctypes.c_int),
@@ -238,6 +240,20 @@ def dsa_sparse_mla_decode_noalloc(q, latent_pages, cache: PagedCache, idx, dims:
                                                ctypes.byref(cache.struct()), _ptr(idx),
                                                ctypes.byref(dims.struct()), _ptr(out), _ptr(lse),
                                                _stream(stream)), "dsa_sparse_mla_decode_noalloc")
+
+
+def forward_launches(op: int, dims: Dims, cache: PagedCache) -> int:
+    """Kernels one fused forward call launches for these shapes on the current device."""
+    return int(lib().dsa_forward_launches(op, ctypes.byref(dims.struct()),
+                                          ctypes.byref(cache.struct())))
+
+
+def noalloc_status(stream=None):
+    """(status, info) of the last no-alloc decode on the current device: its
+    device-side range checks and bounded waits (synchronises the stream)."""
+    info = ctypes.c_uint32(0)
+    st = lib().dsa_noalloc_status(_stream(stream), ctypes.byref(info))
+    return st, info.value
 
 
 def dsa_attention_forward(q_idx, w, k_idx_pages, q, latent_pages, cache: PagedCache, dims: Dims,

@@ -237,13 +237,10 @@ dsa_status_t launch_absorb_impl(const AbsorbLaunch &a, cudaStream_t stream) {
   while (nt > 16 && absorb_smem(K, nt, kProject) > device_max_smem_optin()) nt /= 2;
   if (absorb_smem(K, nt, kProject) > device_max_smem_optin()) return DSA_ERR_UNSUPPORTED;
   if (a.n <= 128) nt = std::min(nt, std::max(16, (a.n + 15) / 16 * 16));
-  static bool attr_set = false;
-  if (!attr_set) {
-    if (cudaFuncSetAttribute(absorb_kernel<kProject>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             static_cast<int>(device_max_smem_optin())) != cudaSuccess)
-      return DSA_ERR_CUDA;
-    attr_set = true;
-  }
+  if (func_attr_once(reinterpret_cast<const void *>(absorb_kernel<kProject>),
+                     cudaFuncAttributeMaxDynamicSharedMemorySize,
+                     static_cast<int>(device_max_smem_optin())) != cudaSuccess)
+    return DSA_ERR_CUDA;
   CUtensorMap tmW;
   // the weights as [H * K rows][M columns]; boxes of 64 columns x min(K, 256) rows
   if (!make_map_2d(&tmW, a.w, static_cast<uint64_t>(a.M), static_cast<uint64_t>(a.H) * K, 64,

@@ -5,6 +5,8 @@
 #include <string.h>
 
 #include <algorithm>
+#include <mutex>
+#include <vector>
 
 #include <cudaTypedefs.h>
 
@@ -126,6 +128,24 @@ size_t device_smem_per_sm() {
   return cached[d];
 }
 
+cudaError_t func_attr_once(const void *kernel, cudaFuncAttribute attr, int value) {
+  struct Entry {
+    int dev;
+    const void *kernel;
+    cudaFuncAttribute attr;
+    int value;
+  };
+  static std::mutex mu;
+  static std::vector<Entry> done;
+  const int d = current_device();
+  std::lock_guard<std::mutex> lock(mu);
+  for (const Entry &e : done)
+    if (e.dev == d && e.kernel == kernel && e.attr == attr && e.value == value) return cudaSuccess;
+  const cudaError_t err = cudaFuncSetAttribute(kernel, attr, value);
+  if (err == cudaSuccess && d >= 0) done.push_back(Entry{d, kernel, attr, value});
+  return err;
+}
+
 namespace {
 
 constexpr size_t kStatusBytes = sizeof(DevStatus);
@@ -145,6 +165,8 @@ int64_t max_keys(const dsa_dims_t &d, const dsa_cache_t &c) {
 int64_t scores_ld(const dsa_dims_t &d, const dsa_cache_t &c) {
   return std::max<int64_t>(4, (max_keys(d, c) + 3) & ~static_cast<int64_t>(3));
 }
+
+}  // namespace
 
 dsa_status_t check_dims_common(const dsa_dims_t *d) {
   if (d == nullptr) return DSA_ERR_INVALID_ARG;
@@ -172,15 +194,6 @@ dsa_status_t check_cache(const dsa_cache_t *c, const dsa_dims_t &d) {
   return DSA_OK;
 }
 
-dsa_status_t check_indexer_dims(const dsa_dims_t &d) {
-  if (d.H_I < 1 || d.H_I > 64) return DSA_ERR_UNSUPPORTED;
-  if (d.D_I != 32 && d.D_I != 64 && d.D_I != 128) return DSA_ERR_UNSUPPORTED;
-  // the indexer walks row groups out of a shared-memory table
-  const int64_t groups = d.causal ? (d.n_q + 3) / 4 : d.n_q;
-  if (groups > 8192) return DSA_ERR_UNSUPPORTED;
-  return DSA_OK;
-}
-
 dsa_status_t check_mla_dims(const dsa_dims_t &d) {
   if (d.topk < 1 || d.topk > 65536) return DSA_ERR_UNSUPPORTED;
   if (d.H < 1 || d.H > 64) return DSA_ERR_UNSUPPORTED;
@@ -188,6 +201,17 @@ dsa_status_t check_mla_dims(const dsa_dims_t &d) {
   if (d.P < 0 || d.P % 16 != 0 || d.R + d.P > 576) return DSA_ERR_UNSUPPORTED;
   if (!isfinite(d.scale)) return DSA_ERR_INVALID_ARG;
   if (d.n_q > 65535) return DSA_ERR_UNSUPPORTED;  // grid.y
+  return DSA_OK;
+}
+
+namespace {
+
+dsa_status_t check_indexer_dims(const dsa_dims_t &d) {
+  if (d.H_I < 1 || d.H_I > 64) return DSA_ERR_UNSUPPORTED;
+  if (d.D_I != 32 && d.D_I != 64 && d.D_I != 128) return DSA_ERR_UNSUPPORTED;
+  // the indexer walks row groups out of a shared-memory table
+  const int64_t groups = d.causal ? (d.n_q + 3) / 4 : d.n_q;
+  if (groups > 8192) return DSA_ERR_UNSUPPORTED;
   return DSA_OK;
 }
 
@@ -420,6 +444,17 @@ size_t dsa_workspace_bytes(dsa_op_t op, const dsa_dims_t *dims, const dsa_cache_
     return 0;
   dsa_cache_t empty = {};
   return ws_bytes_for(op, *dims, cache ? *cache : empty);
+}
+
+int32_t dsa_forward_launches(dsa_op_t op, const dsa_dims_t *dims, const dsa_cache_t *cache) {
+  if (op != DSA_OP_ATTENTION_FORWARD && op != DSA_OP_ATTENTION_FORWARD_K8) return -1;
+  if (check_dims_common(dims) != DSA_OK || check_indexer_dims(*dims) != DSA_OK ||
+      check_mla_dims(*dims) != DSA_OK || check_cache(cache, *dims) != DSA_OK)
+    return -1;
+  if (dims->n_q == 0) return 0;
+  // indexer (+ the E4M3 query split for FP8 keys), top-k, sparse MLA (+ merge)
+  return (op == DSA_OP_ATTENTION_FORWARD_K8 ? 3 : 2) +
+         mla_launch_count(dims->n_q, dims->topk, dims->R, dims->P);
 }
 
 dsa_status_t dsa_workspace_init(void *ws, size_t ws_bytes, dsa_stream_t stream) {

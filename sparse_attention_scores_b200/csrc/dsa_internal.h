@@ -25,6 +25,17 @@ constexpr uint64_t kDrainLimitNs = 1000000000ull;
 
 int device_sm_count();
 
+// Sets a kernel's function attribute (e.g. its dynamic shared-memory opt-in)
+// on the current device, once per (device, kernel, attribute).  Attributes
+// belong to the device's copy of the kernel, so a process that drives several
+// GPUs sets them on each.  Thread-safe.
+cudaError_t func_attr_once(const void *kernel, cudaFuncAttribute attr, int value);
+
+// Host-side argument checks shared by the entry points (dsa_api.cu).
+dsa_status_t check_dims_common(const dsa_dims_t *d);
+dsa_status_t check_mla_dims(const dsa_dims_t &d);
+dsa_status_t check_cache(const dsa_cache_t *c, const dsa_dims_t &d);
+
 // 2-D bf16 tensor map over `rows` rows of `cols` elements (row pitch cols * 2
 // bytes) with a box of box_cols x box_rows and a 128- (aw = 128) or 64-byte
 // (aw = 64) swizzle.  Returns false when the driver entry point is missing or
@@ -170,5 +181,7 @@ struct MlaLaunch {
 int mla_num_splits(int n_q, int topk);
 size_t mla_scratch_bytes(int n_q, int topk, int R);
 dsa_status_t launch_mla(const MlaLaunch &a, cudaStream_t stream);
+// Kernels launch_mla launches for these shapes on the current device (1 or 2).
+int mla_launch_count(int n_q, int topk, int R, int P);
 
 }  // namespace dsa

@@ -577,14 +577,10 @@ dsa_status_t launch_impl(const IndexerLaunch &a, cudaStream_t stream) {
   if (stages < 2) return DSA_ERR_UNSUPPORTED;
   const size_t smem = fixed + stages * stage_bytes;
 
-  static bool attr_set = false;  // per template instantiation
-  if (!attr_set) {
-    if (cudaFuncSetAttribute(indexer_kernel<G, AW, NEG, K8>,
-                             cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             static_cast<int>(max_smem)) != cudaSuccess)
-      return DSA_ERR_CUDA;
-    attr_set = true;
-  }
+  if (func_attr_once(reinterpret_cast<const void *>(indexer_kernel<G, AW, NEG, K8>),
+                     cudaFuncAttributeMaxDynamicSharedMemorySize,
+                     static_cast<int>(max_smem)) != cudaSuccess)
+    return DSA_ERR_CUDA;
   const int64_t max_keys = a.causal ? static_cast<int64_t>(a.q_pos0) + a.n_q : a.max_seq_len;
   const int64_t max_units = static_cast<int64_t>(num_groups) * ((max_keys + kTileKeys - 1) / kTileKeys);
   const int per_sm = (NEG == 1) ? 2 : 1;

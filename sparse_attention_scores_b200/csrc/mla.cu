@@ -148,6 +148,9 @@ __device__ __forceinline__ void cluster_merge_epilogue(const MlaParams &p, uint8
   const int q4 = warp & 3, hh = warp >> 2;
   const int R = p.R;
   const uint32_t C = cluster_nctarank(), me = cluster_ctarank();
+  // every CTA of the cluster arrived (relaxed) at kernel entry: once this wait
+  // returns, all of them have started and their shared memory may be written
+  cluster_wait();
   if (tid < 2 * kHeads) {
     const int h = tid & (kHeads - 1);
     const float v = (tid < kHeads) ? mrun[h] : lrun[h];
@@ -247,6 +250,9 @@ __global__ void __launch_bounds__(kThreads, 1) mla_kernel(const MlaParams p) {
   // cluster merge: every split's (m, l) per head, [kMaxMergeCluster][2][64]
   float *ml_all = reinterpret_cast<float *>(misc + 4);
 
+  // the cluster merge writes into peers' shared memory: arrive now, wait
+  // (for every peer to have started) just before the first remote store
+  if constexpr (kClusterMerge) cluster_arrive_relaxed();
   const int tid = threadIdx.x, warp = warp_id(), lane = lane_id();
   const int q4 = warp & 3;   // tensor-memory lane quadrant: keys / rows 32*q4 ..
   const int hh = warp >> 2;  // head half: heads 32*hh ..
@@ -768,19 +774,27 @@ bool mla_cluster_ok(int size, size_t smem) {
   return cached[dev][size] > 0;
 }
 
+int mla_launch_count(int n_q, int topk, int R, int P) {
+  const SplitPlan sp = plan_splits(n_q, topk);
+  if (sp.merge != kMergeGlobal) return 1;
+  const int nmb = (R + 127) / 128;
+  const int ncb = (nmb > 1 && static_cast<int64_t>(n_q) * sp.nsplit * nmb <= device_sm_count()) ? nmb : 1;
+  const bool cluster = ncb == 1 && sp.nsplit <= kMaxMergeCluster && (nmb * 4) % sp.nsplit == 0 &&
+                       mla_cluster_ok(sp.nsplit, mla_smem_bytes(R, P));
+  return cluster ? 1 : 2;
+}
+
 dsa_status_t launch_mla(const MlaLaunch &a, cudaStream_t stream) {
   const int W = a.R + a.P;
   const size_t smem = mla_smem_bytes(a.R, a.P);
   if (smem > device_max_smem_optin()) return DSA_ERR_UNSUPPORTED;
-  static bool attr_set = false;
-  if (!attr_set) {
-    if (cudaFuncSetAttribute(mla_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             static_cast<int>(device_max_smem_optin())) != cudaSuccess ||
-        cudaFuncSetAttribute(mla_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             static_cast<int>(device_max_smem_optin())) != cudaSuccess)
-      return DSA_ERR_CUDA;
-    attr_set = true;
-  }
+  if (func_attr_once(reinterpret_cast<const void *>(mla_kernel<false>),
+                     cudaFuncAttributeMaxDynamicSharedMemorySize,
+                     static_cast<int>(device_max_smem_optin())) != cudaSuccess ||
+      func_attr_once(reinterpret_cast<const void *>(mla_kernel<true>),
+                     cudaFuncAttributeMaxDynamicSharedMemorySize,
+                     static_cast<int>(device_max_smem_optin())) != cudaSuccess)
+    return DSA_ERR_CUDA;
   const SplitPlan sp = plan_splits(a.n_q, a.topk);
   MlaParams p;
   p.q = a.q;

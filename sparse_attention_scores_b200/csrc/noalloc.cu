@@ -50,25 +50,19 @@ using namespace dsa;
 extern "C" DSA_API dsa_status_t dsa_sparse_mla_decode_noalloc(
     const uint16_t *q, const uint16_t *latent_pages, const dsa_cache_t *cache, const int32_t *idx,
     const dsa_dims_t *dims, float *out, float *lse, dsa_stream_t stream) {
-  if (dims == nullptr || cache == nullptr) return DSA_ERR_INVALID_ARG;
+  // the same host checks as dsa_sparse_mla_decode (decode rows only)
+  dsa_status_t chk = check_dims_common(dims);
+  if (chk != DSA_OK) return chk;
+  if (dims->causal != 0) return DSA_ERR_INVALID_ARG;
+  if ((chk = check_mla_dims(*dims)) != DSA_OK) return chk;
+  if ((chk = check_cache(cache, *dims)) != DSA_OK) return chk;
   const dsa_dims_t &d = *dims;
-  const dsa_cache_t &c = *cache;
-  if (d.n_q < 0 || d.causal != 0 || d.q_pos0 != 0) return DSA_ERR_INVALID_ARG;
-  if (d.topk < 1 || d.topk > 65536 || d.H < 1 || d.H > 64) return DSA_ERR_UNSUPPORTED;
-  if (d.R < 64 || d.R > 512 || d.R % 64 != 0) return DSA_ERR_UNSUPPORTED;
-  if (d.P < 0 || d.P % 16 != 0 || d.R + d.P > 576 || d.n_q > 65535) return DSA_ERR_UNSUPPORTED;
-  if (!isfinite(d.scale)) return DSA_ERR_INVALID_ARG;
-  if (c.seq_lens == nullptr || c.block_table == nullptr || c.page_size != kPageSize)
-    return c.page_size != kPageSize ? DSA_ERR_UNSUPPORTED : DSA_ERR_INVALID_ARG;
-  if (c.num_seqs != d.n_q || c.max_pages < 1 || c.num_pages < 1 || c.max_seq_len < 0 ||
-      static_cast<int64_t>(c.max_seq_len) > static_cast<int64_t>(c.max_pages) * kPageSize)
-    return DSA_ERR_INVALID_ARG;
   if (q == nullptr || latent_pages == nullptr || idx == nullptr || out == nullptr || lse == nullptr)
     return DSA_ERR_INVALID_ARG;
   if (!aligned_to(q, 16) || !aligned_to(latent_pages, 16) || !aligned_to(idx, 4) ||
-      !aligned_to(out, 4) || !aligned_to(lse, 4) || !aligned_to(c.seq_lens, 4) ||
-      !aligned_to(c.block_table, 4))
+      !aligned_to(out, 4) || !aligned_to(lse, 4))
     return DSA_ERR_INVALID_ARG;
+  const dsa_cache_t &c = *cache;
   // the built-in array holds the status block and the split partials
   const size_t need = sizeof(DevStatus) + mla_scratch_bytes(d.n_q, d.topk, d.R);
   if (need > kNoAllocScratchBytes) return DSA_ERR_WORKSPACE;
@@ -105,4 +99,21 @@ extern "C" DSA_API dsa_status_t dsa_sparse_mla_decode_noalloc(
   a.scratch_bytes = kNoAllocScratchBytes - sizeof(DevStatus);
   a.status = reinterpret_cast<DevStatus *>(base);
   return launch_mla(a, s);
+}
+
+extern "C" DSA_API dsa_status_t dsa_noalloc_status(dsa_stream_t stream, uint32_t *info) {
+  int dev = -1;
+  if (cudaGetDevice(&dev) != cudaSuccess) return DSA_ERR_CUDA;
+  dsa_status_t st = DSA_OK;
+  const void *base = scratch_address(dev, &st);
+  if (st != DSA_OK) return st;
+  cudaStream_t s = stream ? reinterpret_cast<cudaStream_t>(stream) : cudaStreamPerThread;
+  DevStatus host;
+  if (cudaMemcpyAsync(&host, base, sizeof(host), cudaMemcpyDeviceToHost, s) != cudaSuccess)
+    return DSA_ERR_CUDA;
+  if (cudaStreamSynchronize(s) != cudaSuccess) return DSA_ERR_CUDA;
+  if (info) *info = host.first;
+  if (host.flags & kErrTimeout) return DSA_ERR_TIMEOUT;
+  if (host.flags != 0u) return DSA_ERR_DEVICE_CHECK;
+  return DSA_OK;
 }

@@ -781,8 +781,8 @@ int max_cluster_of(void (*kern)(const TopkParams), int threads, size_t smem, int
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return 8;
   if (cached[dev] == 0) {
     int best = 8;
-    if (cudaFuncSetAttribute(kern, cudaFuncAttributeNonPortableClusterSizeAllowed, 1) ==
-        cudaSuccess) {
+    if (func_attr_once(reinterpret_cast<const void *>(kern),
+                       cudaFuncAttributeNonPortableClusterSizeAllowed, 1) == cudaSuccess) {
       cudaLaunchConfig_t cfg = {};
       cfg.gridDim = dim3(16, 1, 1);
       cfg.blockDim = dim3(threads, 1, 1);
@@ -813,13 +813,10 @@ dsa_status_t launch_topk(const TopkLaunch &a, cudaStream_t stream) {
   const int max_len = static_cast<int>(
       std::min<int64_t>(INT32_MAX & ~3, (std::max<int64_t>(1, a.max_len) + 3) & ~int64_t{3}));
   const size_t max_smem = device_max_smem_optin();
-  static bool attr_set = false;
-  if (!attr_set) {
-    if (cudaFuncSetAttribute(topk_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             static_cast<int>(max_smem)) != cudaSuccess)
-      return DSA_ERR_CUDA;
-    attr_set = true;
-  }
+  if (func_attr_once(reinterpret_cast<const void *>(topk_kernel),
+                     cudaFuncAttributeMaxDynamicSharedMemorySize,
+                     static_cast<int>(max_smem)) != cudaSuccess)
+    return DSA_ERR_CUDA;
   TopkParams p;
   p.scores = a.scores;
   p.ld = a.ld;
@@ -833,15 +830,13 @@ dsa_status_t launch_topk(const TopkLaunch &a, cudaStream_t stream) {
   p.status = a.status;
   if (max_len <= kSmallMaxLen) {
     // short rows: one CTA per row, keys in registers
-    static bool small_attr = false;
-    if (!small_attr) {
-      if (cudaFuncSetAttribute(topk_small_kernel<4>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                               static_cast<int>(kSmallSmem)) != cudaSuccess ||
-          cudaFuncSetAttribute(topk_small_kernel<8>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                               static_cast<int>(kSmallSmem)) != cudaSuccess)
-        return DSA_ERR_CUDA;
-      small_attr = true;
-    }
+    if (func_attr_once(reinterpret_cast<const void *>(topk_small_kernel<4>),
+                       cudaFuncAttributeMaxDynamicSharedMemorySize,
+                       static_cast<int>(kSmallSmem)) != cudaSuccess ||
+        func_attr_once(reinterpret_cast<const void *>(topk_small_kernel<8>),
+                       cudaFuncAttributeMaxDynamicSharedMemorySize,
+                       static_cast<int>(kSmallSmem)) != cudaSuccess)
+      return DSA_ERR_CUDA;
     void (*kern)(const TopkParams) =
         max_len <= 4 * kSmallThreads ? topk_small_kernel<4> : topk_small_kernel<8>;
     if (launch_pdl(kern, dim3(static_cast<unsigned>(a.n_q)), dim3(kSmallThreads), kSmallSmem, stream,
@@ -854,26 +849,23 @@ dsa_status_t launch_topk(const TopkLaunch &a, cudaStream_t stream) {
   C = std::min(C, std::max(1, device_sm_count() / std::max(1, a.n_q)));
   {
     // segments of at most 16K keys: 1,024 threads per CTA, keys in registers
-    static bool reg_attr = false;
     static int reg_cached[64];
-    if (!reg_attr) {
-      if (cudaFuncSetAttribute(topk_creg_kernel<4>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                               static_cast<int>(kRegSmem)) != cudaSuccess ||
-          cudaFuncSetAttribute(topk_creg_kernel<8>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                               static_cast<int>(kRegSmem)) != cudaSuccess ||
-          cudaFuncSetAttribute(topk_creg_kernel<16>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                               static_cast<int>(kRegSmem)) != cudaSuccess)
+    for (const void *k : {reinterpret_cast<const void *>(topk_creg_kernel<4>),
+                          reinterpret_cast<const void *>(topk_creg_kernel<8>),
+                          reinterpret_cast<const void *>(topk_creg_kernel<16>)})
+      if (func_attr_once(k, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                         static_cast<int>(kRegSmem)) != cudaSuccess)
         return DSA_ERR_CUDA;
-      reg_attr = true;
-    }
     const int Cr = std::max(1, std::min(C, max_cluster_of(topk_creg_kernel<16>, kSmallThreads,
                                                           kRegSmem, reg_cached)));
     const int seg_r = ((max_len + Cr - 1) / Cr + 3) & ~3;
     if (seg_r <= kRegMaxSeg) {
       if (Cr > 8) {
-        cudaFuncSetAttribute(topk_creg_kernel<4>, cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
-        cudaFuncSetAttribute(topk_creg_kernel<8>, cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
-        cudaFuncSetAttribute(topk_creg_kernel<16>, cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
+        for (const void *k : {reinterpret_cast<const void *>(topk_creg_kernel<4>),
+                              reinterpret_cast<const void *>(topk_creg_kernel<8>),
+                              reinterpret_cast<const void *>(topk_creg_kernel<16>)})
+          if (func_attr_once(k, cudaFuncAttributeNonPortableClusterSizeAllowed, 1) != cudaSuccess)
+            return DSA_ERR_CUDA;
       }
       void (*kern)(const TopkParams) = seg_r <= 4 * kSmallThreads   ? topk_creg_kernel<4>
                                        : seg_r <= 8 * kSmallThreads ? topk_creg_kernel<8>

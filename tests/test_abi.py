@@ -27,7 +27,7 @@ def _declared_symbols():
 
 def test_every_declared_symbol_is_exported(L):
     declared = _declared_symbols()
-    assert len(declared) == 21
+    assert len(declared) == 23
     assert sorted(declared) == sorted(dsa.EXPORTED)
     out = subprocess.run(["nm", "-D", "--defined-only", dsa.LIB_PATH], capture_output=True,
                          text=True, check=True).stdout
@@ -94,6 +94,27 @@ def test_noalloc_size_check_host_only(L):
     st = L.dsa_sparse_mla_decode_noalloc(fake, fake, ctypes.byref(c), fake, ctypes.byref(d),
                                          fake, fake, None)
     assert st == 4
+
+
+def test_noalloc_shares_the_workspace_entry_checks(L):
+    _no_device()
+    fake = ctypes.c_void_p(0x300000)
+    # a page pool whose token rows overflow a 32-bit row index: rejected as
+    # unsupported, exactly like the workspace entry point, before any launch
+    big = _cache(num_pages=1 << 25)
+    d = _dims()
+    st_ws = L.dsa_sparse_mla_decode(fake, fake, ctypes.byref(big), fake, ctypes.byref(d), fake,
+                                    fake, ctypes.c_void_p(0x400000), 1 << 30, None)
+    st = L.dsa_sparse_mla_decode_noalloc(fake, fake, ctypes.byref(big), fake, ctypes.byref(d),
+                                         fake, fake, None)
+    assert st_ws == 2 and st == 2
+    # prefill rows, a batch whose sequence count differs from n_q, a bad page size
+    assert L.dsa_sparse_mla_decode_noalloc(fake, fake, ctypes.byref(_cache()), fake,
+                                           ctypes.byref(_dims(causal=1)), fake, fake, None) == 1
+    assert L.dsa_sparse_mla_decode_noalloc(fake, fake, ctypes.byref(_cache(num_seqs=2)), fake,
+                                           ctypes.byref(d), fake, fake, None) == 1
+    assert L.dsa_sparse_mla_decode_noalloc(fake, fake, ctypes.byref(_cache(page_size=32)), fake,
+                                           ctypes.byref(d), fake, fake, None) == 2
 
 
 def test_host_validation_rejects_without_launch(L):

@@ -83,6 +83,47 @@ def test_indexer_scores_prefill_exact(T, q_pos0, H_I, D_I):
         assert np.isnan(got[r, n:]).all()
 
 
+def test_indexer_scores_normal_inputs_within_fp32_bound():
+    # N(0,1) bf16 queries and keys and positive real head weights: the scores
+    # are no longer exact in fp32.  Each bf16 product is exact in fp32; the
+    # D_I-term dot product, the weighting and the H_I-term head sum each add
+    # at most one fp32 rounding (2^-23 relative, allowing truncation) per term,
+    # so |gpu - exact| <= 2^-23 (D_I + H_I + 2) sum_h w_h sum_d |q_hd k_d|.
+    wl = di.small_decode([5000, 1234, 64, 3001], H_I=32, D_I=128, topk=512, H=4, R=64, P=16,
+                         seed=61)
+    inp = di.make_inputs(wl)
+    rng = np.random.default_rng(62)
+    inp["q_idx"] = di.f32_to_bf16_bits(rng.standard_normal(inp["q_idx"].shape).astype(np.float32))
+    inp["k_pages"] = di.f32_to_bf16_bits(rng.standard_normal(inp["k_pages"].shape).astype(np.float32))
+    inp["w"] = np.abs(rng.standard_normal(inp["w"].shape)).astype(np.float32)
+    t = upload(inp)
+    cache, dims = cache_of(inp, t), dims_of(inp)
+    ld = (max(wl.seq_lens) + 3) // 4 * 4
+    scores = torch.full((wl.n_q, ld), float("nan"), device="cuda")
+    ws = dsa.workspace(dsa.OP_INDEXER_SCORES, dims, cache)
+    dsa.dsa_indexer_scores(t["q_idx"], t["w"], t["k_pages"], cache, dims, scores, ws)
+    assert dsa.workspace_check(ws)[0] == 0
+    got = scores.cpu().numpy()
+    # the selection the library makes from those scores
+    idx = torch.full((wl.n_q, wl.topk), -7, dtype=torch.int32, device="cuda")
+    dsa.dsa_topk(scores, t["seq_lens"], 0, wl.topk, idx, ws)
+    assert dsa.workspace_check(ws)[0] == 0
+    idx = idx.cpu().numpy()
+    D_I, H_I = wl.D_I, wl.H_I
+    for b, n in enumerate(wl.seq_lens):
+        k_rows = orc.bf16_to_f64(orc.gather_paged_rows(inp["k_pages"], inp["block_table"][b],
+                                                       range(n)))
+        q = orc.bf16_to_f64(inp["q_idx"][b])
+        w = inp["w"][b].astype(np.float64)
+        ref = orc.indexer_scores(q, inp["w"][b], k_rows)
+        bound = 2.0 ** -23 * (D_I + H_I + 2) * (np.abs(k_rows) @ np.abs(q).T) @ w
+        err = np.abs(got[b, :n].astype(np.float64) - ref)
+        assert np.all(err <= bound), (b, float(np.max(err / np.maximum(bound, 1e-300))))
+        # exact top-k of the GPU's own fp32 scores (both sides decide in fp32)
+        want = orc.topk_select(got[b, :n].astype(np.float64), wl.topk)
+        np.testing.assert_array_equal(idx[b].astype(np.int64), want)
+
+
 # ---------------------------------------------------------------- step 2
 
 def _topk_rows(lengths, k, seed, kind):
