@@ -178,7 +178,7 @@ def small_prefill(T, *, q_pos0=0, H_I=4, D_I=32, topk=64, H=8, R=64, P=16, seed=
                     shuffle_pages=shuffle_pages, q_pos0=q_pos0, value_kind=value_kind)
 
 
-__all__ = ["Workload", "CONFIGS", "CONFIG_ORDER", "make_inputs", "f32_to_bf16_bits",
+__all__ = ["Workload", "CONFIGS", "CONFIG_ORDER", "make_inputs", "f32_to_bf16_bits", "with_fp8_latent",
            "small_decode", "small_prefill", "ragged_lengths", "pages_needed", "PAGE_SIZE",
            "replace", "field"]
 
@@ -200,6 +200,31 @@ def with_fp8_keys(inp: dict, seed: int = 0, max_shift: int = 7) -> dict:
     out = dict(inp)
     out["k8_pages"] = codes.numpy()
     out["k_scale"] = np.exp2(-j).astype(np.float32).reshape(-1)
+    return out
+
+
+def with_fp8_latent(inp: dict, seed: int = 0, max_shift: int = 4) -> dict:
+    """The same inputs with the latent cache held as E4M3 bytes plus one fp32
+    scale per token.  Each token's latent row x (the bf16 values) is stored as
+    the codes of x * 2^j and the scale 2^-j, j drawn per token in
+    [0, max_shift] (seeded); the codes come from torch's float8_e4m3fn
+    conversion (round to nearest even).  The returned "latent_pages" is
+    replaced by the bf16 bits of the rows the codes stand for (exact: every
+    E4M3 value times a power of two in this range is a bf16 value), so the
+    bf16 and the FP8 inputs describe the same latent cache."""
+    import torch
+    lat = (inp["latent_pages"].astype(np.uint32) << 16).view(np.float32)   # bf16 -> f32, exact
+    if np.abs(lat).max() * 2 ** max_shift > 448:
+        raise ValueError("latent values too large for E4M3 at this shift")
+    rng = np.random.default_rng(np.random.PCG64([seed, 0x1A7]))
+    j = rng.integers(0, max_shift + 1, lat.shape[:2])                    # one shift per token
+    scaled = lat * np.exp2(j)[..., None].astype(np.float32)
+    codes = torch.from_numpy(np.ascontiguousarray(scaled)).to(torch.float8_e4m3fn)
+    back = (codes.to(torch.float32).numpy() * np.exp2(-j)[..., None].astype(np.float32))
+    out = dict(inp)
+    out["latent8_pages"] = codes.view(torch.uint8).numpy()
+    out["latent_scale"] = np.exp2(-j).astype(np.float32).reshape(-1)
+    out["latent_pages"] = f32_to_bf16_bits(back)
     return out
 
 

@@ -83,6 +83,15 @@ def dequantize_keys(k8_rows: np.ndarray, scale_rows: np.ndarray) -> np.ndarray:
     return np.asarray(scale_rows, np.float64).reshape(-1, 1) * e4m3_to_f64(k8_rows)
 
 
+def dequantize_latent(l8_rows: np.ndarray, scale_rows: np.ndarray) -> np.ndarray:
+    """Latent rows from E4M3 codes [n, W] and one fp32 scale per token [n]
+    ("GLM on an A100, in Vx", section "INT4, FP8 and BF16": E4M3 bytes with a
+    float32 scale per block; here the block is one token's whole latent row
+    [c_kv | k_rope]).  The dequantized row serves as key and value exactly as a
+    bf16 row does: z uses all W columns, V the first R."""
+    return np.asarray(scale_rows, np.float64).reshape(-1, 1) * e4m3_to_f64(l8_rows)
+
+
 # --------------------------------------------------------------------------
 # paged cache lookup
 # --------------------------------------------------------------------------
@@ -295,6 +304,11 @@ def _query_row(inp, r, table_row, n):
         k_rows = bf16_to_f64(gather_paged_rows(inp["k_pages"], table_row, np.arange(n)))
 
     def latent_of(sel):
+        if "latent8_pages" in inp:   # FP8 latent rows with one scale per token
+            codes = gather_paged_rows(inp["latent8_pages"], table_row, sel)
+            scales = gather_paged_rows(np.asarray(inp["latent_scale"]).reshape(-1, PAGE_SIZE, 1),
+                                       table_row, sel)
+            return dequantize_latent(codes, scales)
         return bf16_to_f64(gather_paged_rows(inp["latent_pages"], table_row, sel))
 
     return dsa_query(bf16_to_f64(inp["q_idx"][r]), np.asarray(inp["w"][r], np.float64),

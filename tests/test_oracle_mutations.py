@@ -192,6 +192,11 @@ def _dequantize_scale_ignored(k8_rows, scale_rows):
     return orc.e4m3_to_f64(k8_rows)
 
 
+def _dequantize_scale_squared(rows, scale_rows):
+    s = np.asarray(scale_rows, np.float64).reshape(-1, 1)
+    return s * s * orc.e4m3_to_f64(rows)
+
+
 def _cp_merge_ties_to_higher_index(cand_s, cand_i, k):
     s = np.asarray(cand_s, np.float64).reshape(-1)
     i = np.asarray(cand_i, np.int64).reshape(-1)
@@ -243,6 +248,9 @@ MUTANTS = {
     "cp: candidate ties to the higher index": ("cp_merge_candidates", _cp_merge_ties_to_higher_index),
     "cp: partials averaged without LSE weights": ("cp_merge_partials", _cp_merge_partials_unweighted),
     "fp8 keys: scale ignored": ("dequantize_keys", _dequantize_scale_ignored),
+    "fp8 latent: scale ignored": ("dequantize_latent", _dequantize_scale_ignored),
+    "fp8 latent: scale applied to the codes' exponent twice": ("dequantize_latent",
+                                                               _dequantize_scale_squared),
     "append: the next token's position": ("append_positions", _append_positions_of_the_next_token),
 }
 

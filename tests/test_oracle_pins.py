@@ -447,6 +447,42 @@ def test_fp8_key_scale_is_a_factor_of_the_score():
     np.testing.assert_allclose(s2, scale * s1, rtol=1e-12)
 
 
+# ---------------------------------------------------------------- FP8 latent cache
+
+def test_fp8_latent_stands_for_the_same_latent_and_attention():
+    # codes of x * 2^j with scale 2^-j stand for the latent x exactly, so the
+    # whole step over the FP8 cache equals the step over the bf16 cache
+    wl = di.small_decode([300, 129], H_I=4, D_I=32, topk=64, H=3, R=64, P=16, seed=33,
+                         shuffle_pages=True)
+    inp = di.with_fp8_latent(di.make_inputs(wl), seed=5)
+    assert inp["latent8_pages"].dtype == np.uint8
+    assert inp["latent_scale"].shape == (inp["latent_pages"].shape[0] * 64,)
+    assert len(set(inp["latent_scale"].tolist())) > 1      # the scales vary per token
+    W = wl.R + wl.P
+    deq = orc.dequantize_latent(inp["latent8_pages"].reshape(-1, W), inp["latent_scale"])
+    np.testing.assert_array_equal(deq, orc.bf16_to_f64(inp["latent_pages"]).reshape(-1, W))
+    bf = {k: v for k, v in inp.items() if k not in ("latent8_pages", "latent_scale")}
+    r_bf, r_l8 = orc.dsa_decode(bf), orc.dsa_decode(inp)
+    for b in r_bf:
+        assert np.array_equal(r_bf[b]["idx"], r_l8[b]["idx"])
+        np.testing.assert_array_equal(r_bf[b]["out"], r_l8[b]["out"])
+        np.testing.assert_array_equal(r_bf[b]["lse"], r_l8[b]["lse"])
+
+
+def test_fp8_latent_single_token_closed_form():
+    # one selected token: out is its dequantized c_kv part, lse its logit
+    rng = np.random.default_rng(43)
+    codes = rng.integers(0, 256, (1, 40)).astype(np.uint8)
+    codes[(codes & 0x7F) == 0x7F] = 0                      # no NaN codes
+    scale = np.array([0.375])
+    q = rng.standard_normal((2, 40))
+    row = orc.dequantize_latent(codes, scale)
+    out, lse, p = orc.mla_attention(q, row, 32, 0.5)
+    np.testing.assert_array_equal(out, np.repeat(0.375 * orc.e4m3_to_f64(codes[:, :32]), 2, axis=0))
+    np.testing.assert_allclose(lse, 0.5 * (q @ (0.375 * orc.e4m3_to_f64(codes[0]))), rtol=1e-12)
+    assert np.all(p == 1.0)
+
+
 # ---------------------------------------------------------------- context-parallel decode
 
 @pytest.mark.parametrize("ranks", [2, 3, 5])
