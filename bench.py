@@ -40,6 +40,8 @@ HEADLINE = "glm5_decode_b32_ragged"
 EXTRA = ["tiny_decode", "glm5_decode_8k", "glm5_prefill_2300", "glm5_decode_4x128k"]
 # the same workloads with the index keys held as E4M3 bytes + one scale per token
 EXTRA_K8 = ["glm5_decode_8k", "glm5_decode_b32_ragged", "glm5_decode_4x128k"]
+# ... and with both caches (index keys and latent rows) in that format
+EXTRA_FP8 = ["glm5_decode_b32_ragged", "glm5_decode_4x128k", "glm5_decode_8k"]
 NOMINAL_HBM_GBS = 8000.0
 FLUSH_BYTES = 512 << 20
 
@@ -67,20 +69,22 @@ def row_lengths(wl):
     return list(wl.seq_lens)
 
 
-def algorithmic(wl, k8=False):
+def algorithmic(wl, k8=False, l8=False):
     """Must-move bytes and flops of one step (scores and page tables excluded).
-    k8: the index keys as E4M3 bytes plus a 4-byte scale per token."""
+    k8: the index keys as E4M3 bytes plus a 4-byte scale per token; l8: the
+    latent rows likewise."""
     lens = row_lengths(wl)
     keys = sum(lens)
     sel = sum(min(wl.topk, n) for n in lens)
     key_bytes = (wl.D_I + 4) if k8 else wl.D_I * 2
+    row_bytes = (wl.W + 4) if l8 else wl.W * 2
     b_keys = keys * key_bytes
-    b_lat = sel * wl.W * 2
+    b_lat = sel * row_bytes
     b_small = wl.n_q * (wl.H * wl.W * 2 + wl.H_I * wl.D_I * 2 + wl.H_I * 4 + wl.H * wl.R * 4
                         + wl.H * 4)
     if wl.mode == "prefill":   # every row reads the same (L2-resident) cache
         b_keys = (wl.q_pos0 + wl.n_q) * key_bytes
-        b_lat = (wl.q_pos0 + wl.n_q) * wl.W * 2
+        b_lat = (wl.q_pos0 + wl.n_q) * row_bytes
     flops_idx = 2 * wl.H_I * wl.D_I * keys
     flops_mla = sel * wl.H * 2 * (wl.W + wl.R)
     # indexer kernel alone: key rows read + fp32 score per key written
@@ -186,11 +190,15 @@ def job_rows_per_s(rows_per_rank: int, world: int, ms_per_step: float) -> float:
 class Case:
     """Device-resident inputs, outputs and workspace of one workload."""
 
-    def __init__(self, wl, torch, dsa, k8=False):
+    def __init__(self, wl, torch, dsa, k8=False, l8=False):
         self.wl = wl
-        self.k8 = k8
+        self.k8 = k8 or l8      # the FP8 latent cache goes with FP8 index keys
+        self.l8 = l8
         self.inp = di.make_inputs(wl)
+        if l8:   # the latent rows as E4M3 bytes with one scale per token
+            self.inp = di.with_fp8_latent(self.inp, seed=wl.seed)
         inp = self.inp
+        k8 = self.k8
         dev = "cuda"
 
         def bf(x):
@@ -205,6 +213,10 @@ class Case:
             self.t["k8_pages"] = torch.from_numpy(k8in["k8_pages"]).to(dev)
             self.t["k_scale"] = torch.from_numpy(k8in["k_scale"]).to(dev)
             del self.t["k_pages"]
+        if l8:
+            self.t["latent8_pages"] = torch.from_numpy(inp["latent8_pages"]).to(dev)
+            self.t["latent_scale"] = torch.from_numpy(inp["latent_scale"]).to(dev)
+            del self.t["latent_pages"]
         self.cache = dsa.PagedCache(self.t["seq_lens"], self.t["block_table"],
                                     num_pages=int(inp["k_pages"].shape[0]),
                                     max_seq_len=int(inp["seq_lens"].max()))
@@ -214,7 +226,8 @@ class Case:
         self.idx = torch.empty((wl.n_q, wl.topk), dtype=torch.int32, device=dev)
         self.out = torch.empty((wl.n_q, wl.H, wl.R), dtype=torch.float32, device=dev)
         self.lse = torch.empty((wl.n_q, wl.H), dtype=torch.float32, device=dev)
-        self.ws = dsa.workspace(dsa.OP_ATTENTION_FORWARD_K8 if k8 else dsa.OP_ATTENTION_FORWARD,
+        self.ws = dsa.workspace(dsa.OP_ATTENTION_FORWARD_FP8 if l8 else
+                                dsa.OP_ATTENTION_FORWARD_K8 if k8 else dsa.OP_ATTENTION_FORWARD,
                                 self.dims, self.cache)
         ld = max(4, (max(row_lengths(wl)) + 3) // 4 * 4)
         self.scores = torch.empty((wl.n_q, ld), dtype=torch.float32, device=dev)
@@ -243,7 +256,12 @@ class Case:
 
     def step(self):
         t = self.t
-        if self.k8:
+        if self.l8:
+            self.dsa.dsa_attention_forward_fp8(t["q_idx"], t["w"], t["k8_pages"], t["k_scale"],
+                                               t["q"], t["latent8_pages"], t["latent_scale"],
+                                               self.cache, self.dims, self.idx, self.out,
+                                               self.lse, self.ws)
+        elif self.k8:
             self.dsa.dsa_attention_forward_k8(t["q_idx"], t["w"], t["k8_pages"], t["k_scale"],
                                               t["q"], t["latent_pages"], self.cache, self.dims,
                                               self.idx, self.out, self.lse, self.ws)
@@ -289,6 +307,12 @@ class Case:
 
     def mla(self):
         t = self.t
+        if self.l8:
+            fn = (self.dsa.dsa_sparse_mla_prefill_l8 if self.wl.mode == "prefill"
+                  else self.dsa.dsa_sparse_mla_decode_l8)
+            fn(t["q"], t["latent8_pages"], t["latent_scale"], self.cache, self.idx, self.dims,
+               self.out, self.lse, self.ws)
+            return
         fn = (self.dsa.dsa_sparse_mla_prefill if self.wl.mode == "prefill"
               else self.dsa.dsa_sparse_mla_decode)
         fn(t["q"], t["latent_pages"], self.cache, self.idx, self.dims, self.out, self.lse,
@@ -296,7 +320,8 @@ class Case:
 
     def launches_per_step(self):
         # the library's own launch plan for these shapes on this device
-        op = self.dsa.OP_ATTENTION_FORWARD_K8 if self.k8 else self.dsa.OP_ATTENTION_FORWARD
+        op = (self.dsa.OP_ATTENTION_FORWARD_FP8 if self.l8 else
+              self.dsa.OP_ATTENTION_FORWARD_K8 if self.k8 else self.dsa.OP_ATTENTION_FORWARD)
         n = self.dsa.forward_launches(op, self.dims, self.cache)
         if n <= 0:
             raise RuntimeError(f"no launch plan for {self.wl.name}")
@@ -338,7 +363,7 @@ def timed_hot(torch, fn, steps, warmup):
 
 def measure(case, torch, steps, warmup, flush_buf, peaks, extras=True):
     wl = case.wl
-    alg = algorithmic(wl, case.k8)
+    alg = algorithmic(wl, case.k8, case.l8)
     ms, _ = timed_events(torch, case.step, steps, warmup, flush_buf)
     ms_hot = timed_hot(torch, case.step, steps, warmup)
     st, info = case.dsa.workspace_check(case.ws)
@@ -354,6 +379,7 @@ def measure(case, torch, steps, warmup, flush_buf, peaks, extras=True):
     s = ms * 1e-3
     res = {
         "workload": wl.name, "mode": wl.mode, "index_keys": "e4m3+scale" if case.k8 else "bf16",
+        "latent_rows": "e4m3+scale" if case.l8 else "bf16",
         "us_per_step": ms * 1e3,
         "tokens_per_s": wl.n_q / s,
         "alg_bytes": alg["bytes"], "alg_gbs": alg["bytes"] / s / 1e9,
@@ -438,6 +464,7 @@ STAGE_KERNELS = {"indexer": "indexer_kernel (tcgen05 + TMA)",
 
 
 def roofline_of(res, wl, peaks, k8=False):
+    # (FP8 variants pass k8=True: the recorded DRAM traffic is of the bf16 caches)
     """Roofline of the stage that takes the longest alone: algorithmic bytes
     (or flops, for the tensor-bound prefill MLA) over its event time."""
     stage = max(res["stage_us"], key=res["stage_us"].get)
@@ -673,6 +700,16 @@ def run_ours(args):
             r["us_per_step"] = max_over_ranks(r["us_per_step"], pg, "cuda")
             r["roofline"] = roofline_of(r, c.wl, peaks, k8=True)
             per_config[name + "+fp8_keys"] = r
+            del c
+            torch.cuda.empty_cache()
+        for name in EXTRA_FP8:
+            c = Case(replica_workload(di.CONFIGS[name], rank), torch, dsa, l8=True)
+            c.step()
+            torch.cuda.synchronize()
+            r = measure(c, torch, args.steps, args.warmup, flush_buf, peaks, extras=False)
+            r["us_per_step"] = max_over_ranks(r["us_per_step"], pg, "cuda")
+            r["roofline"] = roofline_of(r, c.wl, peaks, k8=True)
+            per_config[name + "+fp8_cache"] = r
             del c
             torch.cuda.empty_cache()
 

@@ -213,18 +213,25 @@ def with_fp8_latent(inp: dict, seed: int = 0, max_shift: int = 4) -> dict:
     E4M3 value times a power of two in this range is a bf16 value), so the
     bf16 and the FP8 inputs describe the same latent cache."""
     import torch
-    lat = (inp["latent_pages"].astype(np.uint32) << 16).view(np.float32)   # bf16 -> f32, exact
-    if np.abs(lat).max() * 2 ** max_shift > 448:
-        raise ValueError("latent values too large for E4M3 at this shift")
+    pages = inp["latent_pages"]
     rng = np.random.default_rng(np.random.PCG64([seed, 0x1A7]))
-    j = rng.integers(0, max_shift + 1, lat.shape[:2])                    # one shift per token
-    scaled = lat * np.exp2(j)[..., None].astype(np.float32)
-    codes = torch.from_numpy(np.ascontiguousarray(scaled)).to(torch.float8_e4m3fn)
-    back = (codes.to(torch.float32).numpy() * np.exp2(-j)[..., None].astype(np.float32))
+    j = rng.integers(0, max_shift + 1, pages.shape[:2])                  # one shift per token
+    codes_all = np.empty(pages.shape, np.uint8)
+    bits_all = np.empty(pages.shape, np.uint16)
+    for p0 in range(0, pages.shape[0], 2048):                           # bounded host memory
+        p1 = min(p0 + 2048, pages.shape[0])
+        lat = (pages[p0:p1].astype(np.uint32) << 16).view(np.float32)   # bf16 -> f32, exact
+        if np.abs(lat).max() * 2 ** max_shift > 448:
+            raise ValueError("latent values too large for E4M3 at this shift")
+        scaled = lat * np.exp2(j[p0:p1])[..., None].astype(np.float32)
+        codes = torch.from_numpy(np.ascontiguousarray(scaled)).to(torch.float8_e4m3fn)
+        back = codes.to(torch.float32).numpy() * np.exp2(-j[p0:p1])[..., None].astype(np.float32)
+        codes_all[p0:p1] = codes.view(torch.uint8).numpy()
+        bits_all[p0:p1] = f32_to_bf16_bits(back)
     out = dict(inp)
-    out["latent8_pages"] = codes.view(torch.uint8).numpy()
+    out["latent8_pages"] = codes_all
     out["latent_scale"] = np.exp2(-j).astype(np.float32).reshape(-1)
-    out["latent_pages"] = f32_to_bf16_bits(back)
+    out["latent_pages"] = bits_all
     return out
 
 

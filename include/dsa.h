@@ -117,7 +117,8 @@ typedef enum {
   DSA_OP_CACHE_APPEND = 5,
   DSA_OP_INDEXER_SCORES_K8 = 6,   /* dsa_indexer_scores_k8 */
   DSA_OP_ATTENTION_FORWARD_K8 = 7, /* dsa_attention_forward_k8 */
-  DSA_OP_ATTENTION_FORWARD_HOST = 8 /* dsa_attention_forward_host */
+  DSA_OP_ATTENTION_FORWARD_HOST = 8, /* dsa_attention_forward_host */
+  DSA_OP_ATTENTION_FORWARD_FP8 = 9   /* dsa_attention_forward_fp8 */
 } dsa_op_t;
 
 /* Library version (major * 10000 + minor * 100 + patch). */
@@ -126,13 +127,20 @@ DSA_API int dsa_version(void);
 /* Human-readable name of a status code (static string). */
 DSA_API const char *dsa_status_string(dsa_status_t status);
 
+/* The last CUDA error a call of this library met on the calling thread (a
+ * failed launch or kernel attribute), as "where: message (code)"; an empty
+ * string when there was none.  The text behind a DSA_ERR_CUDA status.  Valid
+ * until the thread's next failing call. */
+DSA_API const char *dsa_last_cuda_error(void);
+
 /* Bytes of device workspace `op` needs for these dims and cache.  Every
  * workspace starts with a 256-byte status block; the rest is scratch whose
  * contents are undefined between calls.  Returns 0 for invalid input. */
 DSA_API size_t dsa_workspace_bytes(dsa_op_t op, const dsa_dims_t *dims, const dsa_cache_t *cache);
 
-/* Number of kernels one dsa_attention_forward (op = DSA_OP_ATTENTION_FORWARD)
- * or dsa_attention_forward_k8 (DSA_OP_ATTENTION_FORWARD_K8) call launches for
+/* Number of kernels one dsa_attention_forward (op = DSA_OP_ATTENTION_FORWARD),
+ * dsa_attention_forward_k8 (DSA_OP_ATTENTION_FORWARD_K8) or
+ * dsa_attention_forward_fp8 (DSA_OP_ATTENTION_FORWARD_FP8) call launches for
  * these dims and cache on the current device: the indexer (plus the E4M3
  * query split for FP8 keys), the top-k, the sparse MLA, and the split merge
  * when a row's partial results meet in global memory.  A query of the launch
@@ -181,9 +189,15 @@ DSA_API dsa_status_t dsa_topk(const float *scores, int64_t ld, int32_t n_q, cons
  *   q            [n_q, H, R + P] bf16 absorbed queries, rows 16-byte aligned
  *   latent_pages [num_pages, 64, R + P] bf16
  *   idx          [n_q, topk] int32 token positions (-1 = unused slot); a position
- *                outside the row's context is skipped and flagged on the device
+ *                outside the row's context is skipped and flagged on the device.
+ *                Row r reads only its first min(topk, len(r)) slots, len(r) the
+ *                number of tokens the row sees (a row keeps at most that many;
+ *                dsa_topk emits them first, then -1)
  *   out          [n_q, H, R] fp32, lse [n_q, H] fp32 (natural log).  A row with
  *                no kept token gets out = 0 and lse = -inf.
+ * Precision: bf16 products of q and the latent rows, accumulated in fp32; the
+ * softmax weights enter the PV product as two bf16 terms (hi + lo, about 16
+ * significant bits). 
  * dims.causal must be 0; row b reads sequence b of the cache. */
 DSA_API dsa_status_t dsa_sparse_mla_decode(const uint16_t *q, const uint16_t *latent_pages,
                                    const dsa_cache_t *cache, const int32_t *idx,
@@ -266,6 +280,38 @@ DSA_API dsa_status_t dsa_attention_forward_k8(const uint16_t *q_idx, const float
                                       int32_t *idx_out, float *out, float *lse, void *ws,
                                       size_t ws_bytes, dsa_stream_t stream);
 
+/* FP8 latent cache: the sparse MLA step, and the whole step with both caches
+ * in FP8, over a latent cache held as E4M3 bytes with one fp32 scale per token
+ * ("GLM on an A100, in Vx", section "INT4, FP8 and BF16": E4M3 bytes with a
+ * float32 scale per block; here a block is one token's whole latent row
+ * [c_kv | k_rope]).  Token row `row` = page * 64 + slot stands for
+ *   L[row, :] = latent_scale[row] * e4m3(latent8_pages[row, :])
+ * and serves as key (all R + P columns) and value (the first R) exactly as a
+ * bf16 row does.
+ *   latent8_pages [num_pages, 64, R + P] uint8 E4M3 codes, 16-byte aligned
+ *   latent_scale  [num_pages * 64] fp32 (finite, any sign), 4-byte aligned
+ * Everything else as dsa_sparse_mla_decode / _prefill (workspaces from
+ * DSA_OP_SPARSE_MLA_DECODE / _PREFILL) and, for dsa_attention_forward_fp8,
+ * as dsa_attention_forward_k8 with the FP8 index keys (workspace from
+ * DSA_OP_ATTENTION_FORWARD_FP8, the same size as DSA_OP_ATTENTION_FORWARD_K8).  The kernel widens each gathered E4M3 row to
+ * bf16 in shared memory (exact) and applies the token's scale to its logit and
+ * to its PV weight, so the latent rows cost 580 bytes per kept token instead
+ * of 1,152. */
+DSA_API dsa_status_t dsa_sparse_mla_decode_l8(const uint16_t *q, const uint8_t *latent8_pages,
+                                      const float *latent_scale, const dsa_cache_t *cache,
+                                      const int32_t *idx, const dsa_dims_t *dims, float *out,
+                                      float *lse, void *ws, size_t ws_bytes, dsa_stream_t stream);
+DSA_API dsa_status_t dsa_sparse_mla_prefill_l8(const uint16_t *q, const uint8_t *latent8_pages,
+                                       const float *latent_scale, const dsa_cache_t *cache,
+                                       const int32_t *idx, const dsa_dims_t *dims, float *out,
+                                       float *lse, void *ws, size_t ws_bytes, dsa_stream_t stream);
+DSA_API dsa_status_t dsa_attention_forward_fp8(const uint16_t *q_idx, const float *w,
+                                       const uint8_t *k8_pages, const float *k_scale,
+                                       const uint16_t *q, const uint8_t *latent8_pages,
+                                       const float *latent_scale, const dsa_cache_t *cache,
+                                       const dsa_dims_t *dims, int32_t *idx_out, float *out,
+                                       float *lse, void *ws, size_t ws_bytes, dsa_stream_t stream);
+
 /* Cache append: write the new tokens' index keys and latent rows into the
  * paged caches, the step in front of the indexer ("Self-contained GLM-5
  * serving stack ...", file list: absorbed MLA decode over compressed
@@ -334,8 +380,8 @@ DSA_API dsa_status_t dsa_project_values(const float *o_lat, const uint16_t *w_uv
  *      [ranks, n_q, k];
  *   3. dsa_cp_select: the exact global top-k of the pairs (the lower global
  *      index wins ties, as in dsa_topk) into gidx [n_q, k] (ascending, -1
- *      padded), and in own_idx [n_q, k] the same slots as this rank's local
- *      positions (-1 for tokens of other ranks); my_offsets / my_lens [n_q]
+ *      padded), and in own_idx [n_q, k] this rank's share of it as local
+ *      positions, ascending, first in the row (-1 after them); my_offsets / my_lens [n_q]
  *      give this rank's key range.  Workspace: dsa_cp_workspace_bytes;
  *   4. dsa_sparse_mla_decode with own_idx over the rank's latent rows, then
  *      the caller all-gathers (out, lse): outs [ranks, n_q, H, dv], lses
@@ -362,19 +408,23 @@ DSA_API dsa_status_t dsa_cp_merge(const float *outs, const float *lses, int32_t 
  * The pages have no counterpart of this entry point: it exists for callers
  * that cannot call cudaMalloc (or any allocator) at the point where they run
  * the step, e.g. code inside a memory pool that must not grow, or a host that
- * hands the library only its input and output buffers.  It computes exactly
- * what dsa_sparse_mla_decode computes (same kernels, same launch shapes) but
- * takes no workspace: its scratch (the per-split partial results and a status
- * block) is a fixed 32 MiB array in the library's own device memory, present
- * on every GPU that loads the library until the process exits.
+ * hands the library only its input and output buffers.  It computes what
+ * dsa_sparse_mla_decode computes, always with the pipelined kernel that call
+ * uses for large batches (results agree within the step's tolerance), and
+ * takes no workspace: its scratch (the
+ * per-split partial results and a status block) is a fixed 16 MiB array in
+ * the library's own device memory, present on every GPU that loads the
+ * library until the process exits.
  *
  *   Arguments as for dsa_sparse_mla_decode, without ws / ws_bytes.
  *   Returns DSA_ERR_WORKSPACE, before launching anything, when the partial
- *   results of this call (n_q * splits * 64 * R' * 4 bytes, R' = R rounded up
- *   to a multiple of 128; rows are split
- *   when there are fewer rows than SMs) would not fit in the 32 MiB array:
- *   a batch of 32 at R = 512 and top-2,048 (16.8 MB) fits; 140 rows of
- *   top-65,536 (two splits each, 36.7 MB) are rejected.
+ *   results of this call would not fit in the 16 MiB array.  Partials exist
+ *   only when few rows hold long selections: each row is then split over more
+ *   CTAs than one cluster holds, and every split leaves n_q * splits * 64 *
+ *   R' * 4 bytes (R' = R rounded up to a multiple of 128).  One row of
+ *   top-8,192 (64 splits, 8.4 MB) fits; two rows of top-65,536 (64 splits
+ *   each, 16.8 MB) are rejected.  Rows split over one cluster (e.g. a batch of
+ *   32 at top-2,048) or not split at all need only the status block.
  *
  * The first call on a device looks up the array's device address (once per
  * device, with that device current); make that first call before any stream

@@ -31,6 +31,7 @@ OP_CACHE_APPEND = 5
 OP_INDEXER_SCORES_K8 = 6
 OP_ATTENTION_FORWARD_K8 = 7
 OP_ATTENTION_FORWARD_HOST = 8
+OP_ATTENTION_FORWARD_FP8 = 9
 
 STATUS_NAMES = {0: "DSA_OK", 1: "DSA_ERR_INVALID_ARG", 2: "DSA_ERR_UNSUPPORTED",
                 3: "DSA_ERR_CUDA", 4: "DSA_ERR_WORKSPACE", 5: "DSA_ERR_TIMEOUT",
@@ -42,13 +43,18 @@ EXPORTED = ["dsa_version", "dsa_status_string", "dsa_workspace_bytes", "dsa_work
             "dsa_cache_append", "dsa_absorb_query", "dsa_project_values",
             "dsa_indexer_scores_k8", "dsa_attention_forward_k8", "dsa_cp_workspace_bytes",
             "dsa_cp_candidates", "dsa_cp_select", "dsa_cp_merge",
-            "dsa_attention_forward_host", "dsa_noalloc_status", "dsa_forward_launches"]
+            "dsa_attention_forward_host", "dsa_noalloc_status", "dsa_forward_launches",
+            "dsa_sparse_mla_decode_l8", "dsa_sparse_mla_prefill_l8", "dsa_attention_forward_fp8",
+            "dsa_last_cuda_error"]
 
 
 class DsaError(RuntimeError):
     def __init__(self, status: int, where: str):
         self.status = status
-        super().__init__(f"{where}: {STATUS_NAMES.get(status, status)}")
+        msg = f"{where}: {STATUS_NAMES.get(status, status)}"
+        if status == 3 and _lib is not None:   # DSA_ERR_CUDA: the CUDA error behind it
+            msg += f" ({_lib.dsa_last_cuda_error().decode()})"
+        super().__init__(msg)
 
 
 class CacheStruct(ctypes.Structure):
@@ -82,6 +88,7 @@ def lib() -> ctypes.CDLL:
         sigs = {
             "dsa_version": ([], ctypes.c_int),
             "dsa_status_string": ([ctypes.c_int], ctypes.c_char_p),
+            "dsa_last_cuda_error": ([], ctypes.c_char_p),
             "dsa_workspace_bytes": ([ctypes.c_int, pd, pc], sz),
             "dsa_workspace_init": ([vp, sz, vp], ctypes.c_int),
             "dsa_workspace_check": ([vp, vp, ctypes.POINTER(ctypes.c_uint32)], ctypes.c_int),
@@ -94,6 +101,10 @@ def lib() -> ctypes.CDLL:
             "dsa_sparse_mla_decode_noalloc": ([vp, vp, pc, vp, pd, vp, vp, vp], ctypes.c_int),
             "dsa_noalloc_status": ([vp, ctypes.POINTER(ctypes.c_uint32)], ctypes.c_int),
             "dsa_forward_launches": ([ctypes.c_int, pd, pc], i32),
+            "dsa_sparse_mla_decode_l8": ([vp, vp, vp, pc, vp, pd, vp, vp, vp, sz, vp], ctypes.c_int),
+            "dsa_sparse_mla_prefill_l8": ([vp, vp, vp, pc, vp, pd, vp, vp, vp, sz, vp], ctypes.c_int),
+            "dsa_attention_forward_fp8": ([vp, vp, vp, vp, vp, vp, vp, pc, pd, vp, vp, vp, vp, sz,
+                                           vp], ctypes.c_int),
             "dsa_cache_append": ([vp, vp, vp, vp, pc, pd, vp, sz, vp], ctypes.c_int),
             "dsa_absorb_query": ([vp, vp, vp, vp, i32, i32, i32, i32, i32, vp, sz, vp],
                                  ctypes.c_int),
@@ -229,6 +240,37 @@ def dsa_sparse_mla_prefill(q, latent_pages, cache: PagedCache, idx, dims: Dims, 
                                         ctypes.byref(dims.struct()), _ptr(out), _ptr(lse),
                                         _ptr(ws), ws.numel(), _stream(stream)),
            "dsa_sparse_mla_prefill")
+
+
+def dsa_sparse_mla_decode_l8(q, latent8_pages, latent_scale, cache: PagedCache, idx, dims: Dims,
+                             out, lse, ws, stream=None) -> None:
+    """Sparse MLA decode over an FP8 latent cache (E4M3 rows, one fp32 scale per token)."""
+    _check(lib().dsa_sparse_mla_decode_l8(_ptr(q), _ptr(latent8_pages), _ptr(latent_scale),
+                                          ctypes.byref(cache.struct()), _ptr(idx),
+                                          ctypes.byref(dims.struct()), _ptr(out), _ptr(lse),
+                                          _ptr(ws), ws.numel(), _stream(stream)),
+           "dsa_sparse_mla_decode_l8")
+
+
+def dsa_sparse_mla_prefill_l8(q, latent8_pages, latent_scale, cache: PagedCache, idx, dims: Dims,
+                              out, lse, ws, stream=None) -> None:
+    _check(lib().dsa_sparse_mla_prefill_l8(_ptr(q), _ptr(latent8_pages), _ptr(latent_scale),
+                                           ctypes.byref(cache.struct()), _ptr(idx),
+                                           ctypes.byref(dims.struct()), _ptr(out), _ptr(lse),
+                                           _ptr(ws), ws.numel(), _stream(stream)),
+           "dsa_sparse_mla_prefill_l8")
+
+
+def dsa_attention_forward_fp8(q_idx, w, k8_pages, k_scale, q, latent8_pages, latent_scale,
+                              cache: PagedCache, dims: Dims, idx_out, out, lse, ws,
+                              stream=None) -> None:
+    """The whole step with both caches in FP8 (E4M3 + one scale per token)."""
+    _check(lib().dsa_attention_forward_fp8(_ptr(q_idx), _ptr(w), _ptr(k8_pages), _ptr(k_scale),
+                                           _ptr(q), _ptr(latent8_pages), _ptr(latent_scale),
+                                           ctypes.byref(cache.struct()),
+                                           ctypes.byref(dims.struct()), _ptr(idx_out), _ptr(out),
+                                           _ptr(lse), _ptr(ws), ws.numel(), _stream(stream)),
+           "dsa_attention_forward_fp8")
 
 
 def dsa_sparse_mla_decode_noalloc(q, latent_pages, cache: PagedCache, idx, dims: Dims, out, lse,

@@ -59,13 +59,14 @@ constexpr int kSelThreads = 1024;
 __global__ void __launch_bounds__(kSelThreads) cp_select_kernel(
     const int32_t *pos, const int32_t *all_i, int R, int n_q, int k, const int32_t *my_off,
     const int32_t *my_len, int32_t *gidx, int32_t *own) {
-  __shared__ int warp_tot[kSelThreads / 32];
-  __shared__ int carry;
+  // per warp: kept picks, and kept picks in this rank's range
+  __shared__ int warp_tot[2][kSelThreads / 32];
+  __shared__ int carry[2];
   griddep_wait();
   griddep_launch_dependents();
   const int r = blockIdx.x, tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int off = my_off[r], len = my_len[r];
-  if (tid == 0) carry = 0;
+  if (tid < 2) carry[tid] = 0;
   __syncthreads();
   for (int base = 0; base < k; base += kSelThreads) {
     const int j = base + tid;
@@ -78,38 +79,42 @@ __global__ void __launch_bounds__(kSelThreads) cp_select_kernel(
       }
     }
     const int v = (g >= 0) ? 1 : 0;
-    int incl = v;
+    const int m = (g >= off && g < off + len) ? 1 : 0;  // one of this rank's tokens
+    int incl = v, incl_m = m;
 #pragma unroll
     for (int o = 1; o < 32; o <<= 1) {
       const int y = __shfl_up_sync(0xffffffffu, incl, o);
-      if (lane >= o) incl += y;
+      const int ym = __shfl_up_sync(0xffffffffu, incl_m, o);
+      if (lane >= o) { incl += y; incl_m += ym; }
     }
-    if (lane == 31) warp_tot[warp] = incl;
+    if (lane == 31) { warp_tot[0][warp] = incl; warp_tot[1][warp] = incl_m; }
     __syncthreads();
-    if (warp == 0) {
-      const int x = warp_tot[lane];
+    if (warp < 2) {
+      const int x = warp_tot[warp][lane];
       int wi = x;
 #pragma unroll
       for (int o = 1; o < 32; o <<= 1) {
         const int y = __shfl_up_sync(0xffffffffu, wi, o);
         if (lane >= o) wi += y;
       }
-      warp_tot[lane] = wi - x;  // exclusive over warps
+      warp_tot[warp][lane] = wi - x;  // exclusive over warps
     }
     __syncthreads();
-    const int dst = carry + warp_tot[warp] + incl - v;
-    if (v) {
-      gidx[static_cast<int64_t>(r) * k + dst] = g;
-      own[static_cast<int64_t>(r) * k + dst] = (g >= off && g < off + len) ? g - off : -1;
+    const int dst = carry[0] + warp_tot[0][warp] + incl - v;
+    const int dst_m = carry[1] + warp_tot[1][warp] + incl_m - m;
+    // the global picks in their global slots; this rank's share compacted to
+    // the front of own (local positions, ascending like the global slots)
+    if (v) gidx[static_cast<int64_t>(r) * k + dst] = g;
+    if (m) own[static_cast<int64_t>(r) * k + dst_m] = g - off;
+    __syncthreads();
+    if (tid == kSelThreads - 1) {
+      carry[0] = dst + v;
+      carry[1] = dst_m + m;
     }
     __syncthreads();
-    if (tid == kSelThreads - 1) carry = dst + v;
-    __syncthreads();
   }
-  for (int j = carry + tid; j < k; j += kSelThreads) {
-    gidx[static_cast<int64_t>(r) * k + j] = -1;
-    own[static_cast<int64_t>(r) * k + j] = -1;
-  }
+  for (int j = carry[0] + tid; j < k; j += kSelThreads) gidx[static_cast<int64_t>(r) * k + j] = -1;
+  for (int j = carry[1] + tid; j < k; j += kSelThreads) own[static_cast<int64_t>(r) * k + j] = -1;
 }
 
 // out = sum_r exp(lse_r - L) out_r, L = log sum_r exp(lse_r); grid (n_q, H).

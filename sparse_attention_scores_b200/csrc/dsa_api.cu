@@ -1,6 +1,7 @@
 // The C ABI of libdsa: argument checks on the host, workspace layout, and the
 // launch sequence of each entry point.  See include/dsa.h for the contract.
 #include <math.h>
+#include <stdio.h>
 #include <stdlib.h>
 #include <string.h>
 
@@ -128,6 +129,16 @@ size_t device_smem_per_sm() {
   return cached[d];
 }
 
+namespace {
+thread_local char g_last_error[256];
+}  // namespace
+
+cudaError_t note_cuda_error(cudaError_t err, const char *where) {
+  snprintf(g_last_error, sizeof(g_last_error), "%s: %s (%d)", where, cudaGetErrorString(err),
+           static_cast<int>(err));
+  return err;
+}
+
 cudaError_t func_attr_once(const void *kernel, cudaFuncAttribute attr, int value) {
   struct Entry {
     int dev;
@@ -139,10 +150,19 @@ cudaError_t func_attr_once(const void *kernel, cudaFuncAttribute attr, int value
   static std::vector<Entry> done;
   const int d = current_device();
   std::lock_guard<std::mutex> lock(mu);
-  for (const Entry &e : done)
-    if (e.dev == d && e.kernel == kernel && e.attr == attr && e.value == value) return cudaSuccess;
+  // one entry per (device, kernel, attribute) holding the value last set: a
+  // kernel has one value per attribute, so a new value is set again
+  Entry *slot = nullptr;
+  for (Entry &e : done)
+    if (e.dev == d && e.kernel == kernel && e.attr == attr) slot = &e;
+  if (slot != nullptr && slot->value == value) return cudaSuccess;
   const cudaError_t err = cudaFuncSetAttribute(kernel, attr, value);
-  if (err == cudaSuccess && d >= 0) done.push_back(Entry{d, kernel, attr, value});
+  if (err != cudaSuccess) {
+    if (slot != nullptr) slot->value = INT32_MIN;  // unknown now: set again next time
+    return note_cuda_error(err, "cudaFuncSetAttribute");
+  }
+  if (slot != nullptr) slot->value = value;
+  else if (d >= 0) done.push_back(Entry{d, kernel, attr, value});
   return err;
 }
 
@@ -282,6 +302,7 @@ size_t ws_bytes_for(dsa_op_t op, const dsa_dims_t &d, const dsa_cache_t &c) {
     case DSA_OP_INDEXER_SCORES_K8:
       return kStatusBytes + k8_region_bytes(d);
     case DSA_OP_ATTENTION_FORWARD_K8:
+    case DSA_OP_ATTENTION_FORWARD_FP8:
       return k8_region_bytes(d) + ws_bytes_for(DSA_OP_ATTENTION_FORWARD, d, c);
     case DSA_OP_SPARSE_MLA_DECODE:
     case DSA_OP_SPARSE_MLA_PREFILL:
@@ -351,13 +372,17 @@ dsa_status_t run_topk(const float *scores, int64_t ld, int n_q, const int32_t *v
   return launch_topk(a, s);
 }
 
+// latent8 != nullptr: E4M3 latent rows with one fp32 scale per row (lat_scale)
 dsa_status_t run_mla(const uint16_t *q, const uint16_t *latent, const dsa_cache_t &c,
                      const int32_t *idx, const dsa_dims_t &d, float *out, float *lse, void *scratch,
-                     size_t scratch_bytes, DevStatus *st, cudaStream_t s, int early_q = 0) {
+                     size_t scratch_bytes, DevStatus *st, cudaStream_t s, int early_q = 0,
+                     const uint8_t *latent8 = nullptr, const float *lat_scale = nullptr) {
   MlaLaunch a;
   a.early_q = early_q;
   a.q = q;
   a.latent = latent;
+  a.latent8 = latent8;
+  a.lat_scale = lat_scale;
   a.idx = idx;
   a.seq_lens = c.seq_lens;
   a.block_table = c.block_table;
@@ -379,17 +404,21 @@ dsa_status_t run_mla(const uint16_t *q, const uint16_t *latent, const dsa_cache_
   return launch_mla(a, s);
 }
 
-dsa_status_t mla_entry(const uint16_t *q, const uint16_t *latent_pages, const dsa_cache_t *cache,
-                       const int32_t *idx, const dsa_dims_t *dims, float *out, float *lse,
-                       void *ws, size_t ws_bytes, dsa_stream_t stream, int want_causal) {
+// the sparse MLA entry for bf16 latent rows (latent_pages) or E4M3 rows
+// (latent8_pages + lat_scale)
+dsa_status_t mla_entry(const uint16_t *q, const uint16_t *latent_pages, const uint8_t *latent8_pages,
+                       const float *lat_scale, const dsa_cache_t *cache, const int32_t *idx,
+                       const dsa_dims_t *dims, float *out, float *lse, void *ws, size_t ws_bytes,
+                       dsa_stream_t stream, int want_causal) {
   DSA_TRY(check_dims_common(dims));
   if (dims->causal != want_causal) return DSA_ERR_INVALID_ARG;
   DSA_TRY(check_mla_dims(*dims));
   DSA_TRY(check_cache(cache, *dims));
-  if (q == nullptr || latent_pages == nullptr || idx == nullptr || out == nullptr || lse == nullptr)
+  const void *lat = latent8_pages ? static_cast<const void *>(latent8_pages) : latent_pages;
+  if (q == nullptr || lat == nullptr || idx == nullptr || out == nullptr || lse == nullptr)
     return DSA_ERR_INVALID_ARG;
-  if (!aligned16(q) || !aligned16(latent_pages) || !aligned4(idx) || !aligned4(out) ||
-      !aligned4(lse))
+  if (!aligned16(q) || !aligned16(lat) || !aligned4(idx) || !aligned4(out) || !aligned4(lse) ||
+      (lat_scale && !aligned4(lat_scale)))
     return DSA_ERR_INVALID_ARG;
   const size_t need = ws_bytes_for(want_causal ? DSA_OP_SPARSE_MLA_PREFILL : DSA_OP_SPARSE_MLA_DECODE,
                                    *dims, *cache);
@@ -397,7 +426,7 @@ dsa_status_t mla_entry(const uint16_t *q, const uint16_t *latent_pages, const ds
   if (dims->n_q == 0) return DSA_OK;
   return run_mla(q, latent_pages, *cache, idx, *dims, out, lse,
                  static_cast<uint8_t *>(ws) + kStatusBytes, ws_bytes - kStatusBytes, status_of(ws),
-                 as_stream(stream));
+                 as_stream(stream), 0, latent8_pages, lat_scale);
 }
 
 dsa_status_t indexer_entry(const uint16_t *q_idx, const float *w, const uint16_t *k_idx_pages,
@@ -408,7 +437,8 @@ dsa_status_t forward_entry(const uint16_t *q_idx, const float *w, const uint16_t
                            const uint8_t *k8_pages, const float *k_scale, const uint16_t *q,
                            const uint16_t *latent_pages, const dsa_cache_t *cache,
                            const dsa_dims_t *dims, int32_t *idx_out, float *out, float *lse,
-                           void *ws, size_t ws_bytes, dsa_stream_t stream);
+                           void *ws, size_t ws_bytes, dsa_stream_t stream,
+                           const uint8_t *latent8_pages = nullptr, const float *lat_scale = nullptr);
 
 }  // namespace
 }  // namespace dsa
@@ -418,6 +448,8 @@ using namespace dsa;
 extern "C" {
 
 int dsa_version(void) { return 100; }
+
+const char *dsa_last_cuda_error(void) { return g_last_error; }
 
 const char *dsa_status_string(dsa_status_t s) {
   switch (s) {
@@ -439,7 +471,7 @@ size_t dsa_workspace_bytes(dsa_op_t op, const dsa_dims_t *dims, const dsa_cache_
   if (op == DSA_OP_INDEXER_SCORES_K8) return ws_bytes_for(op, *dims, dsa_cache_t{});
   if (check_mla_dims(*dims) != DSA_OK) return 0;
   if ((op == DSA_OP_ATTENTION_FORWARD || op == DSA_OP_ATTENTION_FORWARD_K8 ||
-       op == DSA_OP_ATTENTION_FORWARD_HOST) &&
+       op == DSA_OP_ATTENTION_FORWARD_FP8 || op == DSA_OP_ATTENTION_FORWARD_HOST) &&
       (cache == nullptr || check_cache(cache, *dims) != DSA_OK))
     return 0;
   dsa_cache_t empty = {};
@@ -447,14 +479,17 @@ size_t dsa_workspace_bytes(dsa_op_t op, const dsa_dims_t *dims, const dsa_cache_
 }
 
 int32_t dsa_forward_launches(dsa_op_t op, const dsa_dims_t *dims, const dsa_cache_t *cache) {
-  if (op != DSA_OP_ATTENTION_FORWARD && op != DSA_OP_ATTENTION_FORWARD_K8) return -1;
+  if (op != DSA_OP_ATTENTION_FORWARD && op != DSA_OP_ATTENTION_FORWARD_K8 &&
+      op != DSA_OP_ATTENTION_FORWARD_FP8)
+    return -1;
   if (check_dims_common(dims) != DSA_OK || check_indexer_dims(*dims) != DSA_OK ||
       check_mla_dims(*dims) != DSA_OK || check_cache(cache, *dims) != DSA_OK)
     return -1;
   if (dims->n_q == 0) return 0;
   // indexer (+ the E4M3 query split for FP8 keys), top-k, sparse MLA (+ merge)
-  return (op == DSA_OP_ATTENTION_FORWARD_K8 ? 3 : 2) +
-         mla_launch_count(dims->n_q, dims->topk, dims->R, dims->P);
+  return (op == DSA_OP_ATTENTION_FORWARD ? 2 : 3) +
+         mla_launch_count(dims->n_q, dims->topk, dims->R, dims->P,
+                          op == DSA_OP_ATTENTION_FORWARD_FP8);
 }
 
 dsa_status_t dsa_workspace_init(void *ws, size_t ws_bytes, dsa_stream_t stream) {
@@ -514,14 +549,34 @@ dsa_status_t dsa_sparse_mla_decode(const uint16_t *q, const uint16_t *latent_pag
                                    const dsa_cache_t *cache, const int32_t *idx,
                                    const dsa_dims_t *dims, float *out, float *lse, void *ws,
                                    size_t ws_bytes, dsa_stream_t stream) {
-  return mla_entry(q, latent_pages, cache, idx, dims, out, lse, ws, ws_bytes, stream, 0);
+  return mla_entry(q, latent_pages, nullptr, nullptr, cache, idx, dims, out, lse, ws, ws_bytes,
+                   stream, 0);
 }
 
 dsa_status_t dsa_sparse_mla_prefill(const uint16_t *q, const uint16_t *latent_pages,
                                     const dsa_cache_t *cache, const int32_t *idx,
                                     const dsa_dims_t *dims, float *out, float *lse, void *ws,
                                     size_t ws_bytes, dsa_stream_t stream) {
-  return mla_entry(q, latent_pages, cache, idx, dims, out, lse, ws, ws_bytes, stream, 1);
+  return mla_entry(q, latent_pages, nullptr, nullptr, cache, idx, dims, out, lse, ws, ws_bytes,
+                   stream, 1);
+}
+
+dsa_status_t dsa_sparse_mla_decode_l8(const uint16_t *q, const uint8_t *latent8_pages,
+                                      const float *latent_scale, const dsa_cache_t *cache,
+                                      const int32_t *idx, const dsa_dims_t *dims, float *out,
+                                      float *lse, void *ws, size_t ws_bytes, dsa_stream_t stream) {
+  if (latent8_pages == nullptr || latent_scale == nullptr) return DSA_ERR_INVALID_ARG;
+  return mla_entry(q, nullptr, latent8_pages, latent_scale, cache, idx, dims, out, lse, ws,
+                   ws_bytes, stream, 0);
+}
+
+dsa_status_t dsa_sparse_mla_prefill_l8(const uint16_t *q, const uint8_t *latent8_pages,
+                                       const float *latent_scale, const dsa_cache_t *cache,
+                                       const int32_t *idx, const dsa_dims_t *dims, float *out,
+                                       float *lse, void *ws, size_t ws_bytes, dsa_stream_t stream) {
+  if (latent8_pages == nullptr || latent_scale == nullptr) return DSA_ERR_INVALID_ARG;
+  return mla_entry(q, nullptr, latent8_pages, latent_scale, cache, idx, dims, out, lse, ws,
+                   ws_bytes, stream, 1);
 }
 
 dsa_status_t dsa_attention_forward(const uint16_t *q_idx, const float *w,
@@ -614,6 +669,19 @@ dsa_status_t dsa_attention_forward_k8(const uint16_t *q_idx, const float *w,
   if (k8_pages == nullptr || k_scale == nullptr) return DSA_ERR_INVALID_ARG;
   return forward_entry(q_idx, w, nullptr, k8_pages, k_scale, q, latent_pages, cache, dims,
                        idx_out, out, lse, ws, ws_bytes, stream);
+}
+
+dsa_status_t dsa_attention_forward_fp8(const uint16_t *q_idx, const float *w,
+                                       const uint8_t *k8_pages, const float *k_scale,
+                                       const uint16_t *q, const uint8_t *latent8_pages,
+                                       const float *latent_scale, const dsa_cache_t *cache,
+                                       const dsa_dims_t *dims, int32_t *idx_out, float *out,
+                                       float *lse, void *ws, size_t ws_bytes, dsa_stream_t stream) {
+  if (k8_pages == nullptr || k_scale == nullptr || latent8_pages == nullptr ||
+      latent_scale == nullptr)
+    return DSA_ERR_INVALID_ARG;
+  return forward_entry(q_idx, w, nullptr, k8_pages, k_scale, q, nullptr, cache, dims, idx_out,
+                       out, lse, ws, ws_bytes, stream, latent8_pages, latent_scale);
 }
 
 size_t dsa_cp_workspace_bytes(int32_t ranks, int32_t n_q, int32_t k) {
@@ -712,16 +780,19 @@ dsa_status_t forward_entry(const uint16_t *q_idx, const float *w, const uint16_t
                            const uint8_t *k8_pages, const float *k_scale, const uint16_t *q,
                            const uint16_t *latent_pages, const dsa_cache_t *cache,
                            const dsa_dims_t *dims, int32_t *idx_out, float *out, float *lse,
-                           void *ws, size_t ws_bytes, dsa_stream_t stream) {
+                           void *ws, size_t ws_bytes, dsa_stream_t stream,
+                           const uint8_t *latent8_pages, const float *lat_scale) {
   DSA_TRY(check_dims_common(dims));
   DSA_TRY(check_indexer_dims(*dims));
   DSA_TRY(check_mla_dims(*dims));
   DSA_TRY(check_cache(cache, *dims));
   const void *keys = k8_pages ? static_cast<const void *>(k8_pages) : k_idx_pages;
-  if (q_idx == nullptr || w == nullptr || keys == nullptr || q == nullptr ||
-      latent_pages == nullptr || out == nullptr || lse == nullptr)
+  const void *lat = latent8_pages ? static_cast<const void *>(latent8_pages) : latent_pages;
+  if (q_idx == nullptr || w == nullptr || keys == nullptr || q == nullptr || lat == nullptr ||
+      out == nullptr || lse == nullptr)
     return DSA_ERR_INVALID_ARG;
-  if (!aligned16(q_idx) || !aligned16(keys) || !aligned16(q) || !aligned16(latent_pages) ||
+  if ((lat_scale && !aligned4(lat_scale))) return DSA_ERR_INVALID_ARG;
+  if (!aligned16(q_idx) || !aligned16(keys) || !aligned16(q) || !aligned16(lat) ||
       !aligned4(w) || !aligned4(out) || !aligned4(lse) || (idx_out && !aligned4(idx_out)) ||
       (k_scale && !aligned16(k_scale)))
     return DSA_ERR_INVALID_ARG;
@@ -751,7 +822,7 @@ dsa_status_t forward_entry(const uint16_t *q_idx, const float *w, const uint16_t
   DSA_TRY(run_topk(scores, ld, d.n_q, d.causal ? nullptr : c.seq_lens, d.q_pos0, d.topk, idx,
                    static_cast<int>(max_keys(d, c)), st, s));
   return run_mla(q, latent_pages, c, idx, d, out, lse, scratch, scratch_bytes, st, s,
-                 /*early_q=*/1);
+                 /*early_q=*/1, latent8_pages, lat_scale);
 }
 
 }  // namespace

@@ -26,9 +26,11 @@ constexpr uint64_t kDrainLimitNs = 1000000000ull;
 int device_sm_count();
 
 // Sets a kernel's function attribute (e.g. its dynamic shared-memory opt-in)
-// on the current device, once per (device, kernel, attribute).  Attributes
-// belong to the device's copy of the kernel, so a process that drives several
-// GPUs sets them on each.  Thread-safe.
+// on the current device, skipping the call when the same value is already set
+// for this (device, kernel, attribute).  Attributes belong to the device's
+// copy of the kernel, so a process that drives several GPUs sets them on
+// each.  Callers opt kernels into the device's maximum dynamic shared memory,
+// one value per kernel.  Thread-safe.
 cudaError_t func_attr_once(const void *kernel, cudaFuncAttribute attr, int value);
 
 // Host-side argument checks shared by the entry points (dsa_api.cu).
@@ -44,6 +46,10 @@ bool make_map_2d_u8(CUtensorMap *map, const void *base, uint64_t cols, uint64_t 
                     uint32_t box_cols, uint32_t box_rows, int aw);
 bool make_map_2d(CUtensorMap *map, const void *base, uint64_t cols, uint64_t rows,
                  uint32_t box_cols, uint32_t box_rows, int aw);
+
+// Remember a failed CUDA call of this thread (its error and where it came
+// from) for dsa_last_cuda_error(); returns err.
+cudaError_t note_cuda_error(cudaError_t err, const char *where);
 
 // Launch `kernel` on `stream` with programmatic stream serialization (the
 // kernel calls griddep_wait() before its first dependent read), optionally
@@ -70,7 +76,8 @@ cudaError_t launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t s
   }
   cfg.attrs = attr;
   cfg.numAttrs = n;
-  return cudaLaunchKernelEx(&cfg, kernel, std::forward<Args>(args)...);
+  const cudaError_t err = cudaLaunchKernelEx(&cfg, kernel, std::forward<Args>(args)...);
+  return err == cudaSuccess ? err : note_cuda_error(err, "kernel launch");
 }
 size_t device_max_smem_optin();
 size_t device_smem_per_sm();
@@ -161,6 +168,8 @@ dsa_status_t launch_cp_merge(const float *outs, const float *lses, int R, int n_
 struct MlaLaunch {
   const uint16_t *q;
   const uint16_t *latent;
+  const uint8_t *latent8 = nullptr;   // E4M3 latent rows instead of `latent` (with lat_scale)
+  const float *lat_scale = nullptr;   // one fp32 scale per physical latent row
   const int32_t *idx;
   const int32_t *seq_lens;
   const int32_t *block_table;
@@ -176,12 +185,19 @@ struct MlaLaunch {
   // the stream started (the fused forward): the query tile is then loaded
   // before waiting on that kernel, overlapping its tail
   int early_q = 0;
+  // 1: the pipelined kernel whatever the batch (its small batches merge their
+  // splits inside clusters, with no partials in scratch)
+  int force_pipe = 0;
 };
-// Number of key splits the launcher uses and the scratch bytes it needs.
+// Number of key splits the launcher uses, and the scratch bytes it needs
+// (enough for either latent format).
 int mla_num_splits(int n_q, int topk);
 size_t mla_scratch_bytes(int n_q, int topk, int R);
+// the scratch bytes of the pipelined kernel alone (force_pipe)
+size_t mla_pipe_scratch_bytes(int n_q, int topk, int R);
 dsa_status_t launch_mla(const MlaLaunch &a, cudaStream_t stream);
-// Kernels launch_mla launches for these shapes on the current device (1 or 2).
-int mla_launch_count(int n_q, int topk, int R, int P);
+// Kernels launch_mla launches for these shapes on the current device (1 or 2;
+// lat8: FP8 latent rows).
+int mla_launch_count(int n_q, int topk, int R, int P, bool lat8 = false);
 
 }  // namespace dsa

@@ -1,7 +1,8 @@
 // dsa_sparse_mla_decode_noalloc: the sparse MLA decode for callers that
 // cannot allocate device memory.  Its scratch is a fixed file-scope device
-// array instead of a caller-provided workspace; everything else is the
-// regular decode path (same launcher, same kernels).
+// array instead of a caller-provided workspace, and it always runs the
+// pipelined kernel, whose small batches merge their splits inside clusters
+// and so need no partials at all.
 #include <math.h>
 
 #include <mutex>
@@ -11,11 +12,12 @@
 namespace dsa {
 namespace {
 
-// 32 MiB: the status block plus the split partials of, e.g., a batch of 32
-// rows at R = 512 and top-2,048 (4 splits each, 16.8 MB) or one row of
-// top-8,192 (64 splits, 8.4 MB).  Every GPU that loads the library holds it
-// until the process exits.
-constexpr size_t kNoAllocScratchBytes = 32ull << 20;
+// 16 MiB: the status block plus the split partials of, e.g., one row of
+// top-8,192 (64 splits, 8.4 MB).  Rows split over the CTAs of one cluster
+// (a batch of 32 at top-2,048) or not split at all (as many rows as SMs) need
+// no partials.  Every GPU that loads the library holds it until the process
+// exits.
+constexpr size_t kNoAllocScratchBytes = 16ull << 20;
 static __device__ __align__(256) uint8_t g_noalloc_scratch[kNoAllocScratchBytes];
 
 // In host code `g_noalloc_scratch` names a host-side stand-in, not the device
@@ -64,7 +66,7 @@ extern "C" DSA_API dsa_status_t dsa_sparse_mla_decode_noalloc(
     return DSA_ERR_INVALID_ARG;
   const dsa_cache_t &c = *cache;
   // the built-in array holds the status block and the split partials
-  const size_t need = sizeof(DevStatus) + mla_scratch_bytes(d.n_q, d.topk, d.R);
+  const size_t need = sizeof(DevStatus) + mla_pipe_scratch_bytes(d.n_q, d.topk, d.R);
   if (need > kNoAllocScratchBytes) return DSA_ERR_WORKSPACE;
   if (d.n_q == 0) return DSA_OK;
 
@@ -98,6 +100,7 @@ extern "C" DSA_API dsa_status_t dsa_sparse_mla_decode_noalloc(
   a.scratch = base + sizeof(DevStatus);
   a.scratch_bytes = kNoAllocScratchBytes - sizeof(DevStatus);
   a.status = reinterpret_cast<DevStatus *>(base);
+  a.force_pipe = 1;
   return launch_mla(a, s);
 }
 

@@ -27,7 +27,7 @@ def _declared_symbols():
 
 def test_every_declared_symbol_is_exported(L):
     declared = _declared_symbols()
-    assert len(declared) == 23
+    assert len(declared) == 27
     assert sorted(declared) == sorted(dsa.EXPORTED)
     out = subprocess.run(["nm", "-D", "--defined-only", dsa.LIB_PATH], capture_output=True,
                          text=True, check=True).stdout
@@ -42,6 +42,7 @@ def test_version_and_status_strings(L):
     for code in range(7):
         assert L.dsa_status_string(code).decode()
     assert L.dsa_status_string(99).decode() == "unknown status"
+    assert L.dsa_last_cuda_error().decode() == ""
 
 
 def _dims(**kw):
@@ -87,9 +88,9 @@ def _no_device():
 
 def test_noalloc_size_check_host_only(L):
     _no_device()
-    # 140 rows x 2 splits x 64 heads x 512 x 4 B = 36.7 MB > the 32 MiB array
-    d = _dims(n_q=140, topk=65536)
-    c = _cache(num_seqs=140, max_pages=1024, num_pages=1024, max_seq_len=65536)
+    # 2 rows x 64 splits x 64 heads x 512 x 4 B = 16.8 MB > the 16 MiB array
+    d = _dims(n_q=2, topk=65536)
+    c = _cache(num_seqs=2, max_pages=1024, num_pages=1024, max_seq_len=65536)
     fake = ctypes.c_void_p(0x300000)
     st = L.dsa_sparse_mla_decode_noalloc(fake, fake, ctypes.byref(c), fake, ctypes.byref(d),
                                          fake, fake, None)

@@ -129,14 +129,14 @@ def test_noalloc_reports_bad_index():
 
 
 def test_noalloc_rejects_oversize_request():
-    # 140 rows of top-65,536 split in two need 36.7 MB of partials: more than
-    # the 32 MiB array, so the call must return DSA_ERR_WORKSPACE before
+    # two rows of top-65,536 split 64 ways need 16.8 MB of partials: more than
+    # the 16 MiB array, so the call must return DSA_ERR_WORKSPACE before
     # launching.  Real, correctly sized buffers (every slot unused) keep the
     # call memory-safe regardless.
     if not torch.cuda.is_available():
         pytest.skip("no CUDA device")
     L = dsa.lib()
-    B, k, H, R, P = 140, 65536, 64, 512, 64
+    B, k, H, R, P = 2, 65536, 64, 512, 64
     q = torch.zeros((B, H, R + P), dtype=torch.bfloat16, device="cuda")
     latent = torch.zeros((1, 64, R + P), dtype=torch.bfloat16, device="cuda")
     idx = torch.full((B, k), -1, dtype=torch.int32, device="cuda")
