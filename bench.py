@@ -439,6 +439,9 @@ TRAFFIC = {
     # mla_kernel + combine_kernel (the merge reads the split partials)
     ("mla", "glm5_decode_8k"): (2509056 + 4232448, "819a18ad9156f93f"),
     ("mla", "glm5_decode_4x128k"): (9863936 + 16864256, "819a18ad9156f93f"),
+    # mla_pipe_kernel (rows merged inside clusters; prefill rows unsplit)
+    ("mla", "glm5_decode_b32_ragged"): (78270208 + 2242304, "b9c0f12e2375e2fd"),
+    ("mla", "glm5_prefill_2300"): (183166464 + 246434560, "b9c0f12e2375e2fd"),
 }
 
 
@@ -460,19 +463,29 @@ def traffic_of(stage, workload):
 
 STAGE_KERNELS = {"indexer": "indexer_kernel (tcgen05 + TMA)",
                  "topk": "topk_small_kernel / topk_creg_kernel (radix select, keys in registers)",
-                 "mla": "mla_kernel + combine_kernel (tcgen05, cp.async gather, split merge)"}
+                 "mla": "mla_kernel + combine_kernel (tcgen05, cp.async gather, split merge)",
+                 "mla_pipe": "mla_pipe_kernel (gather warps, one tcgen05 issuer, softmax warps; "
+                             "splits merged in clusters)"}
 
 
-def roofline_of(res, wl, peaks, k8=False):
-    # (FP8 variants pass k8=True: the recorded DRAM traffic is of the bf16 caches)
+def mla_kernel_of(wl, sms=148, l8=False):
+    """The sparse MLA kernel the library picks: the pipelined one when the
+    batch's 64-key blocks fill at least two waves of SMs (or for FP8 rows)."""
+    halves = wl.n_q * ((wl.topk + 63) // 64)
+    return "mla_pipe" if (l8 or halves >= 2 * sms) else "mla"
+
+
+def roofline_of(res, wl, peaks, k8=False, l8=False):
     """Roofline of the stage that takes the longest alone: algorithmic bytes
-    (or flops, for the tensor-bound prefill MLA) over its event time."""
+    (or flops, for the tensor-bound prefill MLA) over its event time.  FP8
+    variants (k8) report no recorded traffic: it was captured on bf16 caches."""
     stage = max(res["stage_us"], key=res["stage_us"].get)
     us = res["stage_us"][stage]
+    label = STAGE_KERNELS[mla_kernel_of(wl, l8=l8)] if stage == "mla" else STAGE_KERNELS[stage]
     if wl.mode == "prefill" and stage == "mla":
         alg = algorithmic(wl)
         achieved = alg["flops_mla"] / (us * 1e-6) / 1e12
-        return {"kernel": STAGE_KERNELS[stage], "stage": stage, "bound": "tensor",
+        return {"kernel": label, "stage": stage, "bound": "tensor",
                 "achieved": achieved, "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
                 "frac": achieved / peaks["bf16_tflops"],
                 "traffic": None if k8 else traffic_of(stage, wl.name),
@@ -480,7 +493,7 @@ def roofline_of(res, wl, peaks, k8=False):
                 "launch_us": us}
     b = res["stage_alg_bytes"][stage]
     achieved = b / (us * 1e-6) / 1e9
-    return {"kernel": STAGE_KERNELS[stage], "stage": stage, "bound": "hbm",
+    return {"kernel": label, "stage": stage, "bound": "hbm",
             "achieved": achieved, "peak": peaks["hbm_gbs"], "unit": "GB/s",
             "frac": achieved / peaks["hbm_gbs"],
             "traffic": None if k8 else traffic_of(stage, wl.name),
@@ -708,7 +721,7 @@ def run_ours(args):
             torch.cuda.synchronize()
             r = measure(c, torch, args.steps, args.warmup, flush_buf, peaks, extras=False)
             r["us_per_step"] = max_over_ranks(r["us_per_step"], pg, "cuda")
-            r["roofline"] = roofline_of(r, c.wl, peaks, k8=True)
+            r["roofline"] = roofline_of(r, c.wl, peaks, k8=True, l8=True)
             per_config[name + "+fp8_cache"] = r
             del c
             torch.cuda.empty_cache()
