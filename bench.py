@@ -469,10 +469,11 @@ STAGE_KERNELS = {"indexer": "indexer_kernel (tcgen05 + TMA)",
 
 
 def mla_kernel_of(wl, sms=148, l8=False):
-    """The sparse MLA kernel the library picks: the pipelined one when the
-    batch's 64-key blocks fill at least two waves of SMs (or for FP8 rows)."""
+    """The sparse MLA kernel the library picks for either latent format: the
+    pipelined one when the batch's 64-key blocks fill at least two waves of
+    SMs, else the per-chunk one."""
     halves = wl.n_q * ((wl.topk + 63) // 64)
-    return "mla_pipe" if (l8 or halves >= 2 * sms) else "mla"
+    return "mla_pipe" if halves >= 2 * sms else "mla"
 
 
 def roofline_of(res, wl, peaks, k8=False, l8=False):

@@ -225,7 +225,63 @@ __device__ __forceinline__ void cluster_merge_epilogue(const MlaParams &p, uint8
   }
 }
 
-template <bool kClusterMerge>
+// two E4M3 values (low byte first) as a bf16 pair, exactly: every E4M3 value
+// is an f16 value and a bf16 value
+__device__ __forceinline__ uint32_t e4m3x2_to_bf16x2(uint32_t v16) {
+  uint32_t h;
+  asm("{\n\t.reg .b16 a;\n\tcvt.u16.u32 a, %1;\n\tcvt.rn.f16x2.e4m3x2 %0, a;\n\t}"
+      : "=r"(h)
+      : "r"(v16));
+  const float lo = __half2float(__ushort_as_half(static_cast<unsigned short>(h & 0xFFFFu)));
+  const float hi = __half2float(__ushort_as_half(static_cast<unsigned short>(h >> 16)));
+  const __nv_bfloat162 r = __floats2bfloat162_rn(lo, hi);
+  return *reinterpret_cast<const uint32_t *>(&r);
+}
+__device__ __forceinline__ uint4 ld_shared_v4(uint32_t a) {
+  uint4 v;
+  asm volatile("ld.shared.v4.u32 {%0, %1, %2, %3}, [%4];"
+               : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
+               : "r"(a));
+  return v;
+}
+__device__ __forceinline__ void st_shared_v4(uint32_t a, uint4 v) {
+  asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(a), "r"(v.x), "r"(v.y), "r"(v.z),
+               "r"(v.w)
+               : "memory");
+}
+
+// Widen one 16-byte quarter (jq) of a latent row's E4M3 slices in place: the
+// row's 64-byte slice of atom a sits in bytes [64, 128) of its 128-byte row of
+// that atom (unswizzled); its 64 bf16 values go to the row's swizzled 16-byte
+// units 2 jq and 2 jq + 1.  The four lanes holding a row's quarters must be
+// in one warp, and every lane of the warp must call this together: all of
+// them read before any of them writes.
+__device__ __forceinline__ void widen_e4m3_quarter(uint32_t row_base, uint32_t sw, int jq, int nQ) {
+  uint4 st[9];
+#pragma unroll
+  for (int a = 0; a < 9; ++a)
+    if (a < nQ) st[a] = ld_shared_v4(row_base + a * kAtomL + 64 + 16 * jq);
+  __syncwarp();
+#pragma unroll
+  for (int a = 0; a < 9; ++a) {
+    if (a >= nQ) break;
+    const uint32_t w4[4] = {st[a].x, st[a].y, st[a].z, st[a].w};
+    uint32_t o[8];
+#pragma unroll
+    for (int t = 0; t < 4; ++t) {
+      o[2 * t] = e4m3x2_to_bf16x2(w4[t] & 0xFFFFu);
+      o[2 * t + 1] = e4m3x2_to_bf16x2(w4[t] >> 16);
+    }
+    st_shared_v4(row_base + a * kAtomL + (((2u * jq) ^ sw) << 4), make_uint4(o[0], o[1], o[2], o[3]));
+    st_shared_v4(row_base + a * kAtomL + (((2u * jq + 1u) ^ sw) << 4), make_uint4(o[4], o[5], o[6], o[7]));
+  }
+  __syncwarp();
+}
+
+// kLat8: E4M3 latent rows with one fp32 scale per token, staged and widened
+// in the tile as above; the token's scale multiplies its logit and its PV
+// weight (the dequantized row is scale * e4m3(code)).
+template <bool kClusterMerge, bool kLat8>
 __global__ void __launch_bounds__(kThreads, 1) mla_kernel(const MlaParams p) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
@@ -252,6 +308,7 @@ __global__ void __launch_bounds__(kThreads, 1) mla_kernel(const MlaParams p) {
   uint32_t *misc = reinterpret_cast<uint32_t *>(bar_stall + 1);
   // cluster merge: every split's (m, l) per head, [kMaxMergeCluster][2][64]
   float *ml_all = reinterpret_cast<float *>(misc + 4);
+  float *kscale = ml_all + kMaxMergeCluster * 2 * kHeads;  // [128] per-key scale (kLat8)
 
   // the cluster merge writes into peers' shared memory: arrive now, wait
   // (for every peer to have started) just before the first remote store
@@ -373,6 +430,7 @@ __global__ void __launch_bounds__(kThreads, 1) mla_kernel(const MlaParams p) {
         }
       }
       rowi[tid] = phys;
+      if constexpr (kLat8) kscale[tid] = (phys >= 0) ? p.lat_scale[phys] : 0.f;
       valid = phys >= 0;
       if (tid == 0) misc[1] = 0u;
     }
@@ -386,7 +444,28 @@ __global__ void __launch_bounds__(kThreads, 1) mla_kernel(const MlaParams p) {
     // issuing the logits product atom by atom was slower than one wait.)
     // Rows kc .. 127 of a 64-key chunk are never written: their keys are
     // masked and the PV product stops at key kc.
-    {
+    if constexpr (kLat8) {
+      // E4M3: quarter jq (16 bytes) of each row's 64-byte slice of atom a,
+      // staged in the row's unswizzled 16-byte unit 4 + jq of that atom
+      const uint32_t ls = smem_u32(Ls);
+      for (int a = 0; a < nQ; ++a)
+        for (int pc = tid; pc < kc * 4; pc += kThreads) {
+          const int r = pc >> 2, jq = pc & 3;
+          const int phys = rowi[r];
+          const bool ok = phys >= 0 && a * 64 + 16 * jq < W;
+          const uint8_t *src = ok ? p.latent8 + static_cast<int64_t>(phys) * W + a * 64 + 16 * jq
+                                  : p.latent8;
+          cp_async_16(ls + a * kAtomL + r * 128 + 64 + 16 * jq, src, ok ? 16u : 0u);
+        }
+      cp_async_commit();
+      cp_async_wait_all();
+      __syncthreads();  // every quarter of every row has landed
+      // rows kc * 4 / kThreads at a time per warp, all lanes together
+      for (int pc = tid; pc < kc * 4; pc += kThreads) {
+        const int r = pc >> 2;
+        widen_e4m3_quarter(smem_u32(Ls) + r * 128, static_cast<uint32_t>(r & 7), pc & 3, nQ);
+      }
+    } else {
       const uint32_t ls = smem_u32(Ls);
       const int per_atom = kc * 8;  // pieces of one atom: 8 per row
       for (int a = 0; a < nQ; ++a)
@@ -424,13 +503,16 @@ __global__ void __launch_bounds__(kThreads, 1) mla_kernel(const MlaParams p) {
 
     // logits of key 32*q4 + lane for heads 32*hh .. 32*hh+31, log2 units
     const bool kvalid = rowi[q4 * 32 + lane] >= 0;
+    // (E4M3 rows: the logit of the dequantized row, the key's scale applied)
+    const float wk = kLat8 ? kscale[q4 * 32 + lane] : 1.f;
     float z[32];
     {
       uint32_t v[32];
       tmem_ld_32x32b_x32(tmem_s + lane_off, v);
       tmem_ld_wait();
+      const float zs = p.scale_log2 * wk;
 #pragma unroll
-      for (int i = 0; i < 32; ++i) z[i] = kvalid ? __uint_as_float(v[i]) * p.scale_log2 : -INFINITY;
+      for (int i = 0; i < 32; ++i) z[i] = kvalid ? __uint_as_float(v[i]) * zs : -INFINITY;
     }
     // per-head chunk max over the 128 keys
     red[q4 * kHeads + 32 * hh + lane] = butterfly32<true>([&](int i) { return z[i]; });
@@ -449,12 +531,19 @@ __global__ void __launch_bounds__(kThreads, 1) mla_kernel(const MlaParams p) {
     // probabilities, split into a bf16 head and a bf16 tail: p = hi + lo to
     // about 2^-17, so the PV product keeps near-fp32 weights even when a few
     // keys dominate.  Sums use hi + lo.
+    // (E4M3 rows: the PV weight is p times the key's scale; l sums p)
     uint32_t phi[16], plo[16];  // packed bf16 pairs of heads (2i, 2i+1) of this half
 #pragma unroll
     for (int i = 0; i < 16; ++i) {
       const int h = 32 * hh + 2 * i;
-      const float p0 = (z[2 * i] == -INFINITY) ? 0.f : exp2f(z[2 * i] - mrun[h]);
-      const float p1 = (z[2 * i + 1] == -INFINITY) ? 0.f : exp2f(z[2 * i + 1] - mrun[h + 1]);
+      float p0 = (z[2 * i] == -INFINITY) ? 0.f : exp2f(z[2 * i] - mrun[h]);
+      float p1 = (z[2 * i + 1] == -INFINITY) ? 0.f : exp2f(z[2 * i + 1] - mrun[h + 1]);
+      if constexpr (kLat8) {
+        z[2 * i] = p0;
+        z[2 * i + 1] = p1;
+        p0 *= wk;
+        p1 *= wk;
+      }
       const __nv_bfloat162 hi = __floats2bfloat162_rn(p0, p1);
       const __nv_bfloat162 lo =
           __floats2bfloat162_rn(p0 - __low2float(hi), p1 - __high2float(hi));
@@ -468,7 +557,10 @@ __global__ void __launch_bounds__(kThreads, 1) mla_kernel(const MlaParams p) {
         const uint32_t hc = (i & 1) ? (c & 0xFFFF0000u) : (c << 16);
         return __uint_as_float(ha) + __uint_as_float(hc);
       };
-      red[q4 * kHeads + 32 * hh + lane] = butterfly32<false>(pf);
+      if constexpr (kLat8)
+        red[q4 * kHeads + 32 * hh + lane] = butterfly32<false>([&](int i) { return z[i]; });
+      else
+        red[q4 * kHeads + 32 * hh + lane] = butterfly32<false>(pf);
     }
     __syncthreads();
     if (tid < kHeads) {
@@ -786,31 +878,6 @@ __device__ __forceinline__ bool pipe_wait(uint64_t *bar, uint32_t parity, uint64
   }
 }
 
-// two E4M3 values (low byte first) as a bf16 pair, exactly: every E4M3 value
-// is an f16 value and a bf16 value
-__device__ __forceinline__ uint32_t e4m3x2_to_bf16x2(uint32_t v16) {
-  uint32_t h;
-  asm("{\n\t.reg .b16 a;\n\tcvt.u16.u32 a, %1;\n\tcvt.rn.f16x2.e4m3x2 %0, a;\n\t}"
-      : "=r"(h)
-      : "r"(v16));
-  const float lo = __half2float(__ushort_as_half(static_cast<unsigned short>(h & 0xFFFFu)));
-  const float hi = __half2float(__ushort_as_half(static_cast<unsigned short>(h >> 16)));
-  const __nv_bfloat162 r = __floats2bfloat162_rn(lo, hi);
-  return *reinterpret_cast<const uint32_t *>(&r);
-}
-__device__ __forceinline__ uint4 ld_shared_v4(uint32_t a) {
-  uint4 v;
-  asm volatile("ld.shared.v4.u32 {%0, %1, %2, %3}, [%4];"
-               : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
-               : "r"(a));
-  return v;
-}
-__device__ __forceinline__ void st_shared_v4(uint32_t a, uint4 v) {
-  asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(a), "r"(v.x), "r"(v.y), "r"(v.z),
-               "r"(v.w)
-               : "memory");
-}
-
 // kLat8: the latent cache holds E4M3 rows with one fp32 scale per token.  The
 // gather stages each row's 64-byte E4M3 slice of an atom in the upper half of
 // its 128-byte destination row (cp.async), then widens it in place to bf16;
@@ -1083,43 +1150,12 @@ __global__ void __launch_bounds__(kPipeThreads, 1) mla_pipe_kernel(const MlaPara
       const int phys_next = resolve(j + 2);  // overlaps the copies in flight
       cp_async_wait_all();
       if constexpr (kLat8) {
-        // widen in place: all four quarters of a row's slice are read (same
-        // warp) before any 32-byte bf16 result is written over them
+        // widen in place (the four quarters of a row are lanes of this warp)
         const int jq = lane & 3, rr = lane >> 2;
-        __syncwarp();
 #pragma unroll 1
         for (int k = 0; k < 4; ++k) {
           const int trow = kHalfKeys * g + 32 * wl + rr + 8 * k;
-          const uint32_t row_base = ls + trow * 128;
-          const uint32_t sw = static_cast<uint32_t>(trow & 7);
-          uint4 st[9];
-#pragma unroll
-          for (int a = 0; a < 9; ++a)
-            if (a < nQ)
-              asm volatile("ld.shared.v4.u32 {%0, %1, %2, %3}, [%4];"
-                           : "=r"(st[a].x), "=r"(st[a].y), "=r"(st[a].z), "=r"(st[a].w)
-                           : "r"(row_base + a * kAtomL + 64 + 16 * jq));
-          __syncwarp();
-#pragma unroll
-          for (int a = 0; a < 9; ++a) {
-            if (a >= nQ) break;
-            const uint32_t w4[4] = {st[a].x, st[a].y, st[a].z, st[a].w};
-            uint32_t o[8];
-#pragma unroll
-            for (int t = 0; t < 4; ++t) {
-              o[2 * t] = e4m3x2_to_bf16x2(w4[t] & 0xFFFFu);
-              o[2 * t + 1] = e4m3x2_to_bf16x2(w4[t] >> 16);
-            }
-            const uint32_t u0 = row_base + a * kAtomL + (((2u * jq) ^ sw) << 4);
-            const uint32_t u1 = row_base + a * kAtomL + (((2u * jq + 1u) ^ sw) << 4);
-            asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(u0), "r"(o[0]), "r"(o[1]),
-                         "r"(o[2]), "r"(o[3])
-                         : "memory");
-            asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(u1), "r"(o[4]), "r"(o[5]),
-                         "r"(o[6]), "r"(o[7])
-                         : "memory");
-          }
-          __syncwarp();
+          widen_e4m3_quarter(ls + trow * 128, static_cast<uint32_t>(trow & 7), jq, nQ);
         }
       }
       fence_proxy_async_smem();
@@ -1379,7 +1415,7 @@ size_t mla_smem_bytes(int R, int P) {
   const bool p_overlays = nL > 2 * nmb;
   return 1024 + static_cast<size_t>(nL) * kAtomL + (p_overlays ? 0 : kAtomL) +
          static_cast<size_t>(nQ) * kAtomQ + 4 * kChunk + 4 * (7 * kHeads) +
-         8 * 4 + 16 + 4 * (kMaxMergeCluster * 2 * kHeads);
+         8 * 4 + 16 + 4 * (kMaxMergeCluster * 2 * kHeads) + 4 * kChunk;
 }
 
 struct SplitPlan {
@@ -1509,7 +1545,7 @@ size_t chunk_scratch_bytes(int n_q, int topk, int R) {
 }
 }  // namespace
 
-// enough for either latent format (FP8 rows always take the pipelined kernel)
+// enough for either latent format (both take the same kernel for a shape)
 size_t mla_scratch_bytes(int n_q, int topk, int R) {
   const size_t pipe = mla_pipe_scratch_bytes(n_q, topk, R);
   return use_pipe(n_q, topk) ? pipe : std::max(pipe, chunk_scratch_bytes(n_q, topk, R));
@@ -1537,15 +1573,15 @@ bool mla_cluster_ok(int size, size_t smem) {
     cfg.numAttrs = 1;
     int n = 0;
     const bool ok =
-        cudaOccupancyMaxActiveClusters(&n, mla_kernel<true>, &cfg) == cudaSuccess && n > 0;
+        cudaOccupancyMaxActiveClusters(&n, mla_kernel<true, false>, &cfg) == cudaSuccess && n > 0;
     cudaGetLastError();  // clear a rejected query
     cached[dev][size] = ok ? 1 : -1;
   }
   return cached[dev][size] > 0;
 }
 
-int mla_launch_count(int n_q, int topk, int R, int P, bool lat8) {
-  if (lat8 || use_pipe(n_q, topk)) {
+int mla_launch_count(int n_q, int topk, int R, int P, bool /*lat8: the same kernels*/) {
+  if (use_pipe(n_q, topk)) {
     const PipePlan pl = plan_pipe(n_q, topk, R, P);
     return (pl.nsplit == 1 || pl.cluster) ? 1 : 2;
   }
@@ -1627,23 +1663,23 @@ dsa_status_t launch_mla_pipe(const MlaLaunch &a, cudaStream_t stream) {
   return DSA_OK;
 }
 
-dsa_status_t launch_mla(const MlaLaunch &a, cudaStream_t stream) {
-  if (a.latent8 != nullptr) return launch_mla_pipe<true>(a, stream);
-  if (a.force_pipe || use_pipe(a.n_q, a.topk)) return launch_mla_pipe<false>(a, stream);
+// the per-chunk kernel for a few rows (bf16 or E4M3 latent rows)
+template <bool L8>
+dsa_status_t launch_mla_chunk(const MlaLaunch &a, cudaStream_t stream) {
   const int W = a.R + a.P;
   const size_t smem = mla_smem_bytes(a.R, a.P);
   if (smem > device_max_smem_optin()) return DSA_ERR_UNSUPPORTED;
-  if (func_attr_once(reinterpret_cast<const void *>(mla_kernel<false>),
-                     cudaFuncAttributeMaxDynamicSharedMemorySize,
-                     static_cast<int>(device_max_smem_optin())) != cudaSuccess ||
-      func_attr_once(reinterpret_cast<const void *>(mla_kernel<true>),
-                     cudaFuncAttributeMaxDynamicSharedMemorySize,
-                     static_cast<int>(device_max_smem_optin())) != cudaSuccess)
-    return DSA_ERR_CUDA;
+  for (const void *k : {reinterpret_cast<const void *>(mla_kernel<false, L8>),
+                        reinterpret_cast<const void *>(mla_kernel<true, L8>)})
+    if (func_attr_once(k, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                       static_cast<int>(device_max_smem_optin())) != cudaSuccess)
+      return DSA_ERR_CUDA;
   const SplitPlan sp = plan_splits(a.n_q, a.topk);
   MlaParams p;
   p.q = a.q;
   p.latent = a.latent;
+  p.latent8 = a.latent8;
+  p.lat_scale = a.lat_scale;
   p.idx = a.idx;
   p.seq_lens = a.seq_lens;
   p.block_table = a.block_table;
@@ -1689,9 +1725,9 @@ dsa_status_t launch_mla(const MlaLaunch &a, cudaStream_t stream) {
                         ? 1 : 0;
   const cudaError_t le =
       p.cluster_merge
-          ? launch_pdl(mla_kernel<true>, dim3(sp.nsplit, a.n_q, p.ncb), dim3(kThreads), smem,
+          ? launch_pdl(mla_kernel<true, L8>, dim3(sp.nsplit, a.n_q, p.ncb), dim3(kThreads), smem,
                        stream, static_cast<unsigned>(sp.nsplit), p)
-          : launch_pdl(mla_kernel<false>, dim3(sp.nsplit, a.n_q, p.ncb), dim3(kThreads), smem,
+          : launch_pdl(mla_kernel<false, L8>, dim3(sp.nsplit, a.n_q, p.ncb), dim3(kThreads), smem,
                        stream, 1u, p);
   if (le != cudaSuccess) return DSA_ERR_CUDA;
   if (sp.merge == kMergeGlobal && !p.cluster_merge) {
@@ -1704,6 +1740,13 @@ dsa_status_t launch_mla(const MlaLaunch &a, cudaStream_t stream) {
       return DSA_ERR_CUDA;
   }
   return DSA_OK;
+}
+
+dsa_status_t launch_mla(const MlaLaunch &a, cudaStream_t stream) {
+  const bool l8 = a.latent8 != nullptr;
+  if (a.force_pipe || use_pipe(a.n_q, a.topk))
+    return l8 ? launch_mla_pipe<true>(a, stream) : launch_mla_pipe<false>(a, stream);
+  return l8 ? launch_mla_chunk<true>(a, stream) : launch_mla_chunk<false>(a, stream);
 }
 
 }  // namespace dsa

@@ -57,14 +57,18 @@ def _check_rows(inp, sel, out, lse, rows, table_row_of, R, scale):
         assert np.max(np.abs(lse[r] - ref_lse)) <= LSE_TOL, r
 
 
+# Both MLA kernels take E4M3 rows; the batch decides which one runs (the
+# per-chunk kernel for a few rows, the pipelined one for many).
 @pytest.mark.parametrize("shape,batch", [
-    (dict(H=64, R=512, P=64, k=2048), 5),    # splits merged in a cluster
-    (dict(H=64, R=512, P=64, k=2048), 32),   # clusters of 4
-    (dict(H=64, R=512, P=64, k=256), 160),   # one CTA per row
-    (dict(H=64, R=512, P=64, k=8192), 1),    # many splits, partials through the merge kernel
-    (dict(H=4, R=64, P=16, k=256), 7),       # a narrow row: one 128-column block
-    (dict(H=16, R=192, P=32, k=300), 9),     # a ragged last column block and top-k
-], ids=["c_b5", "c4_b32", "single_b160", "global_b1", "tiny_b7", "r192_b9"])
+    (dict(H=64, R=512, P=64, k=2048), 5),    # per-chunk: 16 splits through the merge kernel
+    (dict(H=64, R=512, P=64, k=1024), 12),   # per-chunk: 8 splits merged in a cluster
+    (dict(H=64, R=512, P=64, k=2048), 32),   # pipelined: clusters of 4
+    (dict(H=64, R=512, P=64, k=256), 160),   # pipelined: one CTA per row
+    (dict(H=64, R=512, P=64, k=8192), 1),    # per-chunk: 64 splits through the merge kernel
+    (dict(H=4, R=64, P=16, k=256), 7),       # per-chunk: a narrow row, 4 splits in a cluster
+    (dict(H=16, R=192, P=32, k=300), 9),     # per-chunk: a ragged last column block and top-k
+], ids=["chunk_b5", "chunk_c8_b12", "pipe_c4_b32", "pipe_b160", "chunk_b1_k8192", "chunk_tiny_b7",
+        "chunk_r192_b9"])
 def test_sparse_mla_decode_l8(shape, batch):
     rng = np.random.default_rng(batch + shape["k"])
     lengths = rng.integers(1, 3 * shape["k"], size=batch).tolist()
