@@ -99,6 +99,26 @@ bool make_map_2d(CUtensorMap *map, const void *base, uint64_t cols, uint64_t row
   return r == CUDA_SUCCESS;
 }
 
+// [d2][d1][d0] elements of `esize` bytes (2: bf16, 4: fp32) with row strides
+// s1 and s2 bytes, boxes of b0 x b1 x b2 elements; 128-byte swizzle (b0 *
+// esize must then be 128) or none
+bool make_map_3d(CUtensorMap *map, const void *base, int esize, uint64_t d0, uint64_t d1,
+                 uint64_t d2, uint64_t s1, uint64_t s2, uint32_t b0, uint32_t b1, uint32_t b2,
+                 bool swizzle) {
+  auto encode = get_encode_fn();
+  if (encode == nullptr || (esize != 2 && esize != 4)) return false;
+  cuuint64_t dims[3] = {d0, d1, d2};
+  cuuint64_t strides[2] = {s1, s2};
+  cuuint32_t box[3] = {b0, b1, b2};
+  cuuint32_t estr[3] = {1, 1, 1};
+  CUresult r = encode(map, esize == 2 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT32,
+                      3, const_cast<void *>(base), dims, strides, box, estr,
+                      CU_TENSOR_MAP_INTERLEAVE_NONE,
+                      swizzle ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_NONE,
+                      CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
 // bytes (the FP8 index keys and query terms); aw = swizzle width, 128 or 64
 bool make_map_2d_u8(CUtensorMap *map, const void *base, uint64_t cols, uint64_t rows,
                     uint32_t box_cols, uint32_t box_rows, int aw) {

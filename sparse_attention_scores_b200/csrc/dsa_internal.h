@@ -46,6 +46,11 @@ bool make_map_2d_u8(CUtensorMap *map, const void *base, uint64_t cols, uint64_t 
                     uint32_t box_cols, uint32_t box_rows, int aw);
 bool make_map_2d(CUtensorMap *map, const void *base, uint64_t cols, uint64_t rows,
                  uint32_t box_cols, uint32_t box_rows, int aw);
+// [d2][d1][d0] elements of esize bytes (2: bf16, 4: fp32), row strides s1, s2
+// bytes; boxes b0 x b1 x b2; 128-byte swizzle (b0 * esize == 128) or none
+bool make_map_3d(CUtensorMap *map, const void *base, int esize, uint64_t d0, uint64_t d1,
+                 uint64_t d2, uint64_t s1, uint64_t s2, uint32_t b0, uint32_t b1, uint32_t b2,
+                 bool swizzle);
 
 // Remember a failed CUDA call of this thread (its error and where it came
 // from) for dsa_last_cuda_error(); returns err.

@@ -92,6 +92,61 @@ def test_project_values_near_fp32(n, H, R, d_v):
         assert norm_err(got[b], ref) <= 1e-4, b
 
 
+def test_absorb_many_items_per_cta():
+    # 1,000 rows of 64 heads: 512 (head, 128-row tile) items over the SMs, so
+    # a CTA walks several items (weight tile kept, stage and accumulator rings
+    # wrapping) and the last tile is ragged (104 rows)
+    rng = np.random.default_rng(41)
+    n, H, d_nope, R, P = 1000, 64, 128, 512, 64
+    qn, qr = _ints(rng, (n, H, d_nope)), _normal(rng, (n, H, P))
+    wk = _ints(rng, (H, d_nope, R))
+    q_abs = torch.empty((n, H, R + P), dtype=torch.bfloat16, device="cuda")
+    ws = dsa.status_workspace()
+    dsa.dsa_absorb_query(bf16_tensor(qn), bf16_tensor(qr), bf16_tensor(wk), q_abs, ws)
+    assert dsa.workspace_check(ws)[0] == 0
+    got = _bits(q_abs)
+    WK = orc.bf16_to_f64(wk)
+    for b in list(range(0, n, 37)) + [127, 128, 895, 896, 999]:
+        ref = orc.absorb_query(orc.bf16_to_f64(qn[b]), orc.bf16_to_f64(qr[b]), WK)
+        assert np.array_equal(got[b, :, :R], _bf16_rne(ref[:, :R])), b
+        assert np.array_equal(got[b, :, R:], qr[b]), b
+
+
+def test_project_many_items_per_cta():
+    # the projection's rings over several items per CTA and a ragged last tile
+    rng = np.random.default_rng(42)
+    n, H, R, d_v = 1000, 64, 512, 128
+    o = rng.standard_normal((n, H, R)).astype(np.float32)
+    wv = _normal(rng, (H, R, d_v), 1 / math.sqrt(R))
+    v = torch.full((n, H, d_v), float("nan"), device="cuda")
+    ws = dsa.status_workspace()
+    dsa.dsa_project_values(torch.from_numpy(o).cuda(), bf16_tensor(wv), v, ws)
+    assert dsa.workspace_check(ws)[0] == 0
+    got = v.cpu().numpy()
+    W = orc.bf16_to_f64(wv)
+    for b in list(range(0, n, 37)) + [127, 128, 895, 896, 999]:
+        ref = orc.project_values(o[b].astype(np.float64), W)
+        assert norm_err(got[b], ref) <= 1e-4, b
+
+
+def test_project_values_unaligned_output():
+    # an output that is 4- but not 16-byte aligned takes scalar stores
+    rng = np.random.default_rng(43)
+    n, H, R, d_v = 130, 4, 128, 64
+    o = rng.standard_normal((n, H, R)).astype(np.float32)
+    wv = _normal(rng, (H, R, d_v), 1 / math.sqrt(R))
+    buf = torch.full((n * H * d_v + 1,), float("nan"), device="cuda")
+    v = buf[1:].view(n, H, d_v)
+    ws = dsa.status_workspace()
+    dsa.dsa_project_values(torch.from_numpy(o).cuda(), bf16_tensor(wv), v, ws)
+    assert dsa.workspace_check(ws)[0] == 0
+    assert np.isnan(buf[0].item())
+    got = v.cpu().numpy()
+    W = orc.bf16_to_f64(wv)
+    for b in range(n):
+        assert norm_err(got[b], orc.project_values(o[b].astype(np.float64), W)) <= 1e-4, b
+
+
 def test_nonabsorbed_block_end_to_end():
     # q_nope, q_rope, W_UK, W_UV, caches -> absorb -> step -> project, against
     # the oracle's non-absorbed attention over the same selected tokens
