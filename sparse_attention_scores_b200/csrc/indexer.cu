@@ -119,12 +119,16 @@ __global__ void __launch_bounds__(threads_of<NEG>(), NEG == 1 ? 2 : 1)
   const int stage_bytes = kStageScales + (K8 ? 1024 : 0);
   const int ncols = G * p.H_I;                  // useful accumulator columns
   const int n_mma = (ncols + 15) & ~15;         // MMA N (multiple of 16)
-  // K8: the hi and lo query terms, each [n_mma rows][D_I bytes]
+  // K8: the hi and lo query terms, each [n_mma rows][D_I bytes], one after
+  // the other; when both fit one MMA (N = 2 n_mma <= 256) they are its B
+  // operand and the two products land side by side (hi, then lo columns)
   const int q_bytes = (K8 ? 2 : 1) * natoms * n_mma * AW;
-  const uint32_t acc_stride = (n_mma + 31) & ~31;
-  // as many accumulators as fit 512 columns (<= 8): the MMA warp runs that
-  // many tiles ahead of the epilogue
-  const int nacc = min(kMaxAcc, static_cast<int>(512u / acc_stride));
+  const bool fuse = K8 && 2 * n_mma <= 256;
+  const uint32_t acc_stride = ((fuse ? 2 * n_mma : n_mma) + 31) & ~31;
+  // as many accumulators as fit this CTA's share of the 512 columns (two CTAs
+  // per SM: 256 each) (<= 8): the MMA warp runs that many tiles ahead of the
+  // epilogue
+  const int nacc = min(kMaxAcc, static_cast<int>((NEG == 1 ? 256u : 512u) / acc_stride));
   uint32_t tmem_cols = 32;
   while (tmem_cols < nacc * acc_stride) tmem_cols <<= 1;
 
@@ -318,8 +322,8 @@ __global__ void __launch_bounds__(threads_of<NEG>(), NEG == 1 ? 2 : 1)
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issuer
     if (lane == 0) {
-      const uint32_t idesc =
-          K8 ? idesc_e4m3_f32(kTileKeys, n_mma) : idesc_bf16_f32(kTileKeys, n_mma, 0, 0);
+      const uint32_t idesc = K8 ? idesc_e4m3_f32(kTileKeys, fuse ? 2 * n_mma : n_mma)
+                                : idesc_bf16_f32(kTileKeys, n_mma, 0, 0);
       int stage = 0, qslot = 0, cur = -1, cur_slot = 0;
       uint32_t phase = 0, qphase = 0;
       bool ok = true;
@@ -344,7 +348,13 @@ __global__ void __launch_bounds__(threads_of<NEG>(), NEG == 1 ? 2 : 1)
         const uint32_t d = tmem_base + acc * acc_stride;
         const uint32_t a_base = smem_u32(stage_base + stage * stage_bytes);
         const uint32_t b_base = smem_u32(q_base + cur_slot * q_bytes);
-        if (K8) {
+        if (K8 && fuse) {
+          // E4M3 keys x [hi | lo] E4M3 query terms in one N = 2 n_mma operand
+          // (one K atom: D_I = 128 bytes), 32 elements (32 bytes) per MMA
+          for (int kk = 0; kk < AW / 32; ++kk)
+            mma_e4m3(d, smem_desc(a_base + kk * 32, 16, 8 * AW, layout),
+                     smem_desc(b_base + kk * 32, 16, 8 * AW, layout), idesc, kk != 0 ? 1u : 0u);
+        } else if (K8) {
           // E4M3 keys x (hi + lo) E4M3 query terms, 32 elements (32 bytes) per MMA
           for (int term = 0; term < 2; ++term)
             for (int a = 0; a < natoms; ++a)
@@ -424,6 +434,14 @@ __global__ void __launch_bounds__(threads_of<NEG>(), NEG == 1 ? 2 : 1)
         uint32_t v[32];
         tmem_ld_32x32b_x32(taddr, v);
         tmem_ld_wait();
+        if (fuse) {
+          // the lo term's products, n_mma columns on
+          uint32_t v2[32];
+          tmem_ld_32x32b_x32(taddr + n_mma, v2);
+          tmem_ld_wait();
+#pragma unroll
+          for (int i = 0; i < 32; ++i) v[i] = __float_as_uint(__uint_as_float(v[i]) + __uint_as_float(v2[i]));
+        }
 #pragma unroll
         for (int i = 0; i < 32; ++i) {
           const float x = __uint_as_float(v[i]);
@@ -440,6 +458,13 @@ __global__ void __launch_bounds__(threads_of<NEG>(), NEG == 1 ? 2 : 1)
           const int nvalid = min(32, p.H_I - h0);
           const float *wrow = p.w + static_cast<int64_t>(min(g * G + j, p.n_q - 1)) * p.H_I + h0;
           tmem_ld_wait();
+          if (fuse) {
+            uint32_t v2[32];
+            tmem_ld_32x32b_x32(taddr + n_mma + c * 32, v2);
+            tmem_ld_wait();
+#pragma unroll
+            for (int i = 0; i < 32; ++i) v[i] = __float_as_uint(__uint_as_float(v[i]) + __uint_as_float(v2[i]));
+          }
           float part = 0.f;
 #pragma unroll
           for (int i = 0; i < 32; ++i) {
