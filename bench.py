@@ -428,20 +428,23 @@ def measure(case, torch, steps, warmup, flush_buf, peaks, extras=True):
 TRAFFIC_SOURCES = {"indexer": ["indexer.cu"], "topk": ["topk.cu"], "mla": ["mla.cu"]}
 TRAFFIC_COMMON = ["dsa_common.cuh", "dsa_internal.h"]
 TRAFFIC = {
-    # (stage, workload): (bytes per launch, digest of the stage's sources)
-    # (the indexer and combine_kernel figures were captured on the same kernel code before a
-    # cluster-store helper was added to the shared header)
-    ("indexer", "glm5_decode_8k"): (2156800, "dbf4a9f82361f435"),
-    ("indexer", "glm5_decode_4x128k"): (139531776, "dbf4a9f82361f435"),
-    # topk_small_kernel at 8,192 keys, topk_creg_kernel at 4 x 131,072
-    ("topk", "glm5_decode_8k"): (51968, "eb45bacdb16e700c"),
-    ("topk", "glm5_decode_4x128k"): (2122240, "eb45bacdb16e700c"),
+    # (stage, workload): (bytes per launch, digest of the stage's sources); the
+    # median of 19 launches of one capture per workload
+    ("indexer", "glm5_decode_b32_ragged"): (279645696, "c1ecacdf680da725"),
+    ("indexer", "glm5_decode_8k"): (2156544, "c1ecacdf680da725"),
+    ("indexer", "glm5_decode_4x128k"): (134889216, "c1ecacdf680da725"),
+    ("indexer", "glm5_prefill_2300"): (19776000, "c1ecacdf680da725"),
+    # topk_creg_kernel (32 rows, 4 x 131,072) and topk_small_kernel (8,192 keys, prefill rows)
+    ("topk", "glm5_decode_b32_ragged"): (4351744, "6895ccb10040898d"),
+    ("topk", "glm5_decode_8k"): (52224, "6895ccb10040898d"),
+    ("topk", "glm5_decode_4x128k"): (2121984, "6895ccb10040898d"),
+    ("topk", "glm5_prefill_2300"): (2234112, "6895ccb10040898d"),
     # mla_kernel + combine_kernel (the merge reads the split partials)
-    ("mla", "glm5_decode_8k"): (2509056 + 4232448, "819a18ad9156f93f"),
-    ("mla", "glm5_decode_4x128k"): (9863936 + 16864256, "819a18ad9156f93f"),
+    ("mla", "glm5_decode_8k"): (2508800 + 4232192, "571e9f8a5da9a90c"),
+    ("mla", "glm5_decode_4x128k"): (9864960 + 16864256, "571e9f8a5da9a90c"),
     # mla_pipe_kernel (rows merged inside clusters; prefill rows unsplit)
-    ("mla", "glm5_decode_b32_ragged"): (78270208 + 2242304, "b9c0f12e2375e2fd"),
-    ("mla", "glm5_prefill_2300"): (183166464 + 246434560, "b9c0f12e2375e2fd"),
+    ("mla", "glm5_decode_b32_ragged"): (78309632, "571e9f8a5da9a90c"),
+    ("mla", "glm5_prefill_2300"): (425383680, "571e9f8a5da9a90c"),
 }
 
 
