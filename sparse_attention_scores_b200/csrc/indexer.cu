@@ -6,9 +6,11 @@
 // every earlier token; section "How do we know it is right?": ReLU per
 // indexer head before the heads are combined.)
 //
-// Design (sm_100a): one persistent CTA per SM walks a contiguous range of
-// work units.  A unit is one tile of 128 keys of one row group (decode: one
-// sequence; causal prefill: G consecutive query rows, which share their keys).
+// Design (sm_100a): persistent CTAs walk the work units, each first a
+// contiguous share of most of them, then small chunks of the rest taken from a
+// counter, so that the CTAs finish together.  A unit is one tile of 128 keys
+// of one row group (decode: one sequence; causal prefill: G consecutive query
+// rows, which share their keys).
 // The key tile is the A operand (M = 128 keys, K = D_I), the queries of the
 // group are the B operand (N = G * H_I), so one MMA chain per tile yields
 // every (key, row, head) dot product in tensor memory.  Warp roles:
@@ -55,7 +57,10 @@ __host__ __device__ constexpr int threads_of() { return 64 + 128 * NEG; }
 constexpr int kMaxStages = 8;
 constexpr int kMaxAcc = 8;         // accumulator buffers in tensor memory
 constexpr int kTileKeys = 128;
-constexpr int kLookahead = 16;  // units whose page ids the producer fetches at once
+constexpr int kBatch = 16;  // units whose pages the producer looks up at once (<= 16)
+constexpr int kStaticPct = 50;  // share of the units split statically over the CTAs
+constexpr int kDynChunk = 8;    // most units per counter chunk after that
+constexpr int kRing = 32;   // entries of the unit ring (> stages + accumulators + 2)
 
 struct IndexerParams {
   const float *w;
@@ -68,9 +73,14 @@ struct IndexerParams {
   int num_groups;
   int stages;
   int q_buffers;   // 1 or 2 query tiles in shared memory
+  int static_pct;  // share of the units split statically, in percent
+  int chunk;       // most units taken from the counter at a time (<= 16)
   uint64_t wait_ns;
   int debug_stall;  // the MMA issuer first waits on a barrier nothing arrives at
   const float *k_scale;  // K8: per physical key row [num_pages * 64]
+  // [0] next unit to hand out, [1] CTAs finished (zero between launches: the
+  // last CTA to finish resets both; the workspace init zeroes them first)
+  int *work;
   DevStatus *status;
 };
 
@@ -145,9 +155,13 @@ __global__ void __launch_bounds__(threads_of<NEG>(), NEG == 1 ? 2 : 1)
   uint32_t *misc = reinterpret_cast<uint32_t *>(drain + 1);  // [0] tmem base, [1] abort
   int *scan_tmp = reinterpret_cast<int *>(misc + 4);          // [kThreads + 32]
   int *tile_start = scan_tmp + kThreads + 32;                 // [num_groups + 1]
+  const int NG = p.num_groups;
+  // (sequence number, unit, group) of this CTA's i-th unit, at [i % kRing]
+  // (16-byte aligned: it is read and written as one vector)
+  volatile int4 *uring = reinterpret_cast<volatile int4 *>(
+      (reinterpret_cast<uintptr_t>(tile_start + NG + 1) + 15) & ~static_cast<uintptr_t>(15));
 
   const int warp = warp_id(), lane = lane_id();
-  const int NG = p.num_groups;
 
   if (threadIdx.x == 0) {
     // K8: a stage is free once the MMA has run and the four epilogue warps that
@@ -157,6 +171,8 @@ __global__ void __launch_bounds__(threads_of<NEG>(), NEG == 1 ? 2 : 1)
     for (int i = 0; i < kMaxAcc; ++i) { mbar_init(&tfull[i], 1); mbar_init(&tempty[i], 4); }
     mbar_init(drain, 1);
     misc[1] = 0u;
+    if (NEG == 2)
+      for (int i = 0; i < kRing; ++i) uring[i].x = -1;
     fence_barrier_init();
   }
   if (warp == 0 && lane == 0) { tma_prefetch_desc(&tmK); tma_prefetch_desc(&tmQ); }
@@ -206,9 +222,40 @@ __global__ void __launch_bounds__(threads_of<NEG>(), NEG == 1 ? 2 : 1)
   volatile uint32_t *abort_flag = &misc[1];
 
   const int total = tile_start[NG];
-  const int u0 = static_cast<int>((static_cast<int64_t>(total) * blockIdx.x) / gridDim.x);
-  const int u1 = static_cast<int>((static_cast<int64_t>(total) * (blockIdx.x + 1)) / gridDim.x);
+  // Work order: this CTA first walks its share of the first p.static_pct % of
+  // the units (a contiguous range, so a row group's query tile is loaded once
+  // per CTA), then takes chunks of at most p.chunk units from a counter shared by all
+  // CTAs until none is left, so CTAs that run slower take fewer of them and
+  // all finish together.  The MMA and epilogue warps know the static range;
+  // the producer publishes each counter unit it issues (the i-th unit of the
+  // CTA in uring[i % kRing]) and an end mark after the last.
+  // (decode CTAs, two per SM with one query buffer each, keep to the static split)
+  const bool dyn = NEG == 2 && p.static_pct < 100;
+  const int st_total = static_cast<int>((static_cast<int64_t>(total) * min(p.static_pct, 100)) / 100);
+  const int s0 = static_cast<int>((static_cast<int64_t>(st_total) * blockIdx.x) / gridDim.x);
+  const int s1 = static_cast<int>((static_cast<int64_t>(st_total) * (blockIdx.x + 1)) / gridDim.x);
+  // counter chunks: about two per CTA of what the static share leaves,
+  // at most p.chunk units (the same value in every CTA)
+  const int chunk = max(1, min(p.chunk, (total - st_total) / (2 * static_cast<int>(gridDim.x))));
   const uint32_t layout = (AW == 128) ? kLayoutSW128 : kLayoutSW64;
+  // (lane 0) wait until uring holds the i-th entry; false on abort or time-out
+  auto ring_get = [&](int i, int4 &e) -> bool {
+    const uint32_t addr = smem_u32(const_cast<int4 *>(&uring[i % kRing]));
+    const uint64_t t0 = global_timer_ns();
+    uint32_t spins = 0;
+    while (true) {
+      asm volatile("ld.volatile.shared.v4.s32 {%0, %1, %2, %3}, [%4];"
+                   : "=r"(e.x), "=r"(e.y), "=r"(e.z), "=r"(e.w)
+                   : "r"(addr)
+                   : "memory");
+      if (e.x == i) return true;
+      if (++spins >= 16) {
+        spins = 0;
+        if (*abort_flag || global_timer_ns() - t0 > p.wait_ns) return false;
+        __nanosleep(32);
+      }
+    }
+  };
 
   if (warp == 0) {
     // ------------------------------------------------------------ producer
@@ -216,13 +263,42 @@ __global__ void __launch_bounds__(threads_of<NEG>(), NEG == 1 ? 2 : 1)
     uint32_t phase = 0, qphase = 0;
     uint32_t armed = 0, armed_par = 0;  // stages with loads in flight, their phase parity
     bool ok = true;
-    // lane-parallel lookahead: lane l resolves page (l & 1) of unit ub + l/2;
-    // the next batch is fetched while the current one is issued
-    auto fetch = [&](int ub_, int &g_, int &id_) {
-      const int my_u = ub_ + (lane >> 1);
+    int seq = 0;  // units issued so far
+    // batches of at most kBatch units: the static range, then counter chunks;
+    // the counter is read one batch ahead so the atomic's latency is hidden
+    int sb = s0;
+    int pend = 0;           // lane 0: a counter value not yet used
+    bool asked = false, dyn_done = false;
+    auto ask = [&]() {
+      if (lane == 0) pend = atomicAdd(p.work, chunk);
+      asked = true;
+    };
+    auto take = [&](int &b_, int &n_) {
+      b_ = total;
+      n_ = 0;
+      if (sb < s1) {
+        b_ = sb;
+        n_ = min(kBatch, s1 - sb);
+        sb += n_;
+        if (sb >= s1 && dyn && !asked) ask();
+        return;
+      }
+      if (!dyn || dyn_done) return;
+      if (!asked) ask();
+      const int c = st_total + __shfl_sync(0xffffffffu, pend, 0);
+      asked = false;
+      if (c >= total) { dyn_done = true; return; }
+      b_ = c;
+      n_ = min(chunk, total - c);
+      ask();
+    };
+    // lane-parallel page lookup: lane l resolves page (l & 1) of unit b_ + l/2;
+    // the next batch is looked up while the current one is issued
+    auto fetch = [&](int b_, int n_, int &g_, int &id_) {
+      const int my_u = b_ + (lane >> 1);
       g_ = -1;
       id_ = -1;
-      if (my_u < u1) {
+      if ((lane >> 1) < n_) {
         g_ = locate(tile_start, NG, my_u);
         const int t = my_u - tile_start[g_];
         const int pg = 2 * t + (lane & 1);
@@ -236,38 +312,50 @@ __global__ void __launch_bounds__(threads_of<NEG>(), NEG == 1 ? 2 : 1)
         }
       }
     };
-    int cur_g, cur_id;
-    fetch(u0, cur_g, cur_id);
-    for (int ub = u0; ub < u1 && ok; ub += kLookahead) {
-      int nxt_g, nxt_id;
-      fetch(ub + kLookahead, nxt_g, nxt_id);
-      const int nb = min(kLookahead, u1 - ub);
-      for (int i = 0; i < nb; ++i) {
+    // (lane 0) the query tile of group gq into the next query buffer, once the
+    // MMAs of the group that held it have completed
+    uint32_t qarmed = 0, qarmed_par = 0;  // query buffers with loads in flight, their parity
+    auto load_q = [&](int gq) -> bool {
+      if (!mbar_wait(&qempty[qslot], qphase ^ 1u, p.wait_ns)) return false;
+      mbar_arrive_expect_tx(&qfull[qslot], static_cast<uint32_t>((K8 ? 2 : 1) * natoms * ncols * AW));
+      if (K8) {
+        // hi plane rows [gq * ncols, ...), lo plane rows n_q * H_I further on
+        uint8_t *qd = q_base + qslot * q_bytes;
+        tma_load_2d(qd, &tmQ, 0, gq * ncols, &qfull[qslot]);
+        tma_load_2d(qd + n_mma * AW, &tmQ, 0, p.n_q * p.H_I + gq * ncols, &qfull[qslot]);
+      } else {
+        for (int a = 0; a < natoms; ++a)
+          tma_load_2d(q_base + qslot * q_bytes + a * n_mma * AW, &tmQ, a * (AW / 2), gq * ncols,
+                      &qfull[qslot]);
+      }
+      qarmed |= 1u << qslot;
+      qarmed_par = (qarmed_par & ~(1u << qslot)) | (qphase << qslot);
+      if (++qslot == nqb) { qslot = 0; qphase ^= 1u; }
+      return true;
+    };
+    int cb, cn, cur_g, cur_id;
+    take(cb, cn);
+    fetch(cb, cn, cur_g, cur_id);
+    while (cn > 0 && ok) {
+      int nb, nn, nxt_g, nxt_id;
+      take(nb, nn);
+      fetch(nb, nn, nxt_g, nxt_id);
+      for (int i = 0; i < cn; ++i) {
         const int g = __shfl_sync(0xffffffffu, cur_g, 2 * i);
         const int id0 = __shfl_sync(0xffffffffu, cur_id, 2 * i);
         const int id1 = __shfl_sync(0xffffffffu, cur_id, 2 * i + 1);
         int okl = 1;
         if (lane == 0) {
           if (*abort_flag) okl = 0;
-          if (okl && g != cur) {
-            if (!mbar_wait(&qempty[qslot], qphase ^ 1u, p.wait_ns)) {
-              okl = 0;
-            } else {
-              mbar_arrive_expect_tx(&qfull[qslot],
-                                    static_cast<uint32_t>((K8 ? 2 : 1) * natoms * ncols * AW));
-              if (K8) {
-                // hi plane rows [g * ncols, ...), lo plane rows n_q * H_I further on
-                uint8_t *qd = q_base + qslot * q_bytes;
-                tma_load_2d(qd, &tmQ, 0, g * ncols, &qfull[qslot]);
-                tma_load_2d(qd + n_mma * AW, &tmQ, 0, p.n_q * p.H_I + g * ncols, &qfull[qslot]);
-              } else {
-                for (int a = 0; a < natoms; ++a)
-                  tma_load_2d(q_base + qslot * q_bytes + a * n_mma * AW, &tmQ, a * (AW / 2),
-                              g * ncols, &qfull[qslot]);
-              }
-            }
-          }
+          if (okl && g != cur && !load_q(g)) okl = 0;
           if (okl && !mbar_wait(&empty[stage], phase ^ 1u, p.wait_ns)) okl = 0;
+          if (okl && dyn) {
+            // publish the unit before its stage is armed (the arrive releases it)
+            asm volatile("st.volatile.shared.v4.s32 [%0], {%1, %2, %3, %4};" ::"r"(
+                             smem_u32(const_cast<int4 *>(&uring[seq % kRing]))),
+                         "r"(seq), "r"(cb + i), "r"(g), "r"(0)
+                         : "memory");
+          }
           if (okl) {
             // K8: each page also brings its 64 scales (256 bytes) into the stage
             const uint32_t page_bytes = kPageSize * p.D_I * kEB + (K8 ? kPageSize * 4 : 0);
@@ -302,22 +390,42 @@ __global__ void __launch_bounds__(threads_of<NEG>(), NEG == 1 ? 2 : 1)
         }
         okl = __shfl_sync(0xffffffffu, okl, 0);
         if (!okl) { ok = false; break; }
-        if (g != cur) {
-          cur = g;
-          if (++qslot == nqb) { qslot = 0; qphase ^= 1u; }
-        }
+        cur = g;
+        ++seq;
         if (++stage == S) { stage = 0; phase ^= 1u; }
       }
+      cb = nb;
+      cn = nn;
       cur_g = nxt_g;
       cur_id = nxt_id;
     }
     if (lane == 0) {
+      if (ok && dyn) {
+        // end of the sequence, once for each epilogue warpgroup
+        for (int k = 0; k < NEG; ++k)
+          asm volatile("st.volatile.shared.v4.s32 [%0], {%1, %2, %3, %4};" ::"r"(
+                           smem_u32(const_cast<int4 *>(&uring[(seq + k) % kRing]))),
+                       "r"(seq + k), "r"(-1), "r"(-1), "r"(0)
+                       : "memory");
+      }
+      if (dyn) {
+        // this CTA reads the counter no more (the fence orders a request still
+        // in flight after an abort); the last CTA to get here leaves both
+        // counters at zero for the next launch, whose reads wait for this grid
+        __threadfence();
+        if (atomicAdd(&p.work[1], 1) == static_cast<int>(gridDim.x) - 1) {
+          atomicExch(&p.work[0], 0);
+          atomicExch(&p.work[1], 0);
+        }
+      }
       if (!ok && !*abort_flag) {
         *abort_flag = 1u;
         report(p.status, kErrTimeout, (kKernIndexer << 24) | 0x1);
       }
       for (int s = 0; s < S; ++s)  // drain loads in flight
         if (armed & (1u << s)) mbar_wait(&full[s], (armed_par >> s) & 1u, kDrainLimitNs);
+      for (int s = 0; s < nqb; ++s)
+        if (qarmed & (1u << s)) mbar_wait(&qfull[s], (qarmed_par >> s) & 1u, kDrainLimitNs);
     }
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issuer
@@ -328,20 +436,33 @@ __global__ void __launch_bounds__(threads_of<NEG>(), NEG == 1 ? 2 : 1)
       uint32_t phase = 0, qphase = 0;
       bool ok = true;
       if (p.debug_stall && !mbar_wait(drain, 0, p.wait_ns)) ok = false;
-      int g = (u0 < u1) ? locate(tile_start, NG, u0) : 0;
-      for (int u = u0; u < u1 && ok; ++u) {
-        while (tile_start[g + 1] <= u) ++g;
-        if (*abort_flag) { ok = false; break; }
+      int gs = (s0 < s1) ? locate(tile_start, NG, s0) : 0;
+      for (int i = 0; ok; ++i) {
+        int g;
+        if (i < s1 - s0) {
+          while (tile_start[gs + 1] <= s0 + i) ++gs;
+          g = gs;
+        } else {
+          if (!dyn) break;
+          int4 e;
+          if (!ring_get(i, e)) { ok = false; break; }
+          if (e.y < 0) break;  // end of the sequence
+          g = e.z;
+        }
         if (g != cur) {
+          // the previous group's query buffer is free once its MMAs complete.
+          // (With the counter the MMA learns of a new group from the ring only
+          // after the producer has loaded its query tile, so that load must not
+          // wait for this commit: the grouped CTAs have a second query buffer.)
+          if (cur >= 0) mma_commit(&qempty[cur_slot]);
           if (!mbar_wait(&qfull[qslot], qphase, p.wait_ns)) { ok = false; break; }
           cur = g;
           cur_slot = qslot;
           if (++qslot == nqb) { qslot = 0; qphase ^= 1u; }
         }
         // accumulator of the i-th unit of this CTA: i % nacc, its (i / nacc)-th use
-        const int i_unit = u - u0;
-        const int acc = i_unit % nacc;
-        const uint32_t aphase = static_cast<uint32_t>(i_unit / nacc) & 1u;
+        const int acc = i % nacc;
+        const uint32_t aphase = static_cast<uint32_t>(i / nacc) & 1u;
         if (!mbar_wait(&full[stage], phase, p.wait_ns)) { ok = false; break; }
         if (!mbar_wait(&tempty[acc], aphase ^ 1u, p.wait_ns)) { ok = false; break; }
         tc_fence_after();
@@ -376,8 +497,6 @@ __global__ void __launch_bounds__(threads_of<NEG>(), NEG == 1 ? 2 : 1)
         }
         mma_commit(&empty[stage]);
         mma_commit(&tfull[acc]);
-        const bool last_of_group = (u + 1 == u1) || (tile_start[g + 1] <= u + 1);
-        if (last_of_group) mma_commit(&qempty[cur_slot]);
         if (++stage == S) { stage = 0; phase ^= 1u; }
       }
       if (!ok && !*abort_flag) {
@@ -399,10 +518,24 @@ __global__ void __launch_bounds__(threads_of<NEG>(), NEG == 1 ? 2 : 1)
     float wreg[32];
     int wgroup = -1;
     bool ok = true;
-    int g = (u0 < u1) ? locate(tile_start, NG, u0) : 0;
-    for (int u = u0 + eg; u < u1; u += NEG) {
-      while (tile_start[g + 1] <= u) ++g;
-      const int i_unit = u - u0;
+    int gs = (s0 < s1) ? locate(tile_start, NG, s0) : 0;
+    for (int i_unit = eg;; i_unit += NEG) {
+      int u, g;
+      if (i_unit < s1 - s0) {
+        u = s0 + i_unit;
+        while (tile_start[gs + 1] <= u) ++gs;
+        g = gs;
+      } else {
+        if (!dyn) break;
+        int4 e = make_int4(0, -1, -1, 0);
+        int got = 1;
+        if (lane == 0) got = ring_get(i_unit, e) ? 1 : 0;
+        got = __shfl_sync(0xffffffffu, got, 0);
+        if (!got) { ok = false; break; }
+        u = __shfl_sync(0xffffffffu, e.y, 0);
+        g = __shfl_sync(0xffffffffu, e.z, 0);
+        if (u < 0) break;  // end of the sequence
+      }
       const int acc = i_unit % nacc;
       const uint32_t aphase = static_cast<uint32_t>(i_unit / nacc) & 1u;
       if (w_in_regs && g != wgroup) {
@@ -594,7 +727,7 @@ dsa_status_t launch_impl(const IndexerLaunch &a, cudaStream_t stream) {
   const int q_buffers = (NEG == 1) ? 1 : 2;
   const size_t fixed = 1024 /*align*/ + q_buffers * q_bytes +
                        8 * (2 * kMaxStages + 4 + 2 * kMaxAcc + 1) + 16 + 4 * (kThreads + 32) +
-                       4 * ((num_groups + 4) & ~3) + 64;
+                       4 * ((num_groups + 4) & ~3) + (NEG == 2 ? 16 + 16 * kRing : 0) + 64;
   const size_t max_smem = device_max_smem_optin();
   const size_t budget = std::min((NEG == 1) ? (device_smem_per_sm() / 2 - 1024) : max_smem, max_smem);
   if (budget <= fixed) return DSA_ERR_UNSUPPORTED;
@@ -628,10 +761,15 @@ dsa_status_t launch_impl(const IndexerLaunch &a, cudaStream_t stream) {
   p.num_groups = num_groups;
   p.stages = stages;
   p.q_buffers = q_buffers;
+  // decode CTAs hold one query tile, so a chunk from another row would stall
+  // the MMA on its query: they keep to their static share (and have no ring)
+  p.static_pct = (NEG == 1) ? 100 : kStaticPct;
+  p.chunk = kDynChunk;
   p.wait_ns = wait_limit_ns();
   p.debug_stall = debug_stall() == kKernIndexer ? 1 : 0;
   p.k_scale = a.k_scale;
   p.status = a.status;
+  p.work = reinterpret_cast<int *>(&a.status->pad[0]);
   if (launch_pdl(indexer_kernel<G, AW, NEG, K8>, dim3(grid), dim3(kThreads), smem, stream, 1, tmK, tmQ,
                  p) != cudaSuccess)
     return DSA_ERR_CUDA;
