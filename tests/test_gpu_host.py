@@ -108,3 +108,43 @@ def test_pageable_host_buffers_take_the_copy_engine():
     assert dsa.workspace_check(hws)[0] == 0
     assert torch.equal(idx_h, idx.cpu()) and torch.equal(out_h, out.cpu())
     assert torch.equal(lse_h, lse.cpu())
+
+
+def test_back_to_back_calls_keep_their_own_queries():
+    # calls queued without a sync between them, through one workspace, on
+    # different queries: each must attend with its own (the next call's input
+    # copy overwrites the staging only after the previous step's MLA has read it)
+    wl = CASES[0]
+    inp = di.make_inputs(wl)
+    t = upload(inp)
+    cache, dims = cache_of(inp, t), dims_of(inp)
+    n, k, H, R = wl.n_q, wl.topk, wl.H, wl.R
+    q_b = -t["q"]   # every sign flipped (exact in bf16)
+    ws = dsa.workspace(dsa.OP_ATTENTION_FORWARD, dims, cache)
+    want = []
+    for q in (t["q"], q_b):
+        out = torch.empty((n, H, R), device="cuda")
+        lse = torch.empty((n, H), device="cuda")
+        dsa.dsa_attention_forward(t["q_idx"], t["w"], t["k_pages"], q, t["latent_pages"], cache,
+                                  dims, None, out, lse, ws)
+        want.append((out.cpu(), lse.cpu()))
+    assert not torch.equal(want[0][0], want[1][0])
+    hin = {name: _pinned(t[name]) for name in ("q_idx", "w", "seq_lens", "block_table")}
+    q_h = [_pinned(t["q"]), _pinned(q_b)]
+    cache_h = dsa.PagedCache(hin["seq_lens"], hin["block_table"], num_pages=cache.num_pages,
+                             max_seq_len=cache.max_seq_len)
+    hws = dsa.workspace(dsa.OP_ATTENTION_FORWARD_HOST, dims, cache_h)
+    got = []
+    for rep in range(3):
+        for q in q_h:
+            out_h = torch.full((n, H, R), float("nan")).pin_memory()
+            lse_h = torch.full((n, H), float("nan")).pin_memory()
+            dsa.dsa_attention_forward_host(hin["q_idx"], hin["w"], t["k_pages"], q,
+                                           t["latent_pages"], cache_h, dims, None, out_h, lse_h,
+                                           hws)
+            got.append((out_h, lse_h))
+    torch.cuda.synchronize()
+    assert dsa.workspace_check(hws)[0] == 0
+    for i, (out_h, lse_h) in enumerate(got):
+        assert torch.equal(out_h, want[i % 2][0]), f"call {i}"
+        assert torch.equal(lse_h, want[i % 2][1]), f"call {i}"
