@@ -60,6 +60,8 @@ constexpr int kTileKeys = 128;
 constexpr int kBatch = 16;  // units whose pages the producer looks up at once (<= 16)
 constexpr int kStaticPct = 50;  // share of the units split statically over the CTAs
 constexpr int kDynChunk = 8;    // most units per counter chunk after that
+constexpr int kDecodeStaticPct = 75;  // the same for decode (100: static only, one query buffer)
+constexpr int kMinDynUnits = 8;       // units per CTA below which the split stays static
 constexpr int kRing = 32;   // entries of the unit ring (> stages + accumulators + 2)
 
 struct IndexerParams {
@@ -171,7 +173,7 @@ __global__ void __launch_bounds__(threads_of<NEG>(), NEG == 1 ? 2 : 1)
     for (int i = 0; i < kMaxAcc; ++i) { mbar_init(&tfull[i], 1); mbar_init(&tempty[i], 4); }
     mbar_init(drain, 1);
     misc[1] = 0u;
-    if (NEG == 2)
+    if (p.static_pct < 100 && nqb == 2)
       for (int i = 0; i < kRing; ++i) uring[i].x = -1;
     fence_barrier_init();
   }
@@ -229,8 +231,10 @@ __global__ void __launch_bounds__(threads_of<NEG>(), NEG == 1 ? 2 : 1)
   // all finish together.  The MMA and epilogue warps know the static range;
   // the producer publishes each counter unit it issues (the i-th unit of the
   // CTA in uring[i % kRing]) and an end mark after the last.
-  // (decode CTAs, two per SM with one query buffer each, keep to the static split)
-  const bool dyn = NEG == 2 && p.static_pct < 100;
+  // (only with two query buffers, see the MMA issuer's group change, and
+  // enough units per CTA for chunks to pay for the counter's latency)
+  const bool dyn = p.static_pct < 100 && nqb == 2 &&
+                   total >= kMinDynUnits * static_cast<int>(gridDim.x);
   const int st_total = static_cast<int>((static_cast<int64_t>(total) * min(p.static_pct, 100)) / 100);
   const int s0 = static_cast<int>((static_cast<int64_t>(st_total) * blockIdx.x) / gridDim.x);
   const int s1 = static_cast<int>((static_cast<int64_t>(st_total) * (blockIdx.x + 1)) / gridDim.x);
@@ -721,13 +725,25 @@ dsa_status_t launch_impl(const IndexerLaunch &a, cudaStream_t stream) {
   }
   (void)natoms;
 
+  const int64_t max_keys = a.causal ? static_cast<int64_t>(a.q_pos0) + a.n_q : a.max_seq_len;
+  const int64_t max_units = static_cast<int64_t>(num_groups) * ((max_keys + kTileKeys - 1) / kTileKeys);
+  const int per_sm = (NEG == 1) ? 2 : 1;
+  const int grid = static_cast<int>(
+      std::max<int64_t>(1, std::min<int64_t>(static_cast<int64_t>(per_sm) * device_sm_count(), max_units)));
   const size_t stage_bytes = static_cast<size_t>(kTileKeys) * a.D_I * kEB + (K8 ? 1024 : 0);
   const size_t q_bytes = static_cast<size_t>(K8 ? 2 : 1) * natoms * n_mma * AW;
-  // two CTAs per SM share the SM's shared memory (one query tile each)
-  const int q_buffers = (NEG == 1) ? 1 : 2;
+  // the counter needs a second query tile; bf16-key decode CTAs (two per SM
+  // sharing its shared memory) take it, at the cost of a key stage (3 -> 2),
+  // only when there can be enough units per CTA (the kernel checks the actual
+  // count).  FP8-key decode CTAs stay static: their sixth stage was worth more
+  // than the balance.
+  const int pct = (NEG == 1) ? (K8 ? 100 : kDecodeStaticPct) : kStaticPct;
+  const bool may_dyn = pct < 100 && max_units >= static_cast<int64_t>(kMinDynUnits) * grid;
+  const int static_pct = may_dyn ? pct : 100;
+  const int q_buffers = (NEG == 1 && !may_dyn) ? 1 : 2;
   const size_t fixed = 1024 /*align*/ + q_buffers * q_bytes +
                        8 * (2 * kMaxStages + 4 + 2 * kMaxAcc + 1) + 16 + 4 * (kThreads + 32) +
-                       4 * ((num_groups + 4) & ~3) + (NEG == 2 ? 16 + 16 * kRing : 0) + 64;
+                       4 * ((num_groups + 4) & ~3) + (static_pct < 100 ? 16 + 16 * kRing : 0) + 64;
   const size_t max_smem = device_max_smem_optin();
   const size_t budget = std::min((NEG == 1) ? (device_smem_per_sm() / 2 - 1024) : max_smem, max_smem);
   if (budget <= fixed) return DSA_ERR_UNSUPPORTED;
@@ -739,11 +755,6 @@ dsa_status_t launch_impl(const IndexerLaunch &a, cudaStream_t stream) {
                      cudaFuncAttributeMaxDynamicSharedMemorySize,
                      static_cast<int>(max_smem)) != cudaSuccess)
     return DSA_ERR_CUDA;
-  const int64_t max_keys = a.causal ? static_cast<int64_t>(a.q_pos0) + a.n_q : a.max_seq_len;
-  const int64_t max_units = static_cast<int64_t>(num_groups) * ((max_keys + kTileKeys - 1) / kTileKeys);
-  const int per_sm = (NEG == 1) ? 2 : 1;
-  const int grid = static_cast<int>(
-      std::max<int64_t>(1, std::min<int64_t>(static_cast<int64_t>(per_sm) * device_sm_count(), max_units)));
 
   IndexerParams p;
   p.w = a.w;
@@ -761,9 +772,7 @@ dsa_status_t launch_impl(const IndexerLaunch &a, cudaStream_t stream) {
   p.num_groups = num_groups;
   p.stages = stages;
   p.q_buffers = q_buffers;
-  // decode CTAs hold one query tile, so a chunk from another row would stall
-  // the MMA on its query: they keep to their static share (and have no ring)
-  p.static_pct = (NEG == 1) ? 100 : kStaticPct;
+  p.static_pct = static_pct;
   p.chunk = kDynChunk;
   p.wait_ns = wait_limit_ns();
   p.debug_stall = debug_stall() == kKernIndexer ? 1 : 0;
