@@ -430,10 +430,10 @@ TRAFFIC_COMMON = ["dsa_common.cuh", "dsa_internal.h"]
 TRAFFIC = {
     # (stage, workload): (bytes per launch, digest of the stage's sources); the
     # median of 19 launches of one capture per workload
-    ("indexer", "glm5_decode_b32_ragged"): (279655936, "f8125f23cea39844"),
-    ("indexer", "glm5_decode_8k"): (2157568, "f8125f23cea39844"),
-    ("indexer", "glm5_decode_4x128k"): (134903296, "f8125f23cea39844"),
-    ("indexer", "glm5_prefill_2300"): (19785728, "f8125f23cea39844"),
+    ("indexer", "glm5_decode_b32_ragged"): (279692032, "b4e568d9f9bf9440"),
+    ("indexer", "glm5_decode_8k"): (2165760, "b4e568d9f9bf9440"),
+    ("indexer", "glm5_decode_4x128k"): (134993664, "b4e568d9f9bf9440"),
+    ("indexer", "glm5_prefill_2300"): (19785728, "b4e568d9f9bf9440"),
     # topk_creg_kernel (32 rows, 4 x 131,072) and topk_small_kernel (8,192 keys, prefill rows)
     ("topk", "glm5_decode_b32_ragged"): (4351744, "6895ccb10040898d"),
     ("topk", "glm5_decode_8k"): (52224, "6895ccb10040898d"),
