@@ -229,7 +229,10 @@ DSA_API dsa_status_t dsa_attention_forward(const uint16_t *q_idx, const float *w
  * one small kernel each way, the SMs reading and writing them over the host
  * link (a copy-engine transfer costs microseconds of latency per buffer);
  * any other host buffer by its own cudaMemcpyAsync, which for pageable memory
- * waits for the host.  The call returns once everything is queued: the host
+ * waits for the host.  A mapped q_h (only the sparse MLA reads it) is copied
+ * by a spare warp of every indexer CTA while the keys are scanned, so that its
+ * transfer over the host link overlaps the scan.  The call returns once
+ * everything is queued: the host
  * results are valid after the stream has passed it (e.g. cudaStreamSynchronize).
  *   q_idx_h [n_q, H_I, D_I] bf16, w_h [n_q, H_I] fp32, q_h [n_q, H, R + P] bf16:
  *             host copies of dsa_attention_forward's inputs (any alignment)

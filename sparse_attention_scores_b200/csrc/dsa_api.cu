@@ -345,7 +345,9 @@ size_t ws_bytes_for(dsa_op_t op, const dsa_dims_t &d, const dsa_cache_t &c) {
 dsa_status_t run_indexer(const uint16_t *q_idx, const float *w, const uint16_t *k_pages,
                          const dsa_cache_t &c, const dsa_dims_t &d, float *scores, int64_t ld,
                          DevStatus *st, cudaStream_t s, const uint8_t *k8_pages = nullptr,
-                         const float *k_scale = nullptr, uint8_t *k8_region = nullptr) {
+                         const float *k_scale = nullptr, uint8_t *k8_region = nullptr,
+                         const void *aux_src = nullptr, void *aux_dst = nullptr,
+                         size_t aux_bytes = 0) {
   IndexerLaunch a;
   a.q_idx = q_idx;
   a.w = w;
@@ -373,6 +375,9 @@ dsa_status_t run_indexer(const uint16_t *q_idx, const float *w, const uint16_t *
   a.num_pages = c.num_pages;
   a.max_seq_len = c.max_seq_len;
   a.status = st;
+  a.aux_src = aux_src;
+  a.aux_dst = aux_dst;
+  a.aux_bytes = aux_bytes;
   return launch_indexer(a, s);
 }
 
@@ -458,7 +463,8 @@ dsa_status_t forward_entry(const uint16_t *q_idx, const float *w, const uint16_t
                            const uint16_t *latent_pages, const dsa_cache_t *cache,
                            const dsa_dims_t *dims, int32_t *idx_out, float *out, float *lse,
                            void *ws, size_t ws_bytes, dsa_stream_t stream,
-                           const uint8_t *latent8_pages = nullptr, const float *lat_scale = nullptr);
+                           const uint8_t *latent8_pages = nullptr, const float *lat_scale = nullptr,
+                           const void *q_src = nullptr, size_t q_copy_bytes = 0);
 
 }  // namespace
 }  // namespace dsa
@@ -663,7 +669,13 @@ dsa_status_t dsa_attention_forward_host(const uint16_t *q_idx_h, const float *w_
   };
   add(in, q_idx_h, q_idx, h.q_idx, q_idx_h, true);
   add(in, w_h, w, h.w, w_h, true);
-  add(in, q_h, q, h.q, q_h, true);
+  // The attention query (most of the input bytes) is read only by the MLA:
+  // from mapped host memory the indexer's copy warps move it while the keys
+  // are scanned, and the host link is otherwise idle
+  const void *q_mapped = mapped_host(q_h);
+  const bool q_by_indexer = q_mapped != nullptr && h.q % 16 == 0 &&
+                            (reinterpret_cast<uintptr_t>(q_mapped) & 15u) == 0;
+  if (!q_by_indexer) add(in, q_h, q, h.q, q_h, true);
   add(in, ch.seq_lens, seq_lens, h.seq_lens, ch.seq_lens, true);
   add(in, ch.block_table, block_table, h.block_table, ch.block_table, true);
   if (!ok) return DSA_ERR_CUDA;
@@ -672,7 +684,8 @@ dsa_status_t dsa_attention_forward_host(const uint16_t *q_idx_h, const float *w_
   cd.seq_lens = seq_lens;
   cd.block_table = block_table;
   DSA_TRY(forward_entry(q_idx, w, k_idx_pages, nullptr, nullptr, q, latent_pages, &cd, dims,
-                        idx_h ? idx : nullptr, out, lse, ws, fwd, stream));
+                        idx_h ? idx : nullptr, out, lse, ws, fwd, stream, nullptr, nullptr,
+                        q_by_indexer ? q_mapped : nullptr, h.q));
   if (idx_h) add(out_l, idx, idx_h, h.idx, idx_h, false);
   add(out_l, out, out_h, h.out, out_h, false);
   add(out_l, lse, lse_h, h.lse, lse_h, false);
@@ -801,7 +814,8 @@ dsa_status_t forward_entry(const uint16_t *q_idx, const float *w, const uint16_t
                            const uint16_t *latent_pages, const dsa_cache_t *cache,
                            const dsa_dims_t *dims, int32_t *idx_out, float *out, float *lse,
                            void *ws, size_t ws_bytes, dsa_stream_t stream,
-                           const uint8_t *latent8_pages, const float *lat_scale) {
+                           const uint8_t *latent8_pages, const float *lat_scale,
+                           const void *q_src, size_t q_copy_bytes) {
   DSA_TRY(check_dims_common(dims));
   DSA_TRY(check_indexer_dims(*dims));
   DSA_TRY(check_mla_dims(*dims));
@@ -837,8 +851,10 @@ dsa_status_t forward_entry(const uint16_t *q_idx, const float *w, const uint16_t
   int32_t *idx = idx_out ? idx_out : idx_ws;
   cudaStream_t s = as_stream(stream);
 
+  // q_src: the attention query is still to be copied into q (q_copy_bytes),
+  // which the indexer does under its key scan (bf16 keys only)
   DSA_TRY(run_indexer(q_idx, w, k_idx_pages, c, d, scores, ld, st, s, k8_pages, k_scale,
-                      k8_region));
+                      k8_region, q_src, const_cast<uint16_t *>(q), q_src ? q_copy_bytes : 0));
   DSA_TRY(run_topk(scores, ld, d.n_q, d.causal ? nullptr : c.seq_lens, d.q_pos0, d.topk, idx,
                    static_cast<int>(max_keys(d, c)), st, s));
   return run_mla(q, latent_pages, c, idx, d, out, lse, scratch, scratch_bytes, st, s,

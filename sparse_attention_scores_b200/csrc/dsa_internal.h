@@ -101,6 +101,13 @@ struct IndexerLaunch {
   int n_q, H_I, D_I, causal, q_pos0;
   int num_seqs, max_pages, num_pages, max_seq_len;
   DevStatus *status;
+  // bf16 keys only: a copy of aux_bytes (a multiple of 16, both ends 16-byte
+  // aligned) from aux_src (device-addressable, e.g. mapped host memory) to
+  // aux_dst, done by a spare warp of every CTA while the keys are scanned;
+  // complete when the indexer grid is
+  const void *aux_src = nullptr;
+  void *aux_dst = nullptr;
+  size_t aux_bytes = 0;
 };
 dsa_status_t launch_indexer(const IndexerLaunch &a, cudaStream_t stream);
 // the E4M3 query terms [2][n_q][H_I][D_I] and scaled weights [n_q][H_I] of the FP8-key indexer

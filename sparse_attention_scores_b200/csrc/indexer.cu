@@ -21,6 +21,8 @@
 //   warps 2+   epilogue warpgroups taking alternate tiles: tcgen05.ld of a
 //              128-lane accumulator, ReLU, head-weighted sum, coalesced fp32
 //              stores; up to 8 accumulators let the MMA run ahead
+//   last warp  (bf16 keys) an optional bulk copy that rides under the scan:
+//              the host-buffer step's attention query, over the host link
 // Decode runs two CTAs per SM (one epilogue warpgroup each) so that one CTA's
 // pipeline bubbles are covered by the other; grouped prefill runs one CTA per
 // SM with two epilogue warpgroups.
@@ -51,9 +53,10 @@ namespace dsa {
 namespace {
 
 // producer warp, MMA warp, NEG epilogue warpgroups (NEG = 2: one CTA per SM;
-// NEG = 1: two CTAs per SM, whose pipelines cover each other's bubbles)
-template <int NEG>
-__host__ __device__ constexpr int threads_of() { return 64 + 128 * NEG; }
+// NEG = 1: two CTAs per SM, whose pipelines cover each other's bubbles), and
+// for bf16 keys a copy warp (an optional bulk copy that runs under the scan)
+template <int NEG, bool K8>
+__host__ __device__ constexpr int threads_of() { return 64 + 128 * NEG + (K8 ? 0 : 32); }
 constexpr int kMaxStages = 8;
 constexpr int kMaxAcc = 8;         // accumulator buffers in tensor memory
 constexpr int kTileKeys = 128;
@@ -83,6 +86,11 @@ struct IndexerParams {
   // [0] next unit to hand out, [1] CTAs finished (zero between launches: the
   // last CTA to finish resets both; the workspace init zeroes them first)
   int *work;
+  // bf16 keys: copy n16 16-byte words from aux_src to aux_dst under the scan
+  // (the host-buffer step's attention query, read from mapped host memory)
+  const uint4 *aux_src;
+  uint4 *aux_dst;
+  int64_t aux_n16;
   DevStatus *status;
 };
 
@@ -115,10 +123,10 @@ __device__ __forceinline__ int locate(const int *tile_start, int ng, int u) {
 }
 
 template <int G, int AW, int NEG, bool K8>
-__global__ void __launch_bounds__(threads_of<NEG>(), NEG == 1 ? 2 : 1)
+__global__ void __launch_bounds__(threads_of<NEG, K8>(), NEG == 1 ? 2 : 1)
     indexer_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmQ,
                    const IndexerParams p) {
-  constexpr int kThreads = threads_of<NEG>();
+  constexpr int kThreads = threads_of<NEG, K8>();
   extern __shared__ uint8_t smem_raw[];
   uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                               ~static_cast<uintptr_t>(1023));
@@ -510,7 +518,7 @@ __global__ void __launch_bounds__(threads_of<NEG>(), NEG == 1 ? 2 : 1)
       mma_commit(drain);  // every MMA issued above has completed once this fires
       mbar_wait(drain, 0, kDrainLimitNs);
     }
-  } else {
+  } else if (warp < 2 + 4 * NEG) {
     // ------------------------------------------------------------ epilogue
     // two warpgroups take alternate tiles; within a group, warp w reads the
     // tensor-memory lane quadrant w % 4 (keys 32*quad .. 32*quad+31 of the tile)
@@ -635,6 +643,25 @@ __global__ void __launch_bounds__(threads_of<NEG>(), NEG == 1 ? 2 : 1)
       *abort_flag = 1u;
       report(p.status, kErrTimeout, (kKernIndexer << 24) | 0x3);
     }
+  } else {
+    // ------------------------------------------------------------ copy warp
+    // this CTA's share of the bulk copy, eight 16-byte loads in flight per
+    // lane (the source may be host memory across the host link)
+    const int64_t n = p.aux_n16;
+    const int64_t beg = (n * blockIdx.x) / gridDim.x, end = (n * (blockIdx.x + 1)) / gridDim.x;
+    for (int64_t i0 = beg; i0 < end; i0 += 32 * 8) {
+      uint4 v[8];
+#pragma unroll
+      for (int u = 0; u < 8; ++u) {
+        const int64_t i = i0 + u * 32 + lane;
+        if (i < end) v[u] = p.aux_src[i];
+      }
+#pragma unroll
+      for (int u = 0; u < 8; ++u) {
+        const int64_t i = i0 + u * 32 + lane;
+        if (i < end) p.aux_dst[i] = v[u];
+      }
+    }
   }
 
   tc_fence_before();
@@ -702,12 +729,17 @@ __global__ void __launch_bounds__(256) q8_prep_kernel(const uint16_t *q_idx, con
 // ---------------------------------------------------------------------------
 template <int G, int AW, int NEG, bool K8 = false>
 dsa_status_t launch_impl(const IndexerLaunch &a, cudaStream_t stream) {
-  constexpr int kThreads = threads_of<NEG>();
+  constexpr int kThreads = threads_of<NEG, K8>();
   constexpr int kEB = K8 ? 1 : 2;
   const int natoms = a.D_I * kEB / AW;
   const int ncols = G * a.H_I;
   const int n_mma = (ncols + 15) & ~15;
   const int num_groups = a.causal ? (a.n_q + G - 1) / G : a.n_q;
+  // the bulk copy rides on the bf16-key kernels' copy warp
+  if (a.aux_bytes != 0 &&
+      (K8 || a.aux_src == nullptr || a.aux_dst == nullptr || a.aux_bytes % 16 != 0 ||
+       ((reinterpret_cast<uintptr_t>(a.aux_src) | reinterpret_cast<uintptr_t>(a.aux_dst)) & 15u) != 0))
+    return DSA_ERR_INVALID_ARG;
   CUtensorMap tmK, tmQ;
   if (K8) {
     // byte keys [pages * 64 rows][D_I]; the query terms [2 * n_q * H_I rows][D_I]
@@ -779,6 +811,9 @@ dsa_status_t launch_impl(const IndexerLaunch &a, cudaStream_t stream) {
   p.k_scale = a.k_scale;
   p.status = a.status;
   p.work = reinterpret_cast<int *>(&a.status->pad[0]);
+  p.aux_src = static_cast<const uint4 *>(a.aux_src);
+  p.aux_dst = static_cast<uint4 *>(a.aux_dst);
+  p.aux_n16 = static_cast<int64_t>(a.aux_bytes / 16);
   if (launch_pdl(indexer_kernel<G, AW, NEG, K8>, dim3(grid), dim3(kThreads), smem, stream, 1, tmK, tmQ,
                  p) != cudaSuccess)
     return DSA_ERR_CUDA;
