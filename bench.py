@@ -430,21 +430,21 @@ TRAFFIC_COMMON = ["dsa_common.cuh", "dsa_internal.h"]
 TRAFFIC = {
     # (stage, workload): (bytes per launch, digest of the stage's sources); the
     # median of 19 launches of one capture per workload
-    ("indexer", "glm5_decode_b32_ragged"): (279692032, "b4e568d9f9bf9440"),
-    ("indexer", "glm5_decode_8k"): (2165760, "b4e568d9f9bf9440"),
-    ("indexer", "glm5_decode_4x128k"): (134993664, "b4e568d9f9bf9440"),
-    ("indexer", "glm5_prefill_2300"): (19785728, "b4e568d9f9bf9440"),
+    ("indexer", "glm5_decode_b32_ragged"): (279740928, "d1281380c8e49492"),
+    ("indexer", "glm5_decode_8k"): (2170624, "d1281380c8e49492"),
+    ("indexer", "glm5_decode_4x128k"): (134988288, "d1281380c8e49492"),
+    ("indexer", "glm5_prefill_2300"): (19788544, "d1281380c8e49492"),
     # topk_creg_kernel (32 rows, 4 x 131,072) and topk_small_kernel (8,192 keys, prefill rows)
-    ("topk", "glm5_decode_b32_ragged"): (4351744, "6895ccb10040898d"),
-    ("topk", "glm5_decode_8k"): (52224, "6895ccb10040898d"),
-    ("topk", "glm5_decode_4x128k"): (2121984, "6895ccb10040898d"),
-    ("topk", "glm5_prefill_2300"): (2234112, "6895ccb10040898d"),
+    ("topk", "glm5_decode_b32_ragged"): (4351488, "86581b1144701485"),
+    ("topk", "glm5_decode_8k"): (52224, "86581b1144701485"),
+    ("topk", "glm5_decode_4x128k"): (2122240, "86581b1144701485"),
+    ("topk", "glm5_prefill_2300"): (2234624, "86581b1144701485"),
     # mla_kernel + combine_kernel (the merge reads the split partials)
-    ("mla", "glm5_decode_8k"): (2508800 + 4232192, "571e9f8a5da9a90c"),
-    ("mla", "glm5_decode_4x128k"): (9864960 + 16864256, "571e9f8a5da9a90c"),
+    ("mla", "glm5_decode_8k"): (2508800 + 4231936, "5514fc61eba92590"),
+    ("mla", "glm5_decode_4x128k"): (9864704 + 16864256, "5514fc61eba92590"),
     # mla_pipe_kernel (rows merged inside clusters; prefill rows unsplit)
-    ("mla", "glm5_decode_b32_ragged"): (78309632, "571e9f8a5da9a90c"),
-    ("mla", "glm5_prefill_2300"): (425383680, "571e9f8a5da9a90c"),
+    ("mla", "glm5_decode_b32_ragged"): (78396672, "5514fc61eba92590"),
+    ("mla", "glm5_prefill_2300"): (425517312, "5514fc61eba92590"),
 }
 
 

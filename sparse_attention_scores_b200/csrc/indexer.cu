@@ -240,8 +240,10 @@ __global__ void __launch_bounds__(threads_of<NEG, K8>(), NEG == 1 ? 2 : 1)
   // the producer publishes each counter unit it issues (the i-th unit of the
   // CTA in uring[i % kRing]) and an end mark after the last.
   // (only with two query buffers, see the MMA issuer's group change, and
-  // enough units per CTA for chunks to pay for the counter's latency)
-  const bool dyn = p.static_pct < 100 && nqb == 2 &&
+  // enough units per CTA for chunks to pay for the counter's latency; never
+  // for FP8-key decode, whose kernel is then built without the counter paths)
+  constexpr bool kMayDyn = NEG == 2 || !K8;
+  const bool dyn = kMayDyn && p.static_pct < 100 && nqb == 2 &&
                    total >= kMinDynUnits * static_cast<int>(gridDim.x);
   const int st_total = static_cast<int>((static_cast<int64_t>(total) * min(p.static_pct, 100)) / 100);
   const int s0 = static_cast<int>((static_cast<int64_t>(st_total) * blockIdx.x) / gridDim.x);
