@@ -135,7 +135,11 @@ DSA_API const char *dsa_last_cuda_error(void);
 
 /* Bytes of device workspace `op` needs for these dims and cache.  Every
  * workspace starts with a 256-byte status block; the rest is scratch whose
- * contents are undefined between calls.  Returns 0 for invalid input. */
+ * contents are undefined between calls.  The status block also holds the
+ * indexer's work counter (CTAs take part of the key tiles from it), which
+ * every indexer launch leaves at zero: a workspace serves one call at a time,
+ * so calls that share one are queued on one stream.  Returns 0 for invalid
+ * input. */
 DSA_API size_t dsa_workspace_bytes(dsa_op_t op, const dsa_dims_t *dims, const dsa_cache_t *cache);
 
 /* Number of kernels one dsa_attention_forward (op = DSA_OP_ATTENTION_FORWARD),
