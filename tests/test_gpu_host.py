@@ -1,7 +1,7 @@
 """The whole step with host buffers (dsa_attention_forward_host) on the GPU:
 its results equal dsa_attention_forward's on the same inputs bit for bit (the
 same kernels run on copies of the same bytes), on two calls in a row through
-one workspace, and its selection equals the oracle's."""
+one workspace, and match the oracle (indices exactly, outputs within 2e-3)."""
 
 import numpy as np
 import pytest
@@ -10,7 +10,7 @@ import torch
 import dsa_inputs as di
 import sparse_attention_scores_b200 as dsa
 from oracle import dsa_oracle as orc
-from dsa_testutil import cache_of, dims_of, upload
+from dsa_testutil import assert_row_matches, cache_of, dims_of, upload
 
 pytestmark = pytest.mark.gpu
 
@@ -54,11 +54,12 @@ def test_host_buffers_equal_device_call(wl):
         assert torch.equal(idx_h, idx.cpu())
         assert torch.equal(out_h, out.cpu())
         assert torch.equal(lse_h, lse.cpu())
-    # and the selection is the oracle's
-    for b in (0, n - 1):
-        ref = orc.dsa_decode(inp, rows=[b])[b]["idx"] if wl.mode == "decode" else None
-        if ref is not None:
-            assert np.array_equal(idx_h[b].numpy().astype(np.int64), ref)
+    # and the host results are the oracle's (rows at both ends): indices exact,
+    # outputs and lse within the tolerances
+    rows = [0, n - 1]
+    ref = orc.dsa_decode(inp, rows=rows) if wl.mode == "decode" else orc.dsa_prefill(inp, rows=rows)
+    for r in rows:
+        assert_row_matches(r, ref[r], idx_h.numpy(), out_h.numpy(), lse_h.numpy())
     assert dsa.workspace_check(ws)[0] == 0
 
 
