@@ -11,7 +11,9 @@ decode (32 sequences, contexts 2,048-65,536, ragged paged caches), the largest
 workload that is a decode on one GPU; every other workload is measured too and
 reported under "per_config".  L2 is flushed (a 512 MB read) before every timed
 step; each step is timed with CUDA events on the launching stream; the same
-step with L2 left warm is reported as "hot".  Multi-GPU runs are independent
+step with L2 left warm is reported as "hot", and through the host-buffer entry
+point (inputs and results in pinned host memory) as "e2e", for the headline
+and every other bf16 workload.  Multi-GPU runs are independent
 replicas (weak scaling) timed as the max over ranks.
 
 `--impl reference` times the float64 CPU oracle on this host's cores on the
@@ -702,6 +704,11 @@ def run_ours(args):
             r = measure(c, torch, args.steps, args.warmup, flush_buf, peaks)
             r["us_per_step"] = max_over_ranks(r["us_per_step"], pg, "cuda")
             r["roofline"] = roofline_of(r, c.wl, peaks)
+            # the same workload through the host-buffer entry point
+            e = measure_e2e(c, torch, args.steps, args.warmup, flush_buf)
+            e["ms_per_step"] = max_over_ranks(e["ms_per_step"], pg, "cuda")
+            e["value"] = job_rows_per_s(c.wl.n_q, world, e["ms_per_step"])
+            r["e2e"] = e
             per_config[name] = r
             del c
             torch.cuda.empty_cache()
