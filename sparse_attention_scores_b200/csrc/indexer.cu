@@ -86,12 +86,15 @@ struct IndexerParams {
   // [0] next unit to hand out, [1] CTAs finished (zero between launches: the
   // last CTA to finish resets both; the workspace init zeroes them first)
   int *work;
-  // bf16 keys: copy n16 16-byte words from aux_src to aux_dst under the scan
-  // (the host-buffer step's attention query, read from mapped host memory)
-  const uint4 *aux_src;
-  uint4 *aux_dst;
-  int64_t aux_n16;
   DevStatus *status;
+};
+
+// bf16 keys: copy n16 16-byte words from src to dst under the scan (the
+// host-buffer step's attention query, read from mapped host memory)
+struct AuxCopy {
+  const uint4 *src;
+  uint4 *dst;
+  int64_t n16;
 };
 
 // Tokens a row group must score (the longest row of the group).
@@ -125,7 +128,7 @@ __device__ __forceinline__ int locate(const int *tile_start, int ng, int u) {
 template <int G, int AW, int NEG, bool K8>
 __global__ void __launch_bounds__(threads_of<NEG, K8>(), NEG == 1 ? 2 : 1)
     indexer_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmQ,
-                   const IndexerParams p) {
+                   const IndexerParams p, const __grid_constant__ AuxCopy aux) {
   constexpr int kThreads = threads_of<NEG, K8>();
   extern __shared__ uint8_t smem_raw[];
   uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
@@ -520,8 +523,9 @@ __global__ void __launch_bounds__(threads_of<NEG, K8>(), NEG == 1 ? 2 : 1)
       mma_commit(drain);  // every MMA issued above has completed once this fires
       mbar_wait(drain, 0, kDrainLimitNs);
     }
-  } else if (warp < 2 + 4 * NEG) {
+  } else if (K8 || warp < 2 + 4 * NEG) {
     // ------------------------------------------------------------ epilogue
+    // (the FP8-key kernels have no copy warp, and are built without its code)
     // two warpgroups take alternate tiles; within a group, warp w reads the
     // tensor-memory lane quadrant w % 4 (keys 32*quad .. 32*quad+31 of the tile)
     const int quad = warp & 3;
@@ -649,19 +653,21 @@ __global__ void __launch_bounds__(threads_of<NEG, K8>(), NEG == 1 ? 2 : 1)
     // ------------------------------------------------------------ copy warp
     // this CTA's share of the bulk copy, eight 16-byte loads in flight per
     // lane (the source may be host memory across the host link)
-    const int64_t n = p.aux_n16;
-    const int64_t beg = (n * blockIdx.x) / gridDim.x, end = (n * (blockIdx.x + 1)) / gridDim.x;
-    for (int64_t i0 = beg; i0 < end; i0 += 32 * 8) {
-      uint4 v[8];
+    if constexpr (!K8) {
+      const int64_t n = aux.n16;
+      const int64_t beg = (n * blockIdx.x) / gridDim.x, end = (n * (blockIdx.x + 1)) / gridDim.x;
+      for (int64_t i0 = beg; i0 < end; i0 += 32 * 8) {
+        uint4 v[8];
 #pragma unroll
-      for (int u = 0; u < 8; ++u) {
-        const int64_t i = i0 + u * 32 + lane;
-        if (i < end) v[u] = p.aux_src[i];
-      }
+        for (int u = 0; u < 8; ++u) {
+          const int64_t i = i0 + u * 32 + lane;
+          if (i < end) v[u] = aux.src[i];
+        }
 #pragma unroll
-      for (int u = 0; u < 8; ++u) {
-        const int64_t i = i0 + u * 32 + lane;
-        if (i < end) p.aux_dst[i] = v[u];
+        for (int u = 0; u < 8; ++u) {
+          const int64_t i = i0 + u * 32 + lane;
+          if (i < end) aux.dst[i] = v[u];
+        }
       }
     }
   }
@@ -813,11 +819,12 @@ dsa_status_t launch_impl(const IndexerLaunch &a, cudaStream_t stream) {
   p.k_scale = a.k_scale;
   p.status = a.status;
   p.work = reinterpret_cast<int *>(&a.status->pad[0]);
-  p.aux_src = static_cast<const uint4 *>(a.aux_src);
-  p.aux_dst = static_cast<uint4 *>(a.aux_dst);
-  p.aux_n16 = static_cast<int64_t>(a.aux_bytes / 16);
+  AuxCopy aux;
+  aux.src = static_cast<const uint4 *>(a.aux_src);
+  aux.dst = static_cast<uint4 *>(a.aux_dst);
+  aux.n16 = static_cast<int64_t>(a.aux_bytes / 16);
   if (launch_pdl(indexer_kernel<G, AW, NEG, K8>, dim3(grid), dim3(kThreads), smem, stream, 1, tmK, tmQ,
-                 p) != cudaSuccess)
+                 p, aux) != cudaSuccess)
     return DSA_ERR_CUDA;
   return DSA_OK;
 }
