@@ -432,10 +432,10 @@ TRAFFIC_COMMON = ["dsa_common.cuh", "dsa_internal.h"]
 TRAFFIC = {
     # (stage, workload): (bytes per launch, digest of the stage's sources); the
     # median of 19 launches of one capture per workload
-    ("indexer", "glm5_decode_b32_ragged"): (279740928, "d1281380c8e49492"),
-    ("indexer", "glm5_decode_8k"): (2170624, "d1281380c8e49492"),
-    ("indexer", "glm5_decode_4x128k"): (134988288, "d1281380c8e49492"),
-    ("indexer", "glm5_prefill_2300"): (19788544, "d1281380c8e49492"),
+    ("indexer", "glm5_decode_b32_ragged"): (279734528, "fc474a6e2ffc96b0"),
+    ("indexer", "glm5_decode_8k"): (2168576, "fc474a6e2ffc96b0"),
+    ("indexer", "glm5_decode_4x128k"): (135001344, "fc474a6e2ffc96b0"),
+    ("indexer", "glm5_prefill_2300"): (19788288, "fc474a6e2ffc96b0"),
     # topk_creg_kernel (32 rows, 4 x 131,072) and topk_small_kernel (8,192 keys, prefill rows)
     ("topk", "glm5_decode_b32_ragged"): (4351488, "86581b1144701485"),
     ("topk", "glm5_decode_8k"): (52224, "86581b1144701485"),
